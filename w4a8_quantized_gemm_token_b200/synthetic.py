@@ -1,0 +1,83 @@
+"""Seeded synthetic inputs for the quantized linear (DiT layer shapes).
+
+This module only draws random numbers: it holds none of the quantization or
+matmul arithmetic, so both the CUDA path and the CPU oracle can take their
+inputs from it.  Recipe (one ``numpy.random.default_rng(seed)`` per case, in
+this draw order):
+
+1. x: float64 standard normals of shape [M, K].  If ``outlier_frac`` > 0,
+   ``round(outlier_frac * K)`` distinct channels are drawn without replacement
+   and multiplied by ``outlier_scale`` (DiT activations carry a few large
+   channels).  Then x is cast to float32 and rounded to bf16 (nearest-even).
+2. W: float64 normals times ``w_std`` of shape [N, K], cast to float32.
+3. bias (when requested): float64 normals times ``b_std`` of shape [N], float32.
+
+bf16 arrays are returned as numpy uint16 bit patterns.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 to bf16 (nearest, ties to even) and return the bit patterns.
+
+    torch's CPU cast does the rounding; it is only used to make the input tensor.
+    """
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclass
+class LinearCase:
+    name: str
+    M: int
+    K: int
+    N: int
+    x_std: float = 1.0
+    outlier_frac: float = 0.0
+    outlier_scale: float = 20.0
+    w_std: float = 0.02
+    bias: bool = True
+    b_std: float = 0.1
+    seed: int = 0
+    extra: dict = field(default_factory=dict)
+
+    def draw(self):
+        """Return (x bf16 bits [M,K], W float32 [N,K], bias float32 [N] or None, outlier channels)."""
+        rng = np.random.default_rng(self.seed)
+        x = rng.standard_normal((self.M, self.K)) * self.x_std
+        chans = np.empty(0, np.int64)
+        if self.outlier_frac > 0:
+            n_out = int(round(self.outlier_frac * self.K))
+            chans = np.sort(rng.choice(self.K, size=n_out, replace=False))
+            x[:, chans] *= self.outlier_scale
+        x_bf16 = f32_to_bf16_bits(x.astype(np.float32))
+        del x
+        W = (rng.standard_normal((self.N, self.K)) * self.w_std).astype(np.float32)
+        b = None
+        if self.bias:
+            b = (rng.standard_normal(self.N) * self.b_std).astype(np.float32)
+        return x_bf16, W, b, chans
+
+
+# The five workloads of the quantized linear, at DiT layer shapes.
+TINY = LinearCase("tiny_w8a8_64x256x128", M=64, K=256, N=128)
+DIT_ATTN = LinearCase("dit_attn_proj_w8a8_4096x3072x3072", M=4096, K=3072, N=3072,
+                      outlier_frac=0.01)
+SWEEP = [
+    LinearCase("sweep_w8a8_2048x4096x4096", M=2048, K=4096, N=4096),
+    LinearCase("sweep_w8a8_2048x4096x12288", M=2048, K=4096, N=12288),
+    LinearCase("sweep_w8a8_2048x12288x4096", M=2048, K=12288, N=4096),
+    LinearCase("sweep_w8a8_2048x5120x48_thin", M=2048, K=5120, N=48),
+]
+DIT_MLP = LinearCase("dit_mlp_w8a8_16384x3072x12288", M=16384, K=3072, N=12288,
+                     outlier_frac=0.01)
+W4A8 = [LinearCase(f"w4a8_g64_{m}x4096x4096", M=m, K=4096, N=4096, bias=False)
+        for m in (1, 8, 16, 4096)]
+
+ALL_W8A8 = [TINY, DIT_ATTN, *SWEEP, DIT_MLP]
