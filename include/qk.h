@@ -1,0 +1,250 @@
+/*
+ * qk.h -- C ABI of libqk, the B200 (sm_100a) W8A8 / W4A8 quantized linear.
+ *
+ * What it computes (by page and section of the sources):
+ *   - "qlip-mlx" README, intro bullet "w8a8_linear / W8A8Linear": a linear
+ *     layer whose activations are quantized per token to int8 on the fly, whose
+ *     weights are quantized offline to int8, an INT8 x INT8 -> INT32 matmul,
+ *     and a dequant + bias step fused behind it.
+ *   - same page, "Quick start" -> "Use it from Python": quantize_weight_int8
+ *     turns an [N, K] weight into int8 codes plus fp32 per-output-channel
+ *     scales; w8a8_linear(x, w_i8, sw, bias) runs the layer.
+ *   - same page, intro bullet "w4a8_linear / W4A8Linear": the same int8 compute
+ *     with the weight stored as packed 4-bit codes, and a separate path for
+ *     M <= 16 rows that runs at weight-bandwidth speed.
+ *   - "MLX PR #4722" (int8-staged quantized matmul), "Selector rules": affine
+ *     4-bit weights with group size 64 along K, K % 64 == 0, K <= 65536.
+ *
+ * Conventions for every call:
+ *   - Matrices are row-major.  x is [M, K] (M tokens, K in-features), a weight
+ *     is [N, K] (N out-features; the nn.Linear orientation), y is [M, N].
+ *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ *   - Every pointer is DEVICE memory on the current CUDA device, owned by the
+ *     caller.  The library keeps no pointer after a call returns.
+ *   - Calls are asynchronous and ordered on `stream` (NULL = the legacy
+ *     default stream).  They are deterministic: the same inputs give the same
+ *     bits.  The caller must not modify inputs or read outputs until the stream
+ *     has reached the call.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns an error code and leaves every output untouched.  A launch
+ *     failure returns QK_ERR_CUDA.  Kernels never trap: a kernel wait that
+ *     gives up records QK_ERR_TIMEOUT in a per-device error word, read by
+ *     qk_check_device_error.
+ *   - Inputs must be finite.  Activation rows whose absmax lies in (0, 2^-121)
+ *     are outside the contract (127 / absmax overflows fp32).
+ *   - Pointer alignment: matrices (x, xq, Wq, Wp, wscale, woffset, xsum, y) and
+ *     the workspace need 16-byte alignment; sx, sw and bias need 16 bytes too
+ *     (the kernels read them as 16-byte vectors).
+ */
+#ifndef QK_H
+#define QK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (a CUDA stream handle); NULL is the legacy stream. */
+typedef struct CUstream_st *qk_stream_t;
+
+typedef enum {
+    QK_OK = 0,
+    QK_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad route    */
+    QK_ERR_UNSUPPORTED_SHAPE = 2, /* K or N outside the shape contract         */
+    QK_ERR_MISALIGNED = 3,        /* a pointer breaks the alignment rule       */
+    QK_ERR_NO_DEVICE = 4,         /* no CUDA device, or it is not sm_100       */
+    QK_ERR_WORKSPACE = 5,         /* workspace too small or misaligned         */
+    QK_ERR_CUDA = 6,              /* a CUDA runtime call or launch failed      */
+    QK_ERR_TIMEOUT = 7            /* a kernel wait gave up (device error word) */
+} qk_status;
+
+/* Routes of the W4A8 product. */
+typedef enum {
+    QK_ROUTE_AUTO = 0, /* GEMV when M <= 16, else GEMM                        */
+    QK_ROUTE_GEMM = 1, /* tensor-core GEMM (tcgen05), any M                   */
+    QK_ROUTE_GEMV = 2  /* weight-streaming GEMV, M <= 16 only                 */
+} qk_route;
+
+/* Static string for a status code (never NULL). */
+const char *qk_status_string(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+int qk_version(void);
+
+/* 1 if `device` exists and is compute capability 10.0 (B200, sm_100a), else 0.
+ * Never fails: a missing driver or device gives 0.  (The qlip-mlx README,
+ * "Key features": is_available() reports False where the INT8 path cannot run.) */
+int qk_is_available(int device);
+
+/*
+ * Shape contract (qk_w8a8_*): 1 <= K <= 65536 with K % 32 == 0; N >= 8 with
+ * N % 8 == 0; M >= 0 (M == 0 returns QK_OK and launches nothing).
+ * W4A8 (qk_w4a8_*, qk_quantize_weights_int4): additionally K % 64 == 0.
+ * A shape outside the contract returns QK_ERR_UNSUPPORTED_SHAPE.
+ */
+
+/* ------------------------------------------------------------- workspace */
+
+/* Bytes of workspace qk_w8a8_linear needs: int8 codes [M, K] and fp32 scales
+ * [M], each 256-byte aligned inside the block. */
+size_t qk_w8a8_workspace_size(int64_t M, int64_t K);
+
+/* Bytes of workspace qk_w4a8_linear needs: codes [M, K], scales [M] and int32
+ * group sums [M, K/64]. */
+size_t qk_w4a8_workspace_size(int64_t M, int64_t K);
+
+/* ------------------------------------------------------ offline weights */
+
+/*
+ * W8 weight quantization ("qlip-mlx" README, "Use it from Python":
+ * quantize_weight_int8, [N, K] -> int8 + fp32 scales).  Per output channel n:
+ * sw[n] = absmax_k |W[n,k]| / 127 and Wq[n,k] = round-half-even(W[n,k] *
+ * (127 / absmax)) clamped to [-127, 127]; an all-zero row gets sw = 1 and zero
+ * codes.  All arithmetic is IEEE fp32.
+ *   W  : fp32 [N, K]          (in)
+ *   Wq : int8 [N, K]          (out)
+ *   sw : fp32 [N]             (out)
+ */
+qk_status qk_quantize_weights_int8(const float *W, int64_t N, int64_t K,
+                                   int8_t *Wq, float *sw, qk_stream_t stream);
+
+/*
+ * W4 affine group-64 quantization ("qlip-mlx" README, "w4a8_linear"; "MLX PR
+ * #4722", "Selector rules").  Per row n and group g of 64 consecutive k: lo =
+ * min, hi = max, wscale = fp16((hi - lo) / 15), woffset = fp16(lo); codes
+ * q = round-half-even((W - float(woffset)) * (1 / float(wscale))) clamped to
+ * [0, 15] (all zero when wscale == 0).  The dequantized weight is
+ * q * wscale + woffset.  Two codes per byte: k = 2j in the low nibble of byte
+ * j, k = 2j + 1 in the high nibble.  |W| must stay below 65504 (fp16 range).
+ *   W       : fp32 [N, K]                (in)
+ *   Wp      : uint8 [N, K/2]             (out)
+ *   wscale  : fp16 bits [N, K/64]        (out)
+ *   woffset : fp16 bits [N, K/64]        (out)
+ */
+qk_status qk_quantize_weights_int4(const float *W, int64_t N, int64_t K,
+                                   uint8_t *Wp, uint16_t *wscale, uint16_t *woffset,
+                                   qk_stream_t stream);
+
+/* ----------------------------------------------------- activation quant */
+
+/*
+ * Per-token dynamic symmetric int8 quantization ("qlip-mlx" README,
+ * "w8a8_linear": activations quantized dynamically, no calibration; "MLX PR
+ * #4722", "SIMD fix": x quantized by a kernel of its own).  Per row m:
+ * sx[m] = absmax / 127, xq = round-half-even(x * (127 / absmax)) clamped to
+ * [-127, 127] (fp32 arithmetic); an all-zero row gets sx = 1, codes 0.
+ * If xsum is not NULL (needs K % 64 == 0) it also writes the int32 sums of the
+ * codes over each group of 64: xsum[m, g] = sum_{k = 64g}^{64g+63} xq[m, k].
+ *   x    : bf16 bits [M, K]  (in)
+ *   xq   : int8 [M, K]       (out)
+ *   sx   : fp32 [M]          (out)
+ *   xsum : int32 [M, K/64]   (out, nullable)
+ */
+qk_status qk_quantize_activations(const uint16_t *x, int64_t M, int64_t K,
+                                  int8_t *xq, float *sx, int32_t *xsum,
+                                  qk_stream_t stream);
+
+/* ------------------------------------------------------------ W8A8 linear */
+
+/*
+ * The W8A8 linear ("qlip-mlx" README, "w8a8_linear / W8A8Linear"):
+ *   y[m, n] = bf16( acc[m, n] * sx[m] * sw[n] + bias[n] ),
+ *   acc[m, n] = sum_k xq[m, k] * Wq[n, k]  (exact int32),
+ * where xq, sx are the per-token quantization of x (qk_quantize_activations).
+ * The dequant is evaluated in fp64 and rounded once to bf16 (nearest even).
+ *   x         : bf16 bits [M, K]   (in)
+ *   Wq, sw    : from qk_quantize_weights_int8 (in)
+ *   bias      : fp32 [N] (in, nullable: no bias)
+ *   y         : bf16 bits [M, N]   (out)
+ *   workspace : device scratch of ws_bytes >= qk_w8a8_workspace_size(M, K),
+ *               or NULL: the call then allocates it stream-ordered
+ *               (cudaMallocAsync / cudaFreeAsync on `stream`).
+ */
+qk_status qk_w8a8_linear(const uint16_t *x, int64_t M, int64_t K,
+                         const int8_t *Wq, const float *sw, const float *bias, int64_t N,
+                         uint16_t *y, void *workspace, size_t ws_bytes,
+                         qk_stream_t stream);
+
+/*
+ * The matmul + dequant half of qk_w8a8_linear, on activations that are already
+ * quantized (xq, sx from qk_quantize_activations).  Lets one quantization feed
+ * several projections of the same input.
+ */
+qk_status qk_w8a8_gemm(const int8_t *xq, const float *sx, int64_t M, int64_t K,
+                       const int8_t *Wq, const float *sw, const float *bias, int64_t N,
+                       uint16_t *y, qk_stream_t stream);
+
+/* ------------------------------------------------------------ W4A8 linear */
+
+/*
+ * The W4A8 linear ("qlip-mlx" README, "w4a8_linear / W4A8Linear"; weights in
+ * the affine group-64 format of qk_quantize_weights_int4).  With G = K / 64,
+ * the dequantized weight q * s + o and the dequantized activation xq * sx:
+ *   acc[m, n, g] = sum_{k in group g} xq[m, k] * q[n, k]    (exact int32)
+ *   y[m, n] = bf16( sx[m] * sum_g ( s[n,g] * acc[m,n,g] + o[n,g] * xsum[m,g] )
+ *                   + bias[n] ),
+ * the fold evaluated in fp64 and rounded once to bf16.
+ * M <= 16 takes the weight-streaming GEMV, larger M the tensor-core GEMM; both
+ * compute the same per-group integers and agree to the fp64 rounding order.
+ *   x                  : bf16 bits [M, K]            (in)
+ *   Wp, wscale, woffset: from qk_quantize_weights_int4 (in)
+ *   bias               : fp32 [N] (nullable)
+ *   y                  : bf16 bits [M, N]            (out)
+ *   workspace          : >= qk_w4a8_workspace_size(M, K) bytes, or NULL
+ *                        (stream-ordered allocation as in qk_w8a8_linear).
+ */
+qk_status qk_w4a8_linear(const uint16_t *x, int64_t M, int64_t K,
+                         const uint8_t *Wp, const uint16_t *wscale, const uint16_t *woffset,
+                         const float *bias, int64_t N,
+                         uint16_t *y, void *workspace, size_t ws_bytes,
+                         qk_stream_t stream);
+
+/*
+ * The product half of qk_w4a8_linear on quantized activations (xq, sx and
+ * xsum from qk_quantize_activations), with an explicit route (qk_route).
+ * QK_ROUTE_GEMV with M > 16 returns QK_ERR_INVALID_ARG.
+ */
+qk_status qk_w4a8_gemm(const int8_t *xq, const float *sx, const int32_t *xsum,
+                       int64_t M, int64_t K,
+                       const uint8_t *Wp, const uint16_t *wscale, const uint16_t *woffset,
+                       const float *bias, int64_t N, uint16_t *y, int route,
+                       qk_stream_t stream);
+
+/* ---------------------------------------------------------------- errors */
+
+/*
+ * Synchronizes `stream`, then reads and clears this device's error word.
+ * Returns QK_ERR_TIMEOUT if a kernel wait gave up since the last check,
+ * QK_ERR_CUDA if the synchronization failed, else QK_OK.
+ */
+qk_status qk_check_device_error(qk_stream_t stream);
+
+/* ------------------------------------------------------------ test hooks */
+
+/*
+ * The W8A8 GEMM mainloop with an epilogue that stores the raw int32
+ * accumulators: acc[m, n] = sum_k xq[m, k] * Wq[n, k], acc int32 [M, N].
+ * Same kernel, tiles and schedule as qk_w8a8_gemm.
+ */
+qk_status qk_debug_w8a8_acc(const int8_t *xq, int64_t M, int64_t K,
+                            const int8_t *Wq, int64_t N, int32_t *acc,
+                            qk_stream_t stream);
+
+/*
+ * The per-group int32 accumulators of the W4A8 product for rows [m0, m1):
+ * acc[(m - m0), n, g] = sum_{k in group g} xq[m, k] * q[n, k], acc int32
+ * [m1 - m0, N, K/64], computed by the mainloop of `route` (QK_ROUTE_GEMM or
+ * QK_ROUTE_GEMV; GEMV needs M <= 16).  xq is the full [M, K] matrix.
+ */
+qk_status qk_debug_w4a8_group_acc(const int8_t *xq, int64_t M, int64_t K,
+                                  const uint8_t *Wp, int64_t N,
+                                  int64_t m0, int64_t m1, int32_t *acc,
+                                  int route, qk_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QK_H */

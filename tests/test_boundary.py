@@ -1,0 +1,111 @@
+"""The C-ABI boundary on the CPU: the library loads without a GPU, exports every
+function include/qk.h declares, and rejects bad arguments on the host with the
+documented status codes before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def qk():
+    from w4a8_quantized_gemm_token_b200 import build
+
+    build.build()
+    from w4a8_quantized_gemm_token_b200 import binding
+
+    return binding
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "qk.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qk_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("qk_quantize_weights_int8", "qk_quantize_weights_int4", "qk_quantize_activations",
+              "qk_w8a8_linear", "qk_w4a8_linear", "qk_check_device_error", "qk_is_available"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(qk):
+    for n in declared_functions():
+        assert hasattr(qk.lib, n), n
+
+
+def test_status_strings(qk):
+    for s in range(8):
+        assert qk.qk_status_string(s).startswith("QK_")
+    assert "unknown" in qk.qk_status_string(99)
+
+
+def test_workspace_sizes(qk):
+    r = lambda b: (b + 255) // 256 * 256
+    assert qk.qk_w8a8_workspace_size(16384, 3072) == r(16384 * 3072) + r(16384 * 4)
+    assert qk.qk_w4a8_workspace_size(17, 4096) == r(17 * 4096) + r(17 * 4) + r(17 * 64 * 4)
+    assert qk.qk_w8a8_workspace_size(0, 256) == 0
+
+
+FAKE = 1 << 20  # a 16-byte aligned, never dereferenced address
+
+
+def call_w8a8(qk, x=FAKE, M=64, K=256, Wq=FAKE, sw=FAKE, bias=None, N=128, y=FAKE,
+              ws=None, ws_bytes=0):
+    return qk.lib.qk_w8a8_linear(x, M, K, Wq, sw, bias, N, y, ws, ws_bytes, None)
+
+
+def test_shape_contract(qk):
+    assert call_w8a8(qk, K=33) == 2
+    assert call_w8a8(qk, K=16) == 2
+    assert call_w8a8(qk, K=65536 + 32) == 2
+    assert call_w8a8(qk, N=12) == 2
+    assert call_w8a8(qk, N=0) == 2
+    assert call_w8a8(qk, M=-1) == 1
+    # W4A8 needs K % 64 == 0
+    assert qk.lib.qk_w4a8_linear(FAKE, 8, 96, FAKE, FAKE, FAKE, None, 64, FAKE, None, 0, None) == 2
+
+
+def test_empty_input_is_a_no_op(qk):
+    assert call_w8a8(qk, M=0, x=None, y=None) == 0
+    assert qk.lib.qk_quantize_activations(None, 0, 64, None, None, None, None) == 0
+
+
+def test_null_and_misaligned_pointers(qk):
+    assert call_w8a8(qk, x=None) == 1
+    assert call_w8a8(qk, Wq=None) == 1
+    assert call_w8a8(qk, y=FAKE + 8) == 3
+    assert call_w8a8(qk, bias=FAKE + 4) == 3
+    assert qk.lib.qk_quantize_activations(FAKE + 2, 4, 64, FAKE, FAKE, None, None) == 3
+
+
+def test_routes_are_checked(qk):
+    args = (FAKE, FAKE, FAKE, 32, 256, FAKE, FAKE, FAKE, None, 64, FAKE)
+    assert qk.lib.qk_w4a8_gemm(*args, 2, None) == 1        # GEMV with M > 16
+    assert qk.lib.qk_w4a8_gemm(*args, 7, None) == 1        # unknown route
+    assert qk.lib.qk_debug_w4a8_group_acc(FAKE, 8, 256, FAKE, 64, 4, 2, FAKE, 1, None) == 1
+
+
+def test_no_device_here(qk):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert qk.qk_is_available(0) is False
+    # valid arguments reach the device check and stop there, launching nothing
+    assert call_w8a8(qk) == 4
+    assert qk.lib.qk_quantize_weights_int8(FAKE, 128, 256, FAKE, FAKE, None) == 4
+
+
+def test_binding_rejects_cpu_tensors(qk):
+    import torch
+
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        qk.qk_quantize_activations(x)
+    with pytest.raises(TypeError):
+        qk.qk_quantize_activations(x.float())

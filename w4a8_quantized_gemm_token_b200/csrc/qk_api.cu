@@ -1,0 +1,390 @@
+// qk_api.cu -- the C ABI of include/qk.h: argument checks, device checks,
+// workspace carving and the kernel launches.  All checks run on the host before
+// any launch; nothing here computes on the CPU.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "qk.h"
+#include "qk_internal.h"
+
+namespace qk {
+
+// The device error word (see sm100.cuh).  One per device: every device that
+// loads the library's module has its own copy.
+__device__ int g_qk_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+int g_cc_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+int* g_err_ptr[kMaxDevices];
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool log_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("QK_LOG");
+    return v != nullptr && v[0] == '1';
+  }();
+  return on;
+}
+
+int current_device() {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t b) { return (b + 255u) & ~size_t(255u); }
+
+// Shape contract shared by every product call.
+qk_status check_shape(int64_t M, int64_t K, int64_t N, bool w4) {
+  if (M < 0 || K < 0 || N < 0) return QK_ERR_INVALID_ARG;
+  if (M > INT32_MAX || N > INT32_MAX) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (K < 32 || K > 65536 || K % 32 != 0) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (w4 && K % 64 != 0) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (N < 8 || N % 8 != 0) return QK_ERR_UNSUPPORTED_SHAPE;
+  return QK_OK;
+}
+
+qk_status check_device() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return QK_ERR_NO_DEVICE;
+  if (g_cc_ok[d] == 0) g_cc_ok[d] = qk_is_available(d) ? 1 : -1;
+  return g_cc_ok[d] == 1 ? QK_OK : QK_ERR_NO_DEVICE;
+}
+
+qk_status from_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return QK_OK;
+  if (log_enabled()) std::fprintf(stderr, "[qk] %s: %s\n", what, cudaGetErrorString(e));
+  return QK_ERR_CUDA;
+}
+
+// Carves xq / sx / xsum out of a workspace block, allocating it stream-ordered
+// when the caller passes none.
+struct Workspace {
+  int8_t* xq = nullptr;
+  float* sx = nullptr;
+  int32_t* xsum = nullptr;
+  void* owned = nullptr;
+  cudaStream_t stream = nullptr;
+
+  qk_status init(void* ws, size_t ws_bytes, int64_t M, int64_t K, bool w4, cudaStream_t s) {
+    const size_t need = w4 ? qk_w4a8_workspace_size(M, K) : qk_w8a8_workspace_size(M, K);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    if (base == nullptr) {
+      cudaError_t e = cudaMallocAsync(&owned, need, s);
+      if (e != cudaSuccess) return from_cuda(e, "cudaMallocAsync(workspace)");
+      stream = s;
+      base = static_cast<uint8_t*>(owned);
+    } else if (ws_bytes < need || (reinterpret_cast<uintptr_t>(base) & 255u) != 0) {
+      return QK_ERR_WORKSPACE;
+    }
+    xq = reinterpret_cast<int8_t*>(base);
+    sx = reinterpret_cast<float*>(base + round256((size_t)M * (size_t)K));
+    if (w4) xsum = reinterpret_cast<int32_t*>(base + round256((size_t)M * (size_t)K) +
+                                               round256((size_t)M * 4u));
+    return QK_OK;
+  }
+  ~Workspace() {
+    if (owned != nullptr) cudaFreeAsync(owned, stream);
+  }
+};
+
+}  // namespace
+
+int* device_error_word() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  if (g_err_ptr[d] == nullptr) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_err_ptr[d] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_qk_error) != cudaSuccess) return nullptr;
+      g_err_ptr[d] = static_cast<int*>(p);
+    }
+  }
+  return g_err_ptr[d];
+}
+
+int num_sms() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 1;
+  if (g_sm_count[d] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    g_sm_count[d] = n > 0 ? n : 1;
+  }
+  return g_sm_count[d];
+}
+
+bool encode_tmap_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* base,
+                    uint64_t inner, uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
+                    uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(out, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace qk
+
+using namespace qk;
+
+extern "C" {
+
+const char* qk_status_string(int status) {
+  switch (status) {
+    case QK_OK: return "QK_OK";
+    case QK_ERR_INVALID_ARG: return "QK_ERR_INVALID_ARG: null pointer, negative size or bad route";
+    case QK_ERR_UNSUPPORTED_SHAPE: return "QK_ERR_UNSUPPORTED_SHAPE: K or N outside the shape contract";
+    case QK_ERR_MISALIGNED: return "QK_ERR_MISALIGNED: a pointer is not 16-byte aligned";
+    case QK_ERR_NO_DEVICE: return "QK_ERR_NO_DEVICE: no CUDA device, or not sm_100";
+    case QK_ERR_WORKSPACE: return "QK_ERR_WORKSPACE: workspace too small or not 256-byte aligned";
+    case QK_ERR_CUDA: return "QK_ERR_CUDA: a CUDA call or kernel launch failed";
+    case QK_ERR_TIMEOUT: return "QK_ERR_TIMEOUT: a kernel wait gave up";
+    default: return "unknown qk_status";
+  }
+}
+
+int qk_version(void) { return (0 << 16) | 1; }
+
+int qk_is_available(int device) {
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || device < 0 || device >= n) {
+    cudaGetLastError();
+    return 0;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess)
+    return 0;
+  return (major == 10 && minor == 0) ? 1 : 0;
+}
+
+size_t qk_w8a8_workspace_size(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return 0;
+  return round256((size_t)M * (size_t)K) + round256((size_t)M * 4u);
+}
+
+size_t qk_w4a8_workspace_size(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return 0;
+  return qk_w8a8_workspace_size(M, K) + round256((size_t)M * (size_t)(K / 64) * 4u);
+}
+
+qk_status qk_quantize_weights_int8(const float* W, int64_t N, int64_t K, int8_t* Wq, float* sw,
+                                   qk_stream_t stream) {
+  if (N < 0 || K < 0) return QK_ERR_INVALID_ARG;
+  if (K < 32 || K > 65536 || K % 32 != 0 || N > INT32_MAX) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0) return QK_OK;
+  if (!W || !Wq || !sw) return QK_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wq) || !aligned16(sw)) return QK_ERR_MISALIGNED;
+  qk_status st = check_device();
+  if (st != QK_OK) return st;
+  return from_cuda(launch_quant_w8(W, N, K, Wq, sw, stream), "quant_w8");
+}
+
+qk_status qk_quantize_weights_int4(const float* W, int64_t N, int64_t K, uint8_t* Wp,
+                                   uint16_t* wscale, uint16_t* woffset, qk_stream_t stream) {
+  if (N < 0 || K < 0) return QK_ERR_INVALID_ARG;
+  if (K < 64 || K > 65536 || K % 64 != 0 || N > INT32_MAX) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0) return QK_OK;
+  if (!W || !Wp || !wscale || !woffset) return QK_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wp) || !aligned16(wscale) || !aligned16(woffset))
+    return QK_ERR_MISALIGNED;
+  qk_status st = check_device();
+  if (st != QK_OK) return st;
+  return from_cuda(launch_quant_w4(W, N, K, Wp, wscale, woffset, stream), "quant_w4");
+}
+
+qk_status qk_quantize_activations(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx,
+                                  int32_t* xsum, qk_stream_t stream) {
+  if (M < 0 || K < 0) return QK_ERR_INVALID_ARG;
+  if (K < 32 || K > 65536 || K % 32 != 0 || M > INT32_MAX) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (xsum != nullptr && K % 64 != 0) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return QK_OK;
+  if (!x || !xq || !sx) return QK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(sx) || (xsum && !aligned16(xsum)))
+    return QK_ERR_MISALIGNED;
+  qk_status st = check_device();
+  if (st != QK_OK) return st;
+  return from_cuda(launch_quant_act(x, M, K, xq, sx, xsum, stream), "quant_act");
+}
+
+qk_status qk_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64_t K, const int8_t* Wq,
+                       const float* sw, const float* bias, int64_t N, uint16_t* y,
+                       qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, false);
+  if (st != QK_OK || M == 0) return st;
+  if (!xq || !sx || !Wq || !sw || !y) return QK_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(Wq) || !aligned16(sw) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return QK_ERR_MISALIGNED;
+  if ((st = check_device()) != QK_OK) return st;
+  return from_cuda(launch_w8a8_gemm(xq, sx, M, K, Wq, sw, bias, N, y, nullptr, false, stream),
+                   "w8a8_gemm");
+}
+
+qk_status qk_w8a8_linear(const uint16_t* x, int64_t M, int64_t K, const int8_t* Wq,
+                         const float* sw, const float* bias, int64_t N, uint16_t* y,
+                         void* workspace, size_t ws_bytes, qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, false);
+  if (st != QK_OK || M == 0) return st;
+  if (!x || !Wq || !sw || !y) return QK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(sw) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return QK_ERR_MISALIGNED;
+  if ((st = check_device()) != QK_OK) return st;
+  Workspace ws;
+  if ((st = ws.init(workspace, ws_bytes, M, K, false, stream)) != QK_OK) return st;
+  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, nullptr, stream), "quant_act")) !=
+      QK_OK)
+    return st;
+  if (log_enabled())
+    std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> quant_act + tcgen05 GEMM\n",
+                 (long long)M, (long long)K, (long long)N);
+  return from_cuda(launch_w8a8_gemm(ws.xq, ws.sx, M, K, Wq, sw, bias, N, y, nullptr, true, stream),
+                   "w8a8_gemm");
+}
+
+static qk_status check_w4_product(const uint8_t* Wp, const uint16_t* wscale,
+                                  const uint16_t* woffset, const float* bias, uint16_t* y) {
+  if (!Wp || !wscale || !woffset || !y) return QK_ERR_INVALID_ARG;
+  if (!aligned16(Wp) || !aligned16(wscale) || !aligned16(woffset) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return QK_ERR_MISALIGNED;
+  return QK_OK;
+}
+
+static cudaError_t run_w4a8(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+                            int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                            const float* bias, int64_t N, uint16_t* y, int route, bool pdl,
+                            cudaStream_t s) {
+  const bool gemv = route == QK_ROUTE_GEMV || (route == QK_ROUTE_AUTO && M <= 16 && K <= kGemvMaxK);
+  if (log_enabled())
+    std::fprintf(stderr, "[qk] w4a8 M=%lld K=%lld N=%lld -> %s\n", (long long)M, (long long)K,
+                 (long long)N, gemv ? "GEMV" : "tcgen05 GEMM");
+  if (gemv)
+    return launch_w4a8_gemv(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, pdl, s);
+  return launch_w4a8_gemm(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, pdl, s);
+}
+
+qk_status qk_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+                       int64_t K, const uint8_t* Wp, const uint16_t* wscale,
+                       const uint16_t* woffset, const float* bias, int64_t N, uint16_t* y,
+                       int route, qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, true);
+  if (st != QK_OK) return st;
+  if (route != QK_ROUTE_AUTO && route != QK_ROUTE_GEMM && route != QK_ROUTE_GEMV)
+    return QK_ERR_INVALID_ARG;
+  if (route == QK_ROUTE_GEMV && M > 16) return QK_ERR_INVALID_ARG;
+  if (route == QK_ROUTE_GEMV && K > kGemvMaxK) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return QK_OK;
+  if (!xq || !sx || !xsum) return QK_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(xsum)) return QK_ERR_MISALIGNED;
+  if ((st = check_w4_product(Wp, wscale, woffset, bias, y)) != QK_OK) return st;
+  if ((st = check_device()) != QK_OK) return st;
+  return from_cuda(run_w4a8(xq, sx, xsum, M, K, Wp, wscale, woffset, bias, N, y, route, false,
+                            stream),
+                   "w4a8");
+}
+
+qk_status qk_w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* Wp,
+                         const uint16_t* wscale, const uint16_t* woffset, const float* bias,
+                         int64_t N, uint16_t* y, void* workspace, size_t ws_bytes,
+                         qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, true);
+  if (st != QK_OK || M == 0) return st;
+  if (!x) return QK_ERR_INVALID_ARG;
+  if (!aligned16(x)) return QK_ERR_MISALIGNED;
+  if ((st = check_w4_product(Wp, wscale, woffset, bias, y)) != QK_OK) return st;
+  if ((st = check_device()) != QK_OK) return st;
+  Workspace ws;
+  if ((st = ws.init(workspace, ws_bytes, M, K, true, stream)) != QK_OK) return st;
+  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, ws.xsum, stream), "quant_act")) !=
+      QK_OK)
+    return st;
+  return from_cuda(run_w4a8(ws.xq, ws.sx, ws.xsum, M, K, Wp, wscale, woffset, bias, N, y,
+                            QK_ROUTE_AUTO, true, stream),
+                   "w4a8");
+}
+
+qk_status qk_check_device_error(qk_stream_t stream) {
+  qk_status st = check_device();
+  if (st != QK_OK) return st;
+  if ((st = from_cuda(cudaStreamSynchronize(stream), "cudaStreamSynchronize")) != QK_OK) return st;
+  int* word = device_error_word();
+  if (word == nullptr) return QK_ERR_CUDA;
+  int h = 0;
+  if ((st = from_cuda(cudaMemcpy(&h, word, sizeof h, cudaMemcpyDeviceToHost), "read error word")) !=
+      QK_OK)
+    return st;
+  if (h != 0) {
+    const int zero = 0;
+    if ((st = from_cuda(cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice),
+                        "clear error word")) != QK_OK)
+      return st;
+    return h == QK_ERR_TIMEOUT ? QK_ERR_TIMEOUT : QK_ERR_CUDA;
+  }
+  return QK_OK;
+}
+
+qk_status qk_debug_w8a8_acc(const int8_t* xq, int64_t M, int64_t K, const int8_t* Wq, int64_t N,
+                            int32_t* acc, qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, false);
+  if (st != QK_OK || M == 0) return st;
+  if (!xq || !Wq || !acc) return QK_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(Wq) || !aligned16(acc)) return QK_ERR_MISALIGNED;
+  if ((st = check_device()) != QK_OK) return st;
+  return from_cuda(
+      launch_w8a8_gemm(xq, nullptr, M, K, Wq, nullptr, nullptr, N, nullptr, acc, false, stream),
+      "w8a8_acc");
+}
+
+qk_status qk_debug_w4a8_group_acc(const int8_t* xq, int64_t M, int64_t K, const uint8_t* Wp,
+                                  int64_t N, int64_t m0, int64_t m1, int32_t* acc, int route,
+                                  qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, true);
+  if (st != QK_OK) return st;
+  if (route != QK_ROUTE_GEMM && route != QK_ROUTE_GEMV) return QK_ERR_INVALID_ARG;
+  if (route == QK_ROUTE_GEMV && M > 16) return QK_ERR_INVALID_ARG;
+  if (route == QK_ROUTE_GEMV && K > kGemvMaxK) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (m0 < 0 || m1 < m0 || m1 > M) return QK_ERR_INVALID_ARG;
+  if (m1 == m0) return QK_OK;
+  if (!xq || !Wp || !acc) return QK_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(Wp) || !aligned16(acc)) return QK_ERR_MISALIGNED;
+  if ((st = check_device()) != QK_OK) return st;
+  cudaError_t e =
+      route == QK_ROUTE_GEMV
+          ? launch_w4a8_gemv(xq, nullptr, nullptr, M, K, Wp, nullptr, nullptr, nullptr, N,
+                             nullptr, acc, m0, m1, false, stream)
+          : launch_w4a8_gemm(xq, nullptr, nullptr, M, K, Wp, nullptr, nullptr, nullptr, N,
+                             nullptr, acc, m0, m1, false, stream);
+  return from_cuda(e, "w4a8_group_acc");
+}
+
+}  // extern "C"

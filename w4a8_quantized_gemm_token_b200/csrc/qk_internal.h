@@ -1,0 +1,61 @@
+// qk_internal.h -- host-side declarations shared by the library's .cu files.
+// Not installed; the public ABI is include/qk.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "qk.h"
+
+namespace qk {
+
+// ------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error.  Arguments are already
+// validated by the C-ABI layer (qk_api.cu).
+
+cudaError_t launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx,
+                             int32_t* xsum, cudaStream_t s);
+
+cudaError_t launch_quant_w8(const float* W, int64_t N, int64_t K, int8_t* Wq, float* sw,
+                            cudaStream_t s);
+
+cudaError_t launch_quant_w4(const float* W, int64_t N, int64_t K, uint8_t* Wp, uint16_t* ws,
+                            uint16_t* wo, cudaStream_t s);
+
+// W8A8 GEMM with the fused dequant + bias epilogue (bf16 out), or the raw int32
+// accumulator epilogue when `acc_out` is not null (y, sx, sw, bias ignored).
+// `pdl` launches it as a programmatic dependent of the previous kernel.
+cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64_t K,
+                             const int8_t* Wq, const float* sw, const float* bias, int64_t N,
+                             uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s);
+
+// W4A8 tensor-core GEMM (any M).  When `acc_out` is not null it stores the
+// per-group int32 accumulators of rows [m0, m1) instead of y.
+cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                             const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
+                             int64_t m0, int64_t m1, bool pdl, cudaStream_t s);
+
+// W4A8 weight-streaming GEMV (M <= 16, K <= kGemvMaxK: the CTA's weight slice
+// must fit shared memory); per-group accumulator dump as above.
+constexpr int64_t kGemvMaxK = 16384;
+cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                             const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
+                             int64_t m0, int64_t m1, bool pdl, cudaStream_t s);
+
+// Address of this device's error word (a __device__ int of the library),
+// resolved once per device with cudaGetSymbolAddress; null on failure.
+int* device_error_word();
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda
+// link dependency).  Returns false if the driver call is unavailable or fails.
+bool encode_tmap_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* base,
+                    uint64_t inner, uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
+                    uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
+}  // namespace qk

@@ -1,0 +1,271 @@
+// quant.cu -- quantization kernels.
+//
+//  * quant_act: per-token dynamic symmetric int8 quantization of bf16
+//    activations ("qlip-mlx" README, "w8a8_linear / W8A8Linear": activations
+//    quantized dynamically inside the op; "MLX PR #4722", "SIMD fix": a kernel
+//    of its own quantizes x).  HBM-bound: 2 bytes read and 1 written per
+//    element.  One warp owns one row; each lane moves 16-byte chunks (8 bf16),
+//    so a warp-wide load covers 512 contiguous bytes.  Rows of up to
+//    32 * 8 * NCH elements stay in registers between the absmax and the
+//    quantize pass; longer rows are read twice (the second read hits L2).
+//  * quant_w8: the same rule per output channel on fp32 weights (offline).
+//  * quant_w4: affine group-64 4-bit weights ("qlip-mlx" README,
+//    "w4a8_linear / W4A8Linear"; "MLX PR #4722", "Selector rules"), offline.
+//
+// Rounding: the scale is absmax / 127 and the multiplier 127 / absmax, both
+// correctly rounded fp32 divisions; each code is round-half-even of the fp32
+// product x * multiplier (no fused multiply-add), clamped to [-127, 127].
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "qk_internal.h"
+#include "sm100.cuh"
+
+namespace qk {
+namespace {
+
+constexpr int kQuantWarps = 8;  // rows per 256-thread block
+
+__device__ __forceinline__ uint32_t bf16x2_absmax_bits(uint32_t acc, uint32_t w) {
+  // |bf16| bit patterns order like the values they encode, so a 16-bit integer
+  // max of the magnitudes is the absmax.
+  return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+
+__device__ __forceinline__ int quant1(float v, float r) {
+  int q = __float2int_rn(__fmul_rn(v, r));
+  return max(-127, min(127, q));
+}
+
+// 8 bf16 (one 16-byte chunk) -> 8 int8 codes packed in a uint2; adds the codes
+// to *sum.
+__device__ __forceinline__ uint2 quant_chunk(uint4 c, float r, int* sum) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  uint32_t out[2];
+  int s = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t packed = 0;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t u = w[2 * h + j];
+      const int q0 = quant1(__uint_as_float(u << 16), r);
+      const int q1 = quant1(__uint_as_float(u & 0xFFFF0000u), r);
+      s += q0 + q1;
+      packed |= ((uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8)) << (16 * j);
+    }
+    out[h] = packed;
+  }
+  *sum += s;
+  return make_uint2(out[0], out[1]);
+}
+
+__device__ __forceinline__ float warp_max_bits_to_float(uint32_t bits2) {
+  uint32_t m = max(bits2 & 0xFFFFu, bits2 >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  return __uint_as_float(m << 16);
+}
+
+// Sum over the 8 lanes that hold one group of 64 codes.
+__device__ __forceinline__ int group8_sum(int v) {
+  v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+  v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+  v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+  return v;
+}
+
+// NCH > 0: the row (<= 256 * NCH elements) stays in registers.
+// NCH == 0: two passes over the row.
+template <int NCH>
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int M,
+                                                        int K, int8_t* __restrict__ xq,
+                                                        float* __restrict__ sx,
+                                                        int32_t* __restrict__ xsum) {
+  // The dependent GEMM may start its prologue now; it waits for this grid's
+  // completion before it reads xq / sx.
+  pdl_launch_dependents();
+  const int row = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (row >= M) return;
+  const int lane = threadIdx.x & 31;
+  const int nch = K >> 3;  // 16-byte chunks per row
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * K);
+  uint2* dst = reinterpret_cast<uint2*>(xq + (size_t)row * K);
+  const int G = K >> 6;
+
+  uint32_t mb = 0;
+  float r;
+  if constexpr (NCH > 0) {
+    uint4 v[NCH];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = i * 32 + lane;
+      if (c < nch) {
+        v[i] = __ldcs(src + c);
+        mb = bf16x2_absmax_bits(mb, v[i].x);
+        mb = bf16x2_absmax_bits(mb, v[i].y);
+        mb = bf16x2_absmax_bits(mb, v[i].z);
+        mb = bf16x2_absmax_bits(mb, v[i].w);
+      }
+    }
+    const float amax = warp_max_bits_to_float(mb);
+    r = (amax == 0.0f) ? 0.0f : __fdiv_rn(127.0f, amax);
+    if (lane == 0) sx[row] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = i * 32 + lane;
+      int s = 0;
+      if (c < nch) dst[c] = quant_chunk(v[i], r, &s);
+      if (xsum != nullptr && i * 32 < nch) {  // warp-uniform
+        s = group8_sum(s);
+        if ((lane & 7) == 0 && c < nch) xsum[(size_t)row * G + (c >> 3)] = s;
+      }
+    }
+  } else {
+    for (int c = lane; c < nch; c += 32) {
+      const uint4 v = __ldg(src + c);
+      mb = bf16x2_absmax_bits(mb, v.x);
+      mb = bf16x2_absmax_bits(mb, v.y);
+      mb = bf16x2_absmax_bits(mb, v.z);
+      mb = bf16x2_absmax_bits(mb, v.w);
+    }
+    const float amax = warp_max_bits_to_float(mb);
+    r = (amax == 0.0f) ? 0.0f : __fdiv_rn(127.0f, amax);
+    if (lane == 0) sx[row] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
+    for (int base = 0; base < nch; base += 32) {  // warp-uniform trip count
+      const int c = base + lane;
+      int s = 0;
+      if (c < nch) dst[c] = quant_chunk(__ldcs(src + c), r, &s);
+      if (xsum != nullptr) {
+        s = group8_sum(s);
+        if ((lane & 7) == 0 && c < nch) xsum[(size_t)row * G + (c >> 3)] = s;
+      }
+    }
+  }
+}
+
+// W8: one warp per output channel, fp32 input, two passes (offline op).
+__global__ void __launch_bounds__(256) quant_w8_kernel(const float* __restrict__ W, int N, int K,
+                                                       int8_t* __restrict__ Wq,
+                                                       float* __restrict__ sw) {
+  const int row = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (row >= N) return;
+  const int lane = threadIdx.x & 31;
+  const float4* src = reinterpret_cast<const float4*>(W + (size_t)row * K);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(Wq + (size_t)row * K);
+  const int nch = K >> 2;
+  float amax = 0.0f;
+  for (int c = lane; c < nch; c += 32) {
+    const float4 v = __ldg(src + c);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  const float r = (amax == 0.0f) ? 0.0f : __fdiv_rn(127.0f, amax);
+  if (lane == 0) sw[row] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
+  for (int c = lane; c < nch; c += 32) {
+    const float4 v = __ldg(src + c);
+    const int q0 = quant1(v.x, r), q1 = quant1(v.y, r), q2 = quant1(v.z, r), q3 = quant1(v.w, r);
+    dst[c] = (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) | ((uint32_t)(q2 & 0xFF) << 16) |
+             ((uint32_t)(q3 & 0xFF) << 24);
+  }
+}
+
+// W4 affine, group 64: eight lanes per group, eight weights per lane.
+__global__ void __launch_bounds__(256) quant_w4_kernel(const float* __restrict__ W, int N, int K,
+                                                       uint8_t* __restrict__ Wp,
+                                                       uint16_t* __restrict__ wscale,
+                                                       uint16_t* __restrict__ woffset) {
+  const int G = K >> 6;
+  const long long total = (long long)N * G;
+  const long long grp = ((long long)blockIdx.x * 256 + threadIdx.x) >> 3;
+  const int t = threadIdx.x & 7;
+  const bool valid = grp < total;  // whole 8-lane teams are valid or not
+  const long long g_safe = valid ? grp : 0;
+  const int n = (int)(g_safe / G), g = (int)(g_safe % G);
+  const float4* src = reinterpret_cast<const float4*>(W + (size_t)n * K + 64 * g + 8 * t);
+  float w[8];
+  if (valid) {
+    const float4 a = __ldg(src), b = __ldg(src + 1);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = 0.0f;
+  }
+  float lo = w[0], hi = w[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    lo = fminf(lo, w[i]);
+    hi = fmaxf(hi, w[i]);
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+  }
+  if (!valid) return;
+  const __half sh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+  const __half oh = __float2half_rn(lo);
+  const float s = __half2float(sh);
+  const float off = __half2float(oh);
+  uint32_t packed = 0;
+  if (s != 0.0f) {
+    const float r = __fdiv_rn(1.0f, s);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int q = __float2int_rn(__fmul_rn(__fsub_rn(w[i], off), r));
+      q = max(0, min(15, q));
+      packed |= (uint32_t)q << (4 * i);  // k = 2j low nibble, 2j + 1 high nibble
+    }
+  }
+  reinterpret_cast<uint32_t*>(Wp + (size_t)n * (K / 2) + 32 * g)[t] = packed;
+  if (t == 0) {
+    wscale[(size_t)n * G + g] = __half_as_ushort(sh);
+    woffset[(size_t)n * G + g] = __half_as_ushort(oh);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx,
+                             int32_t* xsum, cudaStream_t s) {
+  const dim3 grid((unsigned)((M + kQuantWarps - 1) / kQuantWarps)), block(256);
+  const int m = (int)M, k = (int)K;
+  const int per_lane = (int)((K / 8 + 31) / 32);  // 16-byte chunks per lane
+  if (per_lane <= 1)
+    quant_act_kernel<1><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
+  else if (per_lane <= 2)
+    quant_act_kernel<2><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
+  else if (per_lane <= 4)
+    quant_act_kernel<4><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
+  else if (per_lane <= 8)
+    quant_act_kernel<8><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
+  else if (per_lane <= 12)
+    quant_act_kernel<12><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
+  else if (per_lane <= 16)
+    quant_act_kernel<16><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
+  else
+    quant_act_kernel<0><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_w8(const float* W, int64_t N, int64_t K, int8_t* Wq, float* sw,
+                            cudaStream_t s) {
+  const dim3 grid((unsigned)((N + kQuantWarps - 1) / kQuantWarps)), block(256);
+  quant_w8_kernel<<<grid, block, 0, s>>>(W, (int)N, (int)K, Wq, sw);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_w4(const float* W, int64_t N, int64_t K, uint8_t* Wp, uint16_t* ws,
+                            uint16_t* wo, cudaStream_t s) {
+  const long long threads = N * (K / 64) * 8;
+  const dim3 grid((unsigned)((threads + 255) / 256)), block(256);
+  quant_w4_kernel<<<grid, block, 0, s>>>(W, (int)N, (int)K, Wp, ws, wo);
+  return cudaGetLastError();
+}
+
+}  // namespace qk
