@@ -1,0 +1,505 @@
+#!/usr/bin/env python3
+"""Benchmark of the W8A8 / W4A8 quantized linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one call of the linear (activation quant + tcgen05 GEMM with the
+fused dequant epilogue) on one batch of synthetic input already resident in
+HBM.  The default workload is the DiT MLP projection W8A8 linear,
+x [16384, 3072] bf16 -> y [16384, 12288] bf16 (1% outlier channels x20, bias).
+Rank 0 prints one JSON line.  Under torchrun each rank is an independent
+replica (the path needs no collective): per-GPU work is fixed, the value is the
+sum over ranks divided by the slowest rank's time ("scaling": "weak").
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and torch.cuda.synchronize(), CUDA events on the launching stream, max over
+ranks.  Inputs rotate over two full input sets (x and Wq), so every step reads
+its operands from HBM (x 100.7 MB + Wq 37.7 MB per set, y 402.7 MB written per
+step; more than the 126 MB L2).  SM clocks and throttle reasons are sampled
+with NVML during the timed region.
+
+`--impl reference` times the CPU oracle (oracle/, plain C) on the host cores
+for the same metric, one bounded sample of the workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W8A8 linear TOPS incl. act quant at DiT shapes; % of B200 INT8 peak"
+INT8_SPEC_TOPS = 4500.0  # dense INT8, B200 datasheet
+
+WORKLOADS = {
+    "dit_mlp": ("DIT_MLP", None),
+    "dit_attn": ("DIT_ATTN", None),
+    "sweep_4096x4096": ("SWEEP", 0),
+    "sweep_4096x12288": ("SWEEP", 1),
+    "sweep_12288x4096": ("SWEEP", 2),
+    "sweep_thin_5120x48": ("SWEEP", 3),
+    "tiny": ("TINY", None),
+    "w4a8_m1": ("W4A8", 0),
+    "w4a8_m8": ("W4A8", 1),
+    "w4a8_m16": ("W4A8", 2),
+    "w4a8_m4096": ("W4A8", 3),
+}
+
+
+def get_case(name):
+    from w4a8_quantized_gemm_token_b200 import synthetic
+
+    attr, idx = WORKLOADS[name]
+    obj = getattr(synthetic, attr)
+    return obj if idx is None else obj[idx]
+
+
+def is_w4(name):
+    return name.startswith("w4a8")
+
+
+# ------------------------------------------------------------ peaks / clocks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons with NVML every `period` s."""
+
+    def __init__(self, torch_device: int, period: float = 0.02):
+        self.period = period
+        self.samples = []
+        self.handle = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            bus = None
+            props = torch.cuda.get_device_properties(torch_device)
+            if hasattr(props, "pci_bus_id"):
+                bus = f"{getattr(props, 'pci_domain_id', 0):08x}:{props.pci_bus_id:02x}:" \
+                      f"{getattr(props, 'pci_device_id', 0):02x}.0"
+            if bus is not None:
+                try:
+                    self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+                except Exception:
+                    self.handle = None
+            if self.handle is None:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(torch_device)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.handle = None
+            self.max_mhz = None
+
+    def _one(self):
+        nv = self.nv
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+            self.samples.append((sm, rs, pw))
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._one()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.handle is not None:
+            self._one()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.handle is not None:
+            self._stop.set()
+            self._t.join()
+            self._one()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, rs, _ in self.samples:
+            for bit, name in REASON_BITS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": float(statistics.median(s[0] for s in self.samples)),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "power_w_max": round(max(s[2] for s in self.samples), 1),
+                "samples": len(self.samples)}
+
+
+def traffic_from_profile(kernel_tag: str, src_path: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel (matched by a hash of the .cu file)."""
+    import hashlib
+
+    prof = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
+    try:
+        digest = hashlib.sha256(open(src_path, "rb").read()).hexdigest()[:16]
+        fields = {}
+        for line in open(prof):
+            if ":" in line:
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+        if fields.get("source_sha256_16") != digest:
+            return None
+        return float(fields["dram_bytes_per_launch_full_workload"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of `value` over ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def whole_job_value(ops_per_step: float, steps: int, world: int, max_seconds: float) -> float:
+    """Aggregate throughput over all ranks in tera-ops/s (each rank does the same work)."""
+    return ops_per_step * steps * world / max_seconds / 1e12
+
+
+# ------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from w4a8_quantized_gemm_token_b200 import binding as qk
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    case = get_case(args.workload)
+    M, K, N = case.M, case.K, case.N
+    w4 = is_w4(args.workload)
+    xb, W, b, _ = case.draw()
+    x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
+    W_dev = torch.from_numpy(W).to(dev)
+    bias = torch.from_numpy(b).to(dev) if b is not None else None
+
+    nsets = args.sets
+    xs = [x_host.to(dev) for _ in range(nsets)]
+    if w4:
+        weights = [qk.qk_quantize_weights_int4(W_dev) for _ in range(nsets)]
+        ws = torch.empty(qk.qk_w4a8_workspace_size(M, K), dtype=torch.uint8, device=dev)
+    else:
+        weights = [qk.qk_quantize_weights_int8(W_dev) for _ in range(nsets)]
+        ws = torch.empty(qk.qk_w8a8_workspace_size(M, K), dtype=torch.uint8, device=dev)
+    del W_dev
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        wt = weights[i % nsets]
+        if w4:
+            qk.qk_w4a8_linear(xs[i % nsets], *wt, bias, y=y, workspace=ws)
+        else:
+            qk.qk_w8a8_linear(xs[i % nsets], *wt, bias, y=y, workspace=ws)
+
+    ops = 2.0 * M * N * K
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    qk.qk_check_device_error()
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = e0.elapsed_time(e1)
+    qk.qk_check_device_error()
+    max_ms = reduce_max(ms, dev)
+    value = whole_job_value(ops, args.steps, world, max_ms / 1e3)
+
+    # ---- dominant kernel alone (the GEMM on pre-quantized activations)
+    peaks = load_peaks()
+    if w4:
+        xq_sets = [qk.qk_quantize_activations(x, with_xsum=True) for x in xs]
+        route = qk.QK_ROUTE_GEMV if M <= 16 else qk.QK_ROUTE_GEMM
+
+        def kstep(i):
+            xq, sx, xsum = xq_sets[i % nsets]
+            qk.qk_w4a8_gemm(xq, sx, xsum, *weights[i % nsets], bias, y=y, route=route)
+    else:
+        xq_sets = [qk.qk_quantize_activations(x) for x in xs]
+
+        def kstep(i):
+            xq, sx, _ = xq_sets[i % nsets]
+            qk.qk_w8a8_gemm(xq, sx, *weights[i % nsets], bias, y=y)
+    for i in range(args.warmup):
+        kstep(i)
+    torch.cuda.synchronize()
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for i in range(args.steps):
+        kstep(i)
+    k1.record(stream)
+    torch.cuda.synchronize()
+    k_ms = k0.elapsed_time(k1) / args.steps
+    if w4 and M <= 16:
+        # weight-streaming GEMV: bound by HBM; algorithmic bytes per launch
+        G = K // 64
+        kbytes = N * K / 2 + 4 * N * G + M * K + 4 * M + 4 * M * G + 2 * M * N
+        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc", "gemv_w4a8.cu")
+        roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
+                "kernel": "w4a8_gemv_kernel",
+                "traffic": traffic_from_profile("w4a8_gemv_kernel", src)}
+    else:
+        peak = peaks["bf16"] * 2.0
+        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc",
+                           "gemm_w4a8.cu" if w4 else "gemm_w8a8.cu")
+        tag = "w4a8_gemm_kernel" if w4 else "w8a8_gemm_kernel"
+        roof = {"bound": "tensor", "achieved": ops / (k_ms / 1e3) / 1e12, "peak": peak,
+                "unit": "TFLOP/s",
+                "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2, the nominal int8/bf16 "
+                               "ratio (4.5 / 2.25 POPS); int8 ops counted as 2*M*N*K",
+                "kernel": tag, "traffic": traffic_from_profile(tag, src)}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel_ms"] = k_ms
+
+    # ---- end to end through the public call, host buffers in and out
+    e2e = None
+    if not args.no_e2e:
+        x_pin = x_host.pin_memory()
+        y_pin = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        n_e2e = max(3, min(args.steps, args.e2e_steps))
+
+        def e2e_step(i):
+            x_dev.copy_(x_pin, non_blocking=True)
+            wt = weights[i % nsets]
+            if w4:
+                qk.qk_w4a8_linear(x_dev, *wt, bias, y=y, workspace=ws)
+            else:
+                qk.qk_w8a8_linear(x_dev, *wt, bias, y=y, workspace=ws)
+            y_pin.copy_(y, non_blocking=True)
+
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier(dev)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(n_e2e):
+            e2e_step(i)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = reduce_max(a0.elapsed_time(a1), dev)
+        e2e = {"value": whole_job_value(ops, n_e2e, world, e_ms / 1e3), "unit": "TOPS",
+               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+               "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case, seconds=args.cpu_seconds)
+
+    clocks = sampler.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8", "data": "synthetic",
+            "config": {"workload": case.name, "M": M, "K": K, "N": N,
+                       "weights": "W4 affine g64" if w4 else "W8 per-channel",
+                       "bias": bias is not None,
+                       "activations": "bf16 N(0,1)" + (", 1% channels x20" if case.outlier_frac else ""),
+                       "l2": f"{nsets} rotating input sets; inputs + outputs per step exceed the 126 MB L2",
+                       "parallelism": f"replicas x{world} (no collective)"},
+            "pct_of_int8_spec": 100.0 * value / world / INT8_SPEC_TOPS,
+            "roofline": roof, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
+            "gpu_launches": 2 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ oracle legs
+
+class OracleSample:
+    """Inputs for bounded oracle samples of a workload (same recipe as the GPU
+    arm; only the first rows of x are drawn, since a sample never uses more)."""
+
+    def __init__(self, case, w4, max_rows=1024):
+        import dataclasses
+
+        import oracle
+
+        self.case, self.w4 = case, w4
+        small = dataclasses.replace(case, M=min(case.M, max_rows))
+        self.xb, W, self.b, _ = small.draw()
+        if w4:
+            self.Wp, self.s16, self.o16 = oracle.quant_w4(W)
+        else:
+            self.Wq, self.sw = oracle.quant_w8(W)
+
+    def run(self, rows, ncols):
+        """Quantize `rows` activation rows and compute their outputs for the first
+        `ncols` output channels.  Returns (seconds, ops)."""
+        import oracle
+
+        t0 = time.perf_counter()
+        xq, sx = oracle.quant_act(self.xb[:rows])
+        if self.w4:
+            xsum = oracle.group_sums(xq)
+            acc = oracle.w4a8_group_acc(xq, self.Wp[:ncols])
+            oracle.w4a8_dequant(acc, xsum, sx, self.s16[:ncols], self.o16[:ncols], None)
+        else:
+            acc = oracle.w8a8_acc(xq, self.Wq[:ncols])
+            oracle.w8a8_dequant(acc, sx, self.sw[:ncols],
+                                None if self.b is None else self.b[:ncols])
+        return time.perf_counter() - t0, 2.0 * rows * ncols * self.case.K
+
+
+def cpu_baseline(case, seconds=10.0):
+    """The oracle on the host cores over a bounded sample of the same workload."""
+    smp = OracleSample(case, case.name.startswith("w4a8"))
+    dt, _ = smp.run(1, case.N)          # calibrate on one row
+    rows = int(max(1, min(smp.xb.shape[0], seconds / max(dt, 1e-6))))
+    dt, ops = smp.run(rows, case.N)
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of {case.M} rows x all {case.N} output channels "
+                      f"(quant + exact int accumulate + fp64 dequant), single thread, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, world, rank, local):
+    if rank != 0:
+        return  # rank 0 alone runs the oracle
+    case = get_case(args.workload)
+    smp = OracleSample(case, is_w4(args.workload), max_rows=8)
+    # size each step so that warm-up + timed steps take about `budget` seconds
+    budget = args.ref_seconds
+    dt1, _ = smp.run(1, case.N)
+    per_step = budget / max(1, args.steps + args.warmup)
+    ncols = int(max(8, min(case.N, case.N * per_step / max(dt1, 1e-6)))) // 8 * 8
+    for _ in range(args.warmup):
+        smp.run(1, ncols)
+    t_total, ops_total = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, ops = smp.run(1, ncols)
+        t_total += dt
+        ops_total += ops
+    value = ops_total / t_total / 1e12
+    sample = (f"per step: 1 of {case.M} rows x {ncols} of {case.N} output channels "
+              f"(quant + exact int accumulate + fp64 dequant), single thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": case.name, "M": case.M, "K": case.K, "N": case.N},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="dit_mlp")
+    ap.add_argument("--sets", type=int, default=2, help="rotating input sets (L2 defeat)")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world, rank, local = dist_env()
+    if world != args.gpus and world != 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,72 @@
+"""The W4A8 linear on the GPU against the oracle.
+
+Per-group int32 accumulators bit-exact on both routes (weight-streaming GEMV for
+M <= 16, tcgen05 GEMM otherwise); bf16 outputs within 2 bf16 ulp of the
+oracle's fp64 fold rounded to bf16; the two routes agree where both apply."""
+import numpy as np
+import pytest
+import torch
+
+from tests.gpu_common import host, qk, t2bits, to_dev, to_dev_bf16  # noqa: F401
+from tests.helpers import bf16_ulp_distance, sample_rows
+from w4a8_quantized_gemm_token_b200 import synthetic
+
+pytestmark = pytest.mark.gpu
+
+TOL_ULP = 2
+GEMV, GEMM = 2, 1
+
+
+def prepare(qk, orc, case):
+    xb, W, b, _ = case.draw()
+    Wp_o, s_o, o_o = orc.quant_w4(W)
+    Wp, s, o = qk.qk_quantize_weights_int4(to_dev(W))
+    assert np.array_equal(host(Wp), Wp_o)
+    assert np.array_equal(t2bits(s), s_o) and np.array_equal(t2bits(o), o_o)
+    return xb, (Wp, s, o), (Wp_o, s_o, o_o), b
+
+
+GEMV_SHAPES = [(1, 64, 8), (1, 4096, 4096), (8, 4096, 4096), (16, 4096, 4096), (3, 192, 40),
+               (11, 1024, 264), (16, 16384, 128), (5, 640, 2056)]
+
+
+@pytest.mark.parametrize("MKN", GEMV_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_gemv_group_acc_and_output(qk, orc, MKN):
+    M, K, N = MKN
+    case = synthetic.LinearCase("v", M=M, K=K, N=N, bias=(N % 16 == 8), seed=M * 31 + K + N)
+    xb, dev_w, ora_w, b = prepare(qk, orc, case)
+    x = to_dev_bf16(xb)
+    xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
+    acc = qk.qk_debug_w4a8_group_acc(xq, dev_w[0], 0, M, GEMV)
+    bias = to_dev(b) if b is not None else None
+    y = qk.qk_w4a8_linear(x, *dev_w, bias)
+    y2 = qk.qk_w4a8_gemm(xq, sx, xsum, *dev_w, bias, route=GEMV)
+    torch.cuda.synchronize()
+    y_o, xq_o, sx_o, xsum_o, acc_o = orc.w4a8_linear(xb, *ora_w, b)
+    assert np.array_equal(host(xq), xq_o) and np.array_equal(host(xsum), xsum_o)
+    assert np.array_equal(host(acc).astype(np.int64), acc_o)
+    d = bf16_ulp_distance(t2bits(y), y_o)
+    assert d.max() <= TOL_ULP, f"worst {d.max()} ulp"
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    qk.qk_check_device_error()
+
+
+@pytest.mark.parametrize("case", synthetic.W4A8[:3], ids=lambda c: c.name)
+def test_w4a8_gemv_configs(qk, orc, case):
+    xb, dev_w, ora_w, b = prepare(qk, orc, case)
+    y = qk.qk_w4a8_linear(to_dev_bf16(xb), *dev_w)
+    torch.cuda.synchronize()
+    y_o, _, _, _, _ = orc.w4a8_linear(xb, *ora_w, None)
+    d = bf16_ulp_distance(t2bits(y), y_o)
+    print(f"{case.name}: worst={d.max()} ulp histogram={np.bincount(d.ravel(), minlength=3).tolist()}")
+    assert d.max() <= TOL_ULP
+
+
+def test_gemv_deterministic(qk, orc):
+    case = synthetic.LinearCase("det", M=16, K=4096, N=4096, bias=False, seed=77)
+    xb, dev_w, _, _ = prepare(qk, orc, case)
+    x = to_dev_bf16(xb)
+    ys = [qk.qk_w4a8_linear(x, *dev_w) for _ in range(3)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(ys[0].view(torch.int16), y.view(torch.int16))

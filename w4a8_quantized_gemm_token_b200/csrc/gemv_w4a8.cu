@@ -38,11 +38,11 @@ constexpr int kWarps = 8;
 constexpr int kGemvSmemLimit = 227 * 1024;
 
 struct GemvSmem {
-  static int row_stride(int K) { return K / 2 + 16; }
-  static size_t weights(int R, int K) { return (size_t)R * row_stride(K); }
+  __host__ __device__ static int row_stride(int K) { return K / 2 + 16; }
+  __host__ __device__ static size_t weights(int R, int K) { return (size_t)R * row_stride(K); }
   // R = 16 * RT rows; the 8 warps form RT row tiles x (8 / RT) K ranges.
-  static size_t partials(int R) { return (size_t)(kWarps / (R / 16)) * R * 16 * sizeof(double); }
-  static size_t bytes(int R, int K) {
+  __host__ __device__ static size_t partials(int R) { return (size_t)(kWarps / (R / 16)) * R * 16 * sizeof(double); }
+  __host__ __device__ static size_t bytes(int R, int K) {
     const int G = K / 64;
     size_t b = 0;
     b += weights(R, K);                        // packed codes
