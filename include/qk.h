@@ -176,6 +176,40 @@ qk_status qk_w8a8_gemm(const int8_t *xq, const float *sx, int64_t M, int64_t K,
                        const int8_t *Wq, const float *sw, const float *bias, int64_t N,
                        uint16_t *y, qk_stream_t stream);
 
+/*
+ * The W8A8 linear without any device allocation.  The pages have no
+ * counterpart: this exists for callers that may not allocate device memory at
+ * call time and cannot hand over a workspace either (a custom allocator that
+ * owns all device memory, a fixed-budget real-time host, a plugin whose host
+ * forbids allocation in its callbacks).
+ *
+ * Computes exactly what qk_w8a8_linear computes (same kernels), but keeps the
+ * quantized activations in a scratch array built into the library: a
+ * file-scope __device__ array of QK_NOALLOC_SCRATCH_BYTES (64 MiB).  Every GPU
+ * that loads the library's module holds that array until the process exits
+ * (with CUDA's default lazy module loading, from the first call on that
+ * device).  The call itself allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *
+ *   - Problems whose scratch, qk_w8a8_workspace_size(M, K), exceeds
+ *     QK_NOALLOC_SCRATCH_BYTES are rejected with QK_ERR_WORKSPACE before any
+ *     launch (M * K up to about 64 Mi elements; e.g. 16384 x 3072 fits).
+ *   - The first call on a device resolves the scratch's device address
+ *     (cudaGetSymbolAddress) and loads the kernels; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one scratch array, which keeps whatever
+ *     the last call wrote.  Nothing in it needs to start at zero (each call
+ *     overwrites the part it reads).  Calls whose executions overlap on the GPU
+ *     (for example on two streams without ordering between them) race on the
+ *     scratch and give wrong results: order them on one stream or with events.
+ * Arguments, layouts and the other errors are those of qk_w8a8_linear.
+ */
+#define QK_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+qk_status qk_w8a8_linear_noalloc(const uint16_t *x, int64_t M, int64_t K,
+                                 const int8_t *Wq, const float *sw, const float *bias,
+                                 int64_t N, uint16_t *y, qk_stream_t stream);
+
 /* ------------------------------------------------------------ W4A8 linear */
 
 /*
