@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "W8A8 linear TOPS incl. act quant at DiT shapes; % of B200 INT8 peak"
 INT8_SPEC_TOPS = 4500.0  # dense INT8, B200 datasheet
+L2_BYTES = 126 * 1024 * 1024
 
 WORKLOADS = {
     "dit_mlp": ("DIT_MLP", None),
@@ -217,6 +218,23 @@ def whole_job_value(ops_per_step: float, steps: int, world: int, max_seconds: fl
 
 # ------------------------------------------------------------ our arm
 
+def graph_runner(fn, steps):
+    """Capture `steps` calls of fn(i) into one CUDA graph; returns its replay.
+    Used where a step lasts only microseconds, so host launch cost would
+    otherwise be timed instead of the kernels."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for i in range(steps):
+                fn(i)
+    torch.cuda.current_stream().wait_stream(side)
+    return g.replay
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -232,7 +250,9 @@ def run_ours(args, world, rank, local):
     W_dev = torch.from_numpy(W).to(dev)
     bias = torch.from_numpy(b).to(dev) if b is not None else None
 
-    nsets = args.sets
+    # enough rotating input sets that one pass over them exceeds the L2 twice
+    per_set = M * K * 2 + (N * K // 2 + N * (K // 64) * 4 if w4 else N * K + 4 * N)
+    nsets = args.sets or int(min(32, max(2, -(-2 * L2_BYTES // per_set))))
     xs = [x_host.to(dev) for _ in range(nsets)]
     if w4:
         weights = [qk.qk_quantize_weights_int4(W_dev) for _ in range(nsets)]
@@ -257,14 +277,16 @@ def run_ours(args, world, rank, local):
     qk.qk_check_device_error()
 
     stream = torch.cuda.current_stream()
+    use_graph = args.graph == "on" or (args.graph == "auto" and M <= 256)
+    run_steps = graph_runner(step, args.steps) if use_graph else \
+        (lambda: [step(i) for i in range(args.steps)])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     barrier(dev)
     torch.cuda.synchronize()
     with sampler:
         e0.record(stream)
-        for i in range(args.steps):
-            step(i)
+        run_steps()
         e1.record(stream)
         torch.cuda.synchronize()
     barrier(dev)
@@ -291,10 +313,11 @@ def run_ours(args, world, rank, local):
     for i in range(args.warmup):
         kstep(i)
     torch.cuda.synchronize()
+    run_k = graph_runner(kstep, args.steps) if use_graph else \
+        (lambda: [kstep(i) for i in range(args.steps)])
     k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     k0.record(stream)
-    for i in range(args.steps):
-        kstep(i)
+    run_k()
     k1.record(stream)
     torch.cuda.synchronize()
     k_ms = k0.elapsed_time(k1) / args.steps
@@ -367,7 +390,9 @@ def run_ours(args, world, rank, local):
                        "weights": "W4 affine g64" if w4 else "W8 per-channel",
                        "bias": bias is not None,
                        "activations": "bf16 N(0,1)" + (", 1% channels x20" if case.outlier_frac else ""),
-                       "l2": f"{nsets} rotating input sets; inputs + outputs per step exceed the 126 MB L2",
+                       "l2": f"{nsets} rotating input sets of {per_set / 1e6:.1f} MB; "
+                             "one pass over them exceeds twice the 126 MB L2",
+                       "timing": "CUDA graph of the timed steps" if use_graph else "eager launches",
                        "parallelism": f"replicas x{world} (no collective)"},
             "pct_of_int8_spec": 100.0 * value / world / INT8_SPEC_TOPS,
             "roofline": roof, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
@@ -467,7 +492,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="dit_mlp")
-    ap.add_argument("--sets", type=int, default=2, help="rotating input sets (L2 defeat)")
+    ap.add_argument("--sets", type=int, default=0,
+                    help="rotating input sets (default: enough to exceed twice the L2)")
+    ap.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
+                    help="replay the timed steps from a CUDA graph (auto: small M)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

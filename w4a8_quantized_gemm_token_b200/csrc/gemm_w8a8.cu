@@ -6,22 +6,26 @@
 //     y[m, n]   = bf16( acc * sx[m] * sw[n] + bias[n] )      (fp64, one rounding)
 //
 // Design (sm_100a):
-//  * persistent grid, one 128 x 256 output tile at a time per CTA, tiles in a
-//    grouped raster (16 M-tiles per group) so concurrent CTAs share operand
-//    tiles in L2;
-//  * warp 0: TMA producer -- 128 x 128 int8 tiles of xq and 256 x 128 of Wq
-//    (both K-major, 128-byte swizzle) into a 4-stage shared-memory ring;
-//  * warp 1: allocates all 512 TMEM columns and issues tcgen05.mma kind::i8
-//    (M = 128, N = 256, K = 32 per instruction) into one of two 256-column
-//    int32 accumulators, so the epilogue of tile i overlaps the mainloop of
-//    tile i + 1;
-//  * warps 2-5: epilogue -- tcgen05.ld 32 lanes x 32 columns, dequant in fp64
-//    (int32 -> fp64 is exact, acc * sx is exact in fp64, one fused multiply-add
-//    with sw and bias), fp64 -> bf16 rounded once (round-to-odd into fp32, then
-//    nearest-even into bf16, which equals direct nearest-even), staged in a
-//    swizzled shared buffer and written with TMA stores that clip the M and N
-//    edges.
-// Every mbarrier wait is bounded (sm100.cuh) so a fault ends the kernel.
+//  * CTA pairs (clusters of 2) run one tcgen05.mma.cta_group::2 kind::i8 over
+//    both SMs: a pair owns a 256 x 256 output tile, each CTA loads its 128 rows
+//    of xq and its 128 rows of Wq (so each SM moves 32 KiB of operands per
+//    128-deep K block instead of 48 KiB for a 128 x 256 tile on one SM) and
+//    holds a 128 x 256 int32 accumulator in its own TMEM;
+//  * persistent grid (one pair per two SMs), tiles in a grouped raster;
+//  * warp 0: TMA producer into a 5-stage shared-memory ring; both CTAs' loads
+//    complete on the pair leader's (rank 0's) full barrier;
+//  * warp 1 of the leader issues the MMAs (M = 256, N = 256, K = 32 each) into
+//    one of two 256-column accumulators and commits each stage and each
+//    finished accumulator to the barriers of both CTAs;
+//  * warps 2-9 (8 per CTA): epilogue.  tcgen05.ld, then exact int32 -> fp64
+//    (2^52 magic number), acc * sx exact in fp64, one fused multiply-add with
+//    sw and bias (pre-converted to fp64 once per tile in shared memory), and
+//    the fp64 -> bf16 round-to-nearest-even done with integer operations on the
+//    double's bits; rows staged in a swizzled shared buffer and written with TMA
+//    stores that clip the M and N edges.  Conversions avoid the XU pipe, whose
+//    throughput made the epilogue the bottleneck.
+// Every mbarrier wait is bounded (sm100.cuh); no load uses cluster multicast.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -32,23 +36,29 @@
 namespace qk {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
+constexpr int BM = 128;   // rows per CTA (the pair covers 256)
+constexpr int BN = 256;   // columns per tile (each CTA loads 128 rows of Wq)
+constexpr int BK = 128;   // K per stage (bytes = elements)
+constexpr int STAGES = 5;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int A_BYTES = BM * BK;                  // 16 KiB
-constexpr int B_BYTES = BN * BK;                  // 32 KiB
-constexpr int STG_BYTES = 32 * 128;               // 32 rows x 128 B per staging buffer
+constexpr int B_BYTES = (BN / 2) * BK;            // 16 KiB
+constexpr uint32_t STAGE_TX = 2 * (A_BYTES + B_BYTES);  // both CTAs' loads
+constexpr int STG_BYTES = 32 * 128;               // 32 rows x 128 B
+constexpr int TAB_DOUBLES = 2 * BN;               // sw then bias, one tile
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_BYTES;
 constexpr int SMEM_STG = SMEM_B + STAGES * B_BYTES;
-constexpr int SMEM_BAR = SMEM_STG + kEpiWarps * 2 * STG_BYTES;
-constexpr int kNumBars = 2 * STAGES + 4;          // full, empty, tmem_full x2, tmem_empty x2
+constexpr int SMEM_TAB = SMEM_STG + kEpiWarps * STG_BYTES;
+constexpr int SMEM_BAR = SMEM_TAB + 2 * TAB_DOUBLES * 8;  // two tile tables
+constexpr int kNumBars = 2 * STAGES + 6;          // + two table-ready barriers
 constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
 constexpr int SMEM_USED = SMEM_SLOT + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;      // room to align the base to 1024 B
 constexpr int kTmemCols = 2 * BN;                 // two accumulators
-constexpr int kGroupM = 16;
-constexpr uint32_t kIdesc = i8_idesc(BM, BN, true, true);
+constexpr int kGroupM = 8;                        // M tiles per raster group
+constexpr uint32_t kIdesc = i8_idesc(2 * BM, BN, true, true);
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -62,22 +72,36 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   nb = r / gm;
 }
 
-// fp64 -> bf16 with one rounding to nearest-even: round to odd into fp32 (24
-// bits, at least two more than bf16's 8), then nearest-even to bf16.
-__device__ __forceinline__ float f64_to_f32_odd(double v) {
-  float f = __double2float_rz(v);
-  if ((double)f != v) f = __uint_as_float(__float_as_uint(f) | 1u);
-  return f;
+// Exact int32 -> fp64 without a conversion instruction: the double with high
+// word 0x43300000 and low word a + 2^31 is 2^52 + 2^31 + a.
+__device__ __forceinline__ double i32_to_f64(uint32_t a) {
+  return __hiloint2double(0x43300000, (int)(a ^ 0x80000000u)) - 4503601774854144.0;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
+// fp64 -> bf16 with one rounding to nearest-even, for |v| >= 2^-126 by integer
+// operations on the bits (keep the sign, the 11-bit exponent and 7 mantissa
+// bits; round on bit 12 of the high word with the rest as sticky bits), and for
+// smaller magnitudes through round-to-odd into fp32.
+__device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
+  const uint32_t hi = (uint32_t)__double2hiint(v);
+  const uint32_t lo = (uint32_t)__double2loint(v);
+  const uint32_t sign = (hi >> 16) & 0x8000u;
+  const uint32_t mag = hi & 0x7FFFFFFFu;
+  if (mag < 0x38100000u) {  // |v| < 2^-126 (bf16 subnormal range) or zero
+    if ((mag | lo) == 0u) return sign;
+    float f = __double2float_rz(v);
+    if ((double)f != v) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+  }
+  const uint32_t keep = mag >> 13;                          // exponent | 7 mantissa bits
+  const uint32_t low13 = (mag & 0x1FFFu) | min(lo, 1u);     // round bit 12, sticky below
+  const uint32_t up = (low13 + 0x0FFFu + (keep & 1u)) >> 13;
+  const uint32_t bits = min(keep + up - (896u << 7), 0x7F80u);  // rebias 1023 -> 127
+  return sign | bits;
 }
 
 template <bool kAccOut>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const float* __restrict__ sx,
                      const float* __restrict__ sw, const float* __restrict__ bias, int M, int N,
@@ -91,11 +115,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  auto table_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 4 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SMEM_SLOT);
+  double* tab = reinterpret_cast<double*>(smem + SMEM_TAB);
 
+  const uint32_t rank = cluster_ctarank();  // 0 leads the pair
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tiles_m = (M + BM - 1) / BM;
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int tiles_m = (M + 2 * BM - 1) / (2 * BM);
   const int tiles_n = (N + BN - 1) / BN;
   const int num_tiles = tiles_m * tiles_n;
   const int num_kb = (K + BK - 1) / BK;
@@ -110,16 +139,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), kEpiWarps);
+      mbar_init(tempty_bar(a), 2 * kEpiWarps);
+      mbar_init(table_bar(a), 32 * kEpiWarps);
     }
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
   }
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers and TMEM of both CTAs are ready
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -132,17 +163,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
         int mb, nb;
         tile_coords(t, tiles_m, tiles_n, mb, nb);
+        const int arow = mb * 2 * BM + (int)rank * BM;
+        const int brow = nb * BN + (int)rank * (BN / 2);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, err)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(stage), A_BYTES + B_BYTES);
-          tma_load_2d(sbase + SMEM_A + stage * A_BYTES, &tmA, kb * BK, mb * BM, full_bar(stage));
-          tma_load_2d(sbase + SMEM_B + stage * B_BYTES, &tmB, kb * BK, nb * BN, full_bar(stage));
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), STAGE_TX);
+          const uint32_t lead_full = mapa_shared(full_bar(stage), 0);
+          tma_load_2d_pair(sbase + SMEM_A + stage * A_BYTES, &tmA, kb * BK, arow, lead_full);
+          tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES, &tmB, kb * BK, brow, lead_full);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -151,14 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------- MMA issuer (pair leader)
+    if (rank == 0 && lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t aphase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
         if (!mbar_wait(tempty_bar(acc), aphase ^ 1u, err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -172,16 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = sbase + SMEM_B + stage * B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
-            mma_i8(d_tmem, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk),
-                   kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            mma_i8_pair(d_tmem, sw128_kmajor_desc(a_addr + 32 * kk),
+                        sw128_kmajor_desc(b_addr + 32 * kk), kIdesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          mma_commit(empty_bar(stage));  // frees the smem stage when these MMAs finish
+          mma_commit_pair(empty_bar(stage), 0x3);  // frees this stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        mma_commit(tfull_bar(acc));  // accumulator ready for the epilogue
+        mma_commit_pair(tfull_bar(acc), 0x3);  // accumulator ready in both CTAs
         if (++acc == 2) {
           acc = 0;
           aphase ^= 1u;
@@ -190,34 +224,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const uint32_t stg0 = sbase + SMEM_STG + (uint32_t)((warp - 2) * 2 * STG_BYTES);
-    uint8_t* stg0_ptr = smem + SMEM_STG + (warp - 2) * 2 * STG_BYTES;
+    const int e = warp - 2;           // 0..7
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int half = e >> 2;          // column half of the tile
+    const int et = threadIdx.x - 64;  // 0..255
+    const uint32_t stg = sbase + SMEM_STG + (uint32_t)(e * STG_BYTES);
+    uint8_t* stg_ptr = smem + SMEM_STG + e * STG_BYTES;
     int acc = 0;
     uint32_t aphase = 0;
-    int use = 0;  // staging-buffer use counter (alternates the two buffers)
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    int iter = 0;
+    for (int t = pair; t < num_tiles; t += num_pairs, ++iter) {
       int mb, nb;
       tile_coords(t, tiles_m, tiles_n, mb, nb);
+      const int ncol0 = nb * BN;
+      double* tsw = tab + (iter & 1) * TAB_DOUBLES;
+      double* tb = tsw + BN;
+      if constexpr (!kAccOut) {
+        // this tile's sw and bias as fp64 (one column per epilogue thread); the
+        // barrier also tells each thread that all others finished the tile
+        // before the previous one, the last user of this table buffer
+        const int n = ncol0 + et;
+        tsw[et] = n < N ? (double)__ldg(sw + n) : 0.0;
+        tb[et] = (n < N && bias != nullptr) ? (double)__ldg(bias + n) : 0.0;
+        mbar_arrive(table_bar(iter & 1));
+        if (!mbar_wait(table_bar(iter & 1), (uint32_t)(iter >> 1) & 1u, err)) break;
+      }
       if (!mbar_wait(tfull_bar(acc), aphase, err)) break;
       tc_fence_after();
-      const int row0 = mb * BM + q * 32;  // first row of this warp's 32-row slab
+      const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;  // this warp's 32-row slab
       const int row = row0 + lane;
-      const double sxd = (!kAccOut && row < M) ? (double)sx[row] : 0.0;
+      const double sxd = (!kAccOut && row < M) ? (double)__ldg(sx + row) : 0.0;
       const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       constexpr int kChunk = kAccOut ? 32 : 64;  // columns per 128-byte staged row
-      for (int c = 0; c < BN / kChunk; ++c) {
-        const int n0 = nb * BN + c * kChunk;
+      constexpr int kChunks = (BN / 2) / kChunk;
+#pragma unroll 1
+      for (int c = 0; c < kChunks; ++c) {
+        const int col0 = half * (BN / 2) + c * kChunk;
+        const int n0 = ncol0 + col0;
         uint32_t v[kChunk];
-        tmem_ld32(t_lane + (uint32_t)(c * kChunk), *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(t_lane + (uint32_t)col0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
         if constexpr (!kAccOut)
-          tmem_ld32(t_lane + (uint32_t)(c * kChunk + 32), *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          tmem_ld32(t_lane + (uint32_t)(col0 + 32), *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_ld_wait();
-        if (c == BN / kChunk - 1) {
-          // all TMEM reads of this accumulator are done: hand it back
+        if (c == kChunks - 1) {
+          // all TMEM reads of this accumulator are done: hand it back to the leader
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(acc));
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
         }
         if (n0 >= N || row0 >= M) continue;  // whole box outside y
         uint32_t out[32];
@@ -226,31 +279,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) out[j] = v[j];
         } else {
 #pragma unroll
-          for (int j4 = 0; j4 < 16; ++j4) {
-            const int n = n0 + 4 * j4;
-            float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (n < N) {
-              w4 = __ldg(reinterpret_cast<const float4*>(sw + n));
-              if (bias != nullptr) b4 = __ldg(reinterpret_cast<const float4*>(bias + n));
-            }
-            const double p0 = (double)(int)v[4 * j4 + 0] * sxd;
-            const double p1 = (double)(int)v[4 * j4 + 1] * sxd;
-            const double p2 = (double)(int)v[4 * j4 + 2] * sxd;
-            const double p3 = (double)(int)v[4 * j4 + 3] * sxd;
-            const float y0 = f64_to_f32_odd(fma(p0, (double)w4.x, (double)b4.x));
-            const float y1 = f64_to_f32_odd(fma(p1, (double)w4.y, (double)b4.y));
-            const float y2 = f64_to_f32_odd(fma(p2, (double)w4.z, (double)b4.z));
-            const float y3 = f64_to_f32_odd(fma(p3, (double)w4.w, (double)b4.w));
-            out[2 * j4] = pack_bf16x2(y0, y1);
-            out[2 * j4 + 1] = pack_bf16x2(y2, y3);
+          for (int j = 0; j < 64; j += 2) {
+            const double y0 = fma(i32_to_f64(v[j]) * sxd, tsw[col0 + j], tb[col0 + j]);
+            const double y1 = fma(i32_to_f64(v[j + 1]) * sxd, tsw[col0 + j + 1], tb[col0 + j + 1]);
+            out[j >> 1] = f64_to_bf16_bits(y0) | (f64_to_bf16_bits(y1) << 16);
           }
         }
-        // staging buffer: wait until the TMA store that used it two chunks ago
-        // has finished reading it
-        const int buf = use & 1;
-        if (lane == 0) bulk_wait_read<1>();
+        // the TMA store that last read the staging buffer must be done with it
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
-        uint8_t* rowp = stg0_ptr + buf * STG_BYTES + lane * 128;
+        uint8_t* rowp = stg_ptr + lane * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int phys = j ^ (lane & 7);  // 128-byte swizzle of the TMA box
@@ -260,10 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmC, stg0 + (uint32_t)(buf * STG_BYTES), n0, row0);
+          tma_store_2d(&tmC, stg, n0, row0);
           bulk_commit();
         }
-        ++use;
       }
       if (++acc == 2) {
         acc = 0;
@@ -273,10 +310,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) bulk_wait<0>();
   }
 
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // every remote arrival and MMA of the pair is done
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
 bool g_attr_done[2][64];
@@ -291,7 +329,7 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
                       (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K, (uint64_t)N,
-                      (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+                      (uint64_t)K, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (acc_mode) {
     if (!encode_tmap_2d(&tC, CU_TENSOR_MAP_DATA_TYPE_INT32, acc_out, (uint64_t)N, (uint64_t)M,
@@ -313,8 +351,9 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   }
   int* err = device_error_word();
   if (err == nullptr) return cudaErrorUnknown;
-  const long long tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  const long long tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+  const long long pairs = num_sms() / 2;
+  const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

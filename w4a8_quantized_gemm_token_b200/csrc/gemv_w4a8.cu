@@ -231,6 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+size_t g_smem_set[2][64];
+
 }  // namespace
 
 cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
@@ -249,9 +251,15 @@ cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* x
   int* err = device_error_word();
   if (err == nullptr) return cudaErrorUnknown;
   auto kernel = M <= 8 ? w4a8_gemv_kernel<1> : w4a8_gemv_kernel<2>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int tt = M <= 8 ? 0 : 1;
+  if (dev >= 64 || g_smem_set[tt][dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kGemvSmemLimit);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) g_smem_set[tt][dev] = kGemvSmemLimit;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
