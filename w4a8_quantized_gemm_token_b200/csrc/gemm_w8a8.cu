@@ -17,7 +17,7 @@
 //  * warp 1 of the leader issues the MMAs (M = 256, N = 256, K = 32 each) into
 //    one of two 256-column accumulators and commits each stage and each
 //    finished accumulator to the barriers of both CTAs;
-//  * warps 2-9 (8 per CTA): epilogue.  tcgen05.ld, then exact int32 -> fp64
+//  * warps 2-5 (4 per CTA): epilogue.  tcgen05.ld, then exact int32 -> fp64
 //    (2^52 magic number), acc * sx exact in fp64, one fused multiply-add with
 //    sw and bias (pre-converted to fp64 once per tile in shared memory), and
 //    the fp64 -> bf16 round-to-nearest-even done with integer operations on the
@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 
 #include "qk_internal.h"
 #include "sm100.cuh"
@@ -40,33 +41,46 @@ constexpr int BM = 128;   // rows per CTA (the pair covers 256)
 constexpr int BN = 256;   // columns per tile (each CTA loads 128 rows of Wq)
 constexpr int BK = 128;   // K per stage (bytes = elements)
 constexpr int STAGES = 5;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 4;  // 6 warps: at most 2 per SM sub-partition, 255 registers each
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int A_BYTES = BM * BK;                  // 16 KiB
 constexpr int B_BYTES = (BN / 2) * BK;            // 16 KiB
 constexpr uint32_t STAGE_TX = 2 * (A_BYTES + B_BYTES);  // both CTAs' loads
 constexpr int STG_BYTES = 32 * 128;               // 32 rows x 128 B
-constexpr int TAB_DOUBLES = 2 * BN;               // sw then bias, one tile
+constexpr int TAB_BYTES = BN * 16;                // per column {sw, bias, threshold, 0}
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_BYTES;
 constexpr int SMEM_STG = SMEM_B + STAGES * B_BYTES;
-constexpr int SMEM_TAB = SMEM_STG + kEpiWarps * STG_BYTES;
-constexpr int SMEM_BAR = SMEM_TAB + 2 * TAB_DOUBLES * 8;  // two tile tables
+constexpr int SMEM_TAB = SMEM_STG + kEpiWarps * 2 * STG_BYTES;  // two staging buffers per warp
+constexpr int SMEM_BAR = SMEM_TAB + 2 * TAB_BYTES;  // two tile tables
 constexpr int kNumBars = 2 * STAGES + 6;          // + two table-ready barriers
 constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
 constexpr int SMEM_USED = SMEM_SLOT + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;      // room to align the base to 1024 B
 constexpr int kTmemCols = 2 * BN;                 // two accumulators
-constexpr int kGroupM = 8;                        // M tiles per raster group
 constexpr uint32_t kIdesc = i8_idesc(2 * BM, BN, true, true);
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
-__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& mb, int& nb) {
-  const int per_group = kGroupM * tiles_n;
+// An output takes the fp32 fast path when |v32| >= max(kGuard |bias|, kTiny).
+constexpr float kGuard = 0.000244140625f;   // 2^-12
+constexpr float kTiny = 7.888609052210118e-31f;  // 2^-100
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Raster: groups of `group_m` M tiles; inside a group, consecutive tiles walk
+// down the M tiles first, then across N, so the CTA pairs running at the same
+// time share the group's rows of xq (kept in L2) and a few Wq tiles.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int group_m, int& mb,
+                                            int& nb) {
+  const int per_group = group_m * tiles_n;
   const int gid = t / per_group;
-  const int first_m = gid * kGroupM;
-  const int gm = min(tiles_m - first_m, kGroupM);
+  const int first_m = gid * group_m;
+  const int gm = min(tiles_m - first_m, group_m);
   const int r = t - gid * per_group;
   mb = first_m + r % gm;
   nb = r / gm;
@@ -105,7 +119,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const float* __restrict__ sx,
                      const float* __restrict__ sw, const float* __restrict__ bias, int M, int N,
-                     int K, int* err) {
+                     int K, int group_m, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -117,7 +131,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   auto table_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 4 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SMEM_SLOT);
-  double* tab = reinterpret_cast<double*>(smem + SMEM_TAB);
+  float4* tab = reinterpret_cast<float4*>(smem + SMEM_TAB);
 
   const uint32_t rank = cluster_ctarank();  // 0 leads the pair
   const int warp = threadIdx.x >> 5;
@@ -165,7 +179,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += num_pairs) {
         int mb, nb;
-        tile_coords(t, tiles_m, tiles_n, mb, nb);
+        tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
         const int arow = mb * 2 * BM + (int)rank * BM;
         const int brow = nb * BN + (int)rank * (BN / 2);
         for (int kb = 0; kb < num_kb; ++kb) {
@@ -224,28 +238,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;           // 0..7
+    const int e = warp - 2;           // 0..3
     const int q = warp & 3;           // TMEM lane quarter this warp may access
-    const int half = e >> 2;          // column half of the tile
-    const int et = threadIdx.x - 64;  // 0..255
-    const uint32_t stg = sbase + SMEM_STG + (uint32_t)(e * STG_BYTES);
-    uint8_t* stg_ptr = smem + SMEM_STG + e * STG_BYTES;
+    const int et = threadIdx.x - 64;  // 0..127
+    const uint32_t stg0 = sbase + SMEM_STG + (uint32_t)(e * 2 * STG_BYTES);
+    uint8_t* stg0_ptr = smem + SMEM_STG + e * 2 * STG_BYTES;
     int acc = 0;
     uint32_t aphase = 0;
     int iter = 0;
+    int use = 0;  // staging-buffer use counter (alternates the two buffers)
     for (int t = pair; t < num_tiles; t += num_pairs, ++iter) {
       int mb, nb;
-      tile_coords(t, tiles_m, tiles_n, mb, nb);
+      tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
       const int ncol0 = nb * BN;
-      double* tsw = tab + (iter & 1) * TAB_DOUBLES;
-      double* tb = tsw + BN;
+      float4* tcol = tab + (iter & 1) * BN;
       if constexpr (!kAccOut) {
-        // this tile's sw and bias as fp64 (one column per epilogue thread); the
-        // barrier also tells each thread that all others finished the tile
+        // this tile's per-column constants (one column per epilogue thread);
+        // the barrier also tells each thread that all others finished the tile
         // before the previous one, the last user of this table buffer
-        const int n = ncol0 + et;
-        tsw[et] = n < N ? (double)__ldg(sw + n) : 0.0;
-        tb[et] = (n < N && bias != nullptr) ? (double)__ldg(bias + n) : 0.0;
+#pragma unroll
+        for (int k = 0; k < BN / (32 * kEpiWarps); ++k) {
+          const int col = et + 32 * kEpiWarps * k;
+          const int n = ncol0 + col;
+          const float w = n < N ? __ldg(sw + n) : 0.0f;
+          const float b = (n < N && bias != nullptr) ? __ldg(bias + n) : 0.0f;
+          tcol[col] = make_float4(w, b, fmaxf(kGuard * fabsf(b), kTiny), 0.0f);
+        }
         mbar_arrive(table_bar(iter & 1));
         if (!mbar_wait(table_bar(iter & 1), (uint32_t)(iter >> 1) & 1u, err)) break;
       }
@@ -253,42 +271,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;  // this warp's 32-row slab
       const int row = row0 + lane;
-      const double sxd = (!kAccOut && row < M) ? (double)__ldg(sx + row) : 0.0;
+      const float sxf = (!kAccOut && row < M) ? __ldg(sx + row) : 0.0f;
       const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       constexpr int kChunk = kAccOut ? 32 : 64;  // columns per 128-byte staged row
-      constexpr int kChunks = (BN / 2) / kChunk;
+      constexpr int kChunks = BN / kChunk;
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
-        const int col0 = half * (BN / 2) + c * kChunk;
+        const int col0 = c * kChunk;
         const int n0 = ncol0 + col0;
-        uint32_t v[kChunk];
-        tmem_ld32(t_lane + (uint32_t)col0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        if constexpr (!kAccOut)
-          tmem_ld32(t_lane + (uint32_t)(col0 + 32), *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_ld_wait();
-        if (c == kChunks - 1) {
-          // all TMEM reads of this accumulator are done: hand it back to the leader
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
-        }
-        if (n0 >= N || row0 >= M) continue;  // whole box outside y
         uint32_t out[32];
-        if constexpr (kAccOut) {
+        // two 32-column halves per chunk keep the live registers down
 #pragma unroll
-          for (int j = 0; j < 32; ++j) out[j] = v[j];
-        } else {
+        for (int h = 0; h < kChunk / 32; ++h) {
+          uint32_t v[32];
+          tmem_ld32(t_lane + (uint32_t)(col0 + 32 * h), v);
+          tmem_ld_wait();
+          if (c == kChunks - 1 && h == kChunk / 32 - 1) {
+            // all TMEM reads of this accumulator are done: hand it back to the leader
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+          }
+          if constexpr (kAccOut) {
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const double y0 = fma(i32_to_f64(v[j]) * sxd, tsw[col0 + j], tb[col0 + j]);
-            const double y1 = fma(i32_to_f64(v[j + 1]) * sxd, tsw[col0 + j + 1], tb[col0 + j + 1]);
-            out[j >> 1] = f64_to_bf16_bits(y0) | (f64_to_bf16_bits(y1) << 16);
+            for (int j = 0; j < 32; ++j) out[j] = v[j];
+          } else {
+            // fast path in fp32: v32 = fma(fp32(acc) * sx, sw, bias).  Its error
+            // is at most 2^-23 |acc sx sw| + 2^-24 |v32|, below 1/8 bf16 ulp when
+            // |v32| >= 2^-12 |bias|, so it then rounds to within 1 ulp of the
+            // exact value.  Other outputs (cancellation against the bias, or
+            // magnitudes near the fp32 underflow) take the exact fp64 path.
+            const float4* tc = tcol + col0 + 32 * h;
+            uint32_t* o = out + 16 * h;
+            uint32_t slow = 0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float4 c0 = tc[j], c1 = tc[j + 1];
+              const float r0 = __fmaf_rn(__fmul_rn(__int2float_rn((int)v[j]), sxf), c0.x, c0.y);
+              const float r1 = __fmaf_rn(__fmul_rn(__int2float_rn((int)v[j + 1]), sxf), c1.x, c1.y);
+              const bool s0 = !(fabsf(r0) >= c0.z) && v[j] != 0u;
+              const bool s1 = !(fabsf(r1) >= c1.z) && v[j + 1] != 0u;
+              slow |= ((s0 ? 1u : 0u) | (s1 ? 2u : 0u)) << j;
+              o[j >> 1] = pack_bf16x2(r0, r1);
+            }
+            if (__any_sync(0xFFFFFFFFu, slow != 0u)) {
+              const double sxd = (double)sxf;
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                const uint32_t m8 = (slow >> (8 * g)) & 0xFFu;
+                if (__any_sync(0xFFFFFFFFu, m8 != 0u)) {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const int j = 8 * g + i;
+                    if ((m8 >> i) & 1u) {
+                      const float4 cj = tc[j];
+                      const double yj =
+                          fma(i32_to_f64(v[j]) * sxd, (double)cj.x, (double)cj.y);
+                      const uint32_t hb = f64_to_bf16_bits(yj);
+                      o[j >> 1] = (j & 1) ? ((o[j >> 1] & 0x0000FFFFu) | (hb << 16))
+                                          : ((o[j >> 1] & 0xFFFF0000u) | hb);
+                    }
+                  }
+                }
+              }
+            }
           }
         }
-        // the TMA store that last read the staging buffer must be done with it
-        if (lane == 0) bulk_wait_read<0>();
+        if (n0 >= N || row0 >= M) continue;  // whole box outside y
+        // the TMA store that used this staging buffer two chunks ago must be
+        // done reading it
+        const int buf = use & 1;
+        if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
-        uint8_t* rowp = stg_ptr + lane * 128;
+        uint8_t* rowp = stg0_ptr + buf * STG_BYTES + lane * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int phys = j ^ (lane & 7);  // 128-byte swizzle of the TMA box
@@ -298,9 +353,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmC, stg, n0, row0);
+          tma_store_2d(&tmC, stg0 + (uint32_t)(buf * STG_BYTES), n0, row0);
           bulk_commit();
         }
+        ++use;
       }
       if (++acc == 2) {
         acc = 0;
@@ -351,7 +407,13 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   }
   int* err = device_error_word();
   if (err == nullptr) return cudaErrorUnknown;
-  const long long tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+  const long long tiles_m = (M + 2 * BM - 1) / (2 * BM);
+  const long long tiles = tiles_m * ((N + BN - 1) / BN);
+  // A raster group's rows of xq (256 rows x K bytes per M tile) should stay in
+  // L2 while the group sweeps all of Wq: about 40 MB of the 126 MB L2.
+  long long group_m = (40ll << 20) / (2 * BM * K);
+  if (const char* env = std::getenv("QK_GROUP_M")) group_m = std::atoll(env);
+  group_m = group_m < 1 ? 1 : (group_m > tiles_m ? tiles_m : group_m);
   const long long pairs = num_sms() / 2;
   const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
 
@@ -365,7 +427,8 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, tA, tB, tC, sx, sw, bias, (int)M, (int)N, (int)K, err);
+  return cudaLaunchKernelEx(&cfg, kernel, tA, tB, tC, sx, sw, bias, (int)M, (int)N, (int)K,
+                            (int)group_m, err);
 }
 
 }  // namespace qk
