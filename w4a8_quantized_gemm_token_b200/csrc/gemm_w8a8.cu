@@ -12,8 +12,9 @@
 //    128-deep K block instead of 48 KiB for a 128 x 256 tile on one SM) and
 //    holds a 128 x 256 int32 accumulator in its own TMEM;
 //  * persistent grid (one pair per two SMs), tiles in a grouped raster;
-//  * warp 0: TMA producer into a 5-stage shared-memory ring; both CTAs' loads
-//    complete on the pair leader's (rank 0's) full barrier;
+//  * warp 0: TMA producer into a 3-stage shared-memory ring of 256-deep K
+//    blocks (64 KiB per stage per CTA, as two 128-byte-wide swizzled slabs per
+//    operand); both CTAs' loads complete on the pair leader's full barrier;
 //  * warp 1 of the leader issues the MMAs (M = 256, N = 256, K = 32 each) into
 //    one of two 256-column accumulators and commits each stage and each
 //    finished accumulator to the barriers of both CTAs;
@@ -39,19 +40,27 @@ namespace {
 
 constexpr int BM = 128;   // rows per CTA (the pair covers 256)
 constexpr int BN = 256;   // columns per tile (each CTA loads 128 rows of Wq)
-constexpr int BK = 128;   // K per stage (bytes = elements)
-constexpr int STAGES = 5;
+constexpr int BK = 256;   // K per stage (bytes = elements): two 128-byte swizzled slabs
+constexpr int kSlabs = BK / 128;
+#ifndef QK_W8A8_STAGES
+#define QK_W8A8_STAGES 3
+#endif
+#ifndef QK_W8A8_STG_BUFS
+#define QK_W8A8_STG_BUFS 1
+#endif
+constexpr int STAGES = QK_W8A8_STAGES;
 constexpr int kEpiWarps = 4;  // 6 warps: at most 2 per SM sub-partition, 255 registers each
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int A_BYTES = BM * BK;                  // 16 KiB
-constexpr int B_BYTES = (BN / 2) * BK;            // 16 KiB
+constexpr int A_BYTES = BM * BK;                  // 32 KiB
+constexpr int B_BYTES = (BN / 2) * BK;            // 32 KiB
 constexpr uint32_t STAGE_TX = 2 * (A_BYTES + B_BYTES);  // both CTAs' loads
 constexpr int STG_BYTES = 32 * 128;               // 32 rows x 128 B
 constexpr int TAB_BYTES = BN * 16;                // per column {sw, bias, threshold, 0}
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_BYTES;
 constexpr int SMEM_STG = SMEM_B + STAGES * B_BYTES;
-constexpr int SMEM_TAB = SMEM_STG + kEpiWarps * 2 * STG_BYTES;  // two staging buffers per warp
+constexpr int kStgBufs = QK_W8A8_STG_BUFS;        // staging buffers per epilogue warp
+constexpr int SMEM_TAB = SMEM_STG + kEpiWarps * kStgBufs * STG_BYTES;
 constexpr int SMEM_BAR = SMEM_TAB + 2 * TAB_BYTES;  // two tile tables
 constexpr int kNumBars = 2 * STAGES + 6;          // + two table-ready barriers
 constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
@@ -189,8 +198,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), STAGE_TX);
           const uint32_t lead_full = mapa_shared(full_bar(stage), 0);
-          tma_load_2d_pair(sbase + SMEM_A + stage * A_BYTES, &tmA, kb * BK, arow, lead_full);
-          tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES, &tmB, kb * BK, brow, lead_full);
+#pragma unroll
+          for (int sl = 0; sl < kSlabs; ++sl) {  // 128-byte-wide K slabs
+            tma_load_2d_pair(sbase + SMEM_A + stage * A_BYTES + sl * (A_BYTES / kSlabs), &tmA,
+                             kb * BK + 128 * sl, arow, lead_full);
+            tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES + sl * (B_BYTES / kSlabs), &tmB,
+                             kb * BK + 128 * sl, brow, lead_full);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -220,8 +234,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = sbase + SMEM_B + stage * B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
-            mma_i8_pair(d_tmem, sw128_kmajor_desc(a_addr + 32 * kk),
-                        sw128_kmajor_desc(b_addr + 32 * kk), kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            // K step kk: slab kk / 4, 32-byte column (kk % 4) inside the swizzle atom
+            const uint32_t ao = (kk >> 2) * (A_BYTES / kSlabs) + 32 * (kk & 3);
+            const uint32_t bo = (kk >> 2) * (B_BYTES / kSlabs) + 32 * (kk & 3);
+            mma_i8_pair(d_tmem, sw128_kmajor_desc(a_addr + ao),
+                        sw128_kmajor_desc(b_addr + bo), kIdesc, (kb | kk) != 0 ? 1u : 0u);
           }
           mma_commit_pair(empty_bar(stage), 0x3);  // frees this stage in both CTAs
           if (++stage == STAGES) {
@@ -241,8 +258,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int e = warp - 2;           // 0..3
     const int q = warp & 3;           // TMEM lane quarter this warp may access
     const int et = threadIdx.x - 64;  // 0..127
-    const uint32_t stg0 = sbase + SMEM_STG + (uint32_t)(e * 2 * STG_BYTES);
-    uint8_t* stg0_ptr = smem + SMEM_STG + e * 2 * STG_BYTES;
+    const uint32_t stg0 = sbase + SMEM_STG + (uint32_t)(e * kStgBufs * STG_BYTES);
+    uint8_t* stg0_ptr = smem + SMEM_STG + e * kStgBufs * STG_BYTES;
     int acc = 0;
     uint32_t aphase = 0;
     int iter = 0;
@@ -338,10 +355,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         if (n0 >= N || row0 >= M) continue;  // whole box outside y
-        // the TMA store that used this staging buffer two chunks ago must be
-        // done reading it
-        const int buf = use & 1;
-        if (lane == 0) bulk_wait_read<1>();
+        // the TMA store that last used this staging buffer must be done reading it
+        const int buf = use % kStgBufs;
+        if (lane == 0) bulk_wait_read<kStgBufs - 1>();
         __syncwarp();
         uint8_t* rowp = stg0_ptr + buf * STG_BYTES + lane * 128;
 #pragma unroll
@@ -383,9 +399,9 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   const bool acc_mode = acc_out != nullptr;
   CUtensorMap tA, tB, tC;
   if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
-                      (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                      (uint64_t)K, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K, (uint64_t)N,
-                      (uint64_t)K, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+                      (uint64_t)K, 128, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (acc_mode) {
     if (!encode_tmap_2d(&tC, CU_TENSOR_MAP_DATA_TYPE_INT32, acc_out, (uint64_t)N, (uint64_t)M,
