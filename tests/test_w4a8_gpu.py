@@ -70,3 +70,68 @@ def test_gemv_deterministic(qk, orc):
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert torch.equal(ys[0].view(torch.int16), y.view(torch.int16))
+
+
+GEMM_SHAPES = [(17, 64, 8), (129, 192, 72), (300, 1024, 264), (64, 4096, 136), (257, 320, 64),
+               (16, 256, 128)]
+
+
+@pytest.mark.parametrize("MKN", GEMM_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_gemm_group_acc_and_output(qk, orc, MKN):
+    M, K, N = MKN
+    case = synthetic.LinearCase("m", M=M, K=K, N=N, bias=(N % 16 == 8), seed=M * 17 + K + N)
+    xb, dev_w, ora_w, b = prepare(qk, orc, case)
+    x = to_dev_bf16(xb)
+    xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
+    acc = qk.qk_debug_w4a8_group_acc(xq, dev_w[0], 0, M, GEMM)
+    bias = to_dev(b) if b is not None else None
+    y = qk.qk_w4a8_gemm(xq, sx, xsum, *dev_w, bias, route=GEMM)
+    torch.cuda.synchronize()
+    y_o, xq_o, sx_o, xsum_o, acc_o = orc.w4a8_linear(xb, *ora_w, b)
+    assert np.array_equal(host(acc).astype(np.int64), acc_o)
+    d = bf16_ulp_distance(t2bits(y), y_o)
+    assert d.max() <= TOL_ULP, f"worst {d.max()} ulp"
+    if M > 16:  # the public call takes the GEMM route
+        y2 = qk.qk_w4a8_linear(x, *dev_w, bias)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    qk.qk_check_device_error()
+
+
+def test_w4a8_gemm_config_4096(qk, orc):
+    """The M = 4096 W4A8 workload: every code bit-exact, per-group sums and
+    outputs of sampled row blocks (first, last, tile edges) against the oracle."""
+    case = synthetic.W4A8[3]
+    xb, dev_w, ora_w, _ = prepare(qk, orc, case)
+    x = to_dev_bf16(xb)
+    y = qk.qk_w4a8_linear(x, *dev_w)
+    xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
+    torch.cuda.synchronize()
+    xq_o, sx_o = orc.quant_act(xb)
+    assert np.array_equal(host(xq), xq_o) and np.array_equal(host(sx), sx_o)
+    worst = 0
+    for m0, m1 in [(0, 4), (126, 130), (2047, 2051), (4092, 4096)]:
+        acc = qk.qk_debug_w4a8_group_acc(xq, dev_w[0], m0, m1, GEMM)
+        torch.cuda.synchronize()
+        acc_o = orc.w4a8_group_acc(xq_o[m0:m1], ora_w[0])
+        assert np.array_equal(host(acc).astype(np.int64), acc_o)
+        y_o = orc.w4a8_dequant(acc_o, orc.group_sums(xq_o[m0:m1]), sx_o[m0:m1], ora_w[1], ora_w[2])
+        d = bf16_ulp_distance(t2bits(y[m0:m1]), y_o)
+        worst = max(worst, int(d.max()))
+    print(f"{case.name}: sampled worst={worst} ulp")
+    assert worst <= TOL_ULP
+
+
+def test_routes_agree_at_m16(qk, orc):
+    """At M = 16 both routes apply: identical per-group integers, outputs equal
+    up to the fp64 summation order (at most 1 ulp)."""
+    case = synthetic.LinearCase("r", M=16, K=4096, N=1024, bias=True, seed=3)
+    xb, dev_w, _, b = prepare(qk, orc, case)
+    xq, sx, xsum = qk.qk_quantize_activations(to_dev_bf16(xb), with_xsum=True)
+    a_v = qk.qk_debug_w4a8_group_acc(xq, dev_w[0], 0, 16, GEMV)
+    a_m = qk.qk_debug_w4a8_group_acc(xq, dev_w[0], 0, 16, GEMM)
+    y_v = qk.qk_w4a8_gemm(xq, sx, xsum, *dev_w, to_dev(b), route=GEMV)
+    y_m = qk.qk_w4a8_gemm(xq, sx, xsum, *dev_w, to_dev(b), route=GEMM)
+    torch.cuda.synchronize()
+    assert torch.equal(a_v, a_m)
+    assert bf16_ulp_distance(t2bits(y_v), t2bits(y_m)).max() <= 1
