@@ -62,7 +62,7 @@ typedef enum {
 
 /* Routes of the W4A8 product. */
 typedef enum {
-    QK_ROUTE_AUTO = 0, /* GEMV when M <= 16, else GEMM                        */
+    QK_ROUTE_AUTO = 0, /* GEMV when M <= 16 and it fits, else GEMM             */
     QK_ROUTE_GEMM = 1, /* tensor-core GEMM (tcgen05), any M                   */
     QK_ROUTE_GEMV = 2  /* weight-streaming GEMV, M <= 16 only                 */
 } qk_route;
@@ -220,7 +220,8 @@ qk_status qk_w8a8_linear_noalloc(const uint16_t *x, int64_t M, int64_t K,
  *   y[m, n] = bf16( sx[m] * sum_g ( s[n,g] * acc[m,n,g] + o[n,g] * xsum[m,g] )
  *                   + bias[n] ),
  * the fold evaluated in fp64 and rounded once to bf16.
- * M <= 16 takes the weight-streaming GEMV, larger M the tensor-core GEMM; both
+ * M <= 16 takes the weight-streaming GEMV when its per-CTA working set fits
+ * in shared memory (K <= 4096 at M = 16), otherwise the tensor-core GEMM; both
  * compute the same per-group integers and agree to the fp64 rounding order.
  *   x                  : bf16 bits [M, K]            (in)
  *   Wp, wscale, woffset: from qk_quantize_weights_int4 (in)
@@ -238,7 +239,8 @@ qk_status qk_w4a8_linear(const uint16_t *x, int64_t M, int64_t K,
 /*
  * The product half of qk_w4a8_linear on quantized activations (xq, sx and
  * xsum from qk_quantize_activations), with an explicit route (qk_route).
- * QK_ROUTE_GEMV with M > 16 returns QK_ERR_INVALID_ARG.
+ * QK_ROUTE_GEMV with M > 16 returns QK_ERR_INVALID_ARG; with a shape whose
+ * GEMV working set does not fit shared memory, QK_ERR_UNSUPPORTED_SHAPE.
  */
 qk_status qk_w4a8_gemm(const int8_t *xq, const float *sx, const int32_t *xsum,
                        int64_t M, int64_t K,

@@ -27,7 +27,7 @@ def prepare(qk, orc, case):
 
 
 GEMV_SHAPES = [(1, 64, 8), (1, 4096, 4096), (8, 4096, 4096), (16, 4096, 4096), (3, 192, 40),
-               (11, 1024, 264), (16, 16384, 128), (5, 640, 2056)]
+               (11, 1024, 264), (16, 3072, 128), (5, 640, 2056)]
 
 
 @pytest.mark.parametrize("MKN", GEMV_SHAPES, ids=lambda s: "x".join(map(str, s)))
@@ -135,3 +135,19 @@ def test_routes_agree_at_m16(qk, orc):
     torch.cuda.synchronize()
     assert torch.equal(a_v, a_m)
     assert bf16_ulp_distance(t2bits(y_v), t2bits(y_m)).max() <= 1
+
+
+def test_large_k_small_m_routes_to_gemm(qk, orc):
+    """M <= 16 with a K whose GEMV working set does not fit shared memory: the
+    explicit GEMV route is refused, the automatic route takes the GEMM."""
+    case = synthetic.LinearCase("lk", M=4, K=16384, N=64, bias=True, seed=8)
+    xb, dev_w, ora_w, b = prepare(qk, orc, case)
+    x = to_dev_bf16(xb)
+    xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
+    with pytest.raises(qk.QKError) as e:
+        qk.qk_w4a8_gemm(xq, sx, xsum, *dev_w, to_dev(b), route=GEMV)
+    assert e.value.status == 2
+    y = qk.qk_w4a8_linear(x, *dev_w, to_dev(b))
+    torch.cuda.synchronize()
+    y_o, _, _, _, _ = orc.w4a8_linear(xb, *ora_w, b)
+    assert bf16_ulp_distance(t2bits(y), y_o).max() <= TOL_ULP

@@ -111,8 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const uint16_t* __restrict__ woffset, const float* __restrict__ bias, int M,
                      int N, int K, int32_t* __restrict__ acc_out, int m0, int m1, int* err) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem<1024>(smem_raw);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + SMEM_BAR;
   auto full_bar = [&](int i) { return bar0 + 8u * i; };
@@ -167,6 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // The next kernel in the stream may become resident now (it waits for this
+  // grid to finish before it touches anything this grid reads or writes).
+  pdl_launch_dependents();
   pdl_wait();  // xq, sx and xsum come from the activation-quant kernel
 
 

@@ -130,8 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                      const float* __restrict__ sw, const float* __restrict__ bias, int M, int N,
                      int K, int group_m, int* err) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem<1024>(smem_raw);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + SMEM_BAR;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -177,6 +176,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // The next kernel in the stream may become resident now (it waits for this
+  // grid to finish before it touches anything this grid reads or writes).
+  pdl_launch_dependents();
   // Everything below reads what the previous kernel (activation quant) wrote.
   pdl_wait();
 

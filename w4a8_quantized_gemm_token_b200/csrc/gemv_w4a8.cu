@@ -7,20 +7,30 @@
 //   y[m, n] = bf16( sx[m] * sum_g (s[n,g] * acc + o[n,g] * xsum[m,g]) + bias[n] )
 // with the fold in fp64 and one rounding to bf16.
 //
-// Design (HBM-bound: the packed weights are ~97% of the bytes):
+// Design (HBM-bound: the packed weights are ~97% of the bytes; every operand of
+// the inner loop comes from shared memory so the loop never waits on L2):
 //  * each CTA owns R = 16 * RT weight rows; at kernel start, before waiting on
 //    the activation-quant kernel it depends on (programmatic dependent launch),
-//    warp 0 bulk-copies the CTA's whole weight slice (rows padded by 16 bytes
-//    against bank conflicts) and its fp16 scales / offsets into shared memory,
-//    so the weight stream is in flight while the previous kernel finishes;
-//  * the 8 warps split into RT row tiles x (8 / RT) K ranges; each K range has
-//    its own mbarrier so a warp starts as soon as its part has landed;
-//  * nibbles are unpacked in registers (two AND/shift + two byte permutes per
-//    8 codes) straight into the A fragments of mma.sync m16n8k32 u8 x s8
-//    (weights as A, tokens as the N = 8 side); K is permuted identically in A
-//    and B so each lane reads 8 consecutive codes and 8 consecutive xq bytes;
-//  * partial fp64 sums of the K ranges are added in a fixed order (so results
-//    are deterministic), then scaled by sx, biased, rounded and stored.
+//    one thread issues 2-D TMA copies of the CTA's whole weight slice -- boxes
+//    of R rows x 128 packed bytes (four groups), 128-byte swizzled so the
+//    fragment reads are free of bank conflicts -- and bulk copies of its fp16
+//    scales / offsets, one mbarrier per box, so the weight stream is in flight
+//    while the previous kernel finishes (few large copies: per-copy overhead
+//    of many small ones dominated an earlier version);
+//  * after the wait: xq (all M rows, padded rows) by bulk copy, xsum as fp64 and the
+//    scales / offsets as fp64 (converted once per CTA) into padded tables;
+//  * 16 warps = RT row tiles x (16 / RT) K ranges; each warp starts as soon as
+//    its K range has landed;
+//  * nibbles are split in registers (one AND, one shift + AND per 8 codes)
+//    straight into the A fragments of mma.sync m16n8k32 u8 x s8 (weights as A,
+//    tokens as the N = 8 side); K is permuted identically in A and B (xq is
+//    byte-permuted once in shared memory) so a lane reads 16 consecutive codes
+//    and 16 xq bytes per group with one load each;
+//  * per-group sums fold into fp64 (exact int -> fp64 by the 2^52 magic
+//    number); the K ranges' partial sums add in a fixed order (deterministic),
+//    then sx, bias and one rounding to bf16.
+// The route is used only when weights, xq and the tables fit shared memory
+// (K <= 4096 at M = 16); larger K goes to the GEMM.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -33,35 +43,38 @@
 namespace qk {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = 8;
-constexpr int kGemvSmemLimit = 227 * 1024;
+constexpr int kThreads = 512;
+constexpr int kWarps = 16;
+constexpr int kSmemLimit = 227 * 1024;
 
-struct GemvSmem {
-  __host__ __device__ static int row_stride(int K) { return K / 2 + 16; }
-  __host__ __device__ static size_t weights(int R, int K) { return (size_t)R * row_stride(K); }
-  // R = 16 * RT rows; the 8 warps form RT row tiles x (8 / RT) K ranges.
-  __host__ __device__ static size_t partials(int R) { return (size_t)(kWarps / (R / 16)) * R * 16 * sizeof(double); }
-  __host__ __device__ static size_t bytes(int R, int K) {
-    const int G = K / 64;
-    size_t b = 0;
-    b += weights(R, K);                        // packed codes
-    b += (size_t)R * G * 2 * 2;                // fp16 scales + offsets
-    b = (b + 15) & ~size_t(15);
-    b += partials(R);                          // fp64 partial sums of the K ranges
-    b += 16 * 8;                               // mbarriers
-    return b;
+// Shared-memory layout for R weight rows, K, and M token rows.
+struct GemvLayout {
+  int G, KS, Mp, nbox, XS;
+  size_t w, so16, so64, xq, xs, sxo, part, bars, total;
+  __host__ __device__ GemvLayout(int R, int K, int M) {
+    G = K / 64;
+    KS = kWarps / (R / 16);
+    Mp = M <= 8 ? 8 : 16;
+    nbox = (G + 3) / 4;                                    // 128-byte boxes per row
+    size_t off = 0;
+    w = off;    off += (size_t)nbox * R * 128;             // packed codes, swizzled boxes
+    so16 = off; off += (size_t)R * G * 2 * 2;              // fp16 scales then offsets
+    off = (off + 15) & ~size_t(15);
+    so64 = off; off += (size_t)R * (G + 1) * 16;           // {s, o} fp64, padded rows
+    // xq row stride = 64 (mod 128): the two token rows of one 16-byte load
+    // phase fall in opposite halves of the banks
+    XS = (K + 63) / 128 * 128 + 64;
+    xq = off;   off += (size_t)Mp * XS;                    // xq rows (zero past M)
+    off = (off + 15) & ~size_t(15);
+    xs = off;   off += (size_t)Mp * (G + 1) * 8;           // xsum fp64, padded rows
+    sxo = off;  off += 16 * 4;                             // sx
+    // fp64 partial sums [K range][token][row], rows padded to R + 4 so the
+    // reduce (consecutive rows per lane) and the stores are conflict-free
+    part = off; off += (size_t)KS * 16 * (R + 4) * 8;
+    bars = off; off += (size_t)(nbox + 2) * 8;             // mbarriers
+    total = off + 1024;                                    // base alignment slack
   }
 };
-
-__device__ __forceinline__ void unpack8(uint32_t w, uint32_t& lo4, uint32_t& hi4) {
-  // w holds codes c0..c7 (c0 = low nibble of byte 0).  Output bytes:
-  // lo4 = {c0, c1, c2, c3}, hi4 = {c4, c5, c6, c7}.
-  const uint32_t even = w & 0x0F0F0F0Fu;         // c0, c2, c4, c6
-  const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;   // c1, c3, c5, c7
-  lo4 = __byte_perm(even, odd, 0x5140);
-  hi4 = __byte_perm(even, odd, 0x7362);
-}
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
@@ -72,82 +85,134 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ float f64_to_f32_odd(double v) {
-  float f = __double2float_rz(v);
-  if ((double)f != v) f = __uint_as_float(__float_as_uint(f) | 1u);
-  return f;
+__device__ __forceinline__ double i32_to_f64(int a) {
+  return __hiloint2double(0x43300000, a ^ (int)0x80000000) - 4503601774854144.0;
 }
 
+// fp64 -> bf16 bits with one rounding to nearest-even (integer operations on
+// the bits for |v| >= 2^-126, round-to-odd into fp32 below).
 __device__ __forceinline__ uint16_t f64_to_bf16_bits(double v) {
-  return __bfloat16_as_ushort(__float2bfloat16_rn(f64_to_f32_odd(v)));
+  const uint32_t hi = (uint32_t)__double2hiint(v);
+  const uint32_t lo = (uint32_t)__double2loint(v);
+  const uint32_t sign = (hi >> 16) & 0x8000u;
+  const uint32_t mag = hi & 0x7FFFFFFFu;
+  if (mag < 0x38100000u) {
+    if ((mag | lo) == 0u) return (uint16_t)sign;
+    float f = __double2float_rz(v);
+    if ((double)f != v) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+  }
+  const uint32_t keep = mag >> 13;
+  const uint32_t low13 = (mag & 0x1FFFu) | min(lo, 1u);
+  const uint32_t up = (low13 + 0x0FFFu + (keep & 1u)) >> 13;
+  return (uint16_t)(sign | min(keep + up - (896u << 7), 0x7F80u));
 }
 
 // TT token tiles of 8 (M <= 8 * TT).  RT row tiles of 16 per CTA.
 template <int TT>
 __global__ void __launch_bounds__(kThreads, 1)
-    w4a8_gemv_kernel(const int8_t* __restrict__ xq, const float* __restrict__ sx,
+    w4a8_gemv_kernel(const __grid_constant__ CUtensorMap tmW, const int8_t* __restrict__ xq,
+                     const float* __restrict__ sx,
                      const int32_t* __restrict__ xsum, int M, int K,
                      const uint8_t* __restrict__ Wp, const uint16_t* __restrict__ wscale,
                      const uint16_t* __restrict__ woffset, const float* __restrict__ bias, int N,
                      uint16_t* __restrict__ y, int32_t* __restrict__ acc_out, int m0, int m1,
                      int RT, int* err) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int G = K / 64;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = align_smem<1024>(smem_raw);
   const int R = 16 * RT;
-  const int KS = kWarps / RT;  // K ranges
-  const int RS = GemvSmem::row_stride(K);
+  const GemvLayout L(R, K, M);
+  const int G = L.G, KS = L.KS, nbox = L.nbox;
+  const int XS = L.XS;         // xq row stride
   const int n0 = blockIdx.x * R;
   const int rows = min(R, N - n0);  // valid rows of this CTA (a multiple of 8)
+  const bool fold = acc_out == nullptr;
 
-  uint8_t* w_sm = smem;
-  uint16_t* s_sm = reinterpret_cast<uint16_t*>(smem + GemvSmem::weights(R, K));
-  uint16_t* o_sm = s_sm + (size_t)R * G;
-  size_t off = GemvSmem::weights(R, K) + (size_t)R * G * 4;
-  off = (off + 15) & ~size_t(15);
-  double* part = reinterpret_cast<double*>(smem + off);
-  off += GemvSmem::partials(R);
-  const uint32_t bars = smem_u32(smem + off);  // KS weight barriers, then 1 scale barrier
+  uint8_t* w_sm = smem + L.w;
+  const uint16_t* s16 = reinterpret_cast<const uint16_t*>(smem + L.so16);
+  const uint16_t* o16 = s16 + (size_t)R * G;
+  double2* so_sm = reinterpret_cast<double2*>(smem + L.so64);
+  int8_t* xq_sm = reinterpret_cast<int8_t*>(smem + L.xq);
+  double* xs_sm = reinterpret_cast<double*>(smem + L.xs);
+  float* sx_sm = reinterpret_cast<float*>(smem + L.sxo);
+  double* part = reinterpret_cast<double*>(smem + L.part);
+  // one barrier per weight box, then one for the scales, one for the activations
+  const uint32_t bars = smem_u32(smem + L.bars);
+  const uint32_t sbar = bars + 8u * nbox, abar = bars + 8u * (nbox + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto g_lo = [&](int q) { return q * G / KS; };
 
   if (threadIdx.x == 0) {
-    for (int q = 0; q <= KS; ++q) mbar_init(bars + 8u * q, 1);
+    prefetch_tmap(&tmW);
+    for (int q = 0; q < nbox + 2; ++q) mbar_init(bars + 8u * q, 1);
     fence_mbar_init();
   }
   __syncthreads();
 
-  // ---- weight stream: issued before the dependency wait
-  if (warp == 0) {
-    if (lane == 0) {
-      for (int q = 0; q < KS; ++q)
-        mbar_arrive_expect_tx(bars + 8u * q, (uint32_t)(rows * (g_lo(q + 1) - g_lo(q)) * 32));
-      const bool with_scales = acc_out == nullptr;
-      mbar_arrive_expect_tx(bars + 8u * KS, with_scales ? (uint32_t)(rows * G * 2 * 2) : 0u);
-      if (with_scales) {
-        bulk_load(smem_u32(s_sm), wscale + (size_t)n0 * G, (uint32_t)(rows * G * 2), bars + 8u * KS);
-        bulk_load(smem_u32(o_sm), woffset + (size_t)n0 * G, (uint32_t)(rows * G * 2), bars + 8u * KS);
-      }
+  // ---- weight stream: issued before the dependency wait (a box always moves
+  // R rows x 128 bytes; rows past N and bytes past K/2 are zero-filled)
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < nbox; ++j) {
+      mbar_arrive_expect_tx(bars + 8u * j, (uint32_t)(R * 128));
+      tma_load_2d(smem_u32(w_sm + (size_t)j * R * 128), &tmW, 128 * j, n0, bars + 8u * j);
     }
-    __syncwarp();
-    for (int i = lane; i < rows * KS; i += 32) {
-      const int q = i / rows, r = i - q * rows;
-      const int glo = g_lo(q), ghi = g_lo(q + 1);
-      if (ghi > glo)
-        bulk_load(smem_u32(w_sm + (size_t)r * RS + glo * 32),
-                  Wp + (size_t)(n0 + r) * (K / 2) + glo * 32, (uint32_t)((ghi - glo) * 32),
-                  bars + 8u * q);
+    mbar_arrive_expect_tx(sbar, fold ? (uint32_t)(rows * G * 2 * 2) : 0u);
+    if (fold) {
+      bulk_load(smem_u32(smem + L.so16), wscale + (size_t)n0 * G, (uint32_t)(rows * G * 2), sbar);
+      bulk_load(smem_u32(smem + L.so16) + (uint32_t)(R * G * 2), woffset + (size_t)n0 * G,
+                (uint32_t)(rows * G * 2), sbar);
     }
   }
 
+  // The next kernel may start its own prologue now; it waits for this grid to
+  // finish before it touches anything this grid reads or writes.
+  pdl_launch_dependents();
   // ---- activations come from the previous kernel
   pdl_wait();
+  if (warp == 1) {
+    if (lane == 0) mbar_arrive_expect_tx(abar, (uint32_t)(M * K));
+    __syncwarp();
+    for (int m = lane; m < M; m += 32)
+      bulk_load(smem_u32(xq_sm + (size_t)m * XS), xq + (size_t)m * K, (uint32_t)K, abar);
+  }
+  // token rows past M read as zeros
+  for (int i = threadIdx.x; i < (L.Mp - M) * (K / 16); i += kThreads) {
+    const int m = M + i / (K / 16), c = i % (K / 16);
+    *reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (fold) {
+    if (threadIdx.x < M) sx_sm[threadIdx.x] = __ldg(sx + threadIdx.x);
+    for (int m = warp; m < L.Mp; m += kWarps)
+      for (int g = lane; g < G; g += 32)
+        xs_sm[m * (G + 1) + g] = m < M ? i32_to_f64(__ldg(xsum + (size_t)m * G + g)) : 0.0;
+    // scales / offsets to fp64 once (rows beyond `rows` are never read)
+    if (mbar_wait(sbar, 0, err)) {
+      for (int r = warp; r < rows; r += kWarps)
+        for (int g = lane; g < G; g += 32)
+          so_sm[r * (G + 1) + g] =
+              make_double2((double)__half2float(__ushort_as_half(s16[(size_t)r * G + g])),
+                           (double)__half2float(__ushort_as_half(o16[(size_t)r * G + g])));
+    }
+  }
+  // xq: within every 8 bytes put the even k first, then the odd k, to match
+  // the even / odd nibble split of the weight codes (see the K map below)
+  bool ok = mbar_wait(abar, 0, err);
+  if (ok) {
+    for (int i = threadIdx.x; i < M * (K / 16); i += kThreads) {
+      const int m = i / (K / 16), c = i % (K / 16);
+      uint4* v = reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * c);
+      const uint4 x = *v;
+      *v = make_uint4(__byte_perm(x.x, x.y, 0x6420), __byte_perm(x.x, x.y, 0x7531),
+                      __byte_perm(x.z, x.w, 0x6420), __byte_perm(x.z, x.w, 0x7531));
+    }
+  }
+  __syncthreads();
 
   const int rt = warp % RT, q = warp / RT;
   const int grp = lane >> 2, tq = lane & 3;
   const int glo = g_lo(q), ghi = g_lo(q + 1);
-  bool ok = mbar_wait(bars + 8u * q, 0, err);
-  ok = mbar_wait(bars + 8u * KS, 0, err) && ok;
+  for (int j = glo / 4; j <= (ghi - 1) / 4 && ghi > glo; ++j) ok = mbar_wait(bars + 8u * j, 0, err) && ok;
 
   double f[TT][4];
 #pragma unroll
@@ -156,59 +221,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 4; ++i) f[tt][i] = 0.0;
 
   const int rloc = rt * 16 + grp;  // this lane's first weight row (second: +8)
-  const uint8_t* wrow0 = w_sm + (size_t)rloc * RS;
-  const uint8_t* wrow1 = wrow0 + (size_t)8 * RS;
+  // rows past the CTA's valid rows are read clamped (their results are dropped)
+  const int ra = min(rloc, rows - 1), rb = min(rloc + 8, rows - 1);
+  const double2* so_a = so_sm + (size_t)ra * (G + 1);
+  const double2* so_b = so_sm + (size_t)rb * (G + 1);
+  // K map.  For group g, lane (grp, tq) handles the 16 consecutive codes
+  // k = 64 g + 16 tq + 0..15 (8 packed bytes).  Splitting a packed word into its
+  // low nibbles (codes 0, 2, 4, 6) and high nibbles (codes 1, 3, 5, 7) gives the
+  // A registers of one m16n8k32 MMA directly; xq was permuted to the same
+  // even / odd order, so each MMA sums the same 32 k on both sides, and the two
+  // MMAs of a group cover its 64 k once.
+  // Packed byte p of row r sits in box p / 128, 16-byte chunk ((p % 128) / 16)
+  // ^ (r % 8); here p = 32 g + 8 tq, so inside a box the offsets depend only on
+  // g % 4: precompute them per row and walk the groups box by box.
+  uint32_t offa[4], offb[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = 2 * i + (tq >> 1);
+    offa[i] = (uint32_t)(ra * 128 + ((c ^ (ra & 7)) << 4) + 8 * (tq & 1));
+    offb[i] = (uint32_t)(rb * 128 + ((c ^ (rb & 7)) << 4) + 8 * (tq & 1));
+  }
+  const uint32_t box_bytes = (uint32_t)R * 128;
+  const int8_t* xb[TT];
+  const double* xsp[TT];
+#pragma unroll
+  for (int tt = 0; tt < TT; ++tt) {
+    xb[tt] = xq_sm + (size_t)(tt * 8 + grp) * XS + 16 * tq;
+    xsp[tt] = xs_sm + (size_t)(tt * 8 + 2 * tq) * (G + 1);
+  }
 
-  for (int g = glo; g < ghi && ok; ++g) {
-    int acc[TT][4];
+  for (int bx = glo >> 2; ok && ghi > glo && bx <= (ghi - 1) >> 2; ++bx) {
+    const uint8_t* box = w_sm + (size_t)bx * box_bytes;
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[tt][i] = 0;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int kb = 64 * g + 32 * h + 8 * tq;  // this lane's 8 consecutive k
-      uint32_t a[4];
-      const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wrow0 + kb / 2);
-      const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wrow1 + kb / 2);
-      unpack8(w0, a[0], a[2]);
-      unpack8(w1, a[1], a[3]);
+    for (int gi = 0; gi < 4; ++gi) {
+      const int g = 4 * bx + gi;
+      if (g < glo || g >= ghi) continue;  // warp-uniform
+      const uint2 wa = *reinterpret_cast<const uint2*>(box + offa[gi]);
+      const uint2 wb = *reinterpret_cast<const uint2*>(box + offb[gi]);
+      // A registers: {row grp, row grp + 8} x {even codes, odd codes}, per MMA
+      const uint32_t a0[4] = {wa.x & 0x0F0F0F0Fu, wb.x & 0x0F0F0F0Fu, (wa.x >> 4) & 0x0F0F0F0Fu,
+                              (wb.x >> 4) & 0x0F0F0F0Fu};
+      const uint32_t a1[4] = {wa.y & 0x0F0F0F0Fu, wb.y & 0x0F0F0F0Fu, (wa.y >> 4) & 0x0F0F0F0Fu,
+                              (wb.y >> 4) & 0x0F0F0F0Fu};
+      int acc[TT][4];
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt) {
-        const int m = tt * 8 + grp;
-        uint2 b = make_uint2(0u, 0u);
-        if (m < M) b = __ldg(reinterpret_cast<const uint2*>(xq + (size_t)m * K + kb));
-        mma_u8s8(acc[tt], a, b.x, b.y);
+        const uint4 b = *reinterpret_cast<const uint4*>(xb[tt] + 64 * g);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[tt][i] = 0;
+        mma_u8s8(acc[tt], a0, b.x, b.y);
+        mma_u8s8(acc[tt], a1, b.z, b.w);
+      }
+      if (!fold) {
+        // accumulator dump: acc[(m - m0), n, g] for rows m0 <= m < m1
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int m = tt * 8 + 2 * tq + (i & 1);
+            const int r = rloc + (i >> 1) * 8;
+            if (m >= m0 && m < m1 && r < rows)
+              acc_out[((size_t)(m - m0) * N + n0 + r) * G + g] = acc[tt][i];
+          }
+        continue;
+      }
+      const double2 sa = so_a[g], sb = so_b[g];
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt) {
+        const double x0 = xsp[tt][g];
+        const double x1 = xsp[tt][(G + 1) + g];
+        f[tt][0] = fma(sa.y, x0, fma(sa.x, i32_to_f64(acc[tt][0]), f[tt][0]));
+        f[tt][1] = fma(sa.y, x1, fma(sa.x, i32_to_f64(acc[tt][1]), f[tt][1]));
+        f[tt][2] = fma(sb.y, x0, fma(sb.x, i32_to_f64(acc[tt][2]), f[tt][2]));
+        f[tt][3] = fma(sb.y, x1, fma(sb.x, i32_to_f64(acc[tt][3]), f[tt][3]));
       }
     }
-    if (acc_out != nullptr) {
-      // accumulator dump: acc[(m - m0), n, g] for rows m0 <= m < m1
-#pragma unroll
-      for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = tt * 8 + 2 * tq + (i & 1);
-          const int n = n0 + rloc + (i >> 1) * 8;
-          if (m >= m0 && m < m1 && n < N) acc_out[((size_t)(m - m0) * N + n) * G + g] = acc[tt][i];
-        }
-      continue;
-    }
-    const double s_a = (double)__half2float(__ushort_as_half(s_sm[(size_t)rloc * G + g]));
-    const double s_b = (double)__half2float(__ushort_as_half(s_sm[(size_t)(rloc + 8) * G + g]));
-    const double o_a = (double)__half2float(__ushort_as_half(o_sm[(size_t)rloc * G + g]));
-    const double o_b = (double)__half2float(__ushort_as_half(o_sm[(size_t)(rloc + 8) * G + g]));
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      const int m = tt * 8 + 2 * tq;
-      const double x0 = m < M ? (double)__ldg(xsum + (size_t)m * G + g) : 0.0;
-      const double x1 = m + 1 < M ? (double)__ldg(xsum + (size_t)(m + 1) * G + g) : 0.0;
-      f[tt][0] = fma(o_a, x0, fma(s_a, (double)acc[tt][0], f[tt][0]));
-      f[tt][1] = fma(o_a, x1, fma(s_a, (double)acc[tt][1], f[tt][1]));
-      f[tt][2] = fma(o_b, x0, fma(s_b, (double)acc[tt][2], f[tt][2]));
-      f[tt][3] = fma(o_b, x1, fma(s_b, (double)acc[tt][3], f[tt][3]));
-    }
   }
-  if (acc_out != nullptr) return;
+  if (!fold) return;
 
   // ---- partial sums of the K ranges, added in a fixed order
 #pragma unroll
@@ -217,23 +306,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 4; ++i) {
       const int m = tt * 8 + 2 * tq + (i & 1);
       const int r = rloc + (i >> 1) * 8;
-      part[((size_t)q * R + r) * 16 + m] = f[tt][i];
+      part[((size_t)q * 16 + m) * (R + 4) + r] = f[tt][i];
     }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < R * M; idx += kThreads) {
-    const int m = idx / R, r = idx - m * R;  // consecutive threads -> consecutive n
-    const int n = n0 + r;
+  for (int m = threadIdx.x / R; m < M; m += kThreads / R) {
+    const int r = threadIdx.x % R;  // consecutive threads -> consecutive n
     if (r >= rows) continue;
     double acc = 0.0;
-    for (int qq = 0; qq < KS; ++qq) acc += part[((size_t)qq * R + r) * 16 + m];
-    const double v = fma((double)sx[m], acc, bias != nullptr ? (double)bias[n] : 0.0);
-    y[(size_t)m * N + n] = f64_to_bf16_bits(v);
+    for (int qq = 0; qq < KS; ++qq) acc += part[((size_t)qq * 16 + m) * (R + 4) + r];
+    const double v = fma((double)sx_sm[m], acc, bias != nullptr ? (double)bias[n0 + r] : 0.0);
+    y[(size_t)m * N + n0 + r] = f64_to_bf16_bits(v);
   }
 }
 
 size_t g_smem_set[2][64];
 
 }  // namespace
+
+size_t gemv_smem_bytes(int64_t M, int64_t K, int64_t N) {
+  const int sms = num_sms();
+  int RT = 1;
+  while (RT < 4 && (N + 16 * RT - 1) / (16 * RT) > sms &&
+         GemvLayout(32 * RT, (int)K, (int)M).total <= (size_t)kSmemLimit)
+    RT *= 2;
+  return GemvLayout(16 * RT, (int)K, (int)M).total;
+}
 
 cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                              int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
@@ -242,12 +339,16 @@ cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* x
   const int sms = num_sms();
   int RT = 1;  // fewest rows per CTA that still fit all CTAs in one wave
   while (RT < 4 && (N + 16 * RT - 1) / (16 * RT) > sms &&
-         GemvSmem::bytes(32 * RT, (int)K) <= (size_t)kGemvSmemLimit)
+         GemvLayout(32 * RT, (int)K, (int)M).total <= (size_t)kSmemLimit)
     RT *= 2;
   const int R = 16 * RT;
   const unsigned grid = (unsigned)((N + R - 1) / R);
-  const size_t smem = GemvSmem::bytes(R, (int)K);
-  if (smem > (size_t)kGemvSmemLimit) return cudaErrorInvalidValue;
+  const size_t smem = GemvLayout(R, (int)K, (int)M).total;
+  if (smem > (size_t)kSmemLimit) return cudaErrorInvalidValue;
+  CUtensorMap tW;
+  if (!encode_tmap_2d(&tW, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wp, (uint64_t)(K / 2), (uint64_t)N,
+                      (uint64_t)(K / 2), 128, (uint32_t)R, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   int* err = device_error_word();
   if (err == nullptr) return cudaErrorUnknown;
   auto kernel = M <= 8 ? w4a8_gemv_kernel<1> : w4a8_gemv_kernel<2>;
@@ -256,9 +357,9 @@ cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* x
   const int tt = M <= 8 ? 0 : 1;
   if (dev >= 64 || g_smem_set[tt][dev] < smem) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kGemvSmemLimit);
+                                         kSmemLimit);
     if (e != cudaSuccess) return e;
-    if (dev < 64) g_smem_set[tt][dev] = kGemvSmemLimit;
+    if (dev < 64) g_smem_set[tt][dev] = kSmemLimit;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -270,8 +371,8 @@ cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* x
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, xq, sx, xsum, (int)M, (int)K, Wp, ws, wo, bias, (int)N,
-                            y, acc_out, (int)m0, (int)m1, RT, err);
+  return cudaLaunchKernelEx(&cfg, kernel, tW, xq, sx, xsum, (int)M, (int)K, Wp, ws, wo, bias,
+                            (int)N, y, acc_out, (int)m0, (int)m1, RT, err);
 }
 
 }  // namespace qk

@@ -261,8 +261,8 @@ qk_status qk_w8a8_linear(const uint16_t* x, int64_t M, int64_t K, const int8_t* 
   if ((st = check_device()) != QK_OK) return st;
   Workspace ws;
   if ((st = ws.init(workspace, ws_bytes, M, K, false, stream)) != QK_OK) return st;
-  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, nullptr, stream), "quant_act")) !=
-      QK_OK)
+  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, nullptr, stream, true),
+                      "quant_act")) != QK_OK)
     return st;
   if (log_enabled())
     std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> quant_act + tcgen05 GEMM\n",
@@ -284,7 +284,7 @@ static cudaError_t run_w4a8(const int8_t* xq, const float* sx, const int32_t* xs
                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                             const float* bias, int64_t N, uint16_t* y, int route, bool pdl,
                             cudaStream_t s) {
-  const bool gemv = route == QK_ROUTE_GEMV || (route == QK_ROUTE_AUTO && M <= 16 && K <= kGemvMaxK);
+  const bool gemv = route == QK_ROUTE_GEMV || (route == QK_ROUTE_AUTO && gemv_fits(M, K, N));
   if (log_enabled())
     std::fprintf(stderr, "[qk] w4a8 M=%lld K=%lld N=%lld -> %s\n", (long long)M, (long long)K,
                  (long long)N, gemv ? "GEMV" : "tcgen05 GEMM");
@@ -302,7 +302,7 @@ qk_status qk_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, i
   if (route != QK_ROUTE_AUTO && route != QK_ROUTE_GEMM && route != QK_ROUTE_GEMV)
     return QK_ERR_INVALID_ARG;
   if (route == QK_ROUTE_GEMV && M > 16) return QK_ERR_INVALID_ARG;
-  if (route == QK_ROUTE_GEMV && K > kGemvMaxK) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (route == QK_ROUTE_GEMV && M > 0 && !gemv_fits(M, K, N)) return QK_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return QK_OK;
   if (!xq || !sx || !xsum) return QK_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(sx) || !aligned16(xsum)) return QK_ERR_MISALIGNED;
@@ -325,8 +325,8 @@ qk_status qk_w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
   if ((st = check_device()) != QK_OK) return st;
   Workspace ws;
   if ((st = ws.init(workspace, ws_bytes, M, K, true, stream)) != QK_OK) return st;
-  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, ws.xsum, stream), "quant_act")) !=
-      QK_OK)
+  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, ws.xsum, stream, true),
+                      "quant_act")) != QK_OK)
     return st;
   return from_cuda(run_w4a8(ws.xq, ws.sx, ws.xsum, M, K, Wp, wscale, woffset, bias, N, y,
                             QK_ROUTE_AUTO, true, stream),
@@ -372,7 +372,7 @@ qk_status qk_debug_w4a8_group_acc(const int8_t* xq, int64_t M, int64_t K, const 
   if (st != QK_OK) return st;
   if (route != QK_ROUTE_GEMM && route != QK_ROUTE_GEMV) return QK_ERR_INVALID_ARG;
   if (route == QK_ROUTE_GEMV && M > 16) return QK_ERR_INVALID_ARG;
-  if (route == QK_ROUTE_GEMV && K > kGemvMaxK) return QK_ERR_UNSUPPORTED_SHAPE;
+  if (route == QK_ROUTE_GEMV && M > 0 && !gemv_fits(M, K, N)) return QK_ERR_UNSUPPORTED_SHAPE;
   if (m0 < 0 || m1 < m0 || m1 > M) return QK_ERR_INVALID_ARG;
   if (m1 == m0) return QK_OK;
   if (!xq || !Wp || !acc) return QK_ERR_INVALID_ARG;

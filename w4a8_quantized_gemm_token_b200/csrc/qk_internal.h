@@ -14,8 +14,10 @@ namespace qk {
 // Each returns cudaSuccess or the launch error.  Arguments are already
 // validated by the C-ABI layer (qk_api.cu).
 
+// `pdl`: launch as a programmatic dependent of the previous kernel in the
+// stream (the kernel waits for it before reading x or writing xq / sx).
 cudaError_t launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx,
-                             int32_t* xsum, cudaStream_t s);
+                             int32_t* xsum, cudaStream_t s, bool pdl = false);
 
 cudaError_t launch_quant_w8(const float* W, int64_t N, int64_t K, int8_t* Wq, float* sw,
                             cudaStream_t s);
@@ -37,9 +39,13 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
                              int64_t m0, int64_t m1, bool pdl, cudaStream_t s);
 
-// W4A8 weight-streaming GEMV (M <= 16, K <= kGemvMaxK: the CTA's weight slice
-// must fit shared memory); per-group accumulator dump as above.
-constexpr int64_t kGemvMaxK = 16384;
+// W4A8 weight-streaming GEMV (M <= 16; its per-CTA working set -- weight slice,
+// xq, scale tables -- must fit shared memory, see gemv_fits); per-group
+// accumulator dump as above.
+size_t gemv_smem_bytes(int64_t M, int64_t K, int64_t N);
+inline bool gemv_fits(int64_t M, int64_t K, int64_t N) {
+  return M <= 16 && gemv_smem_bytes(M, K, N) <= 227u * 1024u;
+}
 cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                              int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,

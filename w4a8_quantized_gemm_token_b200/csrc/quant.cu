@@ -88,6 +88,9 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   // The dependent GEMM may start its prologue now; it waits for this grid's
   // completion before it reads xq / sx.
   pdl_launch_dependents();
+  // When launched as a programmatic dependent, wait for the previous grid (it
+  // may produce x, or still read the xq / sx this kernel overwrites).
+  pdl_wait();
   const int row = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
   if (row >= M) return;
   const int lane = threadIdx.x & 31;
@@ -232,25 +235,26 @@ __global__ void __launch_bounds__(256) quant_w4_kernel(const float* __restrict__
 }  // namespace
 
 cudaError_t launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx,
-                             int32_t* xsum, cudaStream_t s) {
-  const dim3 grid((unsigned)((M + kQuantWarps - 1) / kQuantWarps)), block(256);
+                             int32_t* xsum, cudaStream_t s, bool pdl) {
   const int m = (int)M, k = (int)K;
   const int per_lane = (int)((K / 8 + 31) / 32);  // 16-byte chunks per lane
-  if (per_lane <= 1)
-    quant_act_kernel<1><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
-  else if (per_lane <= 2)
-    quant_act_kernel<2><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
-  else if (per_lane <= 4)
-    quant_act_kernel<4><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
-  else if (per_lane <= 8)
-    quant_act_kernel<8><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
-  else if (per_lane <= 12)
-    quant_act_kernel<12><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
-  else if (per_lane <= 16)
-    quant_act_kernel<16><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
-  else
-    quant_act_kernel<0><<<grid, block, 0, s>>>(x, m, k, xq, sx, xsum);
-  return cudaGetLastError();
+  auto kernel = per_lane <= 1    ? quant_act_kernel<1>
+                : per_lane <= 2  ? quant_act_kernel<2>
+                : per_lane <= 4  ? quant_act_kernel<4>
+                : per_lane <= 8  ? quant_act_kernel<8>
+                : per_lane <= 12 ? quant_act_kernel<12>
+                : per_lane <= 16 ? quant_act_kernel<16>
+                                 : quant_act_kernel<0>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((M + kQuantWarps - 1) / kQuantWarps));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, x, m, k, xq, sx, xsum);
 }
 
 cudaError_t launch_quant_w8(const float* W, int64_t N, int64_t K, int8_t* Wq, float* sw,

@@ -25,6 +25,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Rounds a dynamic shared-memory base up to kAlign bytes.  Pointer arithmetic
+// on the __shared__ array (no integer round trip) keeps the result in the
+// shared address space, so accesses through it compile to shared-memory
+// loads and stores rather than generic ones.
+template <uint32_t kAlign>
+__device__ __forceinline__ uint8_t* align_smem(uint8_t* base) {
+  return base + ((kAlign - (smem_u32(base) & (kAlign - 1u))) & (kAlign - 1u));
+}
+
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 // ----------------------------------------------------------------- mbarrier
