@@ -223,6 +223,9 @@ qk_status qk_w8a8_linear_noalloc(const uint16_t *x, int64_t M, int64_t K,
  * M <= 16 takes the weight-streaming GEMV when its per-CTA working set fits
  * in shared memory (K <= 4096 at M = 16), otherwise the tensor-core GEMM; both
  * compute the same per-group integers and agree to the fp64 rounding order.
+ * When also M * K <= 65536 the GEMV quantizes x itself (same rule and codes as
+ * qk_quantize_activations) and the call is one kernel; the workspace is then
+ * checked but not used (qk_w4a8_linear_plan tells which case applies).
  *   x                  : bf16 bits [M, K]            (in)
  *   Wp, wscale, woffset: from qk_quantize_weights_int4 (in)
  *   bias               : fp32 [N] (nullable)
@@ -235,6 +238,23 @@ qk_status qk_w4a8_linear(const uint16_t *x, int64_t M, int64_t K,
                          const float *bias, int64_t N,
                          uint16_t *y, void *workspace, size_t ws_bytes,
                          qk_stream_t stream);
+
+/* Kernel plans of qk_w4a8_linear (see qk_w4a8_linear_plan). */
+typedef enum {
+    QK_PLAN_NONE = 0,       /* M == 0: nothing is launched                      */
+    QK_PLAN_GEMV_QUANT = 1, /* one kernel: the GEMV quantizing x itself          */
+    QK_PLAN_QUANT_GEMV = 2, /* activation quantization, then the GEMV            */
+    QK_PLAN_QUANT_GEMM = 3  /* activation quantization, then the tcgen05 GEMM    */
+} qk_plan;
+
+/*
+ * Which kernels qk_w4a8_linear launches for this shape on the current device
+ * (a query of this library's routing; the method itself has no such call).
+ * Returns a qk_plan, or the negated qk_status of an invalid shape.  The GEMV
+ * plans depend on the device's SM count; with no device the count is taken
+ * as 1.
+ */
+int qk_w4a8_linear_plan(int64_t M, int64_t K, int64_t N);
 
 /*
  * The product half of qk_w4a8_linear on quantized activations (xq, sx and

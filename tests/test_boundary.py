@@ -109,3 +109,17 @@ def test_binding_rejects_cpu_tensors(qk):
         qk.qk_quantize_activations(x)
     with pytest.raises(TypeError):
         qk.qk_quantize_activations(x.float())
+
+
+def test_w4a8_linear_plan(qk):
+    """The routing query: one fused kernel for small M * K, quantization + GEMV
+    for larger K at M <= 16, quantization + GEMM above M = 16."""
+    assert qk.qk_w4a8_linear_plan(0, 64, 64) == qk.QK_PLAN_NONE
+    assert qk.qk_w4a8_linear_plan(1, 4096, 4096) == qk.QK_PLAN_GEMV_QUANT
+    assert qk.qk_w4a8_linear_plan(16, 4096, 4096) == qk.QK_PLAN_GEMV_QUANT
+    assert qk.qk_w4a8_linear_plan(16, 4160, 136) == qk.QK_PLAN_QUANT_GEMV
+    assert qk.qk_w4a8_linear_plan(17, 4096, 4096) == qk.QK_PLAN_QUANT_GEMM
+    assert qk.qk_w4a8_linear_plan(4, 32768, 64) == qk.QK_PLAN_QUANT_GEMM
+    with pytest.raises(qk.QKError) as e:
+        qk.qk_w4a8_linear_plan(8, 96, 64)  # K % 64 != 0
+    assert e.value.status == 2

@@ -36,6 +36,7 @@ _SIGS = {
     "qk_w8a8_gemm": (_I, [_P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P]),
     "qk_w4a8_linear": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w4a8_gemm": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I, _P]),
+    "qk_w4a8_linear_plan": (_I, [_I64, _I64, _I64]),
     "qk_check_device_error": (_I, [_P]),
     "qk_debug_w8a8_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P]),
     "qk_debug_w4a8_group_acc": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I, _P]),
@@ -47,6 +48,7 @@ for _name, (_res, _args) in _SIGS.items():
 
 QK_OK = 0
 QK_ROUTE_AUTO, QK_ROUTE_GEMM, QK_ROUTE_GEMV = 0, 1, 2
+QK_PLAN_NONE, QK_PLAN_GEMV_QUANT, QK_PLAN_QUANT_GEMV, QK_PLAN_QUANT_GEMM = 0, 1, 2, 3
 
 
 class QKError(RuntimeError):
@@ -65,6 +67,15 @@ def qk_version() -> int:
 
 def qk_is_available(device: int = 0) -> bool:
     return bool(lib.qk_is_available(device))
+
+
+def qk_w4a8_linear_plan(M: int, K: int, N: int) -> int:
+    """The kernels qk_w4a8_linear launches for this shape (a QK_PLAN_* value);
+    raises QKError for an invalid shape."""
+    r = lib.qk_w4a8_linear_plan(M, K, N)
+    if r < 0:
+        raise QKError(-r, "qk_w4a8_linear_plan")
+    return r
 
 
 def qk_w8a8_workspace_size(M: int, K: int) -> int:

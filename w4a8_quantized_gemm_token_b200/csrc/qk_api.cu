@@ -245,7 +245,7 @@ qk_status qk_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64_t K, 
       (bias && !aligned16(bias)))
     return QK_ERR_MISALIGNED;
   if ((st = check_device()) != QK_OK) return st;
-  return from_cuda(launch_w8a8_gemm(xq, sx, M, K, Wq, sw, bias, N, y, nullptr, false, stream),
+  return from_cuda(launch_w8a8_gemm(xq, sx, M, K, Wq, sw, bias, N, y, nullptr, true, stream),
                    "w8a8_gemm");
 }
 
@@ -293,6 +293,15 @@ static cudaError_t run_w4a8(const int8_t* xq, const float* sx, const int32_t* xs
   return launch_w4a8_gemm(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, pdl, s);
 }
 
+int qk_w4a8_linear_plan(int64_t M, int64_t K, int64_t N) {
+  const qk_status st = check_shape(M, K, N, true);
+  if (st != QK_OK) return -(int)st;
+  if (M == 0) return QK_PLAN_NONE;
+  if (gemv_quant_fits(M, K, N)) return QK_PLAN_GEMV_QUANT;
+  if (gemv_fits(M, K, N)) return QK_PLAN_QUANT_GEMV;
+  return QK_PLAN_QUANT_GEMM;
+}
+
 qk_status qk_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                        int64_t K, const uint8_t* Wp, const uint16_t* wscale,
                        const uint16_t* woffset, const float* bias, int64_t N, uint16_t* y,
@@ -308,7 +317,7 @@ qk_status qk_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, i
   if (!aligned16(xq) || !aligned16(sx) || !aligned16(xsum)) return QK_ERR_MISALIGNED;
   if ((st = check_w4_product(Wp, wscale, woffset, bias, y)) != QK_OK) return st;
   if ((st = check_device()) != QK_OK) return st;
-  return from_cuda(run_w4a8(xq, sx, xsum, M, K, Wp, wscale, woffset, bias, N, y, route, false,
+  return from_cuda(run_w4a8(xq, sx, xsum, M, K, Wp, wscale, woffset, bias, N, y, route, true,
                             stream),
                    "w4a8");
 }
@@ -323,6 +332,18 @@ qk_status qk_w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
   if (!aligned16(x)) return QK_ERR_MISALIGNED;
   if ((st = check_w4_product(Wp, wscale, woffset, bias, y)) != QK_OK) return st;
   if ((st = check_device()) != QK_OK) return st;
+  if (gemv_quant_fits(M, K, N)) {
+    // small M: the GEMV quantizes x itself; the workspace is checked, not used
+    if (workspace != nullptr && (ws_bytes < qk_w4a8_workspace_size(M, K) ||
+                                 (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+      return QK_ERR_WORKSPACE;
+    if (log_enabled())
+      std::fprintf(stderr, "[qk] w4a8 M=%lld K=%lld N=%lld -> GEMV (quantizing x)\n",
+                   (long long)M, (long long)K, (long long)N);
+    return from_cuda(launch_w4a8_gemv_quant(x, M, K, Wp, wscale, woffset, bias, N, y, true,
+                                            stream),
+                     "w4a8 gemv");
+  }
   Workspace ws;
   if ((st = ws.init(workspace, ws_bytes, M, K, true, stream)) != QK_OK) return st;
   if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, ws.xsum, stream, true),

@@ -46,6 +46,12 @@ size_t gemv_smem_bytes(int64_t M, int64_t K, int64_t N);
 inline bool gemv_fits(int64_t M, int64_t K, int64_t N) {
   return M <= 16 && gemv_smem_bytes(M, K, N) <= 227u * 1024u;
 }
+// The same GEMV quantizing bf16 x itself (M * K <= 65536, see gemv_quant_fits):
+// the activation-quant kernel and its launch drop out of the small-M linear.
+bool gemv_quant_fits(int64_t M, int64_t K, int64_t N);
+cudaError_t launch_w4a8_gemv_quant(const uint16_t* x, int64_t M, int64_t K, const uint8_t* Wp,
+                                   const uint16_t* ws, const uint16_t* wo, const float* bias,
+                                   int64_t N, uint16_t* y, bool pdl, cudaStream_t s);
 cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                              int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,

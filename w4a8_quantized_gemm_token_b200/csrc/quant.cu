@@ -12,15 +12,16 @@
 //  * quant_w4: affine group-64 4-bit weights ("qlip-mlx" README,
 //    "w4a8_linear / W4A8Linear"; "MLX PR #4722", "Selector rules"), offline.
 //
-// Rounding: the scale is absmax / 127 and the multiplier 127 / absmax, both
-// correctly rounded fp32 divisions; each code is round-half-even of the fp32
-// product x * multiplier (no fused multiply-add), clamped to [-127, 127].
+// Rounding (act_quant.cuh): the scale is absmax / 127 and the multiplier
+// 127 / absmax, both correctly rounded fp32 divisions; each code is
+// round-half-even of the fp32 product x * multiplier, clamped to [-127, 127].
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
+#include "act_quant.cuh"
 #include "qk_internal.h"
 #include "sm100.cuh"
 
@@ -28,55 +29,6 @@ namespace qk {
 namespace {
 
 constexpr int kQuantWarps = 8;  // rows per 256-thread block
-
-__device__ __forceinline__ uint32_t bf16x2_absmax_bits(uint32_t acc, uint32_t w) {
-  // |bf16| bit patterns order like the values they encode, so a 16-bit integer
-  // max of the magnitudes is the absmax.
-  return __vmaxu2(acc, w & 0x7FFF7FFFu);
-}
-
-__device__ __forceinline__ int quant1(float v, float r) {
-  int q = __float2int_rn(__fmul_rn(v, r));
-  return max(-127, min(127, q));
-}
-
-// 8 bf16 (one 16-byte chunk) -> 8 int8 codes packed in a uint2; adds the codes
-// to *sum.
-__device__ __forceinline__ uint2 quant_chunk(uint4 c, float r, int* sum) {
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-  uint32_t out[2];
-  int s = 0;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t packed = 0;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const uint32_t u = w[2 * h + j];
-      const int q0 = quant1(__uint_as_float(u << 16), r);
-      const int q1 = quant1(__uint_as_float(u & 0xFFFF0000u), r);
-      s += q0 + q1;
-      packed |= ((uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8)) << (16 * j);
-    }
-    out[h] = packed;
-  }
-  *sum += s;
-  return make_uint2(out[0], out[1]);
-}
-
-__device__ __forceinline__ float warp_max_bits_to_float(uint32_t bits2) {
-  uint32_t m = max(bits2 & 0xFFFFu, bits2 >> 16);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  return __uint_as_float(m << 16);
-}
-
-// Sum over the 8 lanes that hold one group of 64 codes.
-__device__ __forceinline__ int group8_sum(int v) {
-  v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
-  v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-  v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
-  return v;
-}
 
 // NCH > 0: the row (<= 256 * NCH elements) stays in registers.
 // NCH == 0: two passes over the row.
@@ -115,8 +67,8 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
       }
     }
     const float amax = warp_max_bits_to_float(mb);
-    r = (amax == 0.0f) ? 0.0f : __fdiv_rn(127.0f, amax);
-    if (lane == 0) sx[row] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
+    r = act_multiplier(amax);
+    if (lane == 0) sx[row] = act_scale(amax);
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = i * 32 + lane;
@@ -136,8 +88,8 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
       mb = bf16x2_absmax_bits(mb, v.w);
     }
     const float amax = warp_max_bits_to_float(mb);
-    r = (amax == 0.0f) ? 0.0f : __fdiv_rn(127.0f, amax);
-    if (lane == 0) sx[row] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
+    r = act_multiplier(amax);
+    if (lane == 0) sx[row] = act_scale(amax);
     for (int base = 0; base < nch; base += 32) {  // warp-uniform trip count
       const int c = base + lane;
       int s = 0;
@@ -167,8 +119,8 @@ __global__ void __launch_bounds__(256) quant_w8_kernel(const float* __restrict__
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-  const float r = (amax == 0.0f) ? 0.0f : __fdiv_rn(127.0f, amax);
-  if (lane == 0) sw[row] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
+  const float r = act_multiplier(amax);
+  if (lane == 0) sw[row] = act_scale(amax);
   for (int c = lane; c < nch; c += 32) {
     const float4 v = __ldg(src + c);
     const int q0 = quant1(v.x, r), q1 = quant1(v.y, r), q2 = quant1(v.z, r), q3 = quant1(v.w, r);
