@@ -7,30 +7,39 @@
 //   y[m, n] = bf16( sx[m] * sum_g (s[n,g] * acc + o[n,g] * xsum[m,g]) + bias[n] )
 // with the fold in fp64 and one rounding to bf16.
 //
-// Design (HBM-bound: the packed weights are ~97% of the bytes; every operand of
-// the inner loop comes from shared memory so the loop never waits on L2):
-//  * each CTA owns R = 16 * RT weight rows; at kernel start, before waiting on
-//    the activation-quant kernel it depends on (programmatic dependent launch),
-//    one thread issues 2-D TMA copies of the CTA's whole weight slice -- boxes
-//    of R rows x 128 packed bytes (four groups), 128-byte swizzled so the
-//    fragment reads are free of bank conflicts -- and bulk copies of its fp16
-//    scales / offsets, one mbarrier per box, so the weight stream is in flight
-//    while the previous kernel finishes (few large copies: per-copy overhead
-//    of many small ones dominated an earlier version);
-//  * after the wait: xq (all M rows, padded rows) by bulk copy, xsum as fp64 and the
-//    scales / offsets as fp64 (converted once per CTA) into padded tables;
-//  * 16 warps = RT row tiles x (16 / RT) K ranges; each warp starts as soon as
-//    its K range has landed;
-//  * nibbles are split in registers (one AND, one shift + AND per 8 codes)
+// Design.  The packed weights are ~97% of the bytes, and a call at
+// N = K = 4096 moves only ~9.5 MB, so a lone launch is dominated by fixed
+// latencies.  The kernel is therefore built for back-to-back calls (the
+// layers of a model, graph replays): while one call computes, the next call's
+// CTAs are already resident and streaming their weights.
+//  * A cluster of C CTAs shares R weight rows; CTA c takes the groups of one
+//    K slice [c GC, (c + 1) GC).  The host picks (R, C) so that a CTA needs at
+//    most ~113 KB of shared memory (two CTAs per SM: this call's and the next
+//    one's) and the grid has at most one CTA per SM.
+//  * At kernel start, before the programmatic-dependency wait, one thread
+//    issues 2-D TMA copies of the CTA's packed codes (boxes of R rows x 128
+//    bytes, 128-byte swizzled, so the fragment reads are conflict-free) and of
+//    its fp16 scales / offsets.  Weights, scales and offsets are therefore read
+//    before the previous kernel in the stream has finished: they must not be
+//    written by a kernel that triggers its dependents early (no kernel of this
+//    library that writes weights does).
+//  * After the wait the CTA either quantizes its K slice of bf16 x itself
+//    (the rule of the stand-alone quantization kernel; with C > 1 the per-row
+//    absmax is exchanged through distributed shared memory) or reads
+//    quantized xq / sx / xsum.
+//  * 8 warps = R/16 row tiles x KW box sets.  Nibbles are split in registers
 //    straight into the A fragments of mma.sync m16n8k32 u8 x s8 (weights as A,
-//    tokens as the N = 8 side); K is permuted identically in A and B (xq is
-//    byte-permuted once in shared memory) so a lane reads 16 consecutive codes
-//    and 16 xq bytes per group with one load each;
-//  * per-group sums fold into fp64 (exact int -> fp64 by the 2^52 magic
-//    number); the K ranges' partial sums add in a fixed order (deterministic),
-//    then sx, bias and one rounding to bf16.
-// The route is used only when weights, xq and the tables fit shared memory
-// (K <= 4096 at M = 16); larger K goes to the GEMM.
+//    tokens as the N = 8 side); K is permuted identically in A and B so each
+//    lane reads 8 packed bytes and 16 activation bytes per group.
+//  * Per-group sums fold into fp64 (exact int -> fp64 by the 2^52 magic
+//    number).  With one token the lanes first gather one group each by
+//    shuffles, so no lane folds an all-zero token column.
+//  * The partial sums of all warps of all CTAs of a cluster go, through
+//    distributed shared memory, to the CTA that owns the row (R / C rows
+//    each), which adds them in a fixed order (deterministic), applies sx and
+//    the bias and rounds once to bf16.
+// Every wait is bounded; a CTA that gives up still takes part in every
+// cluster barrier, so its peers never wait on it forever.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -44,40 +53,48 @@
 namespace qk {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = 16;
+constexpr int kThreads = 256;
+constexpr int kWarps = 8;
 constexpr int kSmemLimit = 227 * 1024;
+// Two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA.
+constexpr int kSmemTwoPerSm = 113 * 1024;
 // In-kernel activation quantization keeps up to this many 16-byte chunks of
-// x per thread in registers (M * K <= kQuantChunks * 8 * kThreads = 65536).
-constexpr int kQuantChunks = 16;
+// x per thread in registers (M * KC <= kQuantChunks * 8 * kThreads = 16384,
+// KC = the K slice of one CTA).
+constexpr int kQuantChunks = 8;
 
-// Shared-memory layout for R weight rows, K, and M token rows.
+// Shared-memory layout of one CTA: R weight rows, cluster of C CTAs along K,
+// M token rows.
 struct GemvLayout {
-  int G, KS, Mp, nbox, XS;
-  size_t w, so16, so64, xq, xs, sxo, amx, part, bars, total;
-  __host__ __device__ GemvLayout(int R, int K, int M) {
+  int R, C, M, G, GC, RT, KW, nbox, XS, RO, Mp;
+  size_t w, s16, xq, xs, sx, amx, part, bars, total;
+  __host__ __device__ GemvLayout(int R_, int C_, int K, int M_) {
+    R = R_;
+    C = C_;
+    M = M_;
     G = K / 64;
-    KS = kWarps / (R / 16);
-    Mp = M <= 8 ? 8 : 16;
-    nbox = (G + 3) / 4;                                    // 128-byte boxes per row
-    size_t off = 0;
-    w = off;    off += (size_t)nbox * R * 128;             // packed codes, swizzled boxes
-    so16 = off; off += (size_t)R * G * 2 * 2;              // fp16 scales then offsets
-    off = (off + 15) & ~size_t(15);
-    so64 = off; off += (size_t)R * (G + 1) * 16;           // {s, o} fp64, padded rows
+    GC = (G + C - 1) / C;      // groups per K slice (C > 1: C divides G)
+    RT = R / 16;               // row tiles
+    KW = kWarps / RT;          // box sets per row tile
+    nbox = (GC + 3) / 4;       // 128-byte boxes per row of the slice
+    RO = R / C;                // rows each CTA finalizes
+    Mp = M <= 8 ? 8 : 16;      // token columns of the MMAs
     // xq row stride = 64 (mod 128): the two token rows of one 16-byte load
     // phase fall in opposite halves of the banks
-    XS = (K + 63) / 128 * 128 + 64;
-    xq = off;   off += (size_t)Mp * XS;                    // xq rows (zero past M)
+    XS = (GC * 64 + 127) / 128 * 128 + 64;
+    size_t off = 0;
+    w = off;    off += (size_t)nbox * R * 128;        // packed codes, swizzled boxes
+    s16 = off;  off += (size_t)R * GC * 2 * 2;        // fp16 scales [R][GC], then offsets
+    off = (off + 127) & ~size_t(127);
+    xq = off;   off += (size_t)M * XS;                // xq rows of the slice (permuted)
     off = (off + 15) & ~size_t(15);
-    xs = off;   off += (size_t)Mp * (G + 1) * 8;           // xsum fp64, padded rows
-    sxo = off;  off += 16 * 4;                             // sx
-    amx = off;  off += 16 * 4;                             // row absmax (in-kernel quant)
-    // fp64 partial sums [K range][token][row], rows padded to R + 4 so the
-    // reduce (consecutive rows per lane) and the stores are conflict-free
-    part = off; off += (size_t)KS * 16 * (R + 4) * 8;
-    bars = off; off += (size_t)(nbox + 2) * 8;             // mbarriers
-    total = off + 1024;                                    // base alignment slack
+    xs = off;   off += (size_t)Mp * (GC + 1) * 8;     // xsum as fp64, zero past M
+    sx = off;   off += 16 * 4;                        // sx
+    amx = off;  off += (size_t)(C + 1) * 16 * 4;      // absmax: [C] exchange slots, local
+    off = (off + 15) & ~size_t(15);
+    part = off; off += (size_t)C * KW * M * RO * 8;   // fp64 partials [slot][token][row]
+    bars = off; off += (size_t)(nbox + 1) * 8;        // mbarriers: boxes, scales
+    total = off + 1024;                               // base alignment slack
   }
 };
 
@@ -92,6 +109,10 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
 
 __device__ __forceinline__ double i32_to_f64(int a) {
   return __hiloint2double(0x43300000, a ^ (int)0x80000000) - 4503601774854144.0;
+}
+
+__device__ __forceinline__ double h2d(uint16_t h) {
+  return (double)__half2float(__ushort_as_half(h));
 }
 
 // fp64 -> bf16 bits with one rounding to nearest-even (integer operations on
@@ -113,99 +134,118 @@ __device__ __forceinline__ uint16_t f64_to_bf16_bits(double v) {
   return (uint16_t)(sign | min(keep + up - (896u << 7), 0x7F80u));
 }
 
-// TT token tiles of 8 (M <= 8 * TT).  RT row tiles of 16 per CTA.  kFold:
-// the product y; otherwise the per-group int32 sums go to acc_out.  kQuantX:
-// the activations arrive as bf16 x and are quantized here (xq, sx, xsum are
-// unused), with the rule of the stand-alone quantization kernel.
-template <int TT, bool kFold, bool kQuantX>
-__global__ void __launch_bounds__(kThreads, 1)
-    w4a8_gemv_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ x,
-                     const int8_t* __restrict__ xq,
-                     const float* __restrict__ sx,
+// ---- distributed shared memory (cluster-window addresses from mapa_shared)
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
+  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
+}
+// Split cluster barrier: every thread of every CTA arrives once, then waits.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bytes 0..7 of an 8-code group of xq reordered: the four even k, then the
+// four odd k (the order in which the nibble split delivers the weight codes).
+__device__ __forceinline__ uint2 even_odd(uint32_t lo, uint32_t hi) {
+  return make_uint2(__byte_perm(lo, hi, 0x6420), __byte_perm(lo, hi, 0x7531));
+}
+
+// TT token tiles of 8 (M <= 8 TT).  kFold: the product y; otherwise the
+// per-group int32 sums of rows [m0, m1) go to acc_out.  kQuantX: the
+// activations arrive as bf16 x and are quantized here (xq, sx, xsum unused).
+// kOne: M == 1, the one-token fold.  C: CTAs per cluster along K.
+// Grid (C, ceil(N / R)), cluster (C, 1, 1).
+template <int TT, bool kFold, bool kQuantX, bool kOne, int C>
+__global__ void __launch_bounds__(kThreads, 2)
+    w4a8_gemv_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
+                     const __grid_constant__ CUtensorMap tmO, const uint16_t* __restrict__ x,
+                     const int8_t* __restrict__ xq, const float* __restrict__ sx,
                      const int32_t* __restrict__ xsum, int M, int K,
-                     const uint8_t* __restrict__ Wp, const uint16_t* __restrict__ wscale,
-                     const uint16_t* __restrict__ woffset, const float* __restrict__ bias, int N,
-                     uint16_t* __restrict__ y, int32_t* __restrict__ acc_out, int m0, int m1,
-                     int RT, int* err) {
+                     const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ woffset,
+                     const float* __restrict__ bias, int N, uint16_t* __restrict__ y,
+                     int32_t* __restrict__ acc_out, int m0, int m1, int R, int early_trigger,
+                     int* err) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
-  const int R = 16 * RT;
-  const GemvLayout L(R, K, M);
-  const int G = L.G, KS = L.KS, nbox = L.nbox;
-  const int XS = L.XS;         // xq row stride
-  const int n0 = blockIdx.x * R;
-  const int rows = min(R, N - n0);  // valid rows of this CTA (a multiple of 8)
+  const GemvLayout L(R, C, K, M);
+  const int G = L.G, GC = L.GC, nbox = L.nbox, RT = L.RT, KW = L.KW, RO = L.RO, XS = L.XS;
+  const int crank = (int)blockIdx.x;  // rank in the cluster = K slice
+  const int n0 = (int)blockIdx.y * R;
+  const int rows = min(R, N - n0);    // valid rows of this row block (a multiple of 8)
+  const int g0 = crank * GC;
+  const int gcount = min(GC, G - g0);  // groups of this slice (GC when C > 1)
 
   uint8_t* w_sm = smem + L.w;
-  const uint16_t* s16 = reinterpret_cast<const uint16_t*>(smem + L.so16);
-  const uint16_t* o16 = s16 + (size_t)R * G;
-  double2* so_sm = reinterpret_cast<double2*>(smem + L.so64);
+  const uint16_t* s16 = reinterpret_cast<const uint16_t*>(smem + L.s16);
+  const uint16_t* o16 = s16 + (size_t)R * GC;
   int8_t* xq_sm = reinterpret_cast<int8_t*>(smem + L.xq);
   double* xs_sm = reinterpret_cast<double*>(smem + L.xs);
-  float* sx_sm = reinterpret_cast<float*>(smem + L.sxo);
+  float* sx_sm = reinterpret_cast<float*>(smem + L.sx);
+  unsigned int* amx_sm = reinterpret_cast<unsigned int*>(smem + L.amx);  // [C][16], local [16]
   double* part = reinterpret_cast<double*>(smem + L.part);
-  // one barrier per weight box, then one for the scales, one for the activations
   const uint32_t bars = smem_u32(smem + L.bars);
-  const uint32_t sbar = bars + 8u * nbox, abar = bars + 8u * (nbox + 1);
-
+  const uint32_t sbar = bars + 8u * nbox;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // ---- weights first: issued before the dependency wait, scales / offsets
+  // (needed first) ahead of the boxes, the boxes in K order.  A box always
+  // moves R rows x 128 bytes; rows past N and bytes past K/2 are zero-filled.
   if (threadIdx.x == 0) {
-    prefetch_tmap(&tmW);
-    for (int q = 0; q < nbox + 2; ++q) mbar_init(bars + 8u * q, 1);
+    for (int q = 0; q <= nbox; ++q) mbar_init(bars + 8u * q, 1);
     fence_mbar_init();
-  }
-  __syncthreads();
-
-  // ---- weights: issued before the dependency wait.  The scales / offsets go
-  // first (small, needed first), then the boxes in K order, so the boxes land
-  // roughly in the order the warps consume them.  A box always moves R rows x
-  // 128 bytes; rows past N and bytes past K/2 are zero-filled.
-  if (threadIdx.x == 0) {
     if (kFold) {
-      mbar_arrive_expect_tx(sbar, (uint32_t)(rows * G * 2 * 2));
-      bulk_load(smem_u32(smem + L.so16), wscale + (size_t)n0 * G, (uint32_t)(rows * G * 2), sbar);
-      bulk_load(smem_u32(smem + L.so16) + (uint32_t)(R * G * 2), woffset + (size_t)n0 * G,
-                (uint32_t)(rows * G * 2), sbar);
+      if (C > 1) {
+        mbar_arrive_expect_tx(sbar, (uint32_t)(2 * R * GC * 2));
+        tma_load_2d(smem_u32(smem + L.s16), &tmS, g0, n0, sbar);
+        tma_load_2d(smem_u32(smem + L.s16) + (uint32_t)(R * GC * 2), &tmO, g0, n0, sbar);
+      } else {
+        mbar_arrive_expect_tx(sbar, (uint32_t)(2 * rows * G * 2));
+        bulk_load(smem_u32(smem + L.s16), wscale + (size_t)n0 * G, (uint32_t)(rows * G * 2), sbar);
+        bulk_load(smem_u32(smem + L.s16) + (uint32_t)(R * G * 2), woffset + (size_t)n0 * G,
+                  (uint32_t)(rows * G * 2), sbar);
+      }
     }
     for (int j = 0; j < nbox; ++j) {
       mbar_arrive_expect_tx(bars + 8u * j, (uint32_t)(R * 128));
-      tma_load_2d(smem_u32(w_sm + (size_t)j * R * 128), &tmW, 128 * j, n0, bars + 8u * j);
+      tma_load_2d(smem_u32(w_sm + (size_t)j * R * 128), &tmW, 32 * g0 + 128 * j, n0, bars + 8u * j);
     }
   }
-  // The next kernel may start its own prologue now; it waits for this grid to
-  // finish before it touches anything this grid reads or writes.
-  pdl_launch_dependents();
+  if (early_trigger) pdl_launch_dependents();
+  // token rows past M: zero xsum (their MMA columns are zero too)
+  for (int i = threadIdx.x; i < (L.Mp - M) * (GC + 1); i += kThreads)
+    xs_sm[(size_t)M * (GC + 1) + i] = 0.0;
+  if (threadIdx.x < 16) amx_sm[C * 16 + threadIdx.x] = 0u;
+  // peers write into this CTA's shared memory only after every CTA of the
+  // cluster has arrived here (it has started)
+  if (C > 1) cluster_arrive_relaxed();
+  __syncthreads();
 
-  // scales / offsets to fp64 once they land (rows beyond `rows` are never read)
-  auto scales_to_fp64 = [&]() {
-    if (!mbar_wait(sbar, 0, err)) return;
-    for (int r = warp; r < rows; r += kWarps)
-      for (int g = lane; g < G; g += 32)
-        so_sm[r * (G + 1) + g] =
-            make_double2((double)__half2float(__ushort_as_half(s16[(size_t)r * G + g])),
-                         (double)__half2float(__ushort_as_half(o16[(size_t)r * G + g])));
-  };
-
-  // ---- activations come from the previous kernel
-  bool ok = true;
+  // ---- activations (they come from the previous kernel)
+  pdl_wait();
+  if (!early_trigger) pdl_launch_dependents();
   if constexpr (kQuantX) {
-    // Every CTA quantizes the whole of x (L2-resident, M * K <= 65536): per
-    // row the absmax, then the codes go straight into xq_sm in the even / odd
-    // order of the K map below, and the group sums into xs_sm.
-    unsigned int* amax_sm = reinterpret_cast<unsigned int*>(smem + L.amx);
-    if (threadIdx.x < 16) amax_sm[threadIdx.x] = 0u;
-    pdl_wait();
-    const int nch = K >> 3;     // 16-byte chunks per row
-    const int total = M * nch;  // chunk c of the flattened rows: row c / nch
+    const int nch = GC * 8;         // 16-byte chunks per row of the slice
+    const int total = M * nch;      // chunk c: row c / nch
     const uint4* src = reinterpret_cast<const uint4*>(x);
     uint4 v[kQuantChunks];
 #pragma unroll
     for (int i = 0; i < kQuantChunks; ++i) {
       const int c = threadIdx.x + kThreads * i;
-      v[i] = c < total ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+      v[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (c < total) {
+        const int m = c / nch;
+        v[i] = __ldg(src + (((size_t)m * K + (size_t)g0 * 64) >> 3) + (c - m * nch));
+      }
     }
-    __syncthreads();  // amax_sm zeroed
+    unsigned int* amx_local = amx_sm + C * 16;
 #pragma unroll
     for (int i = 0; i < kQuantChunks; ++i) {
       if (kThreads * i >= total) break;  // warp-uniform
@@ -219,202 +259,306 @@ __global__ void __launch_bounds__(kThreads, 1)
       // one shared-memory atomic per row present in the warp
       const unsigned same = __match_any_sync(0xFFFFFFFFu, m);
       const unsigned red = __reduce_max_sync(same, m16);
-      if (m >= 0 && lane == __ffs(same) - 1) atomicMax(amax_sm + m, red);
+      if (m >= 0 && lane == __ffs(same) - 1) atomicMax(amx_local + m, red);
     }
     __syncthreads();
+    if (C > 1) {
+      cluster_wait_acquire();  // (the start barrier) every peer is running
+      // this slice's absmax of every row, to every CTA of the cluster
+      if (threadIdx.x < C * M) {
+        const int peer = threadIdx.x / M, m = threadIdx.x - peer * M;
+        st_cluster_u32(mapa_shared(smem_u32(amx_sm + crank * 16 + m), (uint32_t)peer),
+                       amx_local[m]);
+      }
+      __syncwarp();
+      cluster_arrive_release();
+      cluster_wait_acquire();
+    }
+    auto row_amax = [&](int m) -> float {
+      unsigned int b = amx_local[m];
+      if (C > 1) {
+        b = amx_sm[m];
+#pragma unroll
+        for (int q = 1; q < C; ++q) b = max(b, amx_sm[q * 16 + m]);
+      }
+      return __uint_as_float(b << 16);
+    };
 #pragma unroll
     for (int i = 0; i < kQuantChunks; ++i) {
       if (kThreads * i >= total) break;  // warp-uniform
       const int c = threadIdx.x + kThreads * i;
-      int sum = 0, m = 0, col = 0;
+      int sum = 0, m = 0, cc = 0;
       if (c < total) {
         m = c / nch;
-        col = c - m * nch;
-        const float r = act_multiplier(__uint_as_float(amax_sm[m] << 16));
-        const uint2 qc = quant_chunk(v[i], r, &sum);
-        *reinterpret_cast<uint2*>(xq_sm + (size_t)m * XS + 8 * col) =
-            make_uint2(__byte_perm(qc.x, qc.y, 0x6420), __byte_perm(qc.x, qc.y, 0x7531));
+        cc = c - m * nch;
+        const uint2 qc = quant_chunk(v[i], act_multiplier(row_amax(m)), &sum);
+        *reinterpret_cast<uint2*>(xq_sm + (size_t)m * XS + 8 * cc) = even_odd(qc.x, qc.y);
       }
       // the 8 chunks of a group sit in 8 consecutive lanes (nch % 8 == 0)
       sum = group8_sum(sum);
-      if ((lane & 7) == 0 && c < total) xs_sm[m * (G + 1) + (col >> 3)] = i32_to_f64(sum);
+      if ((lane & 7) == 0 && c < total) xs_sm[m * (GC + 1) + (cc >> 3)] = i32_to_f64(sum);
     }
-    if (threadIdx.x < M) sx_sm[threadIdx.x] = act_scale(__uint_as_float(amax_sm[threadIdx.x] << 16));
-    for (int m = M + warp; m < L.Mp; m += kWarps)
-      for (int g = lane; g < G; g += 32) xs_sm[m * (G + 1) + g] = 0.0;
-    scales_to_fp64();
+    if (threadIdx.x < M) sx_sm[threadIdx.x] = act_scale(row_amax(threadIdx.x));
+    __syncthreads();
   } else {
-    if (warp == 1) {
-      pdl_wait();
-      if (lane == 0) mbar_arrive_expect_tx(abar, (uint32_t)(M * K));
-      __syncwarp();
-      for (int m = lane; m < M; m += 32)
-        bulk_load(smem_u32(xq_sm + (size_t)m * XS), xq + (size_t)m * K, (uint32_t)K, abar);
+    // quantized activations: the slice of xq, byte-permuted on the way in
+    const int nc16 = GC * 4;  // 16-byte chunks per row of the slice
+    for (int idx = threadIdx.x; idx < M * nc16; idx += kThreads) {
+      const int m = idx / nc16, cc = idx - m * nc16;
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(xq + (size_t)m * K + (size_t)g0 * 64) + cc);
+      const uint2 a = even_odd(q.x, q.y), b = even_odd(q.z, q.w);
+      *reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * cc) = make_uint4(a.x, a.y, b.x, b.y);
     }
-    // (weights: no dependency wait needed)
-    if (kFold) scales_to_fp64();
-    if (warp != 1) pdl_wait();
     if (kFold) {
+      for (int idx = threadIdx.x; idx < M * GC; idx += kThreads) {
+        const int m = idx / GC, g = idx - m * GC;
+        xs_sm[m * (GC + 1) + g] = g < gcount ? i32_to_f64(__ldg(xsum + (size_t)m * G + g0 + g)) : 0.0;
+      }
       if (threadIdx.x < M) sx_sm[threadIdx.x] = __ldg(sx + threadIdx.x);
-      for (int m = warp; m < L.Mp; m += kWarps)
-        for (int g = lane; g < G; g += 32)
-          xs_sm[m * (G + 1) + g] = m < M ? i32_to_f64(__ldg(xsum + (size_t)m * G + g)) : 0.0;
     }
-    // xq: within every 8 bytes put the even k first, then the odd k, to match
-    // the even / odd nibble split of the weight codes (see the K map below)
-    ok = mbar_wait(abar, 0, err);
-    if (ok) {
-      for (int m = warp; m < M; m += kWarps)
-        for (int c = lane; c < K / 16; c += 32) {
-          uint4* v = reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * c);
-          const uint4 x = *v;
-          *v = make_uint4(__byte_perm(x.x, x.y, 0x6420), __byte_perm(x.x, x.y, 0x7531),
-                          __byte_perm(x.z, x.w, 0x6420), __byte_perm(x.z, x.w, 0x7531));
-        }
-    }
+    __syncthreads();
+    if (C > 1) cluster_wait_acquire();  // the start barrier
   }
-  // token rows past M read as zeros
-  for (int m = M + warp; m < L.Mp; m += kWarps)
-    for (int c = lane; c < K / 16; c += 32)
-      *reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
-  __syncthreads();
 
-  // ---- warp (rt, q): row tile rt, groups g = q, q + KS, q + 2 KS, ...  The
-  // groups interleave so that every box (four consecutive groups) is shared by
-  // KS / 4 ... 4 warps per row tile and all warps work while the boxes land.
-  const int rt = warp % RT, q = warp / RT;
+  // ---- products.  Warp (rt, kw): row tile rt, boxes j = kw, kw + KW, ...
+  const int rt = warp % RT, kw = warp / RT;
   const int grp = lane >> 2, tq = lane & 3;
-  const int rloc = rt * 16 + grp;  // this lane's first weight row (second: +8)
-  // rows past the CTA's valid rows are read clamped (their results are dropped)
-  const int ra = min(rloc, rows - 1), rb = min(rloc + 8, rows - 1);
-  const double2* so_a = so_sm + (size_t)ra * (G + 1);
-  const double2* so_b = so_sm + (size_t)rb * (G + 1);
-  const double* xsp[TT];
+  const int ra = rt * 16 + grp;  // this lane's weight rows: ra and ra + 8
+  // Packed byte p of row r sits in box p / 128, 16-byte chunk
+  // ((p % 128) / 16) ^ (r % 8), and r % 8 == grp for both rows of the lane.
+  const uint32_t offa = (uint32_t)(ra * 128 + 8 * (tq & 1));
+  const uint32_t offb = offa + 8u * 128u;
   const int8_t* xb[TT];
+  bool tv[TT];
 #pragma unroll
   for (int tt = 0; tt < TT; ++tt) {
-    xb[tt] = xq_sm + (size_t)(tt * 8 + grp) * XS + 16 * tq;
-    xsp[tt] = xs_sm + (size_t)(tt * 8 + 2 * tq) * (G + 1);
+    const int t = tt * 8 + grp;  // this lane's token column
+    tv[tt] = t < M;
+    xb[tt] = xq_sm + (size_t)(tv[tt] ? t : 0) * XS + 16 * tq;
   }
 
-  // Offset term first, while the weight boxes are still in flight:
-  // f = sum over this warp's groups of o[n, g] * xsum[m, g].
   double f[TT][4];
 #pragma unroll
   for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) f[tt][i] = 0.0;
-  if (kFold) {
-    for (int g = q; g < G; g += KS) {
-      const double oa = so_a[g].y, ob = so_b[g].y;
+  double fa = 0.0, fb = 0.0;  // one token: rows ra, ra + 8
+  bool ok = true;
+  if (kFold) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, err));
+
+  // K map.  For group g, lane (grp, tq) handles the 16 consecutive codes
+  // k = 64 g + 16 tq + 0..15 (8 packed bytes).  Splitting a packed word into
+  // its low nibbles (codes 0, 2, 4, 6) and high nibbles (codes 1, 3, 5, 7)
+  // gives the A registers of one m16n8k32 MMA directly; xq was permuted to the
+  // same even / odd order, so each MMA sums the same 32 k on both sides, and
+  // the two MMAs of a group cover its 64 k once.
+  for (int j = kw; ok && j < nbox; j += KW) {
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars + 8u * j, 0, err))) {
+      ok = false;
+      break;
+    }
+    const uint8_t* box = w_sm + (size_t)j * R * 128;
+    int A0[4] = {0, 0, 0, 0}, A2[4] = {0, 0, 0, 0};  // one token: the box's group sums
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int gl = 4 * j + u;  // group within the slice
+      if (gl >= gcount) break;   // warp-uniform: a partial last box (C == 1)
+      const uint32_t sw = (uint32_t)(((2 * u + (tq >> 1)) ^ grp) << 4);
+      const uint2 wa = *reinterpret_cast<const uint2*>(box + offa + sw);
+      const uint2 wb = *reinterpret_cast<const uint2*>(box + offb + sw);
+      // A registers: {row grp, row grp + 8} x {even codes, odd codes}, per MMA
+      const uint32_t a0[4] = {wa.x & 0x0F0F0F0Fu, wb.x & 0x0F0F0F0Fu, (wa.x >> 4) & 0x0F0F0F0Fu,
+                              (wb.x >> 4) & 0x0F0F0F0Fu};
+      const uint32_t a1[4] = {wa.y & 0x0F0F0F0Fu, wb.y & 0x0F0F0F0Fu, (wa.y >> 4) & 0x0F0F0F0Fu,
+                              (wb.y >> 4) & 0x0F0F0F0Fu};
+      int acc[TT][4];
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt) {
-        const double x0 = xsp[tt][g], x1 = xsp[tt][(G + 1) + g];
-        f[tt][0] = fma(oa, x0, f[tt][0]);
-        f[tt][1] = fma(oa, x1, f[tt][1]);
-        f[tt][2] = fma(ob, x0, f[tt][2]);
-        f[tt][3] = fma(ob, x1, f[tt][3]);
+        const uint4 b = tv[tt] ? *reinterpret_cast<const uint4*>(xb[tt] + 64 * gl)
+                               : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[tt][i] = 0;
+        mma_u8s8(acc[tt], a0, b.x, b.y);
+        mma_u8s8(acc[tt], a1, b.z, b.w);
+      }
+      if constexpr (!kFold) {
+        // accumulator dump: acc[(m - m0), n, g] for rows m0 <= m < m1
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int m = tt * 8 + 2 * tq + (i & 1);
+            const int r = ra + (i >> 1) * 8;
+            if (m >= m0 && m < m1 && r < rows)
+              acc_out[((size_t)(m - m0) * N + n0 + r) * G + g0 + gl] = acc[tt][i];
+          }
+      } else if constexpr (kOne) {
+        A0[u] = acc[0][0];  // token 0 lives in the lanes with tq == 0
+        A2[u] = acc[0][2];
+      } else {
+        const double sa = h2d(s16[ra * GC + gl]), sb = h2d(s16[(ra + 8) * GC + gl]);
+        const double oa = h2d(o16[ra * GC + gl]), ob = h2d(o16[(ra + 8) * GC + gl]);
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+          const double x0 = xs_sm[(tt * 8 + 2 * tq) * (GC + 1) + gl];
+          const double x1 = xs_sm[(tt * 8 + 2 * tq + 1) * (GC + 1) + gl];
+          f[tt][0] = fma(oa, x0, fma(sa, i32_to_f64(acc[tt][0]), f[tt][0]));
+          f[tt][1] = fma(oa, x1, fma(sa, i32_to_f64(acc[tt][1]), f[tt][1]));
+          f[tt][2] = fma(ob, x0, fma(sb, i32_to_f64(acc[tt][2]), f[tt][2]));
+          f[tt][3] = fma(ob, x1, fma(sb, i32_to_f64(acc[tt][3]), f[tt][3]));
+        }
+      }
+    }
+    if constexpr (kFold && kOne) {
+      // lane (grp, tq) folds group 4 j + tq, gathered from lane (grp, 0)
+      int a0 = 0, a2 = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v0 = __shfl_sync(0xFFFFFFFFu, A0[u], lane & ~3);
+        const int v2 = __shfl_sync(0xFFFFFFFFu, A2[u], lane & ~3);
+        if (tq == u) {
+          a0 = v0;
+          a2 = v2;
+        }
+      }
+      const int gl = 4 * j + tq;
+      if (gl < gcount) {
+        const double x0 = xs_sm[gl];
+        fa = fma(h2d(o16[ra * GC + gl]), x0, fma(h2d(s16[ra * GC + gl]), i32_to_f64(a0), fa));
+        fb = fma(h2d(o16[(ra + 8) * GC + gl]), x0,
+                 fma(h2d(s16[(ra + 8) * GC + gl]), i32_to_f64(a2), fb));
       }
     }
   }
 
-  // K map.  For group g, lane (grp, tq) handles the 16 consecutive codes
-  // k = 64 g + 16 tq + 0..15 (8 packed bytes).  Splitting a packed word into its
-  // low nibbles (codes 0, 2, 4, 6) and high nibbles (codes 1, 3, 5, 7) gives the
-  // A registers of one m16n8k32 MMA directly; xq was permuted to the same
-  // even / odd order, so each MMA sums the same 32 k on both sides, and the two
-  // MMAs of a group cover its 64 k once.
-  // Packed byte p of row r sits in box p / 128, 16-byte chunk ((p % 128) / 16)
-  // ^ (r % 8); here p = 32 g + 8 tq and g % 4 = q % 4 for every group of the
-  // warp (KS is a multiple of 4), so the offsets inside a box are fixed.
-  const int c = 2 * (q & 3) + (tq >> 1);
-  const uint32_t offa = (uint32_t)(ra * 128 + ((c ^ (ra & 7)) << 4) + 8 * (tq & 1));
-  const uint32_t offb = (uint32_t)(rb * 128 + ((c ^ (rb & 7)) << 4) + 8 * (tq & 1));
-  const uint32_t box_bytes = (uint32_t)R * 128;
-
-#pragma unroll 2
-  for (int g = q; g < G; g += KS) {
-    if (!mbar_wait(bars + 8u * (uint32_t)(g >> 2), 0, err)) { ok = false; break; }
-    const uint8_t* box = w_sm + (size_t)(g >> 2) * box_bytes;
-    const uint2 wa = *reinterpret_cast<const uint2*>(box + offa);
-    const uint2 wb = *reinterpret_cast<const uint2*>(box + offb);
-    // A registers: {row grp, row grp + 8} x {even codes, odd codes}, per MMA
-    const uint32_t a0[4] = {wa.x & 0x0F0F0F0Fu, wb.x & 0x0F0F0F0Fu, (wa.x >> 4) & 0x0F0F0F0Fu,
-                            (wb.x >> 4) & 0x0F0F0F0Fu};
-    const uint32_t a1[4] = {wa.y & 0x0F0F0F0Fu, wb.y & 0x0F0F0F0Fu, (wa.y >> 4) & 0x0F0F0F0Fu,
-                            (wb.y >> 4) & 0x0F0F0F0Fu};
-    int acc[TT][4];
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      const uint4 b = *reinterpret_cast<const uint4*>(xb[tt] + 64 * g);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[tt][i] = 0;
-      mma_u8s8(acc[tt], a0, b.x, b.y);
-      mma_u8s8(acc[tt], a1, b.z, b.w);
-    }
-    if constexpr (!kFold) {
-      // accumulator dump: acc[(m - m0), n, g] for rows m0 <= m < m1
+  if constexpr (kFold) {
+    // ---- partial sums to the CTA that owns the rows, slot (slice, box set)
+    const int slot = crank * KW + kw;
+    const int owner = (rt * 16) / RO;
+    const int lr = rt * 16 - owner * RO + grp;  // ra within the owner's rows
+    double* pbase = part + (size_t)slot * M * RO;
+    auto put = [&](double* p, double v) {
+      if (C > 1)
+        st_cluster_f64(mapa_shared(smem_u32(p), (uint32_t)owner), v);
+      else
+        *p = v;
+    };
+    if constexpr (kOne) {
+      fa += __shfl_xor_sync(0xFFFFFFFFu, fa, 1);
+      fb += __shfl_xor_sync(0xFFFFFFFFu, fb, 1);
+      fa += __shfl_xor_sync(0xFFFFFFFFu, fa, 2);
+      fb += __shfl_xor_sync(0xFFFFFFFFu, fb, 2);
+      if (tq == 0) {
+        put(pbase + lr, fa);
+        put(pbase + lr + 8, fb);
+      }
+    } else {
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int m = tt * 8 + 2 * tq + (i & 1);
-          const int r = rloc + (i >> 1) * 8;
-          if (m >= m0 && m < m1 && r < rows)
-            acc_out[((size_t)(m - m0) * N + n0 + r) * G + g] = acc[tt][i];
+          const int t = tt * 8 + 2 * tq + (i & 1);
+          if (t < M) put(pbase + (size_t)t * RO + lr + (i >> 1) * 8, f[tt][i]);
         }
+    }
+    __syncwarp();
+    if (C > 1) {
+      cluster_arrive_release();
+      cluster_wait_acquire();
     } else {
-      const double sa = so_a[g].x, sb = so_b[g].x;
-#pragma unroll
-      for (int tt = 0; tt < TT; ++tt) {
-        f[tt][0] = fma(sa, i32_to_f64(acc[tt][0]), f[tt][0]);
-        f[tt][1] = fma(sa, i32_to_f64(acc[tt][1]), f[tt][1]);
-        f[tt][2] = fma(sb, i32_to_f64(acc[tt][2]), f[tt][2]);
-        f[tt][3] = fma(sb, i32_to_f64(acc[tt][3]), f[tt][3]);
-      }
+      __syncthreads();
     }
-  }
-  if constexpr (kFold) {
-    // ---- partial sums of the warps of a row tile, added in a fixed order
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = tt * 8 + 2 * tq + (i & 1);
-        const int r = rloc + (i >> 1) * 8;
-        part[((size_t)q * 16 + m) * (R + 4) + r] = f[tt][i];
-      }
-    __syncthreads();
-    for (int m = threadIdx.x / R; m < M; m += kThreads / R) {
-      const int r = threadIdx.x % R;  // consecutive threads -> consecutive n
-      if (r >= rows) continue;
-      double acc = 0.0;
-      for (int qq = 0; qq < KS; ++qq) acc += part[((size_t)qq * 16 + m) * (R + 4) + r];
-      const double v = fma((double)sx_sm[m], acc, bias != nullptr ? (double)bias[n0 + r] : 0.0);
-      y[(size_t)m * N + n0 + r] = f64_to_bf16_bits(v);
+    // ---- this CTA's rows [crank RO, crank RO + RO): the slots in a fixed
+    // order, then sx, bias and one rounding
+    const int nslots = C * KW;
+    for (int idx = threadIdx.x; idx < M * RO; idx += kThreads) {
+      const int t = idx / RO, r = idx - t * RO;
+      const int rr = crank * RO + r;
+      if (rr >= rows) continue;
+      double s = 0.0;
+      for (int q = 0; q < nslots; ++q) s += part[((size_t)q * M + t) * RO + r];
+      const int n = n0 + rr;
+      const double v = fma((double)sx_sm[t], s, bias != nullptr ? (double)__ldg(bias + n) : 0.0);
+      y[(size_t)t * N + n] = f64_to_bf16_bits(v);
     }
   }
 }
 
-size_t g_smem_set[6][64];
+// Tiling of one GEMV call: R weight rows per CTA, C CTAs per cluster along K.
+struct GemvPlan {
+  int R = 0, C = 0;
+  size_t smem = 0;
+};
 
-// Rows per CTA: the fewest (16, 32, 64) that still fit all CTAs in one wave.
-int choose_rt(int64_t M, int64_t K, int64_t N) {
+// Picks (R, C) for M <= 16.  In order of preference: a CTA fits two per SM
+// (the next call's CTAs can be resident while this call computes); the grid
+// fits one wave, and within it the most CTAs (the most SMs streaming
+// weights); the smallest cluster.  quant_x: x is quantized in the kernel, so
+// the K slice of the activations must fit the registers.
+bool choose_plan(int64_t M, int64_t K, int64_t N, bool quant_x, GemvPlan* out) {
+  if (M < 1 || M > 16 || K % 64 != 0 || K > 65536) return false;
   const int sms = num_sms();
-  int RT = 1;
-  while (RT < 4 && (N + 16 * RT - 1) / (16 * RT) > sms &&
-         GemvLayout(32 * RT, (int)K, (int)M).total <= (size_t)kSmemLimit)
-    RT *= 2;
-  return RT;
+  const int G = (int)(K / 64);
+  bool found = false;
+  long best[4] = {0, 0, 0, 0};
+  for (int C : {1, 2, 4}) {
+    if (C > 1 && (G % C != 0 || (G / C) % 8 != 0)) continue;
+    for (int R : {32, 64, 128}) {
+      if (R / C < 16) continue;
+      const GemvLayout L(R, C, (int)K, (int)M);
+      if (L.total > (size_t)kSmemLimit) continue;
+      if (quant_x && M * L.GC * 64 > (int64_t)kQuantChunks * 8 * kThreads) continue;
+      const long grid = (long)C * ((N + R - 1) / R);
+      const long one_wave = grid <= sms;
+      const long score[4] = {L.total <= (size_t)kSmemTwoPerSm, one_wave, one_wave ? grid : -grid,
+                             -C};
+      bool better = !found;
+      for (int i = 0; i < 4 && !better; ++i) {
+        if (score[i] != best[i]) {
+          better = score[i] > best[i];
+          break;
+        }
+      }
+      if (better) {
+        found = true;
+        for (int i = 0; i < 4; ++i) best[i] = score[i];
+        out->R = R;
+        out->C = C;
+        out->smem = L.total;
+      }
+    }
+  }
+  return found;
 }
 
-}  // namespace
+using GemvKernel = decltype(&w4a8_gemv_kernel<1, true, false, false, 1>);
 
-size_t gemv_smem_bytes(int64_t M, int64_t K, int64_t N) {
-  return GemvLayout(16 * choose_rt(M, K, N), (int)K, (int)M).total;
+template <int TT, bool kFold, bool kQuantX, bool kOne>
+GemvKernel pick_c(int C) {
+  return C == 1 ? w4a8_gemv_kernel<TT, kFold, kQuantX, kOne, 1>
+       : C == 2 ? w4a8_gemv_kernel<TT, kFold, kQuantX, kOne, 2>
+                : w4a8_gemv_kernel<TT, kFold, kQuantX, kOne, 4>;
 }
 
-namespace {
+GemvKernel pick_kernel(int64_t M, bool fold, bool quant_x, int C, int* id) {
+  // id: a small index of the instantiation, for the once-per-device attribute
+  const int ci = C == 1 ? 0 : C == 2 ? 1 : 2;
+  if (!fold) {
+    *id = 18 + ci * 2 + (M > 8);
+    return M <= 8 ? pick_c<1, false, false, false>(C) : pick_c<2, false, false, false>(C);
+  }
+  const int v = M == 1 ? 0 : M <= 8 ? 1 : 2;
+  *id = (quant_x ? 9 : 0) + ci * 3 + v;
+  if (quant_x)
+    return v == 0 ? pick_c<1, true, true, true>(C)
+         : v == 1 ? pick_c<1, true, true, false>(C) : pick_c<2, true, true, false>(C);
+  return v == 0 ? pick_c<1, true, false, true>(C)
+       : v == 1 ? pick_c<1, true, false, false>(C) : pick_c<2, true, false, false>(C);
+}
+
+constexpr int kKernelIds = 24;
+constexpr int kMaxDevices = 64;
+bool g_attr_set[kKernelIds][kMaxDevices];
 
 // One launcher for both activation forms: x != nullptr quantizes x in the
 // kernel, else xq / sx / xsum come from the caller.
@@ -423,56 +567,73 @@ cudaError_t launch_gemv(const uint16_t* x, const int8_t* xq, const float* sx,
                         const uint16_t* ws, const uint16_t* wo, const float* bias, int64_t N,
                         uint16_t* y, int32_t* acc_out, int64_t m0, int64_t m1, bool pdl,
                         cudaStream_t s) {
-  const int RT = choose_rt(M, K, N);
-  const int R = 16 * RT;
-  const unsigned grid = (unsigned)((N + R - 1) / R);
-  const size_t smem = GemvLayout(R, (int)K, (int)M).total;
-  if (smem > (size_t)kSmemLimit) return cudaErrorInvalidValue;
-  CUtensorMap tW;
-  if (!encode_tmap_2d(&tW, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wp, (uint64_t)(K / 2), (uint64_t)N,
-                      (uint64_t)(K / 2), 128, (uint32_t)R, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  int* err = device_error_word();
-  if (err == nullptr) return cudaErrorUnknown;
   const bool fold = acc_out == nullptr;
   const bool qx = x != nullptr;
-  if (qx && (!fold || M * K > (int64_t)kQuantChunks * 8 * kThreads)) return cudaErrorInvalidValue;
-  decltype(&w4a8_gemv_kernel<1, true, false>) kernel;
-  int variant;
-  if (qx) {
-    kernel = M <= 8 ? w4a8_gemv_kernel<1, true, true> : w4a8_gemv_kernel<2, true, true>;
-    variant = M <= 8 ? 4 : 5;
-  } else {
-    kernel = M <= 8 ? (fold ? w4a8_gemv_kernel<1, true, false> : w4a8_gemv_kernel<1, false, false>)
-                    : (fold ? w4a8_gemv_kernel<2, true, false> : w4a8_gemv_kernel<2, false, false>);
-    variant = (M <= 8 ? 0 : 2) + (fold ? 0 : 1);
+  if (qx && !fold) return cudaErrorInvalidValue;
+  GemvPlan p;
+  if (!choose_plan(M, K, N, qx, &p)) return cudaErrorInvalidValue;
+  const int G = (int)(K / 64), GC = G / p.C;
+  CUtensorMap tW, tS, tO;
+  if (!encode_tmap_2d(&tW, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wp, (uint64_t)(K / 2), (uint64_t)N,
+                      (uint64_t)(K / 2), 128, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  tS = tW;
+  tO = tW;
+  if (p.C > 1 && fold) {
+    // scales / offsets [N, G] fp16: boxes of GC groups x R rows
+    if (!encode_tmap_2d(&tS, CU_TENSOR_MAP_DATA_TYPE_UINT16, ws, (uint64_t)G, (uint64_t)N,
+                        (uint64_t)G * 2, (uint32_t)GC, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tmap_2d(&tO, CU_TENSOR_MAP_DATA_TYPE_UINT16, wo, (uint64_t)G, (uint64_t)N,
+                        (uint64_t)G * 2, (uint32_t)GC, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
   }
+  int* err = device_error_word();
+  if (err == nullptr) return cudaErrorUnknown;
+  int id = 0;
+  const GemvKernel kernel = pick_kernel(M, fold, qx, p.C, &id);
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 64 || g_smem_set[variant][dev] < smem) {
+  if (dev >= kMaxDevices || !g_attr_set[id][dev]) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemLimit);
     if (e != cudaSuccess) return e;
-    if (dev < 64) g_smem_set[variant][dev] = kSmemLimit;
+    if (dev < kMaxDevices) g_attr_set[id][dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = dim3((unsigned)p.C, (unsigned)((N + p.R - 1) / p.R));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = p.smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (p.C > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)p.C;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, tW, x, xq, sx, xsum, (int)M, (int)K, Wp, ws, wo, bias,
-                            (int)N, y, acc_out, (int)m0, (int)m1, RT, err);
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kernel, tW, tS, tO, x, xq, sx, xsum, (int)M, (int)K, ws, wo,
+                            bias, (int)N, y, acc_out, (int)m0, (int)m1, p.R, 0, err);
 }
 
 }  // namespace
 
+size_t gemv_smem_bytes(int64_t M, int64_t K, int64_t N) {
+  GemvPlan p;
+  return choose_plan(M, K, N, false, &p) ? p.smem : ~size_t(0);
+}
+
 bool gemv_quant_fits(int64_t M, int64_t K, int64_t N) {
-  return gemv_fits(M, K, N) && M * K <= (int64_t)kQuantChunks * 8 * kThreads;
+  GemvPlan p;
+  return choose_plan(M, K, N, true, &p);
 }
 
 cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
@@ -491,4 +652,3 @@ cudaError_t launch_w4a8_gemv_quant(const uint16_t* x, int64_t M, int64_t K, cons
 }
 
 }  // namespace qk
-

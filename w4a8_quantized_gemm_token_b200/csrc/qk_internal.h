@@ -39,15 +39,16 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
                              int64_t m0, int64_t m1, bool pdl, cudaStream_t s);
 
-// W4A8 weight-streaming GEMV (M <= 16; its per-CTA working set -- weight slice,
-// xq, scale tables -- must fit shared memory, see gemv_fits); per-group
-// accumulator dump as above.
+// W4A8 weight-streaming GEMV (M <= 16; its per-CTA working set -- the weight
+// slice of R rows x one K slice, xq, scales -- must fit shared memory, see
+// gemv_fits); per-group accumulator dump as above.
 size_t gemv_smem_bytes(int64_t M, int64_t K, int64_t N);
 inline bool gemv_fits(int64_t M, int64_t K, int64_t N) {
   return M <= 16 && gemv_smem_bytes(M, K, N) <= 227u * 1024u;
 }
-// The same GEMV quantizing bf16 x itself (M * K <= 65536, see gemv_quant_fits):
-// the activation-quant kernel and its launch drop out of the small-M linear.
+// The same GEMV quantizing bf16 x itself (each CTA's K slice of x must fit its
+// registers, see gemv_quant_fits): the activation-quant kernel and its launch
+// drop out of the small-M linear.
 bool gemv_quant_fits(int64_t M, int64_t K, int64_t N);
 cudaError_t launch_w4a8_gemv_quant(const uint16_t* x, int64_t M, int64_t K, const uint8_t* Wp,
                                    const uint16_t* ws, const uint16_t* wo, const float* bias,
