@@ -27,11 +27,12 @@ def prepare(qk, orc, case):
 
 
 # 9 x 1024 x 2376: 32-row CTAs with a ragged last CTA.  qk_w4a8_linear
-# quantizes x inside the GEMV when M * K <= 65536; 16 x 4160 x 136 is above
-# that and takes the quantization kernel + GEMV.
+# quantizes x inside the GEMV when one CTA's K slice of x fits its registers;
+# 16 x 3072 x 128 and 12 x 2112 x 136 do not and take the quantization kernel
+# + GEMV (2112 = 33 groups: a partial last group range).
 GEMV_SHAPES = [(1, 64, 8), (1, 4096, 4096), (8, 4096, 4096), (16, 4096, 4096), (3, 192, 40),
                (11, 1024, 264), (16, 3072, 128), (5, 640, 2056), (9, 1024, 2376),
-               (16, 4160, 136)]
+               (12, 2112, 136)]
 
 
 @pytest.mark.parametrize("MKN", GEMV_SHAPES, ids=lambda s: "x".join(map(str, s)))
@@ -142,9 +143,9 @@ def test_routes_agree_at_m16(qk, orc):
 
 
 def test_large_k_small_m_routes_to_gemm(qk, orc):
-    """M <= 16 with a K whose GEMV working set does not fit shared memory: the
+    """M <= 16 with a K whose GEMV tiling does not fit the registers: the
     explicit GEMV route is refused, the automatic route takes the GEMM."""
-    # K = 32768: the 16-row weight slice alone is 256 KB
+    # K = 32768: every tiling leaves a warp more than 16 groups of its rows
     case = synthetic.LinearCase("lk", M=4, K=32768, N=64, bias=True, seed=8)
     xb, dev_w, ora_w, b = prepare(qk, orc, case)
     x = to_dev_bf16(xb)

@@ -11,26 +11,29 @@
 // N = K = 4096 moves only ~9.5 MB, so a lone launch is dominated by fixed
 // latencies.  The kernel is therefore built for back-to-back calls (the
 // layers of a model, graph replays): while one call computes, the next call's
-// CTAs are already resident and streaming their weights.
+// CTAs are already resident with their weights in flight.
 //  * A cluster of C CTAs shares R weight rows; CTA c takes the groups of one
-//    K slice [c GC, (c + 1) GC).  The host picks (R, C) so that a CTA needs at
-//    most ~113 KB of shared memory (two CTAs per SM: this call's and the next
-//    one's) and the grid has at most one CTA per SM.
-//  * At kernel start, before the programmatic-dependency wait, one thread
-//    issues 2-D TMA copies of the CTA's packed codes (boxes of R rows x 128
-//    bytes, 128-byte swizzled, so the fragment reads are conflict-free) and of
-//    its fp16 scales / offsets.  Weights, scales and offsets are therefore read
-//    before the previous kernel in the stream has finished: they must not be
-//    written by a kernel that triggers its dependents early (no kernel of this
-//    library that writes weights does).
+//    K slice [c GC, (c + 1) GC).  The host picks (R, C) so that every warp
+//    holds at most 16 groups of its two weight rows per lane, two CTAs fit an
+//    SM (this call's and the next one's) and the grid is at most one CTA per
+//    SM.
+//  * Register-resident weights: at kernel start, before the programmatic-
+//    dependency wait, every lane issues the 8-byte loads of its packed codes
+//    (per group: 8 bytes of each of its two rows) straight into registers,
+//    and one thread bulk-copies the CTA's fp16 scales / offsets into shared
+//    memory; the bias of the CTA's rows is read too.  Weights, scales,
+//    offsets and bias are therefore read before the previous kernel in the
+//    stream has finished: they must not be written by a kernel that triggers
+//    its dependents early (no kernel of this library that writes weights
+//    does).
 //  * After the wait the CTA either quantizes its K slice of bf16 x itself
 //    (the rule of the stand-alone quantization kernel; with C > 1 the per-row
 //    absmax is exchanged through distributed shared memory) or reads
 //    quantized xq / sx / xsum.
-//  * 8 warps = R/16 row tiles x KW box sets.  Nibbles are split in registers
-//    straight into the A fragments of mma.sync m16n8k32 u8 x s8 (weights as A,
-//    tokens as the N = 8 side); K is permuted identically in A and B so each
-//    lane reads 8 packed bytes and 16 activation bytes per group.
+//  * 8 warps = R/16 row tiles x KW group ranges.  Nibbles are split in
+//    registers straight into the A fragments of mma.sync m16n8k32 u8 x s8
+//    (weights as A, tokens as the N = 8 side); K is permuted identically in A
+//    and B so each lane uses 8 packed bytes and 16 activation bytes per group.
 //  * Per-group sums fold into fp64 (exact int -> fp64 by the 2^52 magic
 //    number).  With one token the lanes first gather one group each by
 //    shuffles, so no lane folds an all-zero token column.
@@ -44,6 +47,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "act_quant.cuh"
@@ -62,12 +66,14 @@ constexpr int kSmemTwoPerSm = 113 * 1024;
 // x per thread in registers (M * KC <= kQuantChunks * 8 * kThreads = 16384,
 // KC = the K slice of one CTA).
 constexpr int kQuantChunks = 8;
+// Groups of 64 codes one warp holds in registers (two rows, 8 bytes each).
+constexpr int kWarpGroups = 16;
 
 // Shared-memory layout of one CTA: R weight rows, cluster of C CTAs along K,
 // M token rows.
 struct GemvLayout {
-  int R, C, M, G, GC, RT, KW, nbox, XS, RO, Mp;
-  size_t w, s16, xq, xs, sx, amx, part, bars, total;
+  int R, C, M, G, GC, RT, KW, GW, RO, Mp, XS;
+  size_t s16, xq, xs, sx, amx, bias, part, bars, total;
   __host__ __device__ GemvLayout(int R_, int C_, int K, int M_) {
     R = R_;
     C = C_;
@@ -75,15 +81,14 @@ struct GemvLayout {
     G = K / 64;
     GC = (G + C - 1) / C;      // groups per K slice (C > 1: C divides G)
     RT = R / 16;               // row tiles
-    KW = kWarps / RT;          // box sets per row tile
-    nbox = (GC + 3) / 4;       // 128-byte boxes per row of the slice
+    KW = kWarps / RT;          // group ranges per row tile
+    GW = (GC + KW - 1) / KW;   // groups per warp (at most kWarpGroups)
     RO = R / C;                // rows each CTA finalizes
     Mp = M <= 8 ? 8 : 16;      // token columns of the MMAs
     // xq row stride = 64 (mod 128): the two token rows of one 16-byte load
     // phase fall in opposite halves of the banks
     XS = (GC * 64 + 127) / 128 * 128 + 64;
     size_t off = 0;
-    w = off;    off += (size_t)nbox * R * 128;        // packed codes, swizzled boxes
     s16 = off;  off += (size_t)R * GC * 2 * 2;        // fp16 scales [R][GC], then offsets
     off = (off + 127) & ~size_t(127);
     xq = off;   off += (size_t)M * XS;                // xq rows of the slice (permuted)
@@ -91,20 +96,23 @@ struct GemvLayout {
     xs = off;   off += (size_t)Mp * (GC + 1) * 8;     // xsum as fp64, zero past M
     sx = off;   off += 16 * 4;                        // sx
     amx = off;  off += (size_t)(C + 1) * 16 * 4;      // absmax: [C] exchange slots, local
+    bias = off; off += (size_t)RO * 4;                // bias of the rows this CTA finalizes
     off = (off + 15) & ~size_t(15);
     part = off; off += (size_t)C * KW * M * RO * 8;   // fp64 partials [slot][token][row]
-    bars = off; off += (size_t)(nbox + 1) * 8;        // mbarriers: boxes, scales
+    bars = off; off += 8;                             // mbarrier of the scales
     total = off + 1024;                               // base alignment slack
   }
 };
 
+// D = A (16 x 32, u8) * B (32 x 8, s8), int32, from a zero accumulator.  Not
+// volatile: it has no side effects, so the compiler may interleave the MMAs
+// of independent groups.
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
 }
 
 __device__ __forceinline__ double i32_to_f64(int a) {
@@ -158,6 +166,15 @@ __device__ __forceinline__ uint2 even_odd(uint32_t lo, uint32_t hi) {
   return make_uint2(__byte_perm(lo, hi, 0x6420), __byte_perm(lo, hi, 0x7531));
 }
 
+// 8-byte load of read-only data that is used once (no L1 allocation).
+__device__ __forceinline__ uint2 ldg_stream_v2(const uint8_t* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+               : "=r"(v.x), "=r"(v.y)
+               : "l"(p));
+  return v;
+}
+
 // TT token tiles of 8 (M <= 8 TT).  kFold: the product y; otherwise the
 // per-group int32 sums of rows [m0, m1) go to acc_out.  kQuantX: the
 // activations arrive as bf16 x and are quantized here (xq, sx, xsum unused).
@@ -165,41 +182,44 @@ __device__ __forceinline__ uint2 even_odd(uint32_t lo, uint32_t hi) {
 // Grid (C, ceil(N / R)), cluster (C, 1, 1).
 template <int TT, bool kFold, bool kQuantX, bool kOne, int C>
 __global__ void __launch_bounds__(kThreads, 2)
-    w4a8_gemv_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
-                     const __grid_constant__ CUtensorMap tmO, const uint16_t* __restrict__ x,
-                     const int8_t* __restrict__ xq, const float* __restrict__ sx,
-                     const int32_t* __restrict__ xsum, int M, int K,
-                     const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ woffset,
-                     const float* __restrict__ bias, int N, uint16_t* __restrict__ y,
-                     int32_t* __restrict__ acc_out, int m0, int m1, int R, int early_trigger,
-                     int* err) {
+    w4a8_gemv_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmO,
+                     const uint16_t* __restrict__ x, const int8_t* __restrict__ xq,
+                     const float* __restrict__ sx, const int32_t* __restrict__ xsum, int M, int K,
+                     const uint8_t* __restrict__ Wp, const uint16_t* __restrict__ wscale,
+                     const uint16_t* __restrict__ woffset, const float* __restrict__ bias, int N,
+                     uint16_t* __restrict__ y, int32_t* __restrict__ acc_out, int m0, int m1, int R,
+                     int early_trigger, int* err) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
   const GemvLayout L(R, C, K, M);
-  const int G = L.G, GC = L.GC, nbox = L.nbox, RT = L.RT, KW = L.KW, RO = L.RO, XS = L.XS;
+  const int G = L.G, GC = L.GC, RT = L.RT, KW = L.KW, RO = L.RO, XS = L.XS;
   const int crank = (int)blockIdx.x;  // rank in the cluster = K slice
   const int n0 = (int)blockIdx.y * R;
   const int rows = min(R, N - n0);    // valid rows of this row block (a multiple of 8)
   const int g0 = crank * GC;
   const int gcount = min(GC, G - g0);  // groups of this slice (GC when C > 1)
 
-  uint8_t* w_sm = smem + L.w;
   const uint16_t* s16 = reinterpret_cast<const uint16_t*>(smem + L.s16);
   const uint16_t* o16 = s16 + (size_t)R * GC;
   int8_t* xq_sm = reinterpret_cast<int8_t*>(smem + L.xq);
   double* xs_sm = reinterpret_cast<double*>(smem + L.xs);
   float* sx_sm = reinterpret_cast<float*>(smem + L.sx);
   unsigned int* amx_sm = reinterpret_cast<unsigned int*>(smem + L.amx);  // [C][16], local [16]
+  float* bias_sm = reinterpret_cast<float*>(smem + L.bias);
   double* part = reinterpret_cast<double*>(smem + L.part);
-  const uint32_t bars = smem_u32(smem + L.bars);
-  const uint32_t sbar = bars + 8u * nbox;
+  const uint32_t sbar = smem_u32(smem + L.bars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rt = warp % RT, kw = warp / RT;
+  const int grp = lane >> 2, tq = lane & 3;
+  const int ra = rt * 16 + grp;  // this lane's weight rows: ra and ra + 8
+  // this warp's groups of the slice: [gbeg, gbeg + gn)
+  const int gbeg = kw * L.GW;
+  const int gn = max(0, min(L.GW, gcount - gbeg));
 
-  // ---- weights first: issued before the dependency wait, scales / offsets
-  // (needed first) ahead of the boxes, the boxes in K order.  A box always
-  // moves R rows x 128 bytes; rows past N and bytes past K/2 are zero-filled.
+  // ---- before the dependency wait: scales / offsets by bulk copy, the
+  // packed codes of this lane's two rows into registers, the bias.
   if (threadIdx.x == 0) {
-    for (int q = 0; q <= nbox; ++q) mbar_init(bars + 8u * q, 1);
+    mbar_init(sbar, 1);
     fence_mbar_init();
     if (kFold) {
       if (C > 1) {
@@ -213,11 +233,27 @@ __global__ void __launch_bounds__(kThreads, 2)
                   (uint32_t)(rows * G * 2), sbar);
       }
     }
-    for (int j = 0; j < nbox; ++j) {
-      mbar_arrive_expect_tx(bars + 8u * j, (uint32_t)(R * 128));
-      tma_load_2d(smem_u32(w_sm + (size_t)j * R * 128), &tmW, 32 * g0 + 128 * j, n0, bars + 8u * j);
+  }
+  // Lane (grp, tq) of group g uses the 8 packed bytes 32 g + 8 tq .. + 7 of
+  // rows ra and ra + 8 (rows past N read row N - 1; their results are dropped).
+  uint2 wr[kWarpGroups][2];
+  {
+    const size_t rb = (size_t)(K / 2);
+    const uint8_t* pa = Wp + (size_t)min(n0 + ra, N - 1) * rb + (size_t)(g0 + gbeg) * 32 + 8 * tq;
+    const uint8_t* pb = Wp + (size_t)min(n0 + ra + 8, N - 1) * rb + (size_t)(g0 + gbeg) * 32 + 8 * tq;
+#pragma unroll
+    for (int i = 0; i < kWarpGroups; ++i) {
+      if (i < gn) {
+        wr[i][0] = ldg_stream_v2(pa + 32 * i);
+        wr[i][1] = ldg_stream_v2(pb + 32 * i);
+      } else {
+        wr[i][0] = make_uint2(0u, 0u);
+        wr[i][1] = make_uint2(0u, 0u);
+      }
     }
   }
+  if (kFold && threadIdx.x < RO && crank * RO + (int)threadIdx.x < rows)
+    bias_sm[threadIdx.x] = bias != nullptr ? __ldg(bias + n0 + crank * RO + threadIdx.x) : 0.0f;
   if (early_trigger) pdl_launch_dependents();
   // token rows past M: zero xsum (their MMA columns are zero too)
   for (int i = threadIdx.x; i < (L.Mp - M) * (GC + 1); i += kThreads)
@@ -302,12 +338,30 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
   } else {
     // quantized activations: the slice of xq, byte-permuted on the way in
+    // (batches of 8 independent loads per thread before any store)
     const int nc16 = GC * 4;  // 16-byte chunks per row of the slice
-    for (int idx = threadIdx.x; idx < M * nc16; idx += kThreads) {
-      const int m = idx / nc16, cc = idx - m * nc16;
-      const uint4 q = __ldg(reinterpret_cast<const uint4*>(xq + (size_t)m * K + (size_t)g0 * 64) + cc);
-      const uint2 a = even_odd(q.x, q.y), b = even_odd(q.z, q.w);
-      *reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * cc) = make_uint4(a.x, a.y, b.x, b.y);
+    const int total = M * nc16;
+    for (int base = 0; base < total; base += 8 * kThreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int idx = base + threadIdx.x + kThreads * i;
+        if (idx < total) {
+          const int m = idx / nc16;
+          v[i] = __ldg(reinterpret_cast<const uint4*>(xq + (size_t)m * K + (size_t)g0 * 64) +
+                       (idx - m * nc16));
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int idx = base + threadIdx.x + kThreads * i;
+        if (idx < total) {
+          const int m = idx / nc16, cc = idx - m * nc16;
+          const uint2 a = even_odd(v[i].x, v[i].y), b = even_odd(v[i].z, v[i].w);
+          *reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * cc) =
+              make_uint4(a.x, a.y, b.x, b.y);
+        }
+      }
     }
     if (kFold) {
       for (int idx = threadIdx.x; idx < M * GC; idx += kThreads) {
@@ -320,14 +374,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (C > 1) cluster_wait_acquire();  // the start barrier
   }
 
-  // ---- products.  Warp (rt, kw): row tile rt, boxes j = kw, kw + KW, ...
-  const int rt = warp % RT, kw = warp / RT;
-  const int grp = lane >> 2, tq = lane & 3;
-  const int ra = rt * 16 + grp;  // this lane's weight rows: ra and ra + 8
-  // Packed byte p of row r sits in box p / 128, 16-byte chunk
-  // ((p % 128) / 16) ^ (r % 8), and r % 8 == grp for both rows of the lane.
-  const uint32_t offa = (uint32_t)(ra * 128 + 8 * (tq & 1));
-  const uint32_t offb = offa + 8u * 128u;
+  // ---- products.  Warp (rt, kw): row tile rt, groups [gbeg, gbeg + gn)
   const int8_t* xb[TT];
   bool tv[TT];
 #pragma unroll
@@ -336,15 +383,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     tv[tt] = t < M;
     xb[tt] = xq_sm + (size_t)(tv[tt] ? t : 0) * XS + 16 * tq;
   }
-
   double f[TT][4];
 #pragma unroll
   for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) f[tt][i] = 0.0;
   double fa = 0.0, fb = 0.0;  // one token: rows ra, ra + 8
-  bool ok = true;
-  if (kFold) ok = __all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, err));
+  const bool ok = !kFold || __all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, err));
 
   // K map.  For group g, lane (grp, tq) handles the 16 consecutive codes
   // k = 64 g + 16 tq + 0..15 (8 packed bytes).  Splitting a packed word into
@@ -352,50 +397,51 @@ __global__ void __launch_bounds__(kThreads, 2)
   // gives the A registers of one m16n8k32 MMA directly; xq was permuted to the
   // same even / odd order, so each MMA sums the same 32 k on both sides, and
   // the two MMAs of a group cover its 64 k once.
-  for (int j = kw; ok && j < nbox; j += KW) {
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars + 8u * j, 0, err))) {
-      ok = false;
-      break;
-    }
-    const uint8_t* box = w_sm + (size_t)j * R * 128;
-    int A0[4] = {0, 0, 0, 0}, A2[4] = {0, 0, 0, 0};  // one token: the box's group sums
+  //
+  // Blocks of four groups with no branch inside a block, so the loads and
+  // MMAs of its groups overlap; groups past gn hold zero codes (see wr) and
+  // their results are dropped.
+#pragma unroll
+  for (int blk = 0; blk < kWarpGroups / 4; ++blk) {
+    if (!ok || 4 * blk >= gn) break;  // warp-uniform
+    int A0[4], A2[4];                 // one token: the block's group sums
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int gl = 4 * j + u;  // group within the slice
-      if (gl >= gcount) break;   // warp-uniform: a partial last box (C == 1)
-      const uint32_t sw = (uint32_t)(((2 * u + (tq >> 1)) ^ grp) << 4);
-      const uint2 wa = *reinterpret_cast<const uint2*>(box + offa + sw);
-      const uint2 wb = *reinterpret_cast<const uint2*>(box + offb + sw);
+      const int i = 4 * blk + u;
+      const int gl = gbeg + min(i, gn - 1);  // group within the slice (clamped)
+      const uint2 wa = wr[i][0], wb = wr[i][1];
       // A registers: {row grp, row grp + 8} x {even codes, odd codes}, per MMA
       const uint32_t a0[4] = {wa.x & 0x0F0F0F0Fu, wb.x & 0x0F0F0F0Fu, (wa.x >> 4) & 0x0F0F0F0Fu,
                               (wb.x >> 4) & 0x0F0F0F0Fu};
       const uint32_t a1[4] = {wa.y & 0x0F0F0F0Fu, wb.y & 0x0F0F0F0Fu, (wa.y >> 4) & 0x0F0F0F0Fu,
                               (wb.y >> 4) & 0x0F0F0F0Fu};
+      // two independent MMAs per token tile (half a group each), then one add
       int acc[TT][4];
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt) {
         const uint4 b = tv[tt] ? *reinterpret_cast<const uint4*>(xb[tt] + 64 * gl)
                                : make_uint4(0u, 0u, 0u, 0u);
+        int h0[4], h1[4];
+        mma_u8s8(h0, a0, b.x, b.y);
+        mma_u8s8(h1, a1, b.z, b.w);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[tt][i] = 0;
-        mma_u8s8(acc[tt], a0, b.x, b.y);
-        mma_u8s8(acc[tt], a1, b.z, b.w);
+        for (int q = 0; q < 4; ++q) acc[tt][q] = h0[q] + h1[q];
       }
       if constexpr (!kFold) {
         // accumulator dump: acc[(m - m0), n, g] for rows m0 <= m < m1
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int m = tt * 8 + 2 * tq + (i & 1);
-            const int r = ra + (i >> 1) * 8;
-            if (m >= m0 && m < m1 && r < rows)
-              acc_out[((size_t)(m - m0) * N + n0 + r) * G + g0 + gl] = acc[tt][i];
+          for (int q = 0; q < 4; ++q) {
+            const int m = tt * 8 + 2 * tq + (q & 1);
+            const int r = ra + (q >> 1) * 8;
+            if (i < gn && m >= m0 && m < m1 && r < rows)
+              acc_out[((size_t)(m - m0) * N + n0 + r) * G + g0 + gl] = acc[tt][q];
           }
       } else if constexpr (kOne) {
         A0[u] = acc[0][0];  // token 0 lives in the lanes with tq == 0
         A2[u] = acc[0][2];
-      } else {
+      } else if (i < gn) {
         const double sa = h2d(s16[ra * GC + gl]), sb = h2d(s16[(ra + 8) * GC + gl]);
         const double oa = h2d(o16[ra * GC + gl]), ob = h2d(o16[(ra + 8) * GC + gl]);
 #pragma unroll
@@ -410,29 +456,31 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     if constexpr (kFold && kOne) {
-      // lane (grp, tq) folds group 4 j + tq, gathered from lane (grp, 0)
-      int a0 = 0, a2 = 0;
+      // lane (grp, tq) folds group 4 blk + tq of the warp, gathered from
+      // lane (grp, 0)
+      int s0 = 0, s2 = 0;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int v0 = __shfl_sync(0xFFFFFFFFu, A0[u], lane & ~3);
         const int v2 = __shfl_sync(0xFFFFFFFFu, A2[u], lane & ~3);
         if (tq == u) {
-          a0 = v0;
-          a2 = v2;
+          s0 = v0;
+          s2 = v2;
         }
       }
-      const int gl = 4 * j + tq;
-      if (gl < gcount) {
-        const double x0 = xs_sm[gl];
-        fa = fma(h2d(o16[ra * GC + gl]), x0, fma(h2d(s16[ra * GC + gl]), i32_to_f64(a0), fa));
-        fb = fma(h2d(o16[(ra + 8) * GC + gl]), x0,
-                 fma(h2d(s16[(ra + 8) * GC + gl]), i32_to_f64(a2), fb));
+      const int ig = 4 * blk + tq;
+      if (ig < gn) {
+        const int g = gbeg + ig;
+        const double x0 = xs_sm[g];
+        fa = fma(h2d(o16[ra * GC + g]), x0, fma(h2d(s16[ra * GC + g]), i32_to_f64(s0), fa));
+        fb = fma(h2d(o16[(ra + 8) * GC + g]), x0,
+                 fma(h2d(s16[(ra + 8) * GC + g]), i32_to_f64(s2), fb));
       }
     }
   }
 
   if constexpr (kFold) {
-    // ---- partial sums to the CTA that owns the rows, slot (slice, box set)
+    // ---- partial sums to the CTA that owns the rows, slot (slice, group range)
     const int slot = crank * KW + kw;
     const int owner = (rt * 16) / RO;
     const int lr = rt * 16 - owner * RO + grp;  // ra within the owner's rows
@@ -456,9 +504,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int t = tt * 8 + 2 * tq + (i & 1);
-          if (t < M) put(pbase + (size_t)t * RO + lr + (i >> 1) * 8, f[tt][i]);
+        for (int q = 0; q < 4; ++q) {
+          const int t = tt * 8 + 2 * tq + (q & 1);
+          if (t < M) put(pbase + (size_t)t * RO + lr + (q >> 1) * 8, f[tt][q]);
         }
     }
     __syncwarp();
@@ -477,9 +525,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (rr >= rows) continue;
       double s = 0.0;
       for (int q = 0; q < nslots; ++q) s += part[((size_t)q * M + t) * RO + r];
-      const int n = n0 + rr;
-      const double v = fma((double)sx_sm[t], s, bias != nullptr ? (double)__ldg(bias + n) : 0.0);
-      y[(size_t)t * N + n] = f64_to_bf16_bits(v);
+      const double v = fma((double)sx_sm[t], s, (double)bias_sm[r]);
+      y[(size_t)t * N + n0 + rr] = f64_to_bf16_bits(v);
     }
   }
 }
@@ -490,30 +537,34 @@ struct GemvPlan {
   size_t smem = 0;
 };
 
-// Picks (R, C) for M <= 16.  In order of preference: a CTA fits two per SM
-// (the next call's CTAs can be resident while this call computes); the grid
-// fits one wave, and within it the most CTAs (the most SMs streaming
-// weights); the smallest cluster.  quant_x: x is quantized in the kernel, so
-// the K slice of the activations must fit the registers.
+// Picks (R, C) for M <= 16.  A warp holds at most kWarpGroups groups of its
+// rows in registers.  In order of preference: a CTA fits two per SM (the
+// next call's CTAs can be resident while this call computes); the grid fits
+// one wave; at most 16 KB of activations per CTA (they are read after the
+// dependency wait, on the critical path); the most CTAs (the most SMs
+// streaming weights); the smallest cluster.  quant_x: x is quantized in the kernel, so the K slice
+// of the activations must fit the registers too.
 bool choose_plan(int64_t M, int64_t K, int64_t N, bool quant_x, GemvPlan* out) {
   if (M < 1 || M > 16 || K % 64 != 0 || K > 65536) return false;
   const int sms = num_sms();
   const int G = (int)(K / 64);
   bool found = false;
-  long best[4] = {0, 0, 0, 0};
+  long best[5] = {0, 0, 0, 0, 0};
   for (int C : {1, 2, 4}) {
     if (C > 1 && (G % C != 0 || (G / C) % 8 != 0)) continue;
     for (int R : {32, 64, 128}) {
       if (R / C < 16) continue;
       const GemvLayout L(R, C, (int)K, (int)M);
-      if (L.total > (size_t)kSmemLimit) continue;
+      if (L.total > (size_t)kSmemLimit || L.GW > kWarpGroups) continue;
       if (quant_x && M * L.GC * 64 > (int64_t)kQuantChunks * 8 * kThreads) continue;
       const long grid = (long)C * ((N + R - 1) / R);
       const long one_wave = grid <= sms;
-      const long score[4] = {L.total <= (size_t)kSmemTwoPerSm, one_wave, one_wave ? grid : -grid,
-                             -C};
+      // activation bytes one CTA reads after the dependency wait, beyond 16 KB
+      const long act_excess = -std::max(0L, (long)(M * L.GC * 64) - 16384L);
+      const long score[5] = {L.total <= (size_t)kSmemTwoPerSm, one_wave, act_excess,
+                             one_wave ? grid : -grid, -C};
       bool better = !found;
-      for (int i = 0; i < 4 && !better; ++i) {
+      for (int i = 0; i < 5 && !better; ++i) {
         if (score[i] != best[i]) {
           better = score[i] > best[i];
           break;
@@ -521,7 +572,7 @@ bool choose_plan(int64_t M, int64_t K, int64_t N, bool quant_x, GemvPlan* out) {
       }
       if (better) {
         found = true;
-        for (int i = 0; i < 4; ++i) best[i] = score[i];
+        for (int i = 0; i < 5; ++i) best[i] = score[i];
         out->R = R;
         out->C = C;
         out->smem = L.total;
@@ -573,14 +624,11 @@ cudaError_t launch_gemv(const uint16_t* x, const int8_t* xq, const float* sx,
   GemvPlan p;
   if (!choose_plan(M, K, N, qx, &p)) return cudaErrorInvalidValue;
   const int G = (int)(K / 64), GC = G / p.C;
-  CUtensorMap tW, tS, tO;
-  if (!encode_tmap_2d(&tW, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wp, (uint64_t)(K / 2), (uint64_t)N,
-                      (uint64_t)(K / 2), 128, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  tS = tW;
-  tO = tW;
+  // scales / offsets [N, G] fp16 as 2-D boxes of GC groups x R rows (C > 1;
+  // one CTA's block is then strided); with C == 1 it is contiguous and goes by
+  // bulk copy, and the maps are unused
+  CUtensorMap tS = {}, tO = {};
   if (p.C > 1 && fold) {
-    // scales / offsets [N, G] fp16: boxes of GC groups x R rows
     if (!encode_tmap_2d(&tS, CU_TENSOR_MAP_DATA_TYPE_UINT16, ws, (uint64_t)G, (uint64_t)N,
                         (uint64_t)G * 2, (uint32_t)GC, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !encode_tmap_2d(&tO, CU_TENSOR_MAP_DATA_TYPE_UINT16, wo, (uint64_t)G, (uint64_t)N,
@@ -620,7 +668,7 @@ cudaError_t launch_gemv(const uint16_t* x, const int8_t* xq, const float* sx,
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kernel, tW, tS, tO, x, xq, sx, xsum, (int)M, (int)K, ws, wo,
+  return cudaLaunchKernelEx(&cfg, kernel, tS, tO, x, xq, sx, xsum, (int)M, (int)K, Wp, ws, wo,
                             bias, (int)N, y, acc_out, (int)m0, (int)m1, p.R, 0, err);
 }
 
