@@ -25,6 +25,12 @@ SHAPES = [  # (M, K, N): tiles of 128 x 256 with K blocks of 128
     (257, 1024, 520),
     (128, 128, 256),
     (513, 384, 776),
+    # N <= 64: the split-K cluster route (K ranges over 1, 2, 4 or 8 CTAs,
+    # ragged M, N and K blocks)
+    (300, 992, 40),
+    (1, 5120, 48),
+    (130, 4096, 64),
+    (129, 384, 16),
 ]
 
 
@@ -102,9 +108,10 @@ def test_w8a8_deterministic_and_api_variants(qk, orc):
         assert torch.equal(y1.view(torch.int16), y.view(torch.int16))
 
 
-def test_w8a8_guard_bands(qk, orc):
+@pytest.mark.parametrize("MKN", [(200, 256, 264), (200, 1024, 40)], ids=["tiles", "splitk"])
+def test_w8a8_guard_bands(qk, orc, MKN):
     """Outputs land only inside y: a sentinel halo around it stays untouched."""
-    M, K, N = 200, 256, 264
+    M, K, N = MKN
     case = synthetic.LinearCase("g", M=M, K=K, N=N, seed=9)
     xb, Wq, sw, _, _, b = prepare(qk, orc, case)
     pad = 4096

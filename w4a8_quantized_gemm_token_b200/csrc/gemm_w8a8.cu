@@ -398,6 +398,8 @@ bool g_attr_done[2][64];
 cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64_t K,
                              const int8_t* Wq, const float* sw, const float* bias, int64_t N,
                              uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s) {
+  if (w8a8_use_skinny(M, K, N))
+    return launch_w8a8_skinny(xq, sx, M, K, Wq, sw, bias, N, y, acc_out, pdl, s);
   const bool acc_mode = acc_out != nullptr;
   CUtensorMap tA, tB, tC;
   if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,

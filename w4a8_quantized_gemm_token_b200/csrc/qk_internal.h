@@ -32,6 +32,14 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
                              const int8_t* Wq, const float* sw, const float* bias, int64_t N,
                              uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s);
 
+// The same product for thin outputs (N <= 64, see w8a8_use_skinny): 128-row
+// tiles split along K over a cluster, exact int32 partial sums reduced through
+// distributed shared memory.  launch_w8a8_gemm routes such shapes here.
+bool w8a8_use_skinny(int64_t M, int64_t K, int64_t N);
+cudaError_t launch_w8a8_skinny(const int8_t* xq, const float* sx, int64_t M, int64_t K,
+                               const int8_t* Wq, const float* sw, const float* bias, int64_t N,
+                               uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s);
+
 // W4A8 tensor-core GEMM (any M).  When `acc_out` is not null it stores the
 // per-group int32 accumulators of rows [m0, m1) instead of y.
 cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
