@@ -389,7 +389,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int i = 0; i < 4; ++i) f[tt][i] = 0.0;
   double fa = 0.0, fb = 0.0;  // one token: rows ra, ra + 8
-  const bool ok = !kFold || __all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, err));
+  // (if the scales never land the results are wrong and the error word is set)
+  if (kFold) __all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, err));
 
   // K map.  For group g, lane (grp, tq) handles the 16 consecutive codes
   // k = 64 g + 16 tq + 0..15 (8 packed bytes).  Splitting a packed word into
@@ -398,12 +399,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   // same even / odd order, so each MMA sums the same 32 k on both sides, and
   // the two MMAs of a group cover its 64 k once.
   //
-  // Blocks of four groups with no branch inside a block, so the loads and
-  // MMAs of its groups overlap; groups past gn hold zero codes (see wr) and
-  // their results are dropped.
+  // All kWarpGroups groups in straight-line code (no branch between them, so
+  // the loads, MMAs and folds of different groups overlap); groups past gn
+  // hold zero codes (see wr) and their results are dropped.
 #pragma unroll
   for (int blk = 0; blk < kWarpGroups / 4; ++blk) {
-    if (!ok || 4 * blk >= gn) break;  // warp-uniform
     int A0[4], A2[4];                 // one token: the block's group sums
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
