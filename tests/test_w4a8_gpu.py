@@ -32,7 +32,10 @@ def prepare(qk, orc, case):
 # + GEMV (2112 = 33 groups: a partial last group range).
 GEMV_SHAPES = [(1, 64, 8), (1, 4096, 4096), (8, 4096, 4096), (16, 4096, 4096), (3, 192, 40),
                (11, 1024, 264), (16, 3072, 128), (5, 640, 2056), (9, 1024, 2376),
-               (12, 2112, 136)]
+               (12, 2112, 136),
+               # one token, K a multiple of 1024: the dp4a kernel (1 to 4 chunks per
+               # lane, ragged last CTA)
+               (1, 1024, 264), (1, 3072, 136), (1, 2048, 40)]
 
 
 @pytest.mark.parametrize("MKN", GEMV_SHAPES, ids=lambda s: "x".join(map(str, s)))

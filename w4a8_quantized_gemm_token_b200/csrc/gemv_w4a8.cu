@@ -621,6 +621,8 @@ cudaError_t launch_gemv(const uint16_t* x, const int8_t* xq, const float* sx,
   const bool fold = acc_out == nullptr;
   const bool qx = x != nullptr;
   if (qx && !fold) return cudaErrorInvalidValue;
+  if (gemv1_fits(M, K, N) && (fold || (m0 == 0 && m1 == 1)))
+    return launch_w4a8_gemv1(x, xq, sx, xsum, K, Wp, ws, wo, bias, N, y, acc_out, pdl, s);
   GemvPlan p;
   if (!choose_plan(M, K, N, qx, &p)) return cudaErrorInvalidValue;
   const int G = (int)(K / 64), GC = G / p.C;

@@ -61,6 +61,14 @@ bool gemv_quant_fits(int64_t M, int64_t K, int64_t N);
 cudaError_t launch_w4a8_gemv_quant(const uint16_t* x, int64_t M, int64_t K, const uint8_t* Wp,
                                    const uint16_t* ws, const uint16_t* wo, const float* bias,
                                    int64_t N, uint16_t* y, bool pdl, cudaStream_t s);
+// One token (M = 1, K a multiple of 1024 up to 4096): a dp4a kernel that keeps
+// every lane busy; launch_w4a8_gemv / launch_w4a8_gemv_quant route such shapes
+// here.  x != nullptr quantizes x in the kernel; acc_out dumps the group sums.
+bool gemv1_fits(int64_t M, int64_t K, int64_t N);
+cudaError_t launch_w4a8_gemv1(const uint16_t* x, const int8_t* xq, const float* sx,
+                              const int32_t* xsum, int64_t K, const uint8_t* Wp,
+                              const uint16_t* ws, const uint16_t* wo, const float* bias, int64_t N,
+                              uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s);
 cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                              int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
