@@ -14,11 +14,11 @@
 //    wait one thread bulk-copies each warp's rows (contiguous, 4 x K/2 bytes)
 //    and the CTA's fp16 scales / offsets into shared memory, and the scales
 //    become an fp64 {s, o} table -- all off the critical path;
-//  * after the wait x is quantized in the CTA (the rule of the stand-alone
-//    kernel) or xq / sx / xsum are read;
 //  * lane l owns the 16-byte chunks l, l + 32, l + 64, ... of a packed row
-//    (one 512-byte, conflict-free shared load per chunk index for the warp)
-//    and holds the matching activation codes in registers for all four rows;
+//    (one 512-byte, conflict-free shared load per chunk index for the warp);
+//    after the wait every lane holds the matching activation codes in
+//    registers -- read straight from xq, or quantized by the CTA from bf16 x
+//    (the rule of the stand-alone kernel);
 //    nibbles split into even / odd codes feed dp4a against xq permuted the same
 //    way; the two halves of a group (lanes 2m, 2m + 1) add by one shuffle;
 //  * even lanes fold s * acc, odd lanes o * xsum, in fp64; a fixed-order
@@ -55,9 +55,9 @@ struct Gemv1Layout {
     w = off;    off += (size_t)kRows * KB;           // packed rows, contiguous
     s16 = off;  off += (size_t)kRows * G * 2 * 2;    // fp16 scales [row][g], then offsets
     so = off;   off += (size_t)kRows * G * 16;       // {s, o} in fp64 [row][g]
-    xq = off;   off += (size_t)K;                    // activation codes, even / odd permuted
-    xs = off;   off += (size_t)G * 8;                // group sums in fp64
-    amx = off;  off += kWarps * 4;                   // per-warp absmax
+    xq = off;   off += (size_t)K;                    // codes (in-kernel quantization only)
+    xs = off;   off += (size_t)G * 8;                // group sums in fp64 (ditto)
+    amx = off;  off += kWarps * 4;                   // per-warp absmax (ditto)
     bias = off; off += kRows * 4;
     off = (off + 15) & ~size_t(15);
     bars = off; off += (kWarps + 1) * 8;             // one per warp's rows, one for the scales
@@ -163,12 +163,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       so_sm[i] = make_double2(h2d(s16[i]), h2d(o16[i]));
   }
 
-  // ---- activations (they come from the previous kernel)
+  // ---- activations (they come from the previous kernel).  Lane l owns chunks
+  // c = l + 32 j, i.e. codes 32 c .. 32 c + 31, of group 16 j + l / 2, and
+  // keeps their codes in registers.  Quantized activations are read by every
+  // warp straight from global memory (no warp waits on another); bf16 x is
+  // quantized by the whole CTA (one absmax) through shared memory.
   pdl_wait();
   if (!early_trigger) pdl_launch_dependents();
+  uint32_t xr[NJ][8];  // codes, even / odd permuted per 8 (the nibble-split order)
+  double xsj[NJ];      // xsum of the lane's group of chunk j
   float sxv = 1.0f;
   if constexpr (kQuantX) {
-    const int nch = K >> 3;  // 16-byte chunks of x
+    // cooperative: every thread quantizes two 16-byte chunks of x (absmax by a
+    // block reduction), the codes go to shared memory in the even / odd order,
+    // then each lane picks up its own
+    const int nch = K >> 3;
     const uint4* src = reinterpret_cast<const uint4*>(x);
     uint4 v[2];
     uint32_t mb = 0u;
@@ -203,31 +212,29 @@ __global__ void __launch_bounds__(kThreads, 2)
       sum = group8_sum(sum);
       if ((lane & 7) == 0 && c < nch) xs_sm[c >> 3] = i32_to_f64(sum);
     }
-  } else {
-    for (int c = threadIdx.x; c < (K >> 4); c += kThreads) {
-      const uint4 q = __ldg(reinterpret_cast<const uint4*>(xq) + c);
-      const uint2 a = even_odd(q.x, q.y), b = even_odd(q.z, q.w);
-      *reinterpret_cast<uint4*>(xq_sm + 16 * c) = make_uint4(a.x, a.y, b.x, b.y);
-    }
-    if (!kDump) {
-      for (int g = threadIdx.x; g < G; g += kThreads) xs_sm[g] = i32_to_f64(__ldg(xsum + g));
-      sxv = __ldg(sx);
-    }
-  }
-  __syncthreads();
-
-  // ---- lane l: chunks c = l + 32 j of every row = codes 32 c .. 32 c + 31,
-  // group 16 j + l / 2; its activation codes stay in registers
-  uint32_t xr[NJ][8];
-  double xsj[NJ];
+    __syncthreads();
 #pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const uint4* p = reinterpret_cast<const uint4*>(xq_sm + 32 * (lane + 32 * j));
-    const uint4 a = p[0], b = p[1];
-    xr[j][0] = a.x; xr[j][1] = a.y; xr[j][2] = a.z; xr[j][3] = a.w;
-    xr[j][4] = b.x; xr[j][5] = b.y; xr[j][6] = b.z; xr[j][7] = b.w;
-    xsj[j] = kDump ? 0.0 : xs_sm[16 * j + (lane >> 1)];
+    for (int j = 0; j < NJ; ++j) {
+      const uint4* p = reinterpret_cast<const uint4*>(xq_sm + 32 * (lane + 32 * j));
+      const uint4 a = p[0], b = p[1];
+      xr[j][0] = a.x; xr[j][1] = a.y; xr[j][2] = a.z; xr[j][3] = a.w;
+      xr[j][4] = b.x; xr[j][5] = b.y; xr[j][6] = b.z; xr[j][7] = b.w;
+      xsj[j] = xs_sm[16 * j + (lane >> 1)];
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const uint4* p = reinterpret_cast<const uint4*>(xq) + 2 * (lane + 32 * j);
+      const uint4 a = __ldg(p), b = __ldg(p + 1);
+      const uint2 e0 = even_odd(a.x, a.y), e1 = even_odd(a.z, a.w);
+      const uint2 e2 = even_odd(b.x, b.y), e3 = even_odd(b.z, b.w);
+      xr[j][0] = e0.x; xr[j][1] = e0.y; xr[j][2] = e1.x; xr[j][3] = e1.y;
+      xr[j][4] = e2.x; xr[j][5] = e2.y; xr[j][6] = e3.x; xr[j][7] = e3.y;
+      xsj[j] = kDump ? 0.0 : i32_to_f64(__ldg(xsum + 16 * j + (lane >> 1)));
+    }
+    if (!kDump) sxv = __ldg(sx);
   }
+
   // A warp's four rows are all valid or all past N (rows is a multiple of 8),
   // so they run as one straight-line block and their chains interleave.
   const int r0 = warp * kRowsPerWarp;
