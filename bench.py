@@ -325,11 +325,22 @@ def run_ours(args, world, rank, local):
         # weight-streaming GEMV: bound by HBM; algorithmic bytes per launch
         G = K // 64
         kbytes = N * K / 2 + 4 * N * G + M * K + 4 * M + 4 * M * G + 2 * M * N
-        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc", "gemv_w4a8.cu")
+        # one token with K a multiple of 1024 (up to 4096) runs the dp4a kernel
+        one = M == 1 and K % 1024 == 0 and K <= 4096
+        tag = "w4a8_gemv1_kernel" if one else "w4a8_gemv_kernel"
+        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc",
+                           "gemv1_w4a8.cu" if one else "gemv_w4a8.cu")
         roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
-                "kernel": "w4a8_gemv_kernel",
-                "traffic": traffic_from_profile("w4a8_gemv_kernel", src)}
+                "kernel": tag, "traffic": traffic_from_profile(tag, src)}
+    elif not w4 and N <= 64 and M <= 8192:
+        # thin W8A8 outputs run the split-K cluster kernel, bound by reading xq
+        kbytes = M * K + N * K + 2 * M * N + 4 * (M + 2 * N)
+        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc", "gemm_w8a8_skinny.cu")
+        roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
+                "kernel": "w8a8_skinny_kernel",
+                "traffic": traffic_from_profile("w8a8_skinny_kernel", src)}
     else:
         peak = peaks["bf16"] * 2.0
         src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc",
