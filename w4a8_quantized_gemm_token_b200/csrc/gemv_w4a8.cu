@@ -14,18 +14,18 @@
 // CTAs are already resident with their weights in flight.
 //  * A cluster of C CTAs shares R weight rows; CTA c takes the groups of one
 //    K slice [c GC, (c + 1) GC).  The host picks (R, C) so that every warp
-//    holds at most 16 groups of its two weight rows per lane, two CTAs fit an
-//    SM (this call's and the next one's) and the grid is at most one CTA per
-//    SM.
-//  * Register-resident weights: at kernel start, before the programmatic-
-//    dependency wait, every lane issues the 8-byte loads of its packed codes
-//    (per group: 8 bytes of each of its two rows) straight into registers,
-//    and one thread bulk-copies the CTA's fp16 scales / offsets into shared
-//    memory; the bias of the CTA's rows is read too.  Weights, scales,
-//    offsets and bias are therefore read before the previous kernel in the
-//    stream has finished: they must not be written by a kernel that triggers
-//    its dependents early (no kernel of this library that writes weights
-//    does).
+//    covers at most 16 groups, two CTAs fit an SM (this call's and the next
+//    one's) and the grid is at most one CTA per SM.
+//  * At kernel start, before the programmatic-dependency wait, one thread
+//    issues 2-D TMA copies of the CTA's packed codes (boxes of R rows x 128
+//    bytes, 128-byte swizzled so the fragment reads are conflict-free) and
+//    bulk / TMA copies of its fp16 scales / offsets; the bias of the CTA's rows
+//    is read too.  (An earlier form loaded the codes into registers with
+//    per-lane loads: the flood of loads then delayed the co-resident CTA's
+//    latency-critical activation loads.)  Weights, scales, offsets and bias
+//    are therefore read before the previous kernel in the stream has
+//    finished: they must not be written by a kernel that triggers its
+//    dependents early (no kernel of this library that writes weights does).
 //  * After the wait the CTA either quantizes its K slice of bf16 x itself
 //    (the rule of the stand-alone quantization kernel; with C > 1 the per-row
 //    absmax is exchanged through distributed shared memory) or reads
@@ -66,14 +66,14 @@ constexpr int kSmemTwoPerSm = 113 * 1024;
 // x per thread in registers (M * KC <= kQuantChunks * 8 * kThreads = 16384,
 // KC = the K slice of one CTA).
 constexpr int kQuantChunks = 8;
-// Groups of 64 codes one warp holds in registers (two rows, 8 bytes each).
+// Groups of 64 codes one warp covers (straight-line code over all of them).
 constexpr int kWarpGroups = 16;
 
 // Shared-memory layout of one CTA: R weight rows, cluster of C CTAs along K,
 // M token rows.
 struct GemvLayout {
-  int R, C, M, G, GC, RT, KW, GW, RO, Mp, XS;
-  size_t s16, xq, xs, sx, amx, bias, part, bars, total;
+  int R, C, M, G, GC, RT, KW, GW, RO, Mp, XS, nbox;
+  size_t w, s16, xq, xs, sx, amx, bias, part, bars, total;
   __host__ __device__ GemvLayout(int R_, int C_, int K, int M_) {
     R = R_;
     C = C_;
@@ -88,18 +88,21 @@ struct GemvLayout {
     // xq row stride = 64 (mod 128): the two token rows of one 16-byte load
     // phase fall in opposite halves of the banks
     XS = (GC * 64 + 127) / 128 * 128 + 64;
+    nbox = (GC + 3) / 4;       // 128-byte weight boxes per row of the slice
     size_t off = 0;
+    w = off;    off += (size_t)nbox * R * 128;        // packed codes, 128-byte-swizzled boxes
     s16 = off;  off += (size_t)R * GC * 2 * 2;        // fp16 scales [R][GC], then offsets
     off = (off + 127) & ~size_t(127);
     xq = off;   off += (size_t)M * XS;                // xq rows of the slice (permuted)
     off = (off + 15) & ~size_t(15);
     xs = off;   off += (size_t)Mp * (GC + 1) * 8;     // xsum as fp64, zero past M
     sx = off;   off += 16 * 4;                        // sx
-    amx = off;  off += (size_t)(C + 1) * 16 * 4;      // absmax: [C] exchange slots, local
+    amx = off;  off += (size_t)(C + 1) * 16 * 4 + 256 * 4 + 16 * 4;  // absmax: [C] exchange slots,
+                                                      // local; group maxima; row multipliers
     bias = off; off += (size_t)RO * 4;                // bias of the rows this CTA finalizes
     off = (off + 15) & ~size_t(15);
     part = off; off += (size_t)C * KW * M * RO * 8;   // fp64 partials [slot][token][row]
-    bars = off; off += 8;                             // mbarrier of the scales
+    bars = off; off += (size_t)(nbox + 1) * 8;        // mbarriers: the boxes, the scales
     total = off + 1024;                               // base alignment slack
   }
 };
@@ -166,14 +169,6 @@ __device__ __forceinline__ uint2 even_odd(uint32_t lo, uint32_t hi) {
   return make_uint2(__byte_perm(lo, hi, 0x6420), __byte_perm(lo, hi, 0x7531));
 }
 
-// 8-byte load of read-only data that is used once (no L1 allocation).
-__device__ __forceinline__ uint2 ldg_stream_v2(const uint8_t* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
-  return v;
-}
 
 // TT token tiles of 8 (M <= 8 TT).  kFold: the product y; otherwise the
 // per-group int32 sums of rows [m0, m1) go to acc_out.  kQuantX: the
@@ -182,7 +177,8 @@ __device__ __forceinline__ uint2 ldg_stream_v2(const uint8_t* p) {
 // Grid (C, ceil(N / R)), cluster (C, 1, 1).
 template <int TT, bool kFold, bool kQuantX, bool kOne, int C>
 __global__ void __launch_bounds__(kThreads, 2)
-    w4a8_gemv_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmO,
+    w4a8_gemv_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
+                     const __grid_constant__ CUtensorMap tmO,
                      const uint16_t* __restrict__ x, const int8_t* __restrict__ xq,
                      const float* __restrict__ sx, const int32_t* __restrict__ xsum, int M, int K,
                      const uint8_t* __restrict__ Wp, const uint16_t* __restrict__ wscale,
@@ -207,7 +203,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   unsigned int* amx_sm = reinterpret_cast<unsigned int*>(smem + L.amx);  // [C][16], local [16]
   float* bias_sm = reinterpret_cast<float*>(smem + L.bias);
   double* part = reinterpret_cast<double*>(smem + L.part);
-  const uint32_t sbar = smem_u32(smem + L.bars);
+  const uint8_t* w_sm = smem + L.w;
+  const uint32_t wbar0 = smem_u32(smem + L.bars);      // box j: wbar0 + 8 j
+  const uint32_t sbar = wbar0 + 8u * (uint32_t)L.nbox;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rt = warp % RT, kw = warp / RT;
   const int grp = lane >> 2, tq = lane & 3;
@@ -219,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ---- before the dependency wait: scales / offsets by bulk copy, the
   // packed codes of this lane's two rows into registers, the bias.
   if (threadIdx.x == 0) {
-    mbar_init(sbar, 1);
+    prefetch_tmap(&tmW);
+    for (int q = 0; q <= L.nbox; ++q) mbar_init(wbar0 + 8u * q, 1);
     fence_mbar_init();
     if (kFold) {
       if (C > 1) {
@@ -234,22 +233,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
-  // Lane (grp, tq) of group g uses the 8 packed bytes 32 g + 8 tq .. + 7 of
-  // rows ra and ra + 8 (rows past N read row N - 1; their results are dropped).
-  uint2 wr[kWarpGroups][2];
-  {
-    const size_t rb = (size_t)(K / 2);
-    const uint8_t* pa = Wp + (size_t)min(n0 + ra, N - 1) * rb + (size_t)(g0 + gbeg) * 32 + 8 * tq;
-    const uint8_t* pb = Wp + (size_t)min(n0 + ra + 8, N - 1) * rb + (size_t)(g0 + gbeg) * 32 + 8 * tq;
-#pragma unroll
-    for (int i = 0; i < kWarpGroups; ++i) {
-      if (i < gn) {
-        wr[i][0] = ldg_stream_v2(pa + 32 * i);
-        wr[i][1] = ldg_stream_v2(pb + 32 * i);
-      } else {
-        wr[i][0] = make_uint2(0u, 0u);
-        wr[i][1] = make_uint2(0u, 0u);
-      }
+  // the packed codes: boxes of R rows x 128 bytes (four groups), 128-byte
+  // swizzled, in K order; rows past N and bytes past K/2 are zero-filled
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < L.nbox; ++j) {
+      mbar_arrive_expect_tx(wbar0 + 8u * j, (uint32_t)(R * 128));
+      tma_load_2d(smem_u32(w_sm + (size_t)j * R * 128), &tmW, 32 * g0 + 128 * j, n0, wbar0 + 8u * j);
     }
   }
   if (kFold && threadIdx.x < RO && crank * RO + (int)threadIdx.x < rows)
@@ -282,6 +271,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     unsigned int* amx_local = amx_sm + C * 16;
+    unsigned int* gmax_sm = amx_sm + (C + 1) * 16;                    // [M][GC] group maxima
+    float* rmul_sm = reinterpret_cast<float*>(gmax_sm + 256);          // [16] row multipliers
+    // Group maxima: the 8 chunks of a group sit in 8 consecutive lanes of one
+    // row (nch % 8 == 0), so three shuffles and one plain store per group.
 #pragma unroll
     for (int i = 0; i < kQuantChunks; ++i) {
       if (kThreads * i >= total) break;  // warp-uniform
@@ -290,12 +283,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       mb = bf16x2_absmax_bits(mb, v[i].y);
       mb = bf16x2_absmax_bits(mb, v[i].z);
       mb = bf16x2_absmax_bits(mb, v[i].w);
-      const uint32_t m16 = max(mb & 0xFFFFu, mb >> 16);
-      const int m = c < total ? c / nch : -1;
-      // one shared-memory atomic per row present in the warp
-      const unsigned same = __match_any_sync(0xFFFFFFFFu, m);
-      const unsigned red = __reduce_max_sync(same, m16);
-      if (m >= 0 && lane == __ffs(same) - 1) atomicMax(amx_local + m, red);
+      uint32_t m16 = max(mb & 0xFFFFu, mb >> 16);
+      m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, 1));
+      m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, 2));
+      m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, 4));
+      if ((lane & 7) == 0 && c < total) gmax_sm[c >> 3] = m16;  // index m * GC + g
+    }
+    __syncthreads();
+    // row maxima over this slice: warp w takes rows w and w + 8
+    for (int m = warp; m < M; m += kWarps) {
+      uint32_t mr = 0u;
+      for (int g = lane; g < GC; g += 32) mr = max(mr, gmax_sm[m * GC + g]);
+      mr = __reduce_max_sync(0xFFFFFFFFu, mr);
+      if (lane == 0) amx_local[m] = mr;
     }
     __syncthreads();
     if (C > 1) {
@@ -310,15 +310,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       cluster_arrive_release();
       cluster_wait_acquire();
     }
-    auto row_amax = [&](int m) -> float {
-      unsigned int b = amx_local[m];
+    // the row's absmax over the whole K, its multiplier and scale (one
+    // division each per row)
+    if (threadIdx.x < M) {
+      unsigned int b = amx_local[threadIdx.x];
       if (C > 1) {
-        b = amx_sm[m];
+        b = amx_sm[threadIdx.x];
 #pragma unroll
-        for (int q = 1; q < C; ++q) b = max(b, amx_sm[q * 16 + m]);
+        for (int q = 1; q < C; ++q) b = max(b, amx_sm[q * 16 + threadIdx.x]);
       }
-      return __uint_as_float(b << 16);
-    };
+      const float amax = __uint_as_float(b << 16);
+      rmul_sm[threadIdx.x] = act_multiplier(amax);
+      sx_sm[threadIdx.x] = act_scale(amax);
+    }
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < kQuantChunks; ++i) {
       if (kThreads * i >= total) break;  // warp-uniform
@@ -327,20 +332,29 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (c < total) {
         m = c / nch;
         cc = c - m * nch;
-        const uint2 qc = quant_chunk(v[i], act_multiplier(row_amax(m)), &sum);
+        const uint2 qc = quant_chunk(v[i], rmul_sm[m], &sum);
         *reinterpret_cast<uint2*>(xq_sm + (size_t)m * XS + 8 * cc) = even_odd(qc.x, qc.y);
       }
       // the 8 chunks of a group sit in 8 consecutive lanes (nch % 8 == 0)
       sum = group8_sum(sum);
       if ((lane & 7) == 0 && c < total) xs_sm[m * (GC + 1) + (cc >> 3)] = i32_to_f64(sum);
     }
-    if (threadIdx.x < M) sx_sm[threadIdx.x] = act_scale(row_amax(threadIdx.x));
     __syncthreads();
   } else {
-    // quantized activations: the slice of xq, byte-permuted on the way in
-    // (batches of 8 independent loads per thread before any store)
+    // quantized activations: the slice of xq, byte-permuted on the way in.
+    // Every global load of this stage (the group sums and sx too) is issued
+    // before any is used: one round trip to L2 instead of several.
     const int nc16 = GC * 4;  // 16-byte chunks per row of the slice
     const int total = M * nc16;
+    constexpr int kXs = 8;    // group sums per thread (M * GC <= 16 * 128 = 2048)
+    int xsv[kXs];
+#pragma unroll
+    for (int i = 0; i < kXs; ++i) {
+      const int idx = threadIdx.x + kThreads * i;
+      const int m = idx / GC, g = idx - (idx / GC) * GC;
+      xsv[i] = (kFold && idx < M * GC && g < gcount) ? __ldg(xsum + (size_t)m * G + g0 + g) : 0;
+    }
+    const float sxl = (kFold && (int)threadIdx.x < M) ? __ldg(sx + threadIdx.x) : 0.0f;
     for (int base = 0; base < total; base += 8 * kThreads) {
       uint4 v[8];
 #pragma unroll
@@ -364,11 +378,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     if (kFold) {
-      for (int idx = threadIdx.x; idx < M * GC; idx += kThreads) {
-        const int m = idx / GC, g = idx - m * GC;
-        xs_sm[m * (GC + 1) + g] = g < gcount ? i32_to_f64(__ldg(xsum + (size_t)m * G + g0 + g)) : 0.0;
+#pragma unroll
+      for (int i = 0; i < kXs; ++i) {
+        const int idx = threadIdx.x + kThreads * i;
+        if (idx < M * GC) xs_sm[(idx / GC) * (GC + 1) + idx % GC] = i32_to_f64(xsv[i]);
       }
-      if (threadIdx.x < M) sx_sm[threadIdx.x] = __ldg(sx + threadIdx.x);
+      if ((int)threadIdx.x < M) sx_sm[threadIdx.x] = sxl;
     }
     __syncthreads();
     if (C > 1) cluster_wait_acquire();  // the start barrier
@@ -389,8 +404,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int i = 0; i < 4; ++i) f[tt][i] = 0.0;
   double fa = 0.0, fb = 0.0;  // one token: rows ra, ra + 8
-  // (if the scales never land the results are wrong and the error word is set)
+  // (if the scales or a box never land the results are wrong and the error
+  // word is set)
   if (kFold) __all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, err));
+  if (gn > 0)
+    for (int j = gbeg / 4; j <= (gbeg + gn - 1) / 4; ++j)
+      __all_sync(0xFFFFFFFFu, mbar_wait(wbar0 + 8u * j, 0, err));
+  // Packed byte p of row r sits in box p / 128, 16-byte chunk
+  // ((p % 128) / 16) ^ (r % 8), and r % 8 == grp for both rows of the lane.
+  const uint32_t offa = (uint32_t)(ra * 128 + 8 * (tq & 1));
+  const uint32_t offb = offa + 8u * 128u;
 
   // K map.  For group g, lane (grp, tq) handles the 16 consecutive codes
   // k = 64 g + 16 tq + 0..15 (8 packed bytes).  Splitting a packed word into
@@ -401,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   //
   // All kWarpGroups groups in straight-line code (no branch between them, so
   // the loads, MMAs and folds of different groups overlap); groups past gn
-  // hold zero codes (see wr) and their results are dropped.
+  // re-read the last group and their results are dropped.
 #pragma unroll
   for (int blk = 0; blk < kWarpGroups / 4; ++blk) {
     int A0[4], A2[4];                 // one token: the block's group sums
@@ -409,7 +432,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int u = 0; u < 4; ++u) {
       const int i = 4 * blk + u;
       const int gl = gbeg + min(i, gn - 1);  // group within the slice (clamped)
-      const uint2 wa = wr[i][0], wb = wr[i][1];
+      const uint8_t* box = w_sm + (size_t)(gl >> 2) * R * 128;
+      const uint32_t sw = (uint32_t)(((2 * (gl & 3) + (tq >> 1)) ^ grp) << 4);
+      const uint2 wa = *reinterpret_cast<const uint2*>(box + offa + sw);
+      const uint2 wb = *reinterpret_cast<const uint2*>(box + offb + sw);
       // A registers: {row grp, row grp + 8} x {even codes, odd codes}, per MMA
       const uint32_t a0[4] = {wa.x & 0x0F0F0F0Fu, wb.x & 0x0F0F0F0Fu, (wa.x >> 4) & 0x0F0F0F0Fu,
                               (wb.x >> 4) & 0x0F0F0F0Fu};
@@ -537,8 +563,7 @@ struct GemvPlan {
   size_t smem = 0;
 };
 
-// Picks (R, C) for M <= 16.  A warp holds at most kWarpGroups groups of its
-// rows in registers.  In order of preference: a CTA fits two per SM (the
+// Picks (R, C) for M <= 16.  A warp covers at most kWarpGroups groups.  In order of preference: a CTA fits two per SM (the
 // next call's CTAs can be resident while this call computes); the grid fits
 // one wave; at most 16 KB of activations per CTA (they are read after the
 // dependency wait, on the critical path); the most CTAs (the most SMs
@@ -629,7 +654,10 @@ cudaError_t launch_gemv(const uint16_t* x, const int8_t* xq, const float* sx,
   // scales / offsets [N, G] fp16 as 2-D boxes of GC groups x R rows (C > 1;
   // one CTA's block is then strided); with C == 1 it is contiguous and goes by
   // bulk copy, and the maps are unused
-  CUtensorMap tS = {}, tO = {};
+  CUtensorMap tW, tS = {}, tO = {};
+  if (!encode_tmap_2d(&tW, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wp, (uint64_t)(K / 2), (uint64_t)N,
+                      (uint64_t)(K / 2), 128, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   if (p.C > 1 && fold) {
     if (!encode_tmap_2d(&tS, CU_TENSOR_MAP_DATA_TYPE_UINT16, ws, (uint64_t)G, (uint64_t)N,
                         (uint64_t)G * 2, (uint32_t)GC, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE) ||
@@ -670,7 +698,7 @@ cudaError_t launch_gemv(const uint16_t* x, const int8_t* xq, const float* sx,
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kernel, tS, tO, x, xq, sx, xsum, (int)M, (int)K, Wp, ws, wo,
+  return cudaLaunchKernelEx(&cfg, kernel, tW, tS, tO, x, xq, sx, xsum, (int)M, (int)K, Wp, ws, wo,
                             bias, (int)N, y, acc_out, (int)m0, (int)m1, p.R, 0, err);
 }
 
