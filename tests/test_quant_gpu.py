@@ -13,7 +13,7 @@ from w4a8_quantized_gemm_token_b200 import synthetic
 pytestmark = pytest.mark.gpu
 
 MS = [1, 2, 3, 15, 16, 17, 63, 64, 65, 129]
-KS = [32, 64, 96, 160, 3072, 4096, 5120, 12288]
+KS = [32, 64, 96, 160, 3072, 4096, 5120, 6144, 8192, 12288]
 
 
 @pytest.mark.parametrize("K", KS)

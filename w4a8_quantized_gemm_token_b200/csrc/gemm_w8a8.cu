@@ -30,7 +30,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <cstdlib>
 
 #include "qk_internal.h"
 #include "sm100.cuh"
@@ -432,7 +431,6 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   // A raster group's rows of xq (256 rows x K bytes per M tile) should stay in
   // L2 while the group sweeps all of Wq: about 40 MB of the 126 MB L2.
   long long group_m = (40ll << 20) / (2 * BM * K);
-  if (const char* env = std::getenv("QK_GROUP_M")) group_m = std::atoll(env);
   group_m = group_m < 1 ? 1 : (group_m > tiles_m ? tiles_m : group_m);
   const long long pairs = num_sms() / 2;
   const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);

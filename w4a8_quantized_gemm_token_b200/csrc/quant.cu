@@ -196,6 +196,9 @@ cudaError_t launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq
                 : per_lane <= 8  ? quant_act_kernel<8>
                 : per_lane <= 12 ? quant_act_kernel<12>
                 : per_lane <= 16 ? quant_act_kernel<16>
+                : per_lane <= 20 ? quant_act_kernel<20>
+                : per_lane <= 24 ? quant_act_kernel<24>
+                : per_lane <= 32 ? quant_act_kernel<32>
                                  : quant_act_kernel<0>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((M + kQuantWarps - 1) / kQuantWarps));
