@@ -52,6 +52,7 @@ def _bind(path: str):
         "oracle_w8a8_acc": (None, [P, I64, I64, P, I64, P]),
         "oracle_w4a8_group_acc": (None, [P, I64, I64, P, I64, P]),
         "oracle_w8a8_dequant": (None, [P, I64, I64, P, P, P, P]),
+        "oracle_w8a8_gated": (None, [P, I64, I64, P, P, P, P, P, P]),
         "oracle_w4a8_dequant": (None, [P, P, I64, I64, I64, P, P, P, P, P]),
         "oracle_w8a8_dequant_f64": (None, [P, I64, I64, P, P, P, P]),
         "oracle_w4a8_dequant_f64": (None, [P, P, I64, I64, I64, P, P, P, P, P]),
@@ -201,6 +202,21 @@ def w8a8_dequant(acc, sx, sw, bias=None) -> np.ndarray:
     return y
 
 
+def w8a8_gated(acc, sx, sw, bias, gate, r_bf16) -> np.ndarray:
+    """bf16 bits [M, N] of r + gate * (acc * sx * sw + bias) in fp64, rounded once."""
+    acc = _c(acc, np.int64)
+    M, N = acc.shape
+    sx = _c(sx, np.float32)
+    sw = _c(sw, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    g = _c(gate, np.float32)
+    r = _c(r_bf16, np.uint16)
+    assert g.shape == (N,) and r.shape == (M, N)
+    out = np.empty((M, N), np.uint16)
+    _load().oracle_w8a8_gated(_p(acc), M, N, _p(sx), _p(sw), _p(b), _p(g), _p(r), _p(out))
+    return out
+
+
 def w8a8_dequant_f64(acc, sx, sw, bias=None) -> np.ndarray:
     """fp64 value [M, N] of acc * sx * sw + bias, before the bf16 rounding."""
     acc = _c(acc, np.int64)
@@ -250,6 +266,13 @@ def w8a8_linear(x_bf16, Wq, sw, bias=None):
     xq, sx = quant_act(x_bf16)
     acc = w8a8_acc(xq, Wq)
     return w8a8_dequant(acc, sx, sw, bias), xq, sx, acc
+
+
+def w8a8_linear_gated(x_bf16, Wq, sw, bias, gate, r_bf16):
+    """The W8A8 linear with the gated residual epilogue: (out bf16 bits, xq, sx, acc)."""
+    xq, sx = quant_act(x_bf16)
+    acc = w8a8_acc(xq, Wq)
+    return w8a8_gated(acc, sx, sw, bias, gate, r_bf16), xq, sx, acc
 
 
 def w4a8_linear(x_bf16, Wp, s16, o16, bias=None):

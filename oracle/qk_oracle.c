@@ -23,6 +23,8 @@
  *   [mlx4722] "MLX PR #4722" (int8-staged quantized matmul), "Selector rules":
  *          affine-quantized weights, group size 64, K % 64 == 0; the
  *          "SIMD fix" bullet: x is quantized to int8 by its own kernel.
+ *   [kquant89] "mlx-kquant PR #89", commit list: a quantized matmul with a
+ *          gated residual epilogue, each element held within 2 ulp.
  *
  * Readings taken where the pages are silent (each is stated where it is used):
  *   R1  codes are rne(x * r) with r = 127 / absmax (one fp32 division per row,
@@ -36,6 +38,9 @@
  *   R6  packing: code k = 2j in the low nibble of byte j, k = 2j + 1 in the high.
  *   R7  W4A8 keeps an exact int32 partial sum per group of 64 and folds the
  *       groups with the scale/offset afterwards.
+ *   R13 the gated residual epilogue is out = r + g[n] * (linear output before
+ *       rounding), r a bf16 [M, N] residual, g one fp32 gate per output channel
+ *       (one sample's adaLN gate of a DiT block).
  *   dequant is evaluated in fp64 and rounded once to bf16 (nearest, ties even).
  */
 #include <stdint.h>
@@ -307,6 +312,28 @@ void oracle_w8a8_dequant(const int64_t *acc, int64_t M, int64_t N,
             y[m * N + n] = oracle_f64_to_bf16(v);
         }
     }
+}
+
+/*
+ * W8A8 with the gated residual epilogue [kquant89], (R13):
+ *   out = r[m,n] + g[n] * (acc * sx[m] * sw[n] + bias[n])
+ * in fp64 with no fused multiply-add (the bracket exactly as
+ * oracle_w8a8_dequant_f64 evaluates it), rounded once to bf16.
+ * r bf16 [M, N], g fp32 [N], bias may be NULL; out bf16 [M, N].
+ */
+void oracle_w8a8_gated(const int64_t *acc, int64_t M, int64_t N,
+                       const float *sx, const float *sw, const float *bias,
+                       const float *gate, const uint16_t *r, uint16_t *out)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double v;
+            oracle_w8a8_dequant_f64(acc + m * N + n, 1, 1, sx + m, sw + n,
+                                    bias ? bias + n : NULL, &v);
+            double t = (double)gate[n] * v;
+            t = t + (double)oracle_bf16_to_f32(r[m * N + n]);
+            out[m * N + n] = oracle_f64_to_bf16(t);
+        }
 }
 
 /*

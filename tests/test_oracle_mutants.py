@@ -28,6 +28,9 @@ MUTANTS = [
     ("w4_sx_dropped", "double r = (double)sx[m] * f;", "double r = f;"),
     ("bf16_truncates", "r = (fmod(units, 2.0) == 0.0) ? lo : hi;", "r = lo;"),
     ("bf16_nearest_up", "if (dlo < dhi)\n        r = lo;", "if (dlo < dhi * 0.5)\n        r = lo;"),
+    ("gated_residual_dropped", "t = t + (double)oracle_bf16_to_f32(r[m * N + n]);", "t = t;"),
+    ("gated_gate_skips_bias", "double t = (double)gate[n] * v;",
+     "double t = (double)gate[n] * (v - (bias ? (double)bias[n] : 0.0)) + (bias ? (double)bias[n] : 0.0);"),
     ("group_sum_window", "for (int64_t k = 64 * g; k < 64 * g + 64; ++k)\n                s += xq[m * K + k];",
      "for (int64_t k = 64 * g; k < 64 * g + 63; ++k)\n                s += xq[m * K + k];"),
 ]

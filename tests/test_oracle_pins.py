@@ -368,3 +368,66 @@ def test_w4a8_within_quantization_bound_of_exact(orc):
     assert np.all(np.abs(yv - exact) <= bound + np.abs(yv) * 2.0 ** -8 + 1e-30)
     rms = lambda a: float(np.sqrt(np.mean(a * a)))
     assert rms(yv - exact) < 0.1 * rms(exact)
+
+
+# ----------------------------------------------- gated residual epilogue
+
+def test_w8a8_gated_integer_closed_form(orc):
+    """Integer x and W with row absmax 127 (sx = sw = 1), an integer bias and
+    residual and power-of-two gates: out = bf16(r + g * (x @ W^T + bias)),
+    computed here in numpy int64 / float32 (exact: every value is a multiple of
+    1/4 below 2^22) and rounded by torch."""
+    import torch
+
+    rng = np.random.default_rng(12)
+    M, K, N = 13, 64, 24
+    x = rng.integers(-127, 128, size=(M, K)).astype(np.float32)
+    x[:, 3] = -127
+    W = rng.integers(-127, 128, size=(N, K)).astype(np.float32)
+    W[:, 5] = 127
+    bias = rng.integers(-1000, 1000, size=N).astype(np.float32)
+    gate = rng.choice(np.array([0.25, -0.5, 1.0, 2.0, -4.0], np.float32), size=N)
+    r = rng.integers(-200, 200, size=(M, N)).astype(np.float32)  # exact in bf16
+    Wq, sw = orc.quant_w8(W)
+    out, xq, sx, acc = orc.w8a8_linear_gated(bf16_bits(x), Wq, sw, bias, gate, bf16_bits(r))
+    exact = x.astype(np.int64) @ W.astype(np.int64).T + bias.astype(np.int64)
+    want_f = (r.astype(np.float64) + gate.astype(np.float64) * exact).astype(np.float32)
+    want = torch.from_numpy(want_f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(out, want)
+
+
+def test_w8a8_gated_zero_gate_and_unit_gate(orc):
+    """A zero gate returns the residual bit for bit; a unit gate with a zero
+    residual returns the plain linear (whose own pins are above)."""
+    case = synthetic.LinearCase("gz", M=7, K=160, N=16, outlier_frac=0.05, seed=13)
+    xb, W, b, _ = case.draw()
+    Wq, sw = orc.quant_w8(W)
+    rng = np.random.default_rng(14)
+    r = bf16_bits(rng.normal(size=(7, 16)).astype(np.float32) * 3)
+    out0, _, _, _ = orc.w8a8_linear_gated(xb, Wq, sw, b, np.zeros(16, np.float32), r)
+    assert np.array_equal(out0, r)
+    out1, _, _, _ = orc.w8a8_linear_gated(xb, Wq, sw, b, np.ones(16, np.float32),
+                                          np.zeros((7, 16), np.uint16))
+    y, _, _, _ = orc.w8a8_linear(xb, Wq, sw, b)
+    assert np.array_equal(out1, y)
+
+
+def test_w8a8_gated_brute_force(orc):
+    """r + g * (sum_k (xq*sx)(wq*sw) + bias), term by term in fp64 and rounded by
+    the (separately pinned) fp64 -> bf16 rounding, agrees with the oracle to
+    within one bf16 ulp (equal unless the two fp64 evaluation orders straddle a
+    rounding boundary)."""
+    case = synthetic.LinearCase("gb", M=9, K=96, N=11, outlier_frac=0.03, seed=15)
+    xb, W, b, _ = case.draw()
+    Wq, sw = orc.quant_w8(W)
+    rng = np.random.default_rng(16)
+    gate = (rng.normal(size=11) * 0.5).astype(np.float32)
+    r = bf16_bits(rng.normal(size=(9, 11)).astype(np.float32))
+    out, xq, sx, _ = orc.w8a8_linear_gated(xb, Wq, sw, b, gate, r)
+    xd = xq.astype(np.float64) * sx.astype(np.float64)[:, None]
+    wd = Wq.astype(np.float64) * sw.astype(np.float64)[:, None]
+    lin = (xd[:, None, :] * wd[None, :, :]).sum(axis=2) + b.astype(np.float64)
+    brute = bf16_val(r).astype(np.float64) + gate.astype(np.float64) * lin
+    want = orc.f64_to_bf16_array(brute)
+    assert np.abs(ordinal(out) - ordinal(want)).max() <= 1
+    assert np.mean(out == want) > 0.95
