@@ -168,6 +168,27 @@ qk_status qk_w8a8_linear(const uint16_t *x, int64_t M, int64_t K,
                          qk_stream_t stream);
 
 /*
+ * The W8A8 linear with a gated residual epilogue ("mlx-kquant PR #89", commit
+ * list: a quantized matmul with a gated residual epilogue, each element held
+ * within 2 ulp), the update of a DiT block's residual stream:
+ *   y[m, n] = bf16( residual[m, n] + gate[n] * (acc[m, n] * sx[m] * sw[n] + bias[n]) )
+ * evaluated in fp64 and rounded once to bf16 (nearest even); the bracket is
+ * the value qk_w8a8_linear rounds.
+ *   x, Wq, sw, bias, workspace : as for qk_w8a8_linear
+ *   gate      : fp32 [N], one gate per output channel (in)
+ *   residual  : bf16 bits [M, N] (in); y may be the residual itself (an
+ *               in-place update: each element is read before it is written)
+ *   y         : bf16 bits [M, N]   (out)
+ * Errors as for qk_w8a8_linear; gate and residual must be non-NULL and
+ * 16-byte aligned.
+ */
+qk_status qk_w8a8_linear_gated(const uint16_t *x, int64_t M, int64_t K,
+                               const int8_t *Wq, const float *sw, const float *bias,
+                               const float *gate, const uint16_t *residual, int64_t N,
+                               uint16_t *y, void *workspace, size_t ws_bytes,
+                               qk_stream_t stream);
+
+/*
  * The matmul + dequant half of qk_w8a8_linear, on activations that are already
  * quantized (xq, sx from qk_quantize_activations).  Lets one quantization feed
  * several projections of the same input.

@@ -34,6 +34,7 @@ _SIGS = {
     "qk_quantize_activations": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "qk_w8a8_linear": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w8a8_gemm": (_I, [_P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P]),
+    "qk_w8a8_linear_gated": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w4a8_linear": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w4a8_gemm": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I, _P]),
     "qk_w4a8_linear_plan": (_I, [_I64, _I64, _I64]),
@@ -179,6 +180,28 @@ def qk_w8a8_linear(x, Wq, sw, bias=None, y=None, workspace=None, stream=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.qk_w8a8_linear(_ptr(x), M, K, _ptr(Wq), _ptr(sw), _ptr(bias), N, _ptr(y),
                               _ptr(workspace), ws_bytes, _stream(stream)), "qk_w8a8_linear")
+    return y
+
+
+def qk_w8a8_linear_gated(x, Wq, sw, bias, gate, residual, y=None, workspace=None, stream=None):
+    """y bf16 [M, N] = bf16(residual + gate * (quant(x) . Wq^T * sx * sw + bias));
+    y may be `residual` itself (an in-place update)."""
+    _need(x, torch.bfloat16, 2, "x")
+    _need(Wq, torch.int8, 2, "Wq")
+    _need(sw, torch.float32, 1, "sw")
+    _need(gate, torch.float32, 1, "gate")
+    _need(residual, torch.bfloat16, 2, "residual")
+    if bias is not None:
+        _need(bias, torch.float32, 1, "bias")
+    M, K = x.shape
+    N = Wq.shape[0]
+    if tuple(residual.shape) != (M, N) or gate.shape[0] != N:
+        raise ValueError("residual must be [M, N] and gate [N]")
+    y = _out(y, (M, N), torch.bfloat16, x.device, "y")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qk_w8a8_linear_gated(_ptr(x), M, K, _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(gate),
+                                    _ptr(residual), N, _ptr(y), _ptr(workspace), ws_bytes,
+                                    _stream(stream)), "qk_w8a8_linear_gated")
     return y
 
 

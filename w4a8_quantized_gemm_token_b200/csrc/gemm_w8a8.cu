@@ -80,6 +80,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// bf16 bits -> fp64, exactly: integer operations on the bits for normal
+// values (rebias the exponent, move the 7 mantissa bits), through fp32 for
+// zeros and subnormals.
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) {
+  const uint32_t e = (b >> 7) & 0xFFu;
+  if (e == 0u) return (double)__uint_as_float(b << 16);
+  const uint32_t hi = ((b & 0x8000u) << 16) | ((e + 896u) << 20) | ((b & 0x7Fu) << 13);
+  return __hiloint2double((int)hi, 0);
+}
+
 // Raster: groups of `group_m` M tiles; inside a group, consecutive tiles walk
 // down the M tiles first, then across N, so the CTA pairs running at the same
 // time share the group's rows of xq (kept in L2) and a few Wq tiles.
@@ -122,11 +132,15 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
   return sign | bits;
 }
 
-template <bool kAccOut>
+// kAccOut: store the int32 sums instead of y.  kGated: the gated residual
+// epilogue ("mlx-kquant PR #89", commit list), y = bf16(residual + gate[n] *
+// (acc * sx * sw + bias)) in fp64 for every output.
+template <bool kAccOut, bool kGated>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const float* __restrict__ sx,
-                     const float* __restrict__ sw, const float* __restrict__ bias, int M, int N,
+                     const float* __restrict__ sw, const float* __restrict__ bias,
+                     const float* __restrict__ gate, const uint16_t* residual, int M, int N,
                      int K, int group_m, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
@@ -280,7 +294,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int n = ncol0 + col;
           const float w = n < N ? __ldg(sw + n) : 0.0f;
           const float b = (n < N && bias != nullptr) ? __ldg(bias + n) : 0.0f;
-          tcol[col] = make_float4(w, b, fmaxf(kGuard * fabsf(b), kTiny), 0.0f);
+          const float g = (kGated && n < N) ? __ldg(gate + n) : 0.0f;
+          tcol[col] = make_float4(w, b, fmaxf(kGuard * fabsf(b), kTiny), g);
         }
         mbar_arrive(table_bar(iter & 1));
         if (!mbar_wait(table_bar(iter & 1), (uint32_t)(iter >> 1) & 1u, err)) break;
@@ -298,6 +313,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int col0 = c * kChunk;
         const int n0 = ncol0 + col0;
         uint32_t out[32];
+        // gated: this row's residual for the chunk (64 bf16 = 8 x 16 bytes),
+        // loaded before the accumulator so the latency overlaps
+        uint4 res[kGated ? kChunk / 8 : 1];
+        if constexpr (kGated) {
+#pragma unroll
+          for (int i = 0; i < kChunk / 8; ++i)
+            res[i] = (row < M && n0 + 8 * i < N)
+                         ? *reinterpret_cast<const uint4*>(residual + (size_t)row * N + n0 + 8 * i)
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
         // two 32-column halves per chunk keep the live registers down
 #pragma unroll
         for (int h = 0; h < kChunk / 32; ++h) {
@@ -313,6 +338,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if constexpr (kAccOut) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) out[j] = v[j];
+          } else if constexpr (kGated) {
+            // every output in fp64: u = acc * sx * sw + bias, y = residual + gate * u
+            const float4* tc = tcol + col0 + 32 * h;
+            const double sxd = (double)sxf;
+            uint32_t* o = out + 16 * h;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const uint4 rq = res[(32 * h + j) / 8];
+              const int w4 = ((32 * h + j) % 8) / 2;  // which 32-bit word of the 16-byte piece
+              const uint32_t rw = w4 == 0 ? rq.x : w4 == 1 ? rq.y : w4 == 2 ? rq.z : rq.w;
+              const float4 c0 = tc[j], c1 = tc[j + 1];
+              const double u0 = fma(i32_to_f64(v[j]) * sxd, (double)c0.x, (double)c0.y);
+              const double u1 = fma(i32_to_f64(v[j + 1]) * sxd, (double)c1.x, (double)c1.y);
+              const uint32_t y0 = f64_to_bf16_bits(fma((double)c0.w, u0, bf16_bits_to_f64(rw & 0xFFFFu)));
+              const uint32_t y1 = f64_to_bf16_bits(fma((double)c1.w, u1, bf16_bits_to_f64(rw >> 16)));
+              o[j >> 1] = y0 | (y1 << 16);
+            }
           } else {
             // fast path in fp32: v32 = fma(fp32(acc) * sx, sw, bias).  Its error
             // is at most 2^-23 |acc sx sw| + 2^-24 |v32|, below 1/8 bf16 ulp when
@@ -390,15 +432,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
-bool g_attr_done[2][64];
+bool g_attr_done[3][64];  // plain, accumulator dump, gated
 
 }  // namespace
 
 cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64_t K,
                              const int8_t* Wq, const float* sw, const float* bias, int64_t N,
-                             uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s) {
+                             uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s,
+                             const float* gate, const uint16_t* residual) {
   if (w8a8_use_skinny(M, K, N))
-    return launch_w8a8_skinny(xq, sx, M, K, Wq, sw, bias, N, y, acc_out, pdl, s);
+    return launch_w8a8_skinny(xq, sx, M, K, Wq, sw, bias, N, y, acc_out, pdl, s, gate, residual);
   const bool acc_mode = acc_out != nullptr;
   CUtensorMap tA, tB, tC;
   if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
@@ -417,12 +460,15 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   }
   int dev = 0;
   cudaGetDevice(&dev);
-  auto kernel = acc_mode ? w8a8_gemm_kernel<true> : w8a8_gemm_kernel<false>;
-  if (dev < 64 && !g_attr_done[acc_mode][dev]) {
+  const bool gated = gate != nullptr;
+  auto kernel = acc_mode ? w8a8_gemm_kernel<true, false>
+                         : (gated ? w8a8_gemm_kernel<false, true> : w8a8_gemm_kernel<false, false>);
+  const int variant = acc_mode ? 1 : (gated ? 2 : 0);
+  if (dev < 64 && !g_attr_done[variant][dev]) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    g_attr_done[acc_mode][dev] = true;
+    g_attr_done[variant][dev] = true;
   }
   int* err = device_error_word();
   if (err == nullptr) return cudaErrorUnknown;
@@ -445,8 +491,8 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, tA, tB, tC, sx, sw, bias, (int)M, (int)N, (int)K,
-                            (int)group_m, err);
+  return cudaLaunchKernelEx(&cfg, kernel, tA, tB, tC, sx, sw, bias, gate, residual, (int)M,
+                            (int)N, (int)K, (int)group_m, err);
 }
 
 }  // namespace qk

@@ -18,7 +18,8 @@
 //    store it, through distributed shared memory, into the slot of this K
 //    range in the CTA that owns the row (128 / S rows per CTA); after a
 //    cluster barrier each CTA adds its rows' S partial sums in a fixed order
-//    (integer addition: exact and deterministic) and applies the dequant.
+//    (integer addition: exact and deterministic) and applies the dequant
+//    (and, with a gate, the gated residual epilogue).
 // Every wait is bounded; a CTA that gives up still takes part in the cluster
 // barrier.  No load uses cluster multicast.
 #include <cuda_bf16.h>
@@ -102,8 +103,9 @@ template <bool kAccOut>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const float* __restrict__ sx, const float* __restrict__ sw,
-                       const float* __restrict__ bias, int M, int N, int K, int S,
-                       uint16_t* __restrict__ y, int32_t* __restrict__ acc_out, int* err) {
+                       const float* __restrict__ bias, const float* __restrict__ gate,
+                       const uint16_t* residual, int M, int N, int K, int S,
+                       uint16_t* y, int32_t* __restrict__ acc_out, int* err) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
   const SkinnyLayout L(N, S);
@@ -227,8 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (kAccOut) {
       acc_out[(size_t)m * N + c] = (int32_t)acc;
     } else {
-      const double v = fma(i32_to_f64(acc) * (double)__ldg(sx + m), (double)__ldg(sw + c),
-                           bias != nullptr ? (double)__ldg(bias + c) : 0.0);
+      double v = fma(i32_to_f64(acc) * (double)__ldg(sx + m), (double)__ldg(sw + c),
+                     bias != nullptr ? (double)__ldg(bias + c) : 0.0);
+      if (gate != nullptr)  // gated residual epilogue: residual + gate * v
+        v = fma((double)__ldg(gate + c), v,
+                (double)__uint_as_float((uint32_t)residual[(size_t)m * N + c] << 16));
       y[(size_t)m * N + c] = f64_to_bf16_bits(v);
     }
   }
@@ -259,7 +264,8 @@ bool w8a8_use_skinny(int64_t M, int64_t K, int64_t N) {
 
 cudaError_t launch_w8a8_skinny(const int8_t* xq, const float* sx, int64_t M, int64_t K,
                                const int8_t* Wq, const float* sw, const float* bias, int64_t N,
-                               uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s) {
+                               uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s,
+                               const float* gate, const uint16_t* residual) {
   const bool acc_mode = acc_out != nullptr;
   const int mtiles = (int)((M + BM - 1) / BM);
   const int nkb = (int)((K + BK - 1) / BK);
@@ -335,8 +341,8 @@ cudaError_t launch_w8a8_skinny(const int8_t* xq, const float* sx, int64_t M, int
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kernel, tA, tB, sx, sw, bias, (int)M, (int)N, (int)K, S, y,
-                            acc_out, err);
+  return cudaLaunchKernelEx(&cfg, kernel, tA, tB, sx, sw, bias, gate, residual, (int)M, (int)N,
+                            (int)K, S, y, acc_out, err);
 }
 
 }  // namespace qk

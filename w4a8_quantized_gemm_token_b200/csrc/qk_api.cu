@@ -271,6 +271,30 @@ qk_status qk_w8a8_linear(const uint16_t* x, int64_t M, int64_t K, const int8_t* 
                    "w8a8_gemm");
 }
 
+qk_status qk_w8a8_linear_gated(const uint16_t* x, int64_t M, int64_t K, const int8_t* Wq,
+                               const float* sw, const float* bias, const float* gate,
+                               const uint16_t* residual, int64_t N, uint16_t* y, void* workspace,
+                               size_t ws_bytes, qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, false);
+  if (st != QK_OK || M == 0) return st;
+  if (!x || !Wq || !sw || !y || !gate || !residual) return QK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(sw) || !aligned16(y) || !aligned16(gate) ||
+      !aligned16(residual) || (bias && !aligned16(bias)))
+    return QK_ERR_MISALIGNED;
+  if ((st = check_device()) != QK_OK) return st;
+  Workspace ws;
+  if ((st = ws.init(workspace, ws_bytes, M, K, false, stream)) != QK_OK) return st;
+  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, nullptr, stream, true),
+                      "quant_act")) != QK_OK)
+    return st;
+  if (log_enabled())
+    std::fprintf(stderr, "[qk] w8a8_linear_gated M=%lld K=%lld N=%lld\n", (long long)M,
+                 (long long)K, (long long)N);
+  return from_cuda(launch_w8a8_gemm(ws.xq, ws.sx, M, K, Wq, sw, bias, N, y, nullptr, true, stream,
+                                    gate, residual),
+                   "w8a8_gemm_gated");
+}
+
 static qk_status check_w4_product(const uint8_t* Wp, const uint16_t* wscale,
                                   const uint16_t* woffset, const float* bias, uint16_t* y) {
   if (!Wp || !wscale || !woffset || !y) return QK_ERR_INVALID_ARG;

@@ -28,9 +28,14 @@ cudaError_t launch_quant_w4(const float* W, int64_t N, int64_t K, uint8_t* Wp, u
 // W8A8 GEMM with the fused dequant + bias epilogue (bf16 out), or the raw int32
 // accumulator epilogue when `acc_out` is not null (y, sx, sw, bias ignored).
 // `pdl` launches it as a programmatic dependent of the previous kernel.
+// With `gate` (fp32 [N]) and `residual` (bf16 [M, N]) the gated residual
+// epilogue: y = bf16(residual + gate[n] * (acc * sx * sw + bias)); y may be the
+// residual buffer itself (each element is read before it is written, by the
+// same thread).
 cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64_t K,
                              const int8_t* Wq, const float* sw, const float* bias, int64_t N,
-                             uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s);
+                             uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s,
+                             const float* gate = nullptr, const uint16_t* residual = nullptr);
 
 // The same product for thin outputs (N <= 64, see w8a8_use_skinny): 128-row
 // tiles split along K over a cluster, exact int32 partial sums reduced through
@@ -38,7 +43,8 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
 bool w8a8_use_skinny(int64_t M, int64_t K, int64_t N);
 cudaError_t launch_w8a8_skinny(const int8_t* xq, const float* sx, int64_t M, int64_t K,
                                const int8_t* Wq, const float* sw, const float* bias, int64_t N,
-                               uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s);
+                               uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s,
+                               const float* gate = nullptr, const uint16_t* residual = nullptr);
 
 // W4A8 tensor-core GEMM (any M).  When `acc_out` is not null it stores the
 // per-group int32 accumulators of rows [m0, m1) instead of y.
