@@ -73,6 +73,8 @@ static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 // An output takes the fp32 fast path when |v32| >= max(kGuard |bias|, kTiny).
 constexpr float kGuard = 0.000244140625f;   // 2^-12
 constexpr float kTiny = 7.888609052210118e-31f;  // 2^-100
+// The gated fast path holds when |y| >= kGuardGate |gate| (|u| + |bias|).
+constexpr float kGuardGate = 0.0009765625f;  // 2^-10
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -339,21 +341,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) out[j] = v[j];
           } else if constexpr (kGated) {
-            // every output in fp64: u = acc * sx * sw + bias, y = residual + gate * u
+            // fast path in fp32: u32 = fma(fp32(acc) * sx, sw, bias) and
+            // y32 = fma(gate, u32, residual).  Their error is below
+            // |gate| (|u32| + |bias|) 2^-22.4 + 2^-24 |y32|, under 1/8 bf16 ulp
+            // when |y32| >= 2^-10 |gate| (|u32| + |bias|); y32 then rounds to
+            // within 1 ulp of the exact value.  Other outputs (the residual
+            // cancelling the update, magnitudes near the fp32 underflow) take
+            // the exact fp64 path; a closed gate or a zero update is exact here.
             const float4* tc = tcol + col0 + 32 * h;
-            const double sxd = (double)sxf;
             uint32_t* o = out + 16 * h;
+            uint32_t slow = 0;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const uint4 rq = res[(32 * h + j) / 8];
               const int w4 = ((32 * h + j) % 8) / 2;  // which 32-bit word of the 16-byte piece
               const uint32_t rw = w4 == 0 ? rq.x : w4 == 1 ? rq.y : w4 == 2 ? rq.z : rq.w;
               const float4 c0 = tc[j], c1 = tc[j + 1];
-              const double u0 = fma(i32_to_f64(v[j]) * sxd, (double)c0.x, (double)c0.y);
-              const double u1 = fma(i32_to_f64(v[j + 1]) * sxd, (double)c1.x, (double)c1.y);
-              const uint32_t y0 = f64_to_bf16_bits(fma((double)c0.w, u0, bf16_bits_to_f64(rw & 0xFFFFu)));
-              const uint32_t y1 = f64_to_bf16_bits(fma((double)c1.w, u1, bf16_bits_to_f64(rw >> 16)));
-              o[j >> 1] = y0 | (y1 << 16);
+              const float u0 = __fmaf_rn(__fmul_rn(__int2float_rn((int)v[j]), sxf), c0.x, c0.y);
+              const float u1 = __fmaf_rn(__fmul_rn(__int2float_rn((int)v[j + 1]), sxf), c1.x, c1.y);
+              const float r0 = __fmaf_rn(c0.w, u0, __uint_as_float(rw << 16));
+              const float r1 = __fmaf_rn(c1.w, u1, __uint_as_float(rw & 0xFFFF0000u));
+              const bool s0 =
+                  !(fabsf(r0) >= fmaxf(kGuardGate * fabsf(c0.w) * (fabsf(u0) + fabsf(c0.y)), kTiny)) &&
+                  (v[j] != 0u || c0.y != 0.0f) && c0.w != 0.0f;
+              const bool s1 =
+                  !(fabsf(r1) >= fmaxf(kGuardGate * fabsf(c1.w) * (fabsf(u1) + fabsf(c1.y)), kTiny)) &&
+                  (v[j + 1] != 0u || c1.y != 0.0f) && c1.w != 0.0f;
+              slow |= ((s0 ? 1u : 0u) | (s1 ? 2u : 0u)) << j;
+              o[j >> 1] = pack_bf16x2(r0, r1);
+            }
+            if (__any_sync(0xFFFFFFFFu, slow != 0u)) {
+              const double sxd = (double)sxf;
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                const uint32_t m8 = (slow >> (8 * g)) & 0xFFu;
+                if (__any_sync(0xFFFFFFFFu, m8 != 0u)) {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const int j = 8 * g + i;
+                    if ((m8 >> i) & 1u) {
+                      const uint4 rq = res[(32 * h + j) / 8];
+                      const int w4 = ((32 * h + j) % 8) / 2;
+                      const uint32_t rw = w4 == 0 ? rq.x : w4 == 1 ? rq.y : w4 == 2 ? rq.z : rq.w;
+                      const uint32_t rb = (j & 1) ? (rw >> 16) : (rw & 0xFFFFu);
+                      const float4 cj = tc[j];
+                      const double u = fma(i32_to_f64(v[j]) * sxd, (double)cj.x, (double)cj.y);
+                      const uint32_t hb = f64_to_bf16_bits(fma((double)cj.w, u, bf16_bits_to_f64(rb)));
+                      o[j >> 1] = (j & 1) ? ((o[j >> 1] & 0x0000FFFFu) | (hb << 16))
+                                          : ((o[j >> 1] & 0xFFFF0000u) | hb);
+                    }
+                  }
+                }
+              }
             }
           } else {
             // fast path in fp32: v32 = fma(fp32(acc) * sx, sw, bias).  Its error
