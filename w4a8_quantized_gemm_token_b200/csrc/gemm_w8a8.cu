@@ -54,7 +54,7 @@ constexpr int A_BYTES = BM * BK;                  // 32 KiB
 constexpr int B_BYTES = (BN / 2) * BK;            // 32 KiB
 constexpr uint32_t STAGE_TX = 2 * (A_BYTES + B_BYTES);  // both CTAs' loads
 constexpr int STG_BYTES = 32 * 128;               // 32 rows x 128 B
-constexpr int TAB_BYTES = BN * 16;                // per column {sw, bias, threshold, 0}
+constexpr int TAB_BYTES = BN * 16;                // per column {sw, bias, guard, gate}
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_BYTES;
 constexpr int SMEM_STG = SMEM_B + STAGES * B_BYTES;
@@ -73,8 +73,8 @@ static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 // An output takes the fp32 fast path when |v32| >= max(kGuard |bias|, kTiny).
 constexpr float kGuard = 0.000244140625f;   // 2^-12
 constexpr float kTiny = 7.888609052210118e-31f;  // 2^-100
-// The gated fast path holds when |y| >= kGuardGate |gate| (|u| + |bias|).
-constexpr float kGuardGate = 0.0009765625f;  // 2^-10
+// The gated fast path holds when |y| >= kGuardGate |gate| (|u| + |bias|) + kTiny.
+constexpr float kGuardGate = 0.0001220703125f;  // 2^-13
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -281,9 +281,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t aphase = 0;
     int iter = 0;
     int use = 0;  // staging-buffer use counter (alternates the two buffers)
+    // gated: each lane sends its row of a tile's residual (up to 512 bytes) to
+    // L2 one tile ahead of the tile's epilogue, so the per-chunk register loads
+    // below meet L2 rather than HBM latency
+    auto prefetch_residual = [&](int tt) {
+      if (tt >= num_tiles) return;
+      int pm, pn;
+      tile_coords(tt, tiles_m, tiles_n, group_m, pm, pn);
+      const int prow = pm * 2 * BM + (int)rank * BM + q * 32 + lane;
+      const int pcol = pn * BN;
+      if (prow < M && pcol < N)
+        bulk_prefetch_l2(residual + (size_t)prow * N + pcol, (uint32_t)(min(BN, N - pcol) * 2));
+    };
+    if constexpr (kGated) prefetch_residual(pair);
     for (int t = pair; t < num_tiles; t += num_pairs, ++iter) {
       int mb, nb;
       tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
+      if constexpr (kGated) prefetch_residual(t + num_pairs);
       const int ncol0 = nb * BN;
       float4* tcol = tab + (iter & 1) * BN;
       if constexpr (!kAccOut) {
@@ -297,7 +311,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const float w = n < N ? __ldg(sw + n) : 0.0f;
           const float b = (n < N && bias != nullptr) ? __ldg(bias + n) : 0.0f;
           const float g = (kGated && n < N) ? __ldg(gate + n) : 0.0f;
-          tcol[col] = make_float4(w, b, fmaxf(kGuard * fabsf(b), kTiny), g);
+          const float z = kGated ? kGuardGate * fabsf(g) : fmaxf(kGuard * fabsf(b), kTiny);
+          tcol[col] = make_float4(w, b, z, g);
         }
         mbar_arrive(table_bar(iter & 1));
         if (!mbar_wait(table_bar(iter & 1), (uint32_t)(iter >> 1) & 1u, err)) break;
@@ -343,11 +358,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           } else if constexpr (kGated) {
             // fast path in fp32: u32 = fma(fp32(acc) * sx, sw, bias) and
             // y32 = fma(gate, u32, residual).  Their error is below
-            // |gate| (|u32| + |bias|) 2^-22.4 + 2^-24 |y32|, under 1/8 bf16 ulp
-            // when |y32| >= 2^-10 |gate| (|u32| + |bias|); y32 then rounds to
-            // within 1 ulp of the exact value.  Other outputs (the residual
-            // cancelling the update, magnitudes near the fp32 underflow) take
-            // the exact fp64 path; a closed gate or a zero update is exact here.
+            // |gate| (|u32| + |bias|) 2^-22.4 + 2^-24 |y32|, under 2^-9 |y32|
+            // (half a bf16 ulp) when |y32| >= 2^-13 |gate| (|u32| + |bias|);
+            // y32 then rounds to within 1 ulp of the exact value.  Other
+            // outputs (the residual cancelling the update, magnitudes near the
+            // fp32 underflow) take the exact fp64 path.
             const float4* tc = tcol + col0 + 32 * h;
             uint32_t* o = out + 16 * h;
             uint32_t slow = 0;
@@ -361,12 +376,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               const float u1 = __fmaf_rn(__fmul_rn(__int2float_rn((int)v[j + 1]), sxf), c1.x, c1.y);
               const float r0 = __fmaf_rn(c0.w, u0, __uint_as_float(rw << 16));
               const float r1 = __fmaf_rn(c1.w, u1, __uint_as_float(rw & 0xFFFF0000u));
-              const bool s0 =
-                  !(fabsf(r0) >= fmaxf(kGuardGate * fabsf(c0.w) * (fabsf(u0) + fabsf(c0.y)), kTiny)) &&
-                  (v[j] != 0u || c0.y != 0.0f) && c0.w != 0.0f;
-              const bool s1 =
-                  !(fabsf(r1) >= fmaxf(kGuardGate * fabsf(c1.w) * (fabsf(u1) + fabsf(c1.y)), kTiny)) &&
-                  (v[j + 1] != 0u || c1.y != 0.0f) && c1.w != 0.0f;
+              // c.z = 2^-13 |gate|
+              const bool s0 = !(fabsf(r0) >= __fmaf_rn(c0.z, fabsf(u0) + fabsf(c0.y), kTiny));
+              const bool s1 = !(fabsf(r1) >= __fmaf_rn(c1.z, fabsf(u1) + fabsf(c1.y), kTiny));
               slow |= ((s0 ? 1u : 0u) | (s1 ? 2u : 0u)) << j;
               o[j >> 1] = pack_bf16x2(r0, r1);
             }

@@ -130,6 +130,14 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+// Bring `bytes` of global memory into L2 ahead of use (16-byte aligned source,
+// size % 16 == 0); nothing waits for it.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (TMA store, tcgen05.mma operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
