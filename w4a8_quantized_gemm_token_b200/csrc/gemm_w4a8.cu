@@ -38,17 +38,25 @@ namespace qk {
 namespace {
 
 constexpr int BM = 128;                   // rows (TMEM lanes)
-constexpr int BN = 64;                    // output columns per tile
+constexpr int BN = 128;                   // output columns per tile
 constexpr int BK = 128;                   // K per stage: two groups of 64
 constexpr int STAGES = 4;
 constexpr int UBUFS = 2;                  // unpacked code tiles
 constexpr int TSLOTS = 4;                 // scale/offset table slots (one per K block)
 constexpr int TBUFS = 4;                  // TMEM group accumulators
 constexpr int kUnpackWarps = 2;
-constexpr int kFoldWarps = 16;            // four per TMEM lane quarter
-constexpr int kFoldCols = BN / (kFoldWarps / 4);  // 16 columns per fold thread
-constexpr int kPiece = 8;                 // TMEM columns loaded at a time
-constexpr int kThreads = 32 * (2 + kUnpackWarps + kFoldWarps);
+constexpr int kFoldWarps = 8;             // two per TMEM lane quarter
+constexpr int kFoldCols = BN / (kFoldWarps / 4);  // 64 columns per fold thread
+constexpr int kThreads = 32 * (2 + kUnpackWarps + kFoldWarps);  // 384: three warpgroups
+// Registers: the block is launched with kRegsLaunch per thread; warpgroup 0
+// (producer, MMA issuer, unpack) keeps kRegsCtl and hands the rest to the two
+// fold warpgroups, whose threads hold 64 fp64 sums each.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsCtl = 56;
+constexpr int kRegsFold = 224;
+static_assert(2 + kUnpackWarps == 4, "warpgroup 0 holds every non-fold warp");
+static_assert(128 * kRegsCtl + 32 * kFoldWarps * kRegsFold <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr int A_BYTES = BM * BK;          // 16 KiB
 constexpr int P_BYTES = BN * (BK / 2);    // 4 KiB of packed nibbles
 constexpr int U_BYTES = BN * BK;          // 8 KiB of unpacked codes
@@ -56,7 +64,7 @@ constexpr int U_BYTES = BN * BK;          // 8 KiB of unpacked codes
 // rows of xsum as fp64
 constexpr int T_SO = 2 * BN * 16;
 constexpr int T_BYTES = T_SO + 2 * BM * 8;
-constexpr int STG_BYTES = 32 * 2 * kFoldCols;  // 32 rows x kFoldCols bf16
+constexpr int STG_BYTES = 32 * 2 * kFoldCols;  // 32 rows x kFoldCols bf16 (128-byte swizzle)
 constexpr int SMEM_A = 0;
 constexpr int SMEM_P = SMEM_A + STAGES * A_BYTES;
 constexpr int SMEM_U = SMEM_P + STAGES * P_BYTES;
@@ -72,6 +80,7 @@ constexpr uint32_t kIdesc = i8_idesc(BM, BN, true, false);
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert(SMEM_U % 1024 == 0 && U_BYTES % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(SMEM_STG % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled output stages too");
 
 __device__ __forceinline__ double i32_to_f64(uint32_t a) {
   return __hiloint2double(0x43300000, (int)(a ^ 0x80000000u)) - 4503601774854144.0;
@@ -172,148 +181,163 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();  // xq, sx and xsum come from the activation-quant kernel
 
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int mb = t % tiles_m, nb = t / tiles_m;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1u, err)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(full_bar(s), A_BYTES + P_BYTES);
-          tma_load_2d(sbase + SMEM_A + s * A_BYTES, &tmA, kb * BK, mb * BM, full_bar(s));
-          tma_load_2d(sbase + SMEM_P + s * P_BYTES, &tmP, kb * (BK / 2), nb * BN, full_bar(s));
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      int it = 0, gc = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
-          const int s = it % STAGES, u = it % UBUFS;
-          ok = mbar_wait(ufull_bar(u), (it / UBUFS) & 1, err) &&
-               mbar_wait(full_bar(s), (it / STAGES) & 1, err);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t a_addr = sbase + SMEM_A + s * A_BYTES;
-          const uint32_t b_addr = sbase + SMEM_U + u * U_BYTES;
-          for (int j = 0; j < 2 && 2 * kb + j < G; ++j, ++gc) {
-            const int b = gc % TBUFS;
-            if (!mbar_wait(tempty_bar(b), ((gc / TBUFS) & 1) ^ 1u, err)) {
+  if (warp < 4) {
+    // warpgroup 0: warp 0 loads, warp 1 issues the MMAs, warps 2-3 unpack;
+    // most of its registers go to the fold warpgroups
+    regs_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+          const int mb = t % tiles_m, nb = t / tiles_m;
+          for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            const int s = it % STAGES;
+            if (!mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1u, err)) {
               ok = false;
               break;
             }
+            mbar_arrive_expect_tx(full_bar(s), A_BYTES + P_BYTES);
+            tma_load_2d(sbase + SMEM_A + s * A_BYTES, &tmA, kb * BK, mb * BM, full_bar(s));
+            tma_load_2d(sbase + SMEM_P + s * P_BYTES, &tmP, kb * (BK / 2), nb * BN, full_bar(s));
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        int it = 0, gc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+          for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
+            const int s = it % STAGES, u = it % UBUFS;
+            ok = mbar_wait(ufull_bar(u), (it / UBUFS) & 1, err) &&
+                 mbar_wait(full_bar(s), (it / STAGES) & 1, err);
+            if (!ok) break;
             tc_fence_after();
+            const uint32_t a_addr = sbase + SMEM_A + s * A_BYTES;
+            const uint32_t b_addr = sbase + SMEM_U + u * U_BYTES;
+            for (int j = 0; j < 2 && 2 * kb + j < G; ++j, ++gc) {
+              const int b = gc % TBUFS;
+              if (!mbar_wait(tempty_bar(b), ((gc / TBUFS) & 1) ^ 1u, err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_i8(tmem_base + (uint32_t)(b * BN), sw128_kmajor_desc(a_addr + 64 * j + 32 * kk),
-                     sw128_kmajor_desc(b_addr + 64 * j + 32 * kk), kIdesc, kk);
-            mma_commit(tfull_bar(b));  // this group's sums are ready
+              for (int kk = 0; kk < 2; ++kk)
+                mma_i8(tmem_base + (uint32_t)(b * BN), sw128_kmajor_desc(a_addr + 64 * j + 32 * kk),
+                       sw128_kmajor_desc(b_addr + 64 * j + 32 * kk), kIdesc, kk);
+              mma_commit(tfull_bar(b));  // this group's sums are ready
+            }
+            mma_commit(empty_bar(s));   // xq and packed tiles free
+            mma_commit(uempty_bar(u));  // unpacked tile free
           }
-          mma_commit(empty_bar(s));   // xq and packed tiles free
-          mma_commit(uempty_bar(u));  // unpacked tile free
         }
       }
-    }
-  } else if (warp < 2 + kUnpackWarps) {
-    // -------------------------------------------------------------- unpack
-    const int r = threadIdx.x - 64;  // tile row (output column) 0..63
-    // scales / offsets of K block (tile t, block kb) for this row, fetched one
-    // block ahead so their global-load latency overlaps the current block
-    auto fetch_so = [&](int t, int kb, uint16_t (&v)[4]) {
-      const int n = (t / tiles_m) * BN + r;
+    } else {
+      // -------------------------------------------------------------- unpack
+      const int r = threadIdx.x - 64;  // tile rows (output columns) r and r + 64
+      // scales / offsets of K block (tile t, block kb) for these rows, fetched
+      // one block ahead so their global-load latency overlaps the current block;
+      // v[4 i + 2 j + {0, 1}] = {s, o} of row r + 64 i, group 2 kb + j
+      auto fetch_so = [&](int t, int kb, uint16_t (&v)[8]) {
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int g = 2 * kb + j;
-        const bool in = t < num_tiles && n < N && g < G;
-        v[2 * j] = in ? __ldg(wscale + (size_t)n * G + g) : (uint16_t)0;
-        v[2 * j + 1] = in ? __ldg(woffset + (size_t)n * G + g) : (uint16_t)0;
-      }
-    };
-    // xsum of K block (tile t, block kb) for rows r and r + 64 of the tile
-    auto fetch_xs = [&](int t, int kb, int (&v)[4]) {
-      const int mrow = (t % tiles_m) * BM + r;
+        for (int i = 0; i < 2; ++i) {
+          const int n = (t / tiles_m) * BN + r + 64 * i;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = mrow + 64 * (i >> 1), g = 2 * kb + (i & 1);
-        v[i] = (t < num_tiles && m < M && g < G) ? __ldg(xsum + (size_t)m * G + g) : 0;
-      }
-    };
-    uint16_t so_next[4] = {0, 0, 0, 0};
-    int xs_next[4] = {0, 0, 0, 0};
-    if (!kAccOut) {
-      fetch_so(blockIdx.x, 0, so_next);
-      fetch_xs(blockIdx.x, 0, xs_next);
-    }
-    int it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
-        const int s = it % STAGES, u = it % UBUFS, ts = it % TSLOTS;
-        uint16_t so_cur[4];
-        int xs_cur[4];
+          for (int j = 0; j < 2; ++j) {
+            const int g = 2 * kb + j;
+            const bool in = t < num_tiles && n < N && g < G;
+            v[4 * i + 2 * j] = in ? __ldg(wscale + (size_t)n * G + g) : (uint16_t)0;
+            v[4 * i + 2 * j + 1] = in ? __ldg(woffset + (size_t)n * G + g) : (uint16_t)0;
+          }
+        }
+      };
+      // xsum of K block (tile t, block kb) for rows r and r + 64 of the tile
+      auto fetch_xs = [&](int t, int kb, int (&v)[4]) {
+        const int mrow = (t % tiles_m) * BM + r;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          so_cur[i] = so_next[i];
-          xs_cur[i] = xs_next[i];
+          const int m = mrow + 64 * (i >> 1), g = 2 * kb + (i & 1);
+          v[i] = (t < num_tiles && m < M && g < G) ? __ldg(xsum + (size_t)m * G + g) : 0;
         }
-        if (!kAccOut) {
-          const bool last = kb + 1 == num_kb;
-          fetch_so(last ? t + (int)gridDim.x : t, last ? 0 : kb + 1, so_next);
-          fetch_xs(last ? t + (int)gridDim.x : t, last ? 0 : kb + 1, xs_next);
-        }
-        ok = mbar_wait(full_bar(s), (it / STAGES) & 1, err) &&
-             mbar_wait(uempty_bar(u), ((it / UBUFS) & 1) ^ 1u, err);
-        if (!ok) break;
-        // 64 packed bytes of row r -> 128 u8 codes, 128-byte-swizzled row
-        const uint4* src = reinterpret_cast<const uint4*>(smem + SMEM_P + s * P_BYTES + r * 64);
-        uint8_t* dst = smem + SMEM_U + u * U_BYTES + r * 128;
+      };
+      uint16_t so_next[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int xs_next[4] = {0, 0, 0, 0};
+      if (!kAccOut) {
+        fetch_so(blockIdx.x, 0, so_next);
+        fetch_xs(blockIdx.x, 0, xs_next);
+      }
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % STAGES, u = it % UBUFS, ts = it % TSLOTS;
+          uint16_t so_cur[8];
+          int xs_cur[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 w = src[i];  // codes 32i .. 32i + 31
-          uint4 c0, c1;
-          unpack8(w.x, c0.x, c0.y);
-          unpack8(w.y, c0.z, c0.w);
-          unpack8(w.z, c1.x, c1.y);
-          unpack8(w.w, c1.z, c1.w);
-          *reinterpret_cast<uint4*>(dst + (((2 * i) ^ (r & 7)) * 16)) = c0;
-          *reinterpret_cast<uint4*>(dst + (((2 * i + 1) ^ (r & 7)) * 16)) = c1;
-        }
-        fence_proxy_async_smem();  // generic writes -> tensor-core reads
-        __syncwarp();
-        if (lane == 0) mbar_arrive(ufull_bar(u));
-        // this K block's scales and offsets in fp64, for the fold warps
-        if (!kAccOut) {
-          if (!mbar_wait(tabempty_bar(ts), ((it / TSLOTS) & 1) ^ 1u, err)) {
-            ok = false;
-            break;
+          for (int i = 0; i < 8; ++i) so_cur[i] = so_next[i];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xs_cur[i] = xs_next[i];
+          if (!kAccOut) {
+            const bool last = kb + 1 == num_kb;
+            fetch_so(last ? t + (int)gridDim.x : t, last ? 0 : kb + 1, so_next);
+            fetch_xs(last ? t + (int)gridDim.x : t, last ? 0 : kb + 1, xs_next);
           }
-          double2* tab = reinterpret_cast<double2*>(smem + SMEM_T + ts * T_BYTES);
+          ok = mbar_wait(full_bar(s), (it / STAGES) & 1, err) &&
+               mbar_wait(uempty_bar(u), ((it / UBUFS) & 1) ^ 1u, err);
+          if (!ok) break;
+          // 64 packed bytes of a row -> 128 u8 codes, 128-byte-swizzled row
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
-            tab[j * BN + r] =
-                make_double2((double)__half2float(__ushort_as_half(so_cur[2 * j])),
-                             (double)__half2float(__ushort_as_half(so_cur[2 * j + 1])));
-          double* xs_tab = reinterpret_cast<double*>(smem + SMEM_T + ts * T_BYTES + T_SO);
+          for (int rr = r; rr < BN; rr += 64) {
+            const uint4* src =
+                reinterpret_cast<const uint4*>(smem + SMEM_P + s * P_BYTES + rr * 64);
+            uint8_t* dst = smem + SMEM_U + u * U_BYTES + rr * 128;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)  // [group][row]
-            xs_tab[(i & 1) * BM + r + 64 * (i >> 1)] = i32_to_f64((uint32_t)xs_cur[i]);
+            for (int i = 0; i < 4; ++i) {
+              const uint4 w = src[i];  // codes 32i .. 32i + 31
+              uint4 c0, c1;
+              unpack8(w.x, c0.x, c0.y);
+              unpack8(w.y, c0.z, c0.w);
+              unpack8(w.z, c1.x, c1.y);
+              unpack8(w.w, c1.z, c1.w);
+              *reinterpret_cast<uint4*>(dst + (((2 * i) ^ (rr & 7)) * 16)) = c0;
+              *reinterpret_cast<uint4*>(dst + (((2 * i + 1) ^ (rr & 7)) * 16)) = c1;
+            }
+          }
+          fence_proxy_async_smem();  // generic writes -> tensor-core reads
           __syncwarp();
-          if (lane == 0) mbar_arrive(tabfull_bar(ts));
+          if (lane == 0) mbar_arrive(ufull_bar(u));
+          // this K block's scales and offsets in fp64, for the fold warps
+          if (!kAccOut) {
+            if (!mbar_wait(tabempty_bar(ts), ((it / TSLOTS) & 1) ^ 1u, err)) {
+              ok = false;
+              break;
+            }
+            double2* tab = reinterpret_cast<double2*>(smem + SMEM_T + ts * T_BYTES);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                tab[j * BN + r + 64 * i] = make_double2(
+                    (double)__half2float(__ushort_as_half(so_cur[4 * i + 2 * j])),
+                    (double)__half2float(__ushort_as_half(so_cur[4 * i + 2 * j + 1])));
+            double* xs_tab = reinterpret_cast<double*>(smem + SMEM_T + ts * T_BYTES + T_SO);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)  // [group][row]
+              xs_tab[(i & 1) * BM + r + 64 * (i >> 1)] = i32_to_f64((uint32_t)xs_cur[i]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tabfull_bar(ts));
+          }
         }
       }
     }
   } else {
     // ---------------------------------------------------------------- fold
-    const int fw = warp - (2 + kUnpackWarps);  // 0..15
+    regs_inc<kRegsFold>();
+    const int fw = warp - (2 + kUnpackWarps);  // 0..7
     const int q = warp & 3;                     // TMEM lane quarter
     const int cpart = fw >> 2;                  // columns [kFoldCols cpart, + kFoldCols)
     uint8_t* stg_ptr = smem + SMEM_STG + fw * STG_BYTES;
@@ -350,28 +374,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const double2* tj = tab + j * BN + cpart * kFoldCols;
-          uint32_t v[kFoldCols];
+          // two 32-column halves keep the live registers down; the buffer goes
+          // back to the MMA issuer once the second half is loaded
 #pragma unroll
-          for (int h = 0; h < kFoldCols / kPiece; ++h)  // all pieces in flight, one wait
-            tmem_ld8(t_lane + (uint32_t)(b * BN + kPiece * h),
-                     *reinterpret_cast<uint32_t(*)[kPiece]>(&v[kPiece * h]));
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(b));
-          if constexpr (kAccOut) {
-            if (row >= m0 && row < m1) {
-#pragma unroll
-              for (int c = 0; c < kFoldCols; ++c) {
-                const int n = n0 + c;
-                if (n < N) acc_out[((size_t)(row - m0) * N + n) * G + g] = (int32_t)v[c];
-              }
+          for (int h = 0; h < 2; ++h) {
+            uint32_t v[32];
+            tmem_ld32(t_lane + (uint32_t)(b * BN + 32 * h), v);
+            tmem_ld_wait();
+            if (h == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty_bar(b));
             }
-          } else {
+            if constexpr (kAccOut) {
+              if (row >= m0 && row < m1) {
 #pragma unroll
-            for (int c = 0; c < kFoldCols; ++c) {
-              const double2 so = tj[c];
-              f[c] = fma(so.y, xs, fma(so.x, i32_to_f64(v[c]), f[c]));
+                for (int c = 0; c < 32; ++c) {
+                  const int n = n0 + 32 * h + c;
+                  if (n < N) acc_out[((size_t)(row - m0) * N + n) * G + g] = (int32_t)v[c];
+                }
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const double2 so = tj[32 * h + c];
+                f[32 * h + c] = fma(so.y, xs, fma(so.x, i32_to_f64(v[c]), f[32 * h + c]));
+              }
             }
           }
         }
@@ -395,10 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
-      uint4* rowp = reinterpret_cast<uint4*>(stg_ptr + lane * 2 * kFoldCols);
+      uint8_t* rowp = stg_ptr + lane * 2 * kFoldCols;  // 128-byte rows, 128-byte swizzle
 #pragma unroll
       for (int i = 0; i < kFoldCols / 8; ++i)
-        rowp[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+        *reinterpret_cast<uint4*>(rowp + 16 * (i ^ (lane & 7))) =
+            make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -434,7 +463,7 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
   if (acc_mode)
     tY = tA;  // unused by the accumulator dump
   else if (!encode_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
-                           (uint64_t)N * 2, kFoldCols, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+                           (uint64_t)N * 2, kFoldCols, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -443,6 +472,11 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SMEM_ALLOC);
     if (e != cudaSuccess) return e;
+    // the fold warpgroups' register increase is only satisfiable with the
+    // launch allocation the split was computed for
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
     g_attr_done[acc_mode][dev] = true;
   }
   int* err = device_error_word();
