@@ -46,7 +46,8 @@ constexpr int TSLOTS = 4;                 // scale/offset table slots (one per K
 constexpr int TBUFS = 4;                  // TMEM group accumulators
 constexpr int kUnpackWarps = 2;
 constexpr int kFoldWarps = 8;             // two per TMEM lane quarter
-constexpr int kFoldCols = BN / (kFoldWarps / 4);  // 64 columns per fold thread
+constexpr int kFoldCols = BN / (kFoldWarps / 4);  // columns per fold thread
+constexpr int kHalf = kFoldCols / 2;              // TMEM columns loaded at a time
 constexpr int kThreads = 32 * (2 + kUnpackWarps + kFoldWarps);  // 384: three warpgroups
 // Registers: the block is launched with kRegsLaunch per thread; warpgroup 0
 // (producer, MMA issuer, unpack) keeps kRegsCtl and hands the rest to the two
@@ -80,6 +81,7 @@ constexpr uint32_t kIdesc = i8_idesc(BM, BN, true, false);
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert(SMEM_U % 1024 == 0 && U_BYTES % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(2 * kFoldCols == 128, "the output stage is 128-byte rows with the 128-byte swizzle");
 static_assert(SMEM_STG % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled output stages too");
 
 __device__ __forceinline__ double i32_to_f64(uint32_t a) {
@@ -103,6 +105,10 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
   const uint32_t up = (low13 + 0x0FFFu + (keep & 1u)) >> 13;
   return sign | min(keep + up - (896u << 7), 0x7F80u);
 }
+
+// 32 lanes x 16 or 32 consecutive TMEM columns.
+__device__ __forceinline__ void tmem_ld_cols(uint32_t a, uint32_t (&v)[32]) { tmem_ld32(a, v); }
+__device__ __forceinline__ void tmem_ld_cols(uint32_t a, uint32_t (&v)[16]) { tmem_ld16(a, v); }
 
 // 8 packed codes (c0 = low nibble of byte 0) -> two words of 4 u8 codes.
 __device__ __forceinline__ void unpack8(uint32_t w, uint32_t& lo4, uint32_t& hi4) {
@@ -374,12 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const double2* tj = tab + j * BN + cpart * kFoldCols;
-          // two 32-column halves keep the live registers down; the buffer goes
-          // back to the MMA issuer once the second half is loaded
+          // two halves keep the live registers down; the buffer goes back to
+          // the MMA issuer once the second half is loaded
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            uint32_t v[32];
-            tmem_ld32(t_lane + (uint32_t)(b * BN + 32 * h), v);
+            uint32_t v[kHalf];
+            tmem_ld_cols(t_lane + (uint32_t)(b * BN + kHalf * h), v);
             tmem_ld_wait();
             if (h == 1) {
               tc_fence_before();
@@ -389,16 +395,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (kAccOut) {
               if (row >= m0 && row < m1) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                  const int n = n0 + 32 * h + c;
+                for (int c = 0; c < kHalf; ++c) {
+                  const int n = n0 + kHalf * h + c;
                   if (n < N) acc_out[((size_t)(row - m0) * N + n) * G + g] = (int32_t)v[c];
                 }
               }
             } else {
 #pragma unroll
-              for (int c = 0; c < 32; ++c) {
-                const double2 so = tj[32 * h + c];
-                f[32 * h + c] = fma(so.y, xs, fma(so.x, i32_to_f64(v[c]), f[32 * h + c]));
+              for (int c = 0; c < kHalf; ++c) {
+                const double2 so = tj[kHalf * h + c];
+                f[kHalf * h + c] = fma(so.y, xs, fma(so.x, i32_to_f64(v[c]), f[kHalf * h + c]));
               }
             }
           }
