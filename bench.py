@@ -43,6 +43,7 @@ L2_BYTES = 126 * 1024 * 1024
 
 WORKLOADS = {
     "dit_mlp": ("DIT_MLP", None),
+    "dit_mlp_gated": ("DIT_MLP", None),
     "dit_attn": ("DIT_ATTN", None),
     "sweep_4096x4096": ("SWEEP", 0),
     "sweep_4096x12288": ("SWEEP", 1),
@@ -66,6 +67,11 @@ def get_case(name):
 
 def is_w4(name):
     return name.startswith("w4a8")
+
+
+def is_gated(name):
+    """The W8A8 linear with the gated residual epilogue y = r + gate * linear."""
+    return name.endswith("_gated")
 
 
 # ------------------------------------------------------------ peaks / clocks
@@ -245,8 +251,17 @@ def run_ours(args, world, rank, local):
     case = get_case(args.workload)
     M, K, N = case.M, case.K, case.N
     w4 = is_w4(args.workload)
+    gated = is_gated(args.workload)
     xb, W, b, _ = case.draw()
     x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
+    if gated:
+        from w4a8_quantized_gemm_token_b200 import synthetic
+
+        gate_np, res_bits = synthetic.gated_inputs(case)
+        gate = torch.from_numpy(gate_np).to(dev)
+        res_host = torch.from_numpy(res_bits.view(np.int16)).view(torch.bfloat16)
+        res = res_host.to(dev)
+        del res_bits
     W_dev = torch.from_numpy(W).to(dev)
     bias = torch.from_numpy(b).to(dev) if b is not None else None
 
@@ -267,6 +282,8 @@ def run_ours(args, world, rank, local):
         wt = weights[i % nsets]
         if w4:
             qk.qk_w4a8_linear(xs[i % nsets], *wt, bias, y=y, workspace=ws)
+        elif gated:
+            qk.qk_w8a8_linear_gated(xs[i % nsets], *wt, bias, gate, res, y=y, workspace=ws)
         else:
             qk.qk_w8a8_linear(xs[i % nsets], *wt, bias, y=y, workspace=ws)
 
@@ -304,6 +321,8 @@ def run_ours(args, world, rank, local):
         def kstep(i):
             xq, sx, xsum = xq_sets[i % nsets]
             qk.qk_w4a8_gemm(xq, sx, xsum, *weights[i % nsets], bias, y=y, route=route)
+    elif gated:
+        kstep = step  # no gated entry on pre-quantized activations: the call (quant + GEMM)
     else:
         xq_sets = [qk.qk_quantize_activations(x) for x in xs]
 
@@ -351,6 +370,9 @@ def run_ours(args, world, rank, local):
                 "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2, the nominal int8/bf16 "
                                "ratio (4.5 / 2.25 POPS); int8 ops counted as 2*M*N*K",
                 "kernel": tag, "traffic": traffic_from_profile(tag, src)}
+        if gated:
+            roof["kernel"] = "w8a8_gemm_kernel (gated) with its activation quant: the timed call"
+            roof["traffic"] = None  # the committed summary covers the plain epilogue
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel_ms"] = k_ms
 
@@ -362,11 +384,17 @@ def run_ours(args, world, rank, local):
         x_dev = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
         n_e2e = max(3, min(args.steps, args.e2e_steps))
 
+        if gated:
+            r_pin = res_host.pin_memory()
+
         def e2e_step(i):
             x_dev.copy_(x_pin, non_blocking=True)
             wt = weights[i % nsets]
             if w4:
                 qk.qk_w4a8_linear(x_dev, *wt, bias, y=y, workspace=ws)
+            elif gated:
+                res.copy_(r_pin, non_blocking=True)
+                qk.qk_w8a8_linear_gated(x_dev, *wt, bias, gate, res, y=y, workspace=ws)
             else:
                 qk.qk_w8a8_linear(x_dev, *wt, bias, y=y, workspace=ws)
             y_pin.copy_(y, non_blocking=True)
@@ -383,12 +411,13 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         e_ms = reduce_max(a0.elapsed_time(a1), dev)
         e2e = {"value": whole_job_value(ops, n_e2e, world, e_ms / 1e3), "unit": "TOPS",
-               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+               "h2d_bytes_per_step": M * K * 2 + (M * N * 2 if gated else 0),
+               "d2h_bytes_per_step": M * N * 2,
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(case, seconds=args.cpu_seconds)
+        cpu = cpu_baseline(case, seconds=args.cpu_seconds, gated=gated)
 
     clocks = sampler.summary()
     if rank == 0:
@@ -397,7 +426,8 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8", "data": "synthetic",
-            "config": {"workload": case.name, "M": M, "K": K, "N": N,
+            "config": {"workload": case.name + ("_gated_residual" if gated else ""),
+                       "M": M, "K": K, "N": N,
                        "weights": "W4 affine g64" if w4 else "W8 per-channel",
                        "bias": bias is not None,
                        "activations": "bf16 N(0,1)" + (", 1% channels x20" if case.outlier_frac else ""),
@@ -418,14 +448,17 @@ class OracleSample:
     """Inputs for bounded oracle samples of a workload (same recipe as the GPU
     arm; only the first rows of x are drawn, since a sample never uses more)."""
 
-    def __init__(self, case, w4, max_rows=1024):
+    def __init__(self, case, w4, max_rows=1024, gated=False):
         import dataclasses
 
         import oracle
+        from w4a8_quantized_gemm_token_b200 import synthetic
 
-        self.case, self.w4 = case, w4
+        self.case, self.w4, self.gated = case, w4, gated
         small = dataclasses.replace(case, M=min(case.M, max_rows))
         self.xb, W, self.b, _ = small.draw()
+        if gated:
+            self.gate, self.res = synthetic.gated_inputs(case, rows=small.M)
         if w4:
             self.Wp, self.s16, self.o16 = oracle.quant_w4(W)
         else:
@@ -442,6 +475,10 @@ class OracleSample:
             xsum = oracle.group_sums(xq)
             acc = oracle.w4a8_group_acc(xq, self.Wp[:ncols])
             oracle.w4a8_dequant(acc, xsum, sx, self.s16[:ncols], self.o16[:ncols], None)
+        elif self.gated:
+            acc = oracle.w8a8_acc(xq, self.Wq[:ncols])
+            oracle.w8a8_gated(acc, sx, self.sw[:ncols], None if self.b is None else self.b[:ncols],
+                              self.gate[:ncols], self.res[:rows, :ncols])
         else:
             acc = oracle.w8a8_acc(xq, self.Wq[:ncols])
             oracle.w8a8_dequant(acc, sx, self.sw[:ncols],
@@ -449,9 +486,9 @@ class OracleSample:
         return time.perf_counter() - t0, 2.0 * rows * ncols * self.case.K
 
 
-def cpu_baseline(case, seconds=10.0):
+def cpu_baseline(case, seconds=10.0, gated=False):
     """The oracle on the host cores over a bounded sample of the same workload."""
-    smp = OracleSample(case, case.name.startswith("w4a8"))
+    smp = OracleSample(case, case.name.startswith("w4a8"), gated=gated)
     dt, _ = smp.run(1, case.N)          # calibrate on one row
     rows = int(max(1, min(smp.xb.shape[0], seconds / max(dt, 1e-6))))
     dt, ops = smp.run(rows, case.N)
@@ -465,7 +502,7 @@ def run_reference(args, world, rank, local):
     if rank != 0:
         return  # rank 0 alone runs the oracle
     case = get_case(args.workload)
-    smp = OracleSample(case, is_w4(args.workload), max_rows=8)
+    smp = OracleSample(case, is_w4(args.workload), max_rows=8, gated=is_gated(args.workload))
     # size each step so that warm-up + timed steps take about `budget` seconds
     budget = args.ref_seconds
     dt1, _ = smp.run(1, case.N)
@@ -486,7 +523,8 @@ def run_reference(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": case.name, "M": case.M, "K": case.K, "N": case.N},
+        "config": {"workload": case.name + ("_gated_residual" if is_gated(args.workload) else ""),
+                   "M": case.M, "K": case.K, "N": case.N},
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -12,6 +12,11 @@ this draw order):
 2. W: float64 normals times ``w_std`` of shape [N, K], cast to float32.
 3. bias (when requested): float64 normals times ``b_std`` of shape [N], float32.
 
+Gated residual epilogue inputs (``gated_inputs``), from their own generator
+``default_rng(seed + 1)``: the gate, float64 normals times 0.5 of shape [N]
+with every 7th channel set to 0 (closed), cast to float32; then the residual
+rows, float64 normals of shape [rows, N] cast to float32 and rounded to bf16.
+
 bf16 arrays are returned as numpy uint16 bit patterns.
 """
 from __future__ import annotations
@@ -63,6 +68,21 @@ class LinearCase:
         if self.bias:
             b = (rng.standard_normal(self.N) * self.b_std).astype(np.float32)
         return x_bf16, W, b, chans
+
+
+def gated_inputs(case: LinearCase, rows: int | None = None):
+    """(gate float32 [N], residual bf16 bits [rows, N]) for the gated residual
+    epilogue of `case` (first `rows` rows of the residual; all M by default)."""
+    rng = np.random.default_rng(case.seed + 1)
+    gate = rng.standard_normal(case.N) * 0.5
+    gate[::7] = 0.0
+    rows = case.M if rows is None else rows
+    res = np.empty((rows, case.N), np.uint16)
+    step = max(1, (1 << 24) // max(case.N, 1))  # bounded host memory per block
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        res[r0:r1] = f32_to_bf16_bits(rng.standard_normal((r1 - r0, case.N)).astype(np.float32))
+    return gate.astype(np.float32), res
 
 
 # The five workloads of the quantized linear, at DiT layer shapes.
