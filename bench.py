@@ -54,6 +54,8 @@ WORKLOADS = {
     "w4a8_m8": ("W4A8", 1),
     "w4a8_m16": ("W4A8", 2),
     "w4a8_m4096": ("W4A8", 3),
+    "quickstart_w8a8": ("QUICKSTART", 0),
+    "quickstart_w4a8": ("QUICKSTART", 1),
 }
 
 
@@ -66,7 +68,7 @@ def get_case(name):
 
 
 def is_w4(name):
-    return name.startswith("w4a8")
+    return "w4a8" in name
 
 
 def is_gated(name):
@@ -488,7 +490,7 @@ class OracleSample:
 
 def cpu_baseline(case, seconds=10.0, gated=False):
     """The oracle on the host cores over a bounded sample of the same workload."""
-    smp = OracleSample(case, case.name.startswith("w4a8"), gated=gated)
+    smp = OracleSample(case, "w4a8" in case.name, gated=gated)
     dt, _ = smp.run(1, case.N)          # calibrate on one row
     rows = int(max(1, min(smp.xb.shape[0], seconds / max(dt, 1e-6))))
     dt, ops = smp.run(rows, case.N)

@@ -106,10 +106,14 @@ def test_gemm_group_acc_and_output(qk, orc, MKN):
     qk.qk_check_device_error()
 
 
-def test_w4a8_gemm_config_4096(qk, orc):
-    """The M = 4096 W4A8 workload: every code bit-exact, per-group sums and
+@pytest.mark.parametrize("case, blocks", [
+    (synthetic.W4A8[3], [(0, 4), (126, 130), (2047, 2051), (4092, 4096)]),
+    # the README's quick-start matmul: ragged M (14040 = 109 tiles of 128 + 88)
+    (synthetic.QUICKSTART[1], [(0, 4), (126, 130), (7040, 7044), (13950, 13954), (14036, 14040)]),
+], ids=lambda v: v.name if hasattr(v, "name") else "")
+def test_w4a8_gemm_config(qk, orc, case, blocks):
+    """A large-M W4A8 workload: every code bit-exact, per-group sums and
     outputs of sampled row blocks (first, last, tile edges) against the oracle."""
-    case = synthetic.W4A8[3]
     xb, dev_w, ora_w, _ = prepare(qk, orc, case)
     x = to_dev_bf16(xb)
     y = qk.qk_w4a8_linear(x, *dev_w)
@@ -118,7 +122,7 @@ def test_w4a8_gemm_config_4096(qk, orc):
     xq_o, sx_o = orc.quant_act(xb)
     assert np.array_equal(host(xq), xq_o) and np.array_equal(host(sx), sx_o)
     worst = 0
-    for m0, m1 in [(0, 4), (126, 130), (2047, 2051), (4092, 4096)]:
+    for m0, m1 in blocks:
         acc = qk.qk_debug_w4a8_group_acc(xq, dev_w[0], m0, m1, GEMM)
         torch.cuda.synchronize()
         acc_o = orc.w4a8_group_acc(xq_o[m0:m1], ora_w[0])

@@ -63,13 +63,14 @@ def test_w8a8_small_full_parity(qk, orc, MKN, with_bias):
 
 
 @pytest.mark.parametrize("case", [synthetic.TINY, synthetic.DIT_ATTN, *synthetic.SWEEP,
-                                  synthetic.DIT_MLP], ids=lambda c: c.name)
+                                  synthetic.DIT_MLP, synthetic.QUICKSTART[0]],
+                         ids=lambda c: c.name)
 def test_w8a8_configs(qk, orc, case):
     """Every DiT config at full size: all codes bit-exact, accumulators and
     outputs of sampled rows against the oracle."""
     xb, Wq, sw, Wq_o, sw_o, b = prepare(qk, orc, case)
     x = to_dev_bf16(xb)
-    bias = to_dev(b)
+    bias = to_dev(b) if b is not None else None
     ws = torch.empty(qk.qk_w8a8_workspace_size(case.M, case.K), dtype=torch.uint8, device="cuda")
     y = qk.qk_w8a8_linear(x, Wq, sw, bias, workspace=ws)
     xq, sx, _ = qk.qk_quantize_activations(x)

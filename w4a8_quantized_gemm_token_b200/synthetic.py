@@ -100,4 +100,9 @@ DIT_MLP = LinearCase("dit_mlp_w8a8_16384x3072x12288", M=16384, K=3072, N=12288,
 W4A8 = [LinearCase(f"w4a8_g64_{m}x4096x4096", M=m, K=4096, N=4096, bias=False)
         for m in (1, 8, 16, 4096)]
 
+# The quick-start matmul of the qlip-mlx README ("Quick start": 14040 tokens x
+# 5120 @ 5120 x 5120, bf16 vs W8A8 vs W4A8 on bare tensors, no bias).
+QUICKSTART = [LinearCase("quickstart_w8a8_14040x5120x5120", M=14040, K=5120, N=5120, bias=False),
+              LinearCase("quickstart_w4a8_14040x5120x5120", M=14040, K=5120, N=5120, bias=False)]
+
 ALL_W8A8 = [TINY, DIT_ATTN, *SWEEP, DIT_MLP]
