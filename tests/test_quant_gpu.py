@@ -13,7 +13,11 @@ from w4a8_quantized_gemm_token_b200 import synthetic
 pytestmark = pytest.mark.gpu
 
 MS = [1, 2, 3, 15, 16, 17, 63, 64, 65, 129]
-KS = [32, 64, 96, 160, 3072, 4096, 5120, 6144, 8192, 12288]
+# one warp per row (K <= 2048), then 2, 4 or 8 warps per row with 5..8 chunks
+# per thread (2112 .. 16384, including K % 64 != 0 without group sums), then
+# the two-pass kernel (20480)
+KS = [32, 64, 96, 160, 2048, 2112, 3072, 3104, 3584, 4096, 5120, 6144, 7168, 8192, 10240,
+      12288, 16384, 20480]
 
 
 @pytest.mark.parametrize("K", KS)

@@ -47,11 +47,17 @@ __device__ __forceinline__ uint2 quant_chunk(uint4 c, float r, int* sum) {
   return make_uint2(out[0], out[1]);
 }
 
-__device__ __forceinline__ float warp_max_bits_to_float(uint32_t bits2) {
+// Warp-wide max of two packed |bf16| bit patterns per lane: the bf16 bits of
+// the absmax (as an integer that orders like the value).
+__device__ __forceinline__ uint32_t warp_max_bits(uint32_t bits2) {
   uint32_t m = max(bits2 & 0xFFFFu, bits2 >> 16);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  return __uint_as_float(m << 16);
+  return m;
+}
+
+__device__ __forceinline__ float warp_max_bits_to_float(uint32_t bits2) {
+  return __uint_as_float(warp_max_bits(bits2) << 16);
 }
 
 // Sum over the 8 lanes that hold one group of 64 codes.

@@ -103,6 +103,62 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 }
 
 // W8: one warp per output channel, fp32 input, two passes (offline op).
+// Long rows: WPR warps share a row (8 / WPR rows per 256-thread block), each
+// thread holding CPT 16-byte chunks (chunk c = i * 32 WPR + thread-in-row) in
+// registers; the row's absmax is combined across its warps through shared
+// memory.  More, lighter warps per SM keep more loads in flight than one warp
+// per row holding the whole row.
+template <int WPR, int CPT>
+__global__ void __launch_bounds__(256) quant_act_split_kernel(const uint16_t* __restrict__ x, int M,
+                                                              int K, int8_t* __restrict__ xq,
+                                                              float* __restrict__ sx,
+                                                              int32_t* __restrict__ xsum) {
+  pdl_launch_dependents();
+  pdl_wait();
+  constexpr int T = 32 * WPR;  // threads per row
+  __shared__ uint32_t red[kQuantWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (kQuantWarps / WPR) + warp / WPR;
+  const int t = (warp % WPR) * 32 + lane;
+  const bool live = row < M;
+  const int nch = K >> 3;
+  const int G = K >> 6;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(live ? row : 0) * K);
+  uint2* dst = reinterpret_cast<uint2*>(xq + (size_t)(live ? row : 0) * K);
+  uint4 v[CPT];
+  uint32_t mb = 0;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = i * T + t;
+    if (live && c < nch) {
+      v[i] = __ldcs(src + c);
+      mb = bf16x2_absmax_bits(mb, v[i].x);
+      mb = bf16x2_absmax_bits(mb, v[i].y);
+      mb = bf16x2_absmax_bits(mb, v[i].z);
+      mb = bf16x2_absmax_bits(mb, v[i].w);
+    }
+  }
+  uint32_t m = warp_max_bits(mb);
+  if (lane == 0) red[warp] = m;
+  __syncthreads();  // every thread of the block reaches it (no early return above)
+#pragma unroll
+  for (int w = 0; w < WPR; ++w) m = max(m, red[(warp / WPR) * WPR + w]);
+  if (!live) return;
+  const float amax = __uint_as_float(m << 16);
+  const float r = act_multiplier(amax);
+  if (t == 0) sx[row] = act_scale(amax);
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = i * T + t;
+    int s = 0;
+    if (c < nch) dst[c] = quant_chunk(v[i], r, &s);
+    if (xsum != nullptr && i * T < nch) {  // warp-uniform
+      s = group8_sum(s);
+      if ((lane & 7) == 0 && c < nch) xsum[(size_t)row * G + (c >> 3)] = s;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) quant_w8_kernel(const float* __restrict__ W, int N, int K,
                                                        int8_t* __restrict__ Wq,
                                                        float* __restrict__ sw) {
@@ -189,19 +245,53 @@ __global__ void __launch_bounds__(256) quant_w4_kernel(const float* __restrict__
 cudaError_t launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* sx,
                              int32_t* xsum, cudaStream_t s, bool pdl) {
   const int m = (int)M, k = (int)K;
-  const int per_lane = (int)((K / 8 + 31) / 32);  // 16-byte chunks per lane
-  auto kernel = per_lane <= 1    ? quant_act_kernel<1>
-                : per_lane <= 2  ? quant_act_kernel<2>
-                : per_lane <= 4  ? quant_act_kernel<4>
-                : per_lane <= 8  ? quant_act_kernel<8>
-                : per_lane <= 12 ? quant_act_kernel<12>
-                : per_lane <= 16 ? quant_act_kernel<16>
-                : per_lane <= 20 ? quant_act_kernel<20>
-                : per_lane <= 24 ? quant_act_kernel<24>
-                : per_lane <= 32 ? quant_act_kernel<32>
-                                 : quant_act_kernel<0>;
+  const int nch = (int)(K / 8);                    // 16-byte chunks per row
+  const int per_lane = (nch + 31) / 32;            // ... per lane of one warp
+  using Kern = void (*)(const uint16_t*, int, int, int8_t*, float*, int32_t*);
+  Kern kernel = nullptr;
+  int rows_per_block = kQuantWarps;
+  // rows of up to 8 chunks per lane: one warp per row; longer rows: 2, 4 or 8
+  // warps per row with at most 8 chunks per thread; beyond 16384 elements,
+  // one warp per row reading the row twice
+  auto split = [&](int wpr) -> Kern {
+    const int cpt = (nch + 32 * wpr - 1) / (32 * wpr);
+    rows_per_block = kQuantWarps / wpr;
+    switch (wpr * 16 + cpt) {
+      case 2 * 16 + 5: return quant_act_split_kernel<2, 5>;
+      case 2 * 16 + 6: return quant_act_split_kernel<2, 6>;
+      case 2 * 16 + 7: return quant_act_split_kernel<2, 7>;
+      case 2 * 16 + 8: return quant_act_split_kernel<2, 8>;
+      case 4 * 16 + 5: return quant_act_split_kernel<4, 5>;
+      case 4 * 16 + 6: return quant_act_split_kernel<4, 6>;
+      case 4 * 16 + 7: return quant_act_split_kernel<4, 7>;
+      case 4 * 16 + 8: return quant_act_split_kernel<4, 8>;
+      case 8 * 16 + 5: return quant_act_split_kernel<8, 5>;
+      case 8 * 16 + 6: return quant_act_split_kernel<8, 6>;
+      case 8 * 16 + 7: return quant_act_split_kernel<8, 7>;
+      case 8 * 16 + 8: return quant_act_split_kernel<8, 8>;
+      default: return nullptr;
+    }
+  };
+  if (per_lane <= 1)
+    kernel = quant_act_kernel<1>;
+  else if (per_lane <= 2)
+    kernel = quant_act_kernel<2>;
+  else if (per_lane <= 4)
+    kernel = quant_act_kernel<4>;
+  else if (per_lane <= 8)
+    kernel = quant_act_kernel<8>;
+  else if (per_lane <= 16)
+    kernel = split(2);
+  else if (per_lane <= 32)
+    kernel = split(4);
+  else if (per_lane <= 64)
+    kernel = split(8);
+  if (kernel == nullptr) {
+    kernel = quant_act_kernel<0>;
+    rows_per_block = kQuantWarps;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((M + kQuantWarps - 1) / kQuantWarps));
+  cfg.gridDim = dim3((unsigned)((M + rows_per_block - 1) / rows_per_block));
   cfg.blockDim = dim3(256);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
