@@ -160,7 +160,9 @@ qk_status qk_quantize_activations(const uint16_t *x, int64_t M, int64_t K,
  *   y         : bf16 bits [M, N]   (out)
  *   workspace : device scratch of ws_bytes >= qk_w8a8_workspace_size(M, K),
  *               or NULL: the call then allocates it stream-ordered
- *               (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *               (cudaMallocAsync / cudaFreeAsync on `stream`).  Two calls
+ *               that may run at the same time need separate workspaces; the
+ *               codes and scales of x are left in it.
  */
 qk_status qk_w8a8_linear(const uint16_t *x, int64_t M, int64_t K,
                          const int8_t *Wq, const float *sw, const float *bias, int64_t N,

@@ -101,12 +101,18 @@ def test_w8a8_deterministic_and_api_variants(qk, orc):
     xq, sx, _ = qk.qk_quantize_activations(x)
     y3 = qk.qk_w8a8_gemm(xq, sx, Wq, sw, bias)                    # split API
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())  # the same workspace: not concurrently
     with torch.cuda.stream(s):
         y4 = qk.qk_w8a8_linear(x, Wq, sw, bias, workspace=ws)     # another stream
     s.synchronize()
     torch.cuda.synchronize()
     for y in (y2, y3, y4):
         assert torch.equal(y1.view(torch.int16), y.view(torch.int16))
+    # the one-kernel route leaves the activation codes and scales in the workspace
+    wq = ws[: 777 * 1024].view(torch.int8).view(777, 1024)
+    off = (777 * 1024 + 255) // 256 * 256
+    wsx = ws[off: off + 777 * 4].view(torch.float32)
+    assert torch.equal(wq, xq) and torch.equal(wsx.view(torch.int32), sx.view(torch.int32))
 
 
 @pytest.mark.parametrize("MKN", [(200, 256, 264), (200, 1024, 40)], ids=["tiles", "splitk"])
