@@ -281,6 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t aphase = 0;
     int iter = 0;
     int use = 0;  // staging-buffer use counter (alternates the two buffers)
+    const uint64_t y_policy = l2_policy_evict_first();
     // gated: each lane sends its row of a tile's residual (up to 512 bytes) to
     // L2 one tile ahead of the tile's epilogue, so the per-chunk register loads
     // below meet L2 rather than HBM latency
@@ -463,7 +464,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmC, stg0 + (uint32_t)(buf * STG_BYTES), n0, row0);
+          // y is written once and never read here: evict it first from L2
+          tma_store_2d_hint(&tmC, stg0 + (uint32_t)(buf * STG_BYTES), n0, row0, y_policy);
           bulk_commit();
         }
         ++use;
