@@ -322,6 +322,17 @@ qk_status qk_debug_w4a8_group_acc(const int8_t *xq, int64_t M, int64_t K,
                                   int64_t m0, int64_t m1, int32_t *acc,
                                   int route, qk_stream_t stream);
 
+/*
+ * The timeout path of the library's bounded waits, for tests: launches one
+ * single-thread kernel that waits on an mbarrier no thread arrives at and on
+ * a device word no thread sets.  Each wait gives up after limit_cycles SM
+ * clock cycles (1 <= limit_cycles <= 2^31), records QK_ERR_TIMEOUT in the
+ * device error word and the kernel returns; qk_check_device_error then
+ * returns QK_ERR_TIMEOUT once, and the context stays usable.  Nothing traps.
+ * Returns QK_ERR_INVALID_ARG for a limit out of range.
+ */
+qk_status qk_debug_wait_timeout(int64_t limit_cycles, qk_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

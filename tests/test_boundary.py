@@ -88,6 +88,9 @@ def test_routes_are_checked(qk):
     assert qk.lib.qk_w4a8_gemm(*args, 2, None) == 1        # GEMV with M > 16
     assert qk.lib.qk_w4a8_gemm(*args, 7, None) == 1        # unknown route
     assert qk.lib.qk_debug_w4a8_group_acc(FAKE, 8, 256, FAKE, 64, 4, 2, FAKE, 1, None) == 1
+    # the timeout test hook checks its limit on the host
+    assert qk.lib.qk_debug_wait_timeout(0, None) == 1
+    assert qk.lib.qk_debug_wait_timeout((1 << 31) + 1, None) == 1
 
 
 def test_no_device_here(qk):
@@ -99,6 +102,7 @@ def test_no_device_here(qk):
     # valid arguments reach the device check and stop there, launching nothing
     assert call_w8a8(qk) == 4
     assert qk.lib.qk_quantize_weights_int8(FAKE, 128, 256, FAKE, FAKE, None) == 4
+    assert qk.lib.qk_debug_wait_timeout(1000, None) == 4
 
 
 def test_binding_rejects_cpu_tensors(qk):

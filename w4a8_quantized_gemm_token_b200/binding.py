@@ -41,6 +41,7 @@ _SIGS = {
     "qk_check_device_error": (_I, [_P]),
     "qk_debug_w8a8_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P]),
     "qk_debug_w4a8_group_acc": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I, _P]),
+    "qk_debug_wait_timeout": (_I, [_I64, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -280,3 +281,10 @@ def qk_debug_w4a8_group_acc(xq, Wp, m0, m1, route, acc=None, stream=None):
     _check(lib.qk_debug_w4a8_group_acc(_ptr(xq), M, K, _ptr(Wp), N, m0, m1, _ptr(acc), int(route),
                                        _stream(stream)), "qk_debug_w4a8_group_acc")
     return acc
+
+
+def qk_debug_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Launch the test kernel whose waits can never complete; each gives up
+    after `limit_cycles` SM cycles and records QK_ERR_TIMEOUT for
+    qk_check_device_error."""
+    _check(lib.qk_debug_wait_timeout(int(limit_cycles), _stream(stream)), "qk_debug_wait_timeout")

@@ -398,6 +398,13 @@ qk_status qk_check_device_error(qk_stream_t stream) {
   return QK_OK;
 }
 
+qk_status qk_debug_wait_timeout(int64_t limit_cycles, qk_stream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 31)) return QK_ERR_INVALID_ARG;
+  qk_status st = check_device();
+  if (st != QK_OK) return st;
+  return from_cuda(launch_wait_timeout_probe((long long)limit_cycles, stream), "wait_timeout_probe");
+}
+
 qk_status qk_debug_w8a8_acc(const int8_t* xq, int64_t M, int64_t K, const int8_t* Wq, int64_t N,
                             int32_t* acc, qk_stream_t stream) {
   qk_status st = check_shape(M, K, N, false);

@@ -41,6 +41,10 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
 // tiles split along K over a cluster, exact int32 partial sums reduced through
 // distributed shared memory.  launch_w8a8_gemm routes such shapes here.
 bool w8a8_use_skinny(int64_t M, int64_t K, int64_t N);
+
+// Test hook: one kernel whose two waits can never complete, each bounded by
+// `limit_cycles`; both record QK_ERR_TIMEOUT (debug_wait.cu).
+cudaError_t launch_wait_timeout_probe(long long limit_cycles, cudaStream_t s);
 cudaError_t launch_w8a8_skinny(const int8_t* xq, const float* sx, int64_t M, int64_t K,
                                const int8_t* Wq, const float* sw, const float* bias, int64_t N,
                                uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s,

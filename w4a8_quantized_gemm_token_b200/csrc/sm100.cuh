@@ -69,16 +69,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Waits until the phase with the given parity has completed.  Returns false
 // (and records a timeout) if that takes longer than QK_WAIT_LIMIT_CYCLES.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, int* err,
+                                                long long limit_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > QK_WAIT_LIMIT_CYCLES) {
+    if (clock64() - t0 > limit_cycles) {
       record_timeout(err);
       return false;
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+  return mbar_wait_limit(bar, parity, err, QK_WAIT_LIMIT_CYCLES);
 }
 
 // ---------------------------------------------------------------- TMA copies
