@@ -56,6 +56,7 @@ def _bind(path: str):
         "oracle_w4a8_dequant": (None, [P, P, I64, I64, I64, P, P, P, P, P]),
         "oracle_w8a8_dequant_f64": (None, [P, I64, I64, P, P, P, P]),
         "oracle_w4a8_dequant_f64": (None, [P, P, I64, I64, I64, P, P, P, P, P]),
+        "oracle_sage_attention": (None, [P, P, P, P, P, I64, I64, ctypes.c_double, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -281,3 +282,37 @@ def w4a8_linear(x_bf16, Wp, s16, o16, bias=None):
     xsum = group_sums(xq)
     acc_g = w4a8_group_acc(xq, Wp)
     return w4a8_dequant(acc_g, xsum, sx, s16, o16, bias), xq, sx, xsum, acc_g
+
+
+def sage_attention_head(q_bf16, k_bf16, v_bf16, scale, with_f64=False):
+    """INT8 attention of one head ("qlip-mlx" README, "sage_attention"; R14):
+    q, k, v bf16 bits [L, D].  q and k are quantized per token (quant_act),
+    scores and softmax and P V in fp64, the output rounded once to bf16.
+    Returns bf16 bits [L, D] (and the fp64 output when `with_f64`)."""
+    q = _c(q_bf16, np.uint16)
+    k = _c(k_bf16, np.uint16)
+    v = _c(v_bf16, np.uint16)
+    L, D = q.shape
+    assert k.shape == (L, D) and v.shape == (L, D)
+    qc, sq = quant_act(q)
+    kc, sk = quant_act(k)
+    out = np.empty((L, D), np.uint16)
+    o64 = np.empty((L, D), np.float64) if with_f64 else None
+    _load().oracle_sage_attention(_p(qc), _p(sq), _p(kc), _p(sk), _p(v), L, D, float(scale),
+                                  _p(o64) if with_f64 else None, _p(out))
+    return (out, o64) if with_f64 else out
+
+
+def sage_attention(q_bf16, k_bf16, v_bf16, scale, with_f64=False):
+    """sage_attention_head over [B, H, L, D] bf16 bits, head by head."""
+    B, H, L, D = q_bf16.shape
+    out = np.empty((B, H, L, D), np.uint16)
+    o64 = np.empty((B, H, L, D), np.float64) if with_f64 else None
+    for b in range(B):
+        for h in range(H):
+            r = sage_attention_head(q_bf16[b, h], k_bf16[b, h], v_bf16[b, h], scale, with_f64)
+            if with_f64:
+                out[b, h], o64[b, h] = r
+            else:
+                out[b, h] = r
+    return (out, o64) if with_f64 else out

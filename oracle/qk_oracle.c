@@ -25,6 +25,10 @@
  *          "SIMD fix" bullet: x is quantized to int8 by its own kernel.
  *   [kquant89] "mlx-kquant PR #89", commit list: a quantized matmul with a
  *          gated residual epilogue, each element held within 2 ulp.
+ *   [qlip-sage] "qlip-mlx" README, intro bullet "sage_attention" and the
+ *          "Exact where it matters" bullet: INT8 Q K^T inside a flash-attention
+ *          structure, exact online softmax, per-token / per-block scales, and
+ *          softmax and P V kept in floating point; head dim 128, no mask.
  *
  * Readings taken where the pages are silent (each is stated where it is used):
  *   R1  codes are rne(x * r) with r = 127 / absmax (one fp32 division per row,
@@ -41,6 +45,10 @@
  *   R13 the gated residual epilogue is out = r + g[n] * (linear output before
  *       rounding), r a bf16 [M, N] residual, g one fp32 gate per output channel
  *       (one sample's adaLN gate of a DiT block).
+ *   R14 INT8 attention: q and k rows (tokens) are quantized per token by the
+ *       activation rule (R1-R3); scores s[i, j] = (q_i . k_j exact) * sq[i] *
+ *       sk[j] * scale; softmax over all keys (no mask); o_i = sum_j p_ij v_j
+ *       (v bf16); the exact result is rounded once to bf16.  No smoothing of k.
  *   dequant is evaluated in fp64 and rounded once to bf16 (nearest, ties even).
  */
 #include <stdint.h>
@@ -378,4 +386,48 @@ void oracle_w4a8_dequant(const int64_t *acc, const int32_t *xsum,
                                     bias ? bias + n : NULL, &v);
             y[m * N + n] = oracle_f64_to_bf16(v);
         }
+}
+
+/*
+ * INT8 attention of one head [qlip-sage], (R14), for L queries and L keys of
+ * head dim D: q and k are given as their per-token codes and scales (from
+ * oracle_quant_act_bf16), v as bf16 bits [L, D].  Everything after the integer
+ * dot products is fp64: s = dot * sq[i] * sk[j] * scale, p = exp(s - max_j s),
+ * o = (sum_j p v_j) / (sum_j p).  out_f64 (nullable) receives o before the
+ * rounding; out receives it rounded to bf16.
+ */
+void oracle_sage_attention(const int8_t *qc, const float *sq, const int8_t *kc,
+                           const float *sk, const uint16_t *v, int64_t L, int64_t D,
+                           double scale, double *out_f64, uint16_t *out)
+{
+    double *s = (double *)malloc((size_t)L * sizeof(double));
+    double *o = (double *)malloc((size_t)D * sizeof(double));
+    for (int64_t i = 0; i < L; ++i) {
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < L; ++j) {
+            int64_t dot = 0;
+            for (int64_t d = 0; d < D; ++d)
+                dot += (int64_t)qc[i * D + d] * (int64_t)kc[j * D + d];
+            s[j] = (double)dot * (double)sq[i] * (double)sk[j] * scale;
+            if (s[j] > mx)
+                mx = s[j];
+        }
+        double l = 0.0;
+        for (int64_t d = 0; d < D; ++d)
+            o[d] = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+            double p = exp(s[j] - mx);
+            l += p;
+            for (int64_t d = 0; d < D; ++d)
+                o[d] += p * (double)oracle_bf16_to_f32(v[j * D + d]);
+        }
+        for (int64_t d = 0; d < D; ++d) {
+            double r = o[d] / l;
+            if (out_f64)
+                out_f64[i * D + d] = r;
+            out[i * D + d] = oracle_f64_to_bf16(r);
+        }
+    }
+    free(s);
+    free(o);
 }

@@ -33,6 +33,15 @@ MUTANTS = [
      "double t = (double)gate[n] * (v - (bias ? (double)bias[n] : 0.0)) + (bias ? (double)bias[n] : 0.0);"),
     ("group_sum_window", "for (int64_t k = 64 * g; k < 64 * g + 64; ++k)\n                s += xq[m * K + k];",
      "for (int64_t k = 64 * g; k < 64 * g + 63; ++k)\n                s += xq[m * K + k];"),
+    ("sage_scale_dropped", "s[j] = (double)dot * (double)sq[i] * (double)sk[j] * scale;",
+     "s[j] = (double)dot * (double)sq[i] * (double)sk[j];"),
+    ("sage_key_scale_of_query", "s[j] = (double)dot * (double)sq[i] * (double)sk[j] * scale;",
+     "s[j] = (double)dot * (double)sq[i] * (double)sk[i] * scale;"),
+    ("sage_key_index_is_query", "dot += (int64_t)qc[i * D + d] * (int64_t)kc[j * D + d];",
+     "dot += (int64_t)qc[i * D + d] * (int64_t)kc[i * D + d];"),
+    ("sage_value_transposed", "o[d] += p * (double)oracle_bf16_to_f32(v[j * D + d]);",
+     "o[d] += p * (double)oracle_bf16_to_f32(v[d * L + j]);"),
+    ("sage_normalizer_dropped", "double r = o[d] / l;", "double r = o[d];"),
 ]
 
 

@@ -431,3 +431,72 @@ def test_w8a8_gated_brute_force(orc):
     want = orc.f64_to_bf16_array(brute)
     assert np.abs(ordinal(out) - ordinal(want)).max() <= 1
     assert np.mean(out == want) > 0.95
+
+
+# ------------------------------------------------- INT8 attention (R14)
+
+def _qkv(L, D, seed, scale_q=1.0):
+    rng = np.random.default_rng(seed)
+    q = bf16_bits(rng.normal(size=(L, D)) * scale_q)
+    k = bf16_bits(rng.normal(size=(L, D)))
+    v = bf16_bits(rng.normal(size=(L, D)))
+    return q, k, v
+
+
+def test_sage_single_key_returns_its_value(orc):
+    """One key: its softmax weight is 1, so the output is that value row."""
+    q, k, v = _qkv(1, 128, 21)
+    assert np.array_equal(orc.sage_attention_head(q, k, v, 128 ** -0.5), v)
+
+
+def test_sage_zero_scale_averages_the_values(orc):
+    """scale = 0 makes every score 0: uniform weights, the output is the mean of
+    the value rows (closed form), whatever q and k are."""
+    q, k, v = _qkv(37, 128, 22)
+    out = orc.sage_attention_head(q, k, v, 0.0)
+    want = orc.f64_to_bf16_array(bf16_val(v).astype(np.float64).mean(axis=0))
+    assert np.abs(ordinal(out) - ordinal(np.broadcast_to(want, out.shape))).max() <= 1
+    assert np.mean(out == want[None, :]) > 0.95
+
+
+def test_sage_key_permutation_invariance(orc):
+    """Permuting the keys together with their values leaves every output."""
+    q, k, v = _qkv(48, 128, 23)
+    perm = np.random.default_rng(24).permutation(48)
+    o1, f1 = orc.sage_attention_head(q, k, v, 128 ** -0.5, with_f64=True)
+    o2, f2 = orc.sage_attention_head(q, k[perm], v[perm], 128 ** -0.5, with_f64=True)
+    assert np.allclose(f1, f2, rtol=1e-12, atol=1e-15)
+    assert np.abs(ordinal(o1) - ordinal(o2)).max() <= 1
+
+
+def test_sage_dominant_key_selects_its_value(orc):
+    """A key aligned with query 0 and far larger than the others takes all of
+    query 0's weight (the next weight is below exp(-60))."""
+    q, k, v = _qkv(16, 128, 25)
+    k = k.copy()
+    k[5] = bf16_bits(bf16_val(q[0]) * 64.0)
+    others = np.delete(np.arange(16), 5)
+    k[others] = bf16_bits(bf16_val(k[others]) * 0.01)
+    out = orc.sage_attention_head(q, k, v, 1.0)
+    assert np.array_equal(out[0], v[5])
+
+
+def test_sage_close_to_unquantized_attention(orc):
+    """The pages quote ~1 % total quantization error against fp32 attention;
+    with Gaussian q, k, v (head dim 128, 256 tokens) the INT8 scores keep the
+    output within 5 % (relative, max over elements) of fp64 attention on the
+    unquantized inputs, and far from attention with the keys shuffled."""
+    L, D = 256, 128
+    q, k, v = _qkv(L, D, 26, scale_q=2.0)
+    _, o64 = orc.sage_attention_head(q, k, v, D ** -0.5, with_f64=True)
+    qf, kf, vf = (bf16_val(t).astype(np.float64) for t in (q, k, v))
+    s = qf @ kf.T * D ** -0.5
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    ref = (p @ vf) / p.sum(axis=1, keepdims=True)
+    err = np.abs(o64 - ref).max() / np.abs(ref).max()
+    assert err < 0.05
+    perm = np.random.default_rng(27).permutation(L)
+    s2 = qf @ kf[perm].T * D ** -0.5
+    p2 = np.exp(s2 - s2.max(axis=1, keepdims=True))
+    wrong = (p2 @ vf) / p2.sum(axis=1, keepdims=True)
+    assert np.abs(o64 - wrong).max() / np.abs(ref).max() > 10 * err
