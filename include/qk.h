@@ -300,6 +300,41 @@ qk_status qk_w4a8_gemm(const int8_t *xq, const float *sx, const int32_t *xsum,
  */
 qk_status qk_check_device_error(qk_stream_t stream);
 
+/* ------------------------------------------------------- INT8 attention */
+
+/* Bytes of workspace qk_sage_attention needs: the INT8 codes and fp32 scales
+ * of q and k and a transposed copy of v, each part 256-byte aligned. */
+size_t qk_sage_attention_workspace_size(int64_t B, int64_t H, int64_t L);
+
+/*
+ * INT8 attention of a diffusion transformer block ("qlip-mlx" README, intro
+ * bullet "sage_attention" and the "Exact where it matters" bullet: INT8 Q K^T
+ * inside a flash-attention structure with exact online softmax, per-token
+ * scales, softmax and P V in floating point; head dim 128; no mask):
+ *   qc, sq = per-token quantization of q (the qk_quantize_activations rule on
+ *            each 128-element row), likewise kc, sk for k;
+ *   s[i, j] = (qc_i . kc_j) * sq[i] * sk[j] * scale;
+ *   out_i   = sum_j softmax_j(s[i, :]) v_j.
+ * Scores and the softmax are evaluated in fp32 (2^x by the hardware
+ * approximation), the weights rounded to bf16 for P V (bf16 tensor-core
+ * products, fp32 sums) and normalised by the sum of the rounded weights; out
+ * is rounded to bf16.  Relative to the same formula in exact arithmetic the
+ * error per element stays below about 2^-8 (max_j |v_j| + |out_i|).
+ *   q, k, v   : bf16 bits [B, H, L, 128], contiguous (in)
+ *   D         : head dim, must be 128
+ *   scale     : the softmax scale (e.g. 1 / sqrt(128))
+ *   out       : bf16 bits [B, H, L, 128] (out; must not alias q, k or v)
+ *   workspace : >= qk_sage_attention_workspace_size(B, H, L) bytes, or NULL
+ *               (allocated stream-ordered on `stream`).
+ * Shape contract: B, H >= 1, L >= 1, L % 8 == 0, B * H * L <= 2^31 / 128.
+ * Kernels: the activation quantization twice (q, k), a transpose of v, and
+ * the attention kernel (tcgen05 kind::i8 for Q K^T, kind::f16 for P V).
+ */
+qk_status qk_sage_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            int64_t B, int64_t H, int64_t L, int64_t D, float scale,
+                            uint16_t *out, void *workspace, size_t ws_bytes,
+                            qk_stream_t stream);
+
 /* ------------------------------------------------------------ test hooks */
 
 /*

@@ -57,6 +57,8 @@ def _bind(path: str):
         "oracle_w8a8_dequant_f64": (None, [P, I64, I64, P, P, P, P]),
         "oracle_w4a8_dequant_f64": (None, [P, P, I64, I64, I64, P, P, P, P, P]),
         "oracle_sage_attention": (None, [P, P, P, P, P, I64, I64, ctypes.c_double, P, P]),
+        "oracle_sage_attention_rows": (None, [P, P, P, P, P, I64, I64, ctypes.c_double, P, I64,
+                                              P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -301,6 +303,23 @@ def sage_attention_head(q_bf16, k_bf16, v_bf16, scale, with_f64=False):
     _load().oracle_sage_attention(_p(qc), _p(sq), _p(kc), _p(sk), _p(v), L, D, float(scale),
                                   _p(o64) if with_f64 else None, _p(out))
     return (out, o64) if with_f64 else out
+
+
+def sage_attention_rows(q_bf16, k_bf16, v_bf16, scale, rows):
+    """sage_attention_head for the query rows `rows` only: (bf16 bits, fp64)
+    outputs [len(rows), D] (same arithmetic, for sampled rows of long heads)."""
+    q = _c(q_bf16, np.uint16)
+    k = _c(k_bf16, np.uint16)
+    v = _c(v_bf16, np.uint16)
+    L, D = q.shape
+    rows = _c(np.asarray(rows), np.int64)
+    qc, sq = quant_act(q)
+    kc, sk = quant_act(k)
+    out = np.empty((len(rows), D), np.uint16)
+    o64 = np.empty((len(rows), D), np.float64)
+    _load().oracle_sage_attention_rows(_p(qc), _p(sq), _p(kc), _p(sk), _p(v), L, D, float(scale),
+                                       _p(rows), len(rows), _p(o64), _p(out))
+    return out, o64
 
 
 def sage_attention(q_bf16, k_bf16, v_bf16, scale, with_f64=False):

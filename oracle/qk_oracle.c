@@ -389,20 +389,23 @@ void oracle_w4a8_dequant(const int64_t *acc, const int32_t *xsum,
 }
 
 /*
- * INT8 attention of one head [qlip-sage], (R14), for L queries and L keys of
- * head dim D: q and k are given as their per-token codes and scales (from
- * oracle_quant_act_bf16), v as bf16 bits [L, D].  Everything after the integer
- * dot products is fp64: s = dot * sq[i] * sk[j] * scale, p = exp(s - max_j s),
- * o = (sum_j p v_j) / (sum_j p).  out_f64 (nullable) receives o before the
- * rounding; out receives it rounded to bf16.
+ * INT8 attention of one head [qlip-sage], (R14), for the query rows `rows`
+ * (nrows of them) against all L keys, head dim D: q and k are given as their
+ * per-token codes and scales (from oracle_quant_act_bf16), v as bf16 bits
+ * [L, D].  Everything after the integer dot products is fp64:
+ * s = dot * sq[i] * sk[j] * scale, p = exp(s - max_j s),
+ * o = (sum_j p v_j) / (sum_j p).  out_f64 (nullable, [nrows, D]) receives o
+ * before the rounding; out ([nrows, D]) receives it rounded to bf16.
  */
-void oracle_sage_attention(const int8_t *qc, const float *sq, const int8_t *kc,
-                           const float *sk, const uint16_t *v, int64_t L, int64_t D,
-                           double scale, double *out_f64, uint16_t *out)
+void oracle_sage_attention_rows(const int8_t *qc, const float *sq, const int8_t *kc,
+                                const float *sk, const uint16_t *v, int64_t L, int64_t D,
+                                double scale, const int64_t *rows, int64_t nrows,
+                                double *out_f64, uint16_t *out)
 {
     double *s = (double *)malloc((size_t)L * sizeof(double));
     double *o = (double *)malloc((size_t)D * sizeof(double));
-    for (int64_t i = 0; i < L; ++i) {
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t i = rows[r];
         double mx = -INFINITY;
         for (int64_t j = 0; j < L; ++j) {
             int64_t dot = 0;
@@ -422,12 +425,24 @@ void oracle_sage_attention(const int8_t *qc, const float *sq, const int8_t *kc,
                 o[d] += p * (double)oracle_bf16_to_f32(v[j * D + d]);
         }
         for (int64_t d = 0; d < D; ++d) {
-            double r = o[d] / l;
+            double res = o[d] / l;
             if (out_f64)
-                out_f64[i * D + d] = r;
-            out[i * D + d] = oracle_f64_to_bf16(r);
+                out_f64[r * D + d] = res;
+            out[r * D + d] = oracle_f64_to_bf16(res);
         }
     }
     free(s);
     free(o);
+}
+
+/* The same for every query row 0 .. L - 1 (outputs [L, D]). */
+void oracle_sage_attention(const int8_t *qc, const float *sq, const int8_t *kc,
+                           const float *sk, const uint16_t *v, int64_t L, int64_t D,
+                           double scale, double *out_f64, uint16_t *out)
+{
+    int64_t *rows = (int64_t *)malloc((size_t)L * sizeof(int64_t));
+    for (int64_t i = 0; i < L; ++i)
+        rows[i] = i;
+    oracle_sage_attention_rows(qc, sq, kc, sk, v, L, D, scale, rows, L, out_f64, out);
+    free(rows);
 }

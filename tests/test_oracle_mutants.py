@@ -41,7 +41,7 @@ MUTANTS = [
      "dot += (int64_t)qc[i * D + d] * (int64_t)kc[i * D + d];"),
     ("sage_value_transposed", "o[d] += p * (double)oracle_bf16_to_f32(v[j * D + d]);",
      "o[d] += p * (double)oracle_bf16_to_f32(v[d * L + j]);"),
-    ("sage_normalizer_dropped", "double r = o[d] / l;", "double r = o[d];"),
+    ("sage_normalizer_dropped", "double res = o[d] / l;", "double res = o[d];"),
 ]
 
 

@@ -42,6 +42,8 @@ _SIGS = {
     "qk_debug_w8a8_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P]),
     "qk_debug_w4a8_group_acc": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I, _P]),
     "qk_debug_wait_timeout": (_I, [_I64, _P]),
+    "qk_sage_attention_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "qk_sage_attention": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -288,3 +290,23 @@ def qk_debug_wait_timeout(limit_cycles: int, stream=None) -> None:
     after `limit_cycles` SM cycles and records QK_ERR_TIMEOUT for
     qk_check_device_error."""
     _check(lib.qk_debug_wait_timeout(int(limit_cycles), _stream(stream)), "qk_debug_wait_timeout")
+
+
+def qk_sage_attention_workspace_size(B: int, H: int, L: int) -> int:
+    return int(lib.qk_sage_attention_workspace_size(B, H, L))
+
+
+def qk_sage_attention(q, k, v, scale=None, out=None, workspace=None, stream=None):
+    """INT8 attention over bf16 [B, H, L, 128] q, k, v; returns bf16 [B, H, L, 128]."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, 4, name)
+    B, H, L, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k and v must have the same shape [B, H, L, 128]")
+    out = _out(out, (B, H, L, D), torch.bfloat16, q.device, "out")
+    if scale is None:
+        scale = D ** -0.5
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qk_sage_attention(_ptr(q), _ptr(k), _ptr(v), B, H, L, D, float(scale), _ptr(out),
+                                 _ptr(workspace), ws_bytes, _stream(stream)), "qk_sage_attention")
+    return out

@@ -398,6 +398,68 @@ qk_status qk_check_device_error(qk_stream_t stream) {
   return QK_OK;
 }
 
+// INT8 attention workspace: qc, kc [BH L 128] int8; sq [BH L] fp32; sk
+// [BH L + 128] fp32 (the last key block reads 128 entries from its start);
+// vt [BH, 128, L] bf16.
+static size_t sage_parts(int64_t BH, int64_t L, size_t off[5]) {
+  const size_t n = (size_t)BH * (size_t)L;
+  size_t o = 0;
+  off[0] = o; o += round256(n * 128);
+  off[1] = o; o += round256(n * 128);
+  off[2] = o; o += round256(n * 4);
+  off[3] = o; o += round256((n + 128) * 4);
+  off[4] = o; o += round256(n * 128 * 2);
+  return o;
+}
+
+size_t qk_sage_attention_workspace_size(int64_t B, int64_t H, int64_t L) {
+  if (B <= 0 || H <= 0 || L <= 0) return 0;
+  size_t off[5];
+  return sage_parts(B * H, L, off);
+}
+
+qk_status qk_sage_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t B,
+                            int64_t H, int64_t L, int64_t D, float scale, uint16_t* out,
+                            void* workspace, size_t ws_bytes, qk_stream_t stream) {
+  if (B < 1 || H < 1 || L < 1) return QK_ERR_INVALID_ARG;
+  if (D != 128 || L % 8 != 0 || B * H * L > (int64_t(1) << 31) / 128)
+    return QK_ERR_UNSUPPORTED_SHAPE;
+  if (!q || !k || !v || !out) return QK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return QK_ERR_MISALIGNED;
+  qk_status st = check_device();
+  if (st != QK_OK) return st;
+  const int64_t BH = B * H;
+  size_t off[5];
+  const size_t need = sage_parts(BH, L, off);
+  void* owned = nullptr;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  if (base == nullptr) {
+    if ((st = from_cuda(cudaMallocAsync(&owned, need, stream), "cudaMallocAsync(workspace)")) !=
+        QK_OK)
+      return st;
+    base = static_cast<uint8_t*>(owned);
+  } else if (ws_bytes < need || (reinterpret_cast<uintptr_t>(base) & 255u) != 0) {
+    return QK_ERR_WORKSPACE;
+  }
+  int8_t* qc = reinterpret_cast<int8_t*>(base + off[0]);
+  int8_t* kc = reinterpret_cast<int8_t*>(base + off[1]);
+  float* sq = reinterpret_cast<float*>(base + off[2]);
+  float* sk = reinterpret_cast<float*>(base + off[3]);
+  uint16_t* vt = reinterpret_cast<uint16_t*>(base + off[4]);
+  if (log_enabled())
+    std::fprintf(stderr, "[qk] sage_attention B=%lld H=%lld L=%lld\n", (long long)B, (long long)H,
+                 (long long)L);
+  if ((st = from_cuda(launch_quant_act(q, BH * L, 128, qc, sq, nullptr, stream), "quant_q")) ==
+          QK_OK &&
+      (st = from_cuda(launch_quant_act(k, BH * L, 128, kc, sk, nullptr, stream), "quant_k")) ==
+          QK_OK &&
+      (st = from_cuda(launch_transpose_v(v, BH, L, vt, stream), "transpose_v")) == QK_OK)
+    st = from_cuda(launch_sage_attention(qc, sq, kc, sk, vt, BH, L, scale, out, stream),
+                   "sage_attention");
+  if (owned != nullptr) cudaFreeAsync(owned, stream);
+  return st;
+}
+
 qk_status qk_debug_wait_timeout(int64_t limit_cycles, qk_stream_t stream) {
   if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 31)) return QK_ERR_INVALID_ARG;
   qk_status st = check_device();

@@ -42,6 +42,16 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
 // distributed shared memory.  launch_w8a8_gemm routes such shapes here.
 bool w8a8_use_skinny(int64_t M, int64_t K, int64_t N);
 
+// INT8 attention of BH heads of L tokens (head dim 128): per-token codes and
+// scales of q and k ([BH * L, 128] int8, [BH * L] fp32; sk readable for 128
+// entries past BH * L), v^T ([BH, 128, L] bf16), out [BH, L, 128] bf16.
+cudaError_t launch_sage_attention(const int8_t* qc, const float* sq, const int8_t* kc,
+                                  const float* sk, const uint16_t* vt, int64_t BH, int64_t L,
+                                  float scale, uint16_t* out, cudaStream_t s);
+// v [BH, L, 128] bf16 -> vt [BH, 128, L] bf16.
+cudaError_t launch_transpose_v(const uint16_t* v, int64_t BH, int64_t L, uint16_t* vt,
+                               cudaStream_t s);
+
 // Test hook: one kernel whose two waits can never complete, each bounded by
 // `limit_cycles`; both record QK_ERR_TIMEOUT (debug_wait.cu).
 cudaError_t launch_wait_timeout_probe(long long limit_cycles, cudaStream_t s);

@@ -1,0 +1,391 @@
+// sage_attn.cu -- INT8 attention (scores from INT8 q and k, softmax and P V in
+// floating point), head dim 128, no mask.
+//
+// Computes ("qlip-mlx" README, intro bullet "sage_attention" and the "Exact
+// where it matters" bullet: INT8 Q K^T inside a flash-attention structure,
+// exact online softmax, per-token scales, softmax and P V in floating point),
+// per batch b, head h, query i:
+//     s[i, j] = (qc_i . kc_j) * sq[i] * sk[j] * scale       (integer dot, exact)
+//     o_i     = sum_j softmax_j(s[i, :]) v_j                 (bf16 out)
+// where qc, sq and kc, sk are the per-token INT8 codes and scales of q and k
+// (the activation rule of act_quant.cuh, one 128-element row per token).
+//
+// Design (sm_100a), one CTA per (128-query block, head), 8 warps:
+//  * warp 0: TMA producer -- the query block's codes once, then per 128-key
+//    block the key codes (128 x 128 B, 128-byte swizzle), the value block
+//    transposed (v^T: 128 dims x 128 keys bf16, two 128-byte slabs) and the
+//    block's key scales, into a 2-stage ring;
+//  * warp 1: MMA issuer -- S_j = Q K_j^T by tcgen05.mma kind::i8 (M = N = 128,
+//    K = 32 x 4) into one of two int32 TMEM buffers, then, once the softmax
+//    warps have written P_j (bf16, K-major, swizzled) to shared memory,
+//    O_j = P_j V_j by tcgen05.mma kind::f16 (bf16 in, fp32 accumulate, K = 16
+//    x 8) into one of two fp32 TMEM buffers;
+//  * warps 4-7 (one query row per thread): read S_j twice from TMEM (row
+//    maximum, then p = 2^(s log2 e - m)), keep the running maximum m and sum l
+//    in fp32, write P_j as bf16, and fold the previous block's O_{j-1} into
+//    the output accumulator held in registers, o = 2^(m_{j-2} - m_{j-1}) o +
+//    O_{j-1}, one block behind so the tensor cores are never waited for; at
+//    the end o / l is rounded to bf16.
+// Keys past L (the last block) get p = 0.  Every mbarrier wait is bounded
+// (sm100.cuh); no load uses cluster multicast.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "qk_internal.h"
+#include "sm100.cuh"
+
+namespace qk {
+namespace {
+
+constexpr int D = 128;          // head dim (bytes of a code row)
+constexpr int BQ = 128;         // queries per CTA (TMEM lanes)
+constexpr int BKV = 128;        // keys per block
+constexpr int kStages = 2;
+constexpr int Q_BYTES = BQ * D;                 // 16 KiB of codes
+constexpr int K_BYTES = BKV * D;                // 16 KiB of codes
+constexpr int VT_BYTES = D * BKV * 2;           // 32 KiB: 128 dims x 128 keys bf16
+constexpr int P_BYTES = BQ * BKV * 2;           // 32 KiB: 128 queries x 128 keys bf16
+constexpr int SK_BYTES = BKV * 4;
+constexpr int SMEM_Q = 0;
+constexpr int SMEM_K = SMEM_Q + Q_BYTES;
+constexpr int SMEM_VT = SMEM_K + kStages * K_BYTES;
+constexpr int SMEM_P = SMEM_VT + kStages * VT_BYTES;
+constexpr int SMEM_SK = SMEM_P + kStages * P_BYTES;
+constexpr int SMEM_BAR = SMEM_SK + kStages * SK_BYTES;
+// qfull, kvfull[2], kvempty[2], sfull[2], sfree[2], pfull[2], pfree[2], ofull[2], ofree[2]
+constexpr int kNumBars = 1 + 8 * kStages;
+constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
+constexpr int SMEM_ALLOC = SMEM_SLOT + 16 + 1024;
+constexpr int kThreads = 256;
+constexpr int kSoftWarps = 4;   // warps 4-7
+constexpr uint32_t KV_TX = K_BYTES + VT_BYTES + SK_BYTES;
+constexpr uint32_t kIdescS = i8_idesc(BQ, BKV, true, true);
+// kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A and B bf16 (bits
+// 7-9, 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(D >> 3) << 17) |
+                              ((uint32_t)(BQ >> 4) << 24);
+
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(SMEM_K % 1024 == 0 && SMEM_VT % 1024 == 0 && SMEM_P % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one K = 16 step of bf16 operands.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 2^x by the hardware approximation (relative error below 2^-22).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// v [BH, L, 128] bf16 -> vt [BH, 128, L] bf16 (64 x 64 tiles through shared
+// memory; L % 8 == 0).
+__global__ void __launch_bounds__(256) transpose_v_kernel(const uint16_t* __restrict__ v,
+                                                          uint16_t* __restrict__ vt, int L) {
+  __shared__ uint16_t tile[64][66];
+  const int bh = blockIdx.z;
+  const int l0 = blockIdx.x * 64, d0 = blockIdx.y * 64;
+  const uint16_t* src = v + (size_t)bh * L * D;
+  uint16_t* dst = vt + (size_t)bh * D * L;
+  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
+  for (int r = ty; r < 64; r += 4) {
+    const int l = l0 + r;
+    tile[r][tx] = l < L ? src[(size_t)l * D + d0 + tx] : (uint16_t)0;
+  }
+  __syncthreads();
+  for (int r = ty; r < 64; r += 4) {
+    const int l = l0 + tx;
+    if (l < L) dst[(size_t)(d0 + r) * L + l] = tile[tx][r];
+  }
+}
+
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sage_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmVt, const float* __restrict__ sq,
+                     const float* __restrict__ sk, uint16_t* __restrict__ out, int L,
+                     float scale_log2e, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_smem<1024>(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + SMEM_BAR;
+  const uint32_t qfull = bar0;
+  auto kvfull = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto kvempty = [&](int s) { return bar0 + 8u * (3 + s); };
+  auto sfull = [&](int s) { return bar0 + 8u * (5 + s); };
+  auto sfree = [&](int s) { return bar0 + 8u * (7 + s); };
+  auto pfull = [&](int s) { return bar0 + 8u * (9 + s); };
+  auto pfree = [&](int s) { return bar0 + 8u * (11 + s); };
+  auto ofull = [&](int s) { return bar0 + 8u * (13 + s); };
+  auto ofree = [&](int s) { return bar0 + 8u * (15 + s); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SMEM_SLOT);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int q0 = blockIdx.x * BQ;             // first query of this block, within the head
+  const int nkb = (L + BKV - 1) / BKV;
+  const int row_base = bh * L;                // this head's first row of the [BH * L] arrays
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmVt);
+    mbar_init(qfull, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(kvfull(s), 1);
+      mbar_init(kvempty(s), 1);
+      mbar_init(sfull(s), 1);
+      mbar_init(sfree(s), kSoftWarps);
+      mbar_init(pfull(s), kSoftWarps);
+      mbar_init(pfree(s), 1);
+      mbar_init(ofull(s), 1);
+      mbar_init(ofree(s), kSoftWarps);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);  // S: columns 0-255, O: 256-511
+    tmem_relinquish();
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();  // codes, scales and v^T come from the preparation kernels
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(qfull, Q_BYTES);
+      tma_load_2d(sbase + SMEM_Q, &tmQ, 0, row_base + q0, qfull);
+      for (int j = 0; j < nkb; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(kvempty(s), ((j >> 1) & 1) ^ 1u, err)) break;
+        mbar_arrive_expect_tx(kvfull(s), KV_TX);
+        tma_load_2d(sbase + SMEM_K + s * K_BYTES, &tmK, 0, row_base + j * BKV, kvfull(s));
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl)  // keys [64 sl, 64 sl + 64) of the block
+          tma_load_2d(sbase + SMEM_VT + s * VT_BYTES + sl * (VT_BYTES / 2), &tmVt,
+                      j * BKV + 64 * sl, bh * D, kvfull(s));
+        bulk_load(sbase + SMEM_SK + s * SK_BYTES, sk + row_base + j * BKV, SK_BYTES, kvfull(s));
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T (int32)
+        const int s = j & 1;
+        if (!mbar_wait(kvfull(s), (j >> 1) & 1, err)) return false;
+        if (!mbar_wait(sfree(s), ((j >> 1) & 1) ^ 1u, err)) return false;
+        tc_fence_after();
+        const uint32_t a = sbase + SMEM_Q, b = sbase + SMEM_K + s * K_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk)
+          mma_i8(tmem_base + (uint32_t)(s * BKV), sw128_kmajor_desc(a + 32 * kk),
+                 sw128_kmajor_desc(b + 32 * kk), kIdescS, kk);
+        mma_commit(sfull(s));
+        return true;
+      };
+      bool ok = mbar_wait(qfull, 0, err) && issue_s(0);
+      for (int j = 0; j < nkb && ok; ++j) {
+        if (j + 1 < nkb && !issue_s(j + 1)) break;  // the next scores overlap this softmax
+        const int s = j & 1;
+        if (!mbar_wait(pfull(s), (j >> 1) & 1, err)) break;
+        if (!mbar_wait(ofree(s), ((j >> 1) & 1) ^ 1u, err)) break;
+        tc_fence_after();
+        const uint32_t a = sbase + SMEM_P + s * P_BYTES, b = sbase + SMEM_VT + s * VT_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)  // K = 16 keys per step: slab kk / 4, 32 B in
+          mma_bf16(tmem_base + (uint32_t)(256 + s * D),
+                   sw128_kmajor_desc(a + (kk >> 2) * (P_BYTES / 2) + 32 * (kk & 3)),
+                   sw128_kmajor_desc(b + (kk >> 2) * (VT_BYTES / 2) + 32 * (kk & 3)), kIdescPV,
+                   kk);
+        mma_commit(ofull(s));    // O_j ready
+        mma_commit(pfree(s));    // P_j read
+        mma_commit(kvempty(s));  // K_j and v^T_j read
+      }
+    }
+  } else if (warp >= 8 - kSoftWarps) {
+    // ------------------------------------------------- softmax and output
+    const int q = warp & 3;                  // TMEM lane quarter
+    const int row = q * 32 + lane;           // query row of the block (TMEM lane)
+    const int qi = q0 + row;
+    const bool live = qi < L;
+    const float cq = live ? __ldg(sq + row_base + qi) * scale_log2e : 0.0f;
+    const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16);
+    float o[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) o[d] = 0.0f;
+    float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+    bool ok = true;
+    // o = alpha o + O_jo (the PV product of block jo), then hand the buffer back
+    auto fold_o = [&](int jo, float alpha) -> bool {
+      const int sp = jo & 1;
+      if (!mbar_wait(ofull(sp), (jo >> 1) & 1, err)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(t_lane + (uint32_t)(256 + sp * D + 32 * c), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(alpha, o[32 * c + i], __uint_as_float(v[i]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ofree(sp));
+      return true;
+    };
+    for (int j = 0; j < nkb; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait(sfull(s), (j >> 1) & 1, err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* skb = reinterpret_cast<const float*>(smem + SMEM_SK + s * SK_BYTES);
+      const int kvalid = min(BKV, L - j * BKV);  // keys of this block inside the head
+      const uint32_t t_s = t_lane + (uint32_t)(s * BKV);
+      // pass 1: the block's maximum score (log2 units)
+      float mb = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BKV / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(t_s + (uint32_t)(32 * c), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int key = 32 * c + i;
+          const float x = __int2float_rn((int)v[i]) * skb[key] * cq;
+          if (key < kvalid) mb = fmaxf(mb, x);
+        }
+      }
+      const float m_new = fmaxf(m, mb);
+      const float alpha = ex2(m - m_new);  // 0 on the first block (m = -inf)
+      // pass 2: p = 2^(x - m_new) rounded to bf16, its row sum, P_j to shared
+      // memory (K-major, 128-byte swizzle; keys 64 sl .. 64 sl + 63 in slab sl)
+      if (!mbar_wait(pfree(s), ((j >> 1) & 1) ^ 1u, err)) {
+        ok = false;
+        break;
+      }
+      uint8_t* prow = smem + SMEM_P + s * P_BYTES + row * 128;
+      float rs = 0.0f;
+#pragma unroll
+      for (int c = 0; c < BKV / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(t_s + (uint32_t)(32 * c), v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int key = 32 * c + i;
+          const float x0 = __int2float_rn((int)v[i]) * skb[key] * cq;
+          const float x1 = __int2float_rn((int)v[i + 1]) * skb[key + 1] * cq;
+          const float p0 = key < kvalid ? ex2(x0 - m_new) : 0.0f;
+          const float p1 = key + 1 < kvalid ? ex2(x1 - m_new) : 0.0f;
+          const uint32_t w = pack_bf16x2(p0, p1);
+          rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);  // the weights P V uses
+          pk[i >> 1] = w;
+        }
+        uint8_t* srow = prow + (c >> 1) * (P_BYTES / 2);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int ch = (c & 1) * 4 + u;  // 16-byte chunk of the 128-byte row
+          *reinterpret_cast<uint4*>(srow + ((ch ^ (row & 7)) * 16)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sfree(s));  // S_j read
+      fence_proxy_async_smem();              // P_j stores before the tensor cores read them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull(s));
+      l = alpha * l + rs;
+      if (j >= 1 && !fold_o(j - 1, alpha_prev)) {  // one block behind
+        ok = false;
+        break;
+      }
+      alpha_prev = alpha;
+      m = m_new;
+    }
+    if (ok && nkb >= 1) ok = fold_o(nkb - 1, alpha_prev);
+    if (ok && live) {
+      const float inv = 1.0f / l;
+      uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(row_base + qi) * D);
+#pragma unroll
+      for (int u = 0; u < D / 8; ++u)
+        dst[u] = make_uint4(pack_bf16x2(o[8 * u] * inv, o[8 * u + 1] * inv),
+                            pack_bf16x2(o[8 * u + 2] * inv, o[8 * u + 3] * inv),
+                            pack_bf16x2(o[8 * u + 4] * inv, o[8 * u + 5] * inv),
+                            pack_bf16x2(o[8 * u + 6] * inv, o[8 * u + 7] * inv));
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+bool g_attr_done[64];
+
+}  // namespace
+
+cudaError_t launch_sage_attention(const int8_t* qc, const float* sq, const int8_t* kc,
+                                  const float* sk, const uint16_t* vt, int64_t BH, int64_t L,
+                                  float scale, uint16_t* out, cudaStream_t s) {
+  CUtensorMap tQ, tK, tV;
+  if (!encode_tmap_2d(&tQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, qc, (uint64_t)D, (uint64_t)(BH * L),
+                      (uint64_t)D, D, BQ, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tK, CU_TENSOR_MAP_DATA_TYPE_UINT8, kc, (uint64_t)D, (uint64_t)(BH * L),
+                      (uint64_t)D, D, BKV, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vt, (uint64_t)L, (uint64_t)(BH * D),
+                      (uint64_t)L * 2, 64, D, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !g_attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(sage_attn_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    g_attr_done[dev] = true;
+  }
+  int* err = device_error_word();
+  if (err == nullptr) return cudaErrorUnknown;
+  const float scale_log2e = scale * 1.4426950408889634f;
+  dim3 grid((unsigned)((L + BQ - 1) / BQ), (unsigned)BH);
+  sage_attn_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tQ, tK, tV, sq, sk, out, (int)L, scale_log2e,
+                                                      err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_v(const uint16_t* v, int64_t BH, int64_t L, uint16_t* vt,
+                               cudaStream_t s) {
+  dim3 grid((unsigned)((L + 63) / 64), (unsigned)(D / 64), (unsigned)BH);
+  transpose_v_kernel<<<grid, 256, 0, s>>>(v, vt, (int)L);
+  return cudaGetLastError();
+}
+
+}  // namespace qk
