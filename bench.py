@@ -56,7 +56,9 @@ WORKLOADS = {
     "w4a8_m4096": ("W4A8", 3),
     "quickstart_w8a8": ("QUICKSTART", 0),
     "quickstart_w4a8": ("QUICKSTART", 1),
+    "sage_attn": ("SAGE_QUICKSTART", None),
 }
+ATTN_METRIC = "INT8 attention TFLOP/s (4 B H L^2 D ops) at DiT shapes"
 
 
 def get_case(name):
@@ -69,6 +71,10 @@ def get_case(name):
 
 def is_w4(name):
     return "w4a8" in name
+
+
+def is_attention(name):
+    return name.startswith("sage")
 
 
 def is_gated(name):
@@ -241,6 +247,121 @@ def graph_runner(fn, steps):
                 fn(i)
     torch.cuda.current_stream().wait_stream(side)
     return g.replay
+
+
+def run_attention(args, world, rank, local):
+    """The INT8 attention (qk_sage_attention) on the quick-start shape."""
+    import torch
+
+    from w4a8_quantized_gemm_token_b200 import binding as qk
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    case = get_case(args.workload)
+    B, H, L, D = case.B, case.H, case.L, case.D
+    qb, kb, vb = case.draw()
+    hosts = [torch.from_numpy(t.view(np.int16)).view(torch.bfloat16) for t in (qb, kb, vb)]
+    del qb, kb, vb
+    q, k, v = (t.to(dev) for t in hosts)  # 3 x 144 MB: each step reads more than the L2
+    out = torch.empty_like(q)
+    ws = torch.empty(qk.qk_sage_attention_workspace_size(B, H, L), dtype=torch.uint8, device=dev)
+    flops = 4.0 * B * H * L * L * D
+
+    def step(i):
+        qk.qk_sage_attention(q, k, v, out=out, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    qk.qk_check_device_error()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = e0.elapsed_time(e1)
+    qk.qk_check_device_error()
+    max_ms = reduce_max(ms, dev)
+    value = whole_job_value(flops, args.steps, world, max_ms / 1e3)
+    # Roofline: Q K^T at the INT8 rate, P V at the bf16 rate (measured bf16 x 2 and
+    # measured bf16); the bound is the sum of the two times.
+    peaks = load_peaks()
+    t_bound = (flops / 2) / (2 * peaks["bf16"] * 1e12) + (flops / 2) / (peaks["bf16"] * 1e12)
+    achieved = flops / (max_ms / args.steps / 1e3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": flops / t_bound / 1e12,
+            "unit": "TFLOP/s",
+            "peak_source": f"{peaks['source']} bf16_tflops (burst): Q K^T at x2 (INT8), P V at x1",
+            "kernel": "sage_attn_kernel with its q/k quantization and v transpose (the call)",
+            "traffic": None, "frac": None, "kernel_ms": max_ms / args.steps}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    e2e = None
+    if not args.no_e2e:
+        pins = [t.pin_memory() for t in hosts]
+        o_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        n_e2e = max(3, min(args.steps, 5))
+
+        def e2e_step():
+            for dst, src in zip((q, k, v), pins):
+                dst.copy_(src, non_blocking=True)
+            qk.qk_sage_attention(q, k, v, out=out, workspace=ws)
+            o_pin.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = reduce_max(a0.elapsed_time(a1), dev)
+        e2e = {"value": whole_job_value(flops, n_e2e, world, e_ms / 1e3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+               "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = attention_cpu_baseline(case, args.cpu_seconds)
+    clocks = sampler.summary()
+    if rank == 0:
+        line = {
+            "metric": ATTN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 scores, bf16 P V", "data": "synthetic",
+            "config": {"workload": case.name, "B": B, "H": H, "L": L, "D": D,
+                       "l2": "q, k, v of 144 MB each: every step reads more than the L2",
+                       "timing": "eager launches",
+                       "parallelism": f"replicas x{world} (no collective)"},
+            "roofline": roof, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
+            "gpu_launches": 4 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def attention_cpu_baseline(case, seconds=10.0):
+    """The oracle on the host cores: sampled query rows of head 0 against every key."""
+    import oracle
+
+    qb, kb, vb = case.draw(heads=1)
+    q, k, v = qb[0, 0], kb[0, 0], vb[0, 0]
+    t0 = time.perf_counter()
+    oracle.sage_attention_rows(q, k, v, case.D ** -0.5, np.arange(2))
+    dt = max(time.perf_counter() - t0, 1e-6)
+    rows = int(max(2, min(case.L, 2 * seconds / dt)))
+    t0 = time.perf_counter()
+    oracle.sage_attention_rows(q, k, v, case.D ** -0.5, np.arange(rows))
+    dt = time.perf_counter() - t0
+    ops = 4.0 * rows * case.L * case.D
+    return {"value": ops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} query rows of head 0 x all {case.L} keys (quantization of the "
+                      f"head's q and k included), single thread, {dt:.1f} s"}
 
 
 def run_ours(args, world, rank, local):
@@ -534,6 +655,24 @@ def run_reference(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_attention_reference(args, world):
+    """The oracle's INT8 attention on the host cores, a bounded sample per step."""
+    case = get_case(args.workload)
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)
+    cpu = attention_cpu_baseline(case, seconds=budget)
+    line = {
+        "impl": "reference", "metric": ATTN_METRIC, "value": cpu["value"], "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 scores, fp64 softmax and P V", "data": "synthetic",
+        "config": {"workload": case.name, "B": case.B, "H": case.H, "L": case.L, "D": case.D},
+        "cpu_baseline": cpu,
+        "e2e": {"value": cpu["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main
 
 def main(argv=None):
@@ -561,6 +700,10 @@ def main(argv=None):
         print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
 
     if args.impl == "reference":
+        if is_attention(args.workload):
+            if rank == 0:
+                run_attention_reference(args, world)
+            return
         run_reference(args, world, rank, local)
         return
 
@@ -574,7 +717,10 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     try:
-        run_ours(args, world, rank, local)
+        if is_attention(args.workload):
+            run_attention(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
     finally:
         if world > 1 and dist.is_initialized():
             dist.destroy_process_group()

@@ -105,4 +105,34 @@ W4A8 = [LinearCase(f"w4a8_g64_{m}x4096x4096", M=m, K=4096, N=4096, bias=False)
 QUICKSTART = [LinearCase("quickstart_w8a8_14040x5120x5120", M=14040, K=5120, N=5120, bias=False),
               LinearCase("quickstart_w4a8_14040x5120x5120", M=14040, K=5120, N=5120, bias=False)]
 
+@dataclass
+class AttentionCase:
+    """q, k, v bf16 [B, H, L, 128], float64 standard normals (q times q_std)
+    from default_rng(seed) in the order q, k, v, rounded to bf16."""
+    name: str
+    B: int
+    H: int
+    L: int
+    D: int = 128
+    q_std: float = 1.0
+    seed: int = 0
+
+    def draw(self, heads=None):
+        """(q, k, v) bf16 bits; `heads` limits the draw to the first heads."""
+        rng = np.random.default_rng(self.seed)
+        H = self.H if heads is None else heads
+        shape = (self.B, H, self.L, self.D)
+        out = []
+        for std in (self.q_std, 1.0, 1.0):
+            t = np.empty(shape, np.uint16)
+            for h in range(H):  # bounded host memory per draw
+                t[:, h] = f32_to_bf16_bits((rng.standard_normal((self.B, self.L, self.D)) * std)
+                                           .astype(np.float32))
+            out.append(t)
+        return tuple(out)
+
+
+# The README's quick-start attention (40 heads x 14040 tokens, head dim 128).
+SAGE_QUICKSTART = AttentionCase("sage_attn_40x14040x128", B=1, H=40, L=14040)
+
 ALL_W8A8 = [TINY, DIT_ATTN, *SWEEP, DIT_MLP]
