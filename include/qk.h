@@ -322,7 +322,7 @@ size_t qk_sage_attention_workspace_size(int64_t B, int64_t H, int64_t L);
  * error per element stays below about 2^-8 (max_j |v_j| + |out_i|).
  *   q, k, v   : bf16 bits [B, H, L, 128], contiguous (in)
  *   D         : head dim, must be 128
- *   scale     : the softmax scale (e.g. 1 / sqrt(128))
+ *   scale     : the softmax scale, finite and >= 0 (e.g. 1 / sqrt(128))
  *   out       : bf16 bits [B, H, L, 128] (out; must not alias q, k or v)
  *   workspace : >= qk_sage_attention_workspace_size(B, H, L) bytes, or NULL
  *               (allocated stream-ordered on `stream`).

@@ -106,3 +106,6 @@ def test_sage_attention_rejects_bad_shapes(qk):
     y = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(qk.QKError):
         qk.qk_sage_attention(y, y, y)  # head dim 64
+    z = torch.zeros(1, 1, 16, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(qk.QKError):
+        qk.qk_sage_attention(z, z, z, scale=-1.0)  # negative scale

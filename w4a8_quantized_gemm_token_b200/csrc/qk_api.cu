@@ -421,7 +421,7 @@ size_t qk_sage_attention_workspace_size(int64_t B, int64_t H, int64_t L) {
 qk_status qk_sage_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t B,
                             int64_t H, int64_t L, int64_t D, float scale, uint16_t* out,
                             void* workspace, size_t ws_bytes, qk_stream_t stream) {
-  if (B < 1 || H < 1 || L < 1) return QK_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || L < 1 || !(scale >= 0.0f) || !(scale < INFINITY)) return QK_ERR_INVALID_ARG;
   if (D != 128 || L % 8 != 0 || B * H * L > (int64_t(1) << 31) / 128)
     return QK_ERR_UNSUPPORTED_SHAPE;
   if (!q || !k || !v || !out) return QK_ERR_INVALID_ARG;

@@ -20,8 +20,9 @@
 //    warps have written P_j (bf16, K-major, swizzled) to shared memory,
 //    O_j = P_j V_j by tcgen05.mma kind::f16 (bf16 in, fp32 accumulate, K = 16
 //    x 8) into one of two fp32 TMEM buffers;
-//  * warps 4-7 (one query row per thread): read S_j twice from TMEM (row
-//    maximum, then p = 2^(s log2 e - m)), keep the running maximum m and sum l
+//  * warps 4-7 (one query row per thread): read S_j twice from TMEM (the row
+//    maximum of acc sk, then p = 2^(s log2 e - m) with s log2 e = cq acc sk and
+//    cq = sq scale log2 e >= 0), keep the running maximum m and sum l
 //    in fp32, write P_j as bf16, and fold the previous block's O_{j-1} into
 //    the output accumulator held in registers, o = 2^(m_{j-2} - m_{j-1}) o +
 //    O_{j-1}, one block behind so the tensor cores are never waited for; at
@@ -93,6 +94,75 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Pass 1 over a block's scores: max over the keys (those < kvalid when masked)
+// of y = acc * sk, with acc the int32 dot products in TMEM.
+template <bool kMasked>
+__device__ __forceinline__ float block_max(uint32_t t_s, const float* skb, int kvalid) {
+  float my = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < BKV / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32(t_s + (uint32_t)(32 * c), v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float4 s4 = reinterpret_cast<const float4*>(skb)[(32 * c + i) >> 2];
+      const float y0 = __int2float_rn((int)v[i]) * s4.x;
+      const float y1 = __int2float_rn((int)v[i + 1]) * s4.y;
+      const float y2 = __int2float_rn((int)v[i + 2]) * s4.z;
+      const float y3 = __int2float_rn((int)v[i + 3]) * s4.w;
+      const int key = 32 * c + i;
+      if (!kMasked || key < kvalid) my = fmaxf(my, y0);
+      if (!kMasked || key + 1 < kvalid) my = fmaxf(my, y1);
+      if (!kMasked || key + 2 < kvalid) my = fmaxf(my, y2);
+      if (!kMasked || key + 3 < kvalid) my = fmaxf(my, y3);
+    }
+  }
+  return my;
+}
+
+// Pass 2: p = 2^(cq y + neg_m) rounded to bf16 (0 for masked keys), written as
+// this row of P (K-major, 128-byte swizzle, two slabs of 64 keys); returns the
+// sum of the rounded weights, the ones P V uses.
+template <bool kMasked>
+__device__ __forceinline__ float block_p(uint32_t t_s, const float* skb, int kvalid, float cq,
+                                         float neg_m, uint8_t* prow, int row) {
+  float rs = 0.0f;
+#pragma unroll
+  for (int c = 0; c < BKV / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32(t_s + (uint32_t)(32 * c), v);
+    tmem_ld_wait();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float4 s4 = reinterpret_cast<const float4*>(skb)[(32 * c + i) >> 2];
+      const int key = 32 * c + i;
+      float p[4];
+      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float y = __int2float_rn((int)v[i + e]) * sv[e];
+        p[e] = (!kMasked || key + e < kvalid) ? ex2(fmaf(cq, y, neg_m)) : 0.0f;
+      }
+      const uint32_t w0 = pack_bf16x2(p[0], p[1]);
+      const uint32_t w1 = pack_bf16x2(p[2], p[3]);
+      rs += (__uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xFFFF0000u)) +
+            (__uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xFFFF0000u));
+      pk[i >> 1] = w0;
+      pk[(i >> 1) + 1] = w1;
+    }
+    uint8_t* srow = prow + (c >> 1) * (P_BYTES / 2);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int ch = (c & 1) * 4 + u;  // 16-byte chunk of the 128-byte row
+      *reinterpret_cast<uint4*>(srow + ((ch ^ (row & 7)) * 16)) =
+          make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+    }
+  }
+  return rs;
 }
 
 // v [BH, L, 128] bf16 -> vt [BH, 128, L] bf16 (64 x 64 tiles through shared
@@ -266,55 +336,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* skb = reinterpret_cast<const float*>(smem + SMEM_SK + s * SK_BYTES);
       const int kvalid = min(BKV, L - j * BKV);  // keys of this block inside the head
       const uint32_t t_s = t_lane + (uint32_t)(s * BKV);
-      // pass 1: the block's maximum score (log2 units)
-      float mb = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BKV / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(t_s + (uint32_t)(32 * c), v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = 32 * c + i;
-          const float x = __int2float_rn((int)v[i]) * skb[key] * cq;
-          if (key < kvalid) mb = fmaxf(mb, x);
-        }
-      }
-      const float m_new = fmaxf(m, mb);
+      // pass 1: the block's maximum of y = acc * sk (scores are cq * y, cq >= 0)
+      const float my = kvalid == BKV ? block_max<false>(t_s, skb, kvalid)
+                                     : block_max<true>(t_s, skb, kvalid);
+      const float m_new = fmaxf(m, cq * my);
       const float alpha = ex2(m - m_new);  // 0 on the first block (m = -inf)
-      // pass 2: p = 2^(x - m_new) rounded to bf16, its row sum, P_j to shared
+      // pass 2: p = 2^(cq y - m_new) rounded to bf16, its row sum, P_j to shared
       // memory (K-major, 128-byte swizzle; keys 64 sl .. 64 sl + 63 in slab sl)
       if (!mbar_wait(pfree(s), ((j >> 1) & 1) ^ 1u, err)) {
         ok = false;
         break;
       }
       uint8_t* prow = smem + SMEM_P + s * P_BYTES + row * 128;
-      float rs = 0.0f;
-#pragma unroll
-      for (int c = 0; c < BKV / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(t_s + (uint32_t)(32 * c), v);
-        tmem_ld_wait();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int key = 32 * c + i;
-          const float x0 = __int2float_rn((int)v[i]) * skb[key] * cq;
-          const float x1 = __int2float_rn((int)v[i + 1]) * skb[key + 1] * cq;
-          const float p0 = key < kvalid ? ex2(x0 - m_new) : 0.0f;
-          const float p1 = key + 1 < kvalid ? ex2(x1 - m_new) : 0.0f;
-          const uint32_t w = pack_bf16x2(p0, p1);
-          rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);  // the weights P V uses
-          pk[i >> 1] = w;
-        }
-        uint8_t* srow = prow + (c >> 1) * (P_BYTES / 2);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int ch = (c & 1) * 4 + u;  // 16-byte chunk of the 128-byte row
-          *reinterpret_cast<uint4*>(srow + ((ch ^ (row & 7)) * 16)) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
-      }
+      const float rs = kvalid == BKV ? block_p<false>(t_s, skb, kvalid, cq, -m_new, prow, row)
+                                     : block_p<true>(t_s, skb, kvalid, cq, -m_new, prow, row);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sfree(s));  // S_j read
