@@ -41,27 +41,36 @@ namespace qk {
 namespace {
 
 constexpr int D = 128;          // head dim (bytes of a code row)
-constexpr int BQ = 128;         // queries per CTA (TMEM lanes)
+constexpr int BQ = 128;         // queries per tile (TMEM lanes)
+constexpr int kTiles = 2;       // query tiles per CTA, one softmax warpgroup each
 constexpr int BKV = 128;        // keys per block
 constexpr int kStages = 2;
-constexpr int Q_BYTES = BQ * D;                 // 16 KiB of codes
+constexpr int Q_BYTES = BQ * D;                 // 16 KiB of codes per tile
 constexpr int K_BYTES = BKV * D;                // 16 KiB of codes
 constexpr int VT_BYTES = D * BKV * 2;           // 32 KiB: 128 dims x 128 keys bf16
 constexpr int P_BYTES = BQ * BKV * 2;           // 32 KiB: 128 queries x 128 keys bf16
 constexpr int SK_BYTES = BKV * 4;
 constexpr int SMEM_Q = 0;
-constexpr int SMEM_K = SMEM_Q + Q_BYTES;
+constexpr int SMEM_K = SMEM_Q + kTiles * Q_BYTES;
 constexpr int SMEM_VT = SMEM_K + kStages * K_BYTES;
-constexpr int SMEM_P = SMEM_VT + kStages * VT_BYTES;
-constexpr int SMEM_SK = SMEM_P + kStages * P_BYTES;
+constexpr int SMEM_P = SMEM_VT + kStages * VT_BYTES;  // one P buffer per tile
+constexpr int SMEM_SK = SMEM_P + kTiles * P_BYTES;
 constexpr int SMEM_BAR = SMEM_SK + kStages * SK_BYTES;
-// qfull, kvfull[2], kvempty[2], sfull[2], sfree[2], pfull[2], pfree[2], ofull[2], ofree[2]
-constexpr int kNumBars = 1 + 8 * kStages;
+// qfull, kvfull[2], kvempty[2], then per tile sfull, sfree, pfull, pfree, ofull, ofree
+constexpr int kNumBars = 1 + 2 * kStages + 6 * kTiles;
 constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
 constexpr int SMEM_ALLOC = SMEM_SLOT + 16 + 1024;
-constexpr int kThreads = 256;
-constexpr int kSoftWarps = 4;   // warps 4-7
+constexpr int kThreads = 128 * (1 + kTiles);  // warpgroup 0: producer, MMA, 2 idle
+constexpr int kSoftWarps = 4;                 // per tile
+// Registers: launched with kRegsLaunch per thread; warpgroup 0 keeps kRegsCtl
+// and the softmax warpgroups (o[128] in registers) take the rest.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsCtl = 56;
+constexpr int kRegsSoft = 224;
+static_assert(128 * kRegsCtl + 128 * kTiles * kRegsSoft <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr uint32_t KV_TX = K_BYTES + VT_BYTES + SK_BYTES;
+static_assert(kTiles * 2 * 128 <= 512, "S and O of every tile fit the 512 TMEM columns");
 constexpr uint32_t kIdescS = i8_idesc(BQ, BKV, true, true);
 // kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A and B bf16 (bits
 // 7-9, 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
@@ -199,18 +208,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t qfull = bar0;
   auto kvfull = [&](int s) { return bar0 + 8u * (1 + s); };
   auto kvempty = [&](int s) { return bar0 + 8u * (3 + s); };
-  auto sfull = [&](int s) { return bar0 + 8u * (5 + s); };
-  auto sfree = [&](int s) { return bar0 + 8u * (7 + s); };
-  auto pfull = [&](int s) { return bar0 + 8u * (9 + s); };
-  auto pfree = [&](int s) { return bar0 + 8u * (11 + s); };
-  auto ofull = [&](int s) { return bar0 + 8u * (13 + s); };
-  auto ofree = [&](int s) { return bar0 + 8u * (15 + s); };
+  // per query tile t: 0 sfull, 1 sfree, 2 pfull, 3 pfree, 4 ofull, 5 ofree
+  auto tbar = [&](int t, int which) { return bar0 + 8u * (5 + 6 * t + which); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SMEM_SLOT);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * BQ;             // first query of this block, within the head
+  const int q0 = blockIdx.x * (kTiles * BQ);  // first query of this CTA, within the head
   const int nkb = (L + BKV - 1) / BKV;
   const int row_base = bh * L;                // this head's first row of the [BH * L] arrays
 
@@ -222,17 +227,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(kvfull(s), 1);
       mbar_init(kvempty(s), 1);
-      mbar_init(sfull(s), 1);
-      mbar_init(sfree(s), kSoftWarps);
-      mbar_init(pfull(s), kSoftWarps);
-      mbar_init(pfree(s), 1);
-      mbar_init(ofull(s), 1);
-      mbar_init(ofree(s), kSoftWarps);
+    }
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(tbar(t, 0), 1);           // S ready (MMA commit)
+      mbar_init(tbar(t, 1), kSoftWarps);  // S read
+      mbar_init(tbar(t, 2), kSoftWarps);  // P written
+      mbar_init(tbar(t, 3), 1);           // P read (MMA commit)
+      mbar_init(tbar(t, 4), 1);           // O ready (MMA commit)
+      mbar_init(tbar(t, 5), kSoftWarps);  // O read
     }
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 512);  // S: columns 0-255, O: 256-511
+    tmem_alloc(smem_u32(tmem_slot), 512);  // S of tile t: columns 128 t; O: 256 + 128 t
     tmem_relinquish();
   }
   __syncwarp();
@@ -243,119 +250,135 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   pdl_wait();  // codes, scales and v^T come from the preparation kernels
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(qfull, Q_BYTES);
-      tma_load_2d(sbase + SMEM_Q, &tmQ, 0, row_base + q0, qfull);
-      for (int j = 0; j < nkb; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(kvempty(s), ((j >> 1) & 1) ^ 1u, err)) break;
-        mbar_arrive_expect_tx(kvfull(s), KV_TX);
-        tma_load_2d(sbase + SMEM_K + s * K_BYTES, &tmK, 0, row_base + j * BKV, kvfull(s));
+  if (warp < 4) {
+    // warpgroup 0: warp 0 loads, warp 1 issues the MMAs, warps 2-3 idle; most
+    // of its registers go to the softmax warpgroups
+    regs_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        mbar_arrive_expect_tx(qfull, kTiles * Q_BYTES);
+        for (int t = 0; t < kTiles; ++t)
+          tma_load_2d(sbase + SMEM_Q + t * Q_BYTES, &tmQ, 0, row_base + q0 + t * BQ, qfull);
+        for (int j = 0; j < nkb; ++j) {
+          const int s = j & 1;
+          if (!mbar_wait(kvempty(s), ((j >> 1) & 1) ^ 1u, err)) break;
+          mbar_arrive_expect_tx(kvfull(s), KV_TX);
+          tma_load_2d(sbase + SMEM_K + s * K_BYTES, &tmK, 0, row_base + j * BKV, kvfull(s));
 #pragma unroll
-        for (int sl = 0; sl < 2; ++sl)  // keys [64 sl, 64 sl + 64) of the block
-          tma_load_2d(sbase + SMEM_VT + s * VT_BYTES + sl * (VT_BYTES / 2), &tmVt,
-                      j * BKV + 64 * sl, bh * D, kvfull(s));
-        bulk_load(sbase + SMEM_SK + s * SK_BYTES, sk + row_base + j * BKV, SK_BYTES, kvfull(s));
+          for (int sl = 0; sl < 2; ++sl)  // keys [64 sl, 64 sl + 64) of the block
+            tma_load_2d(sbase + SMEM_VT + s * VT_BYTES + sl * (VT_BYTES / 2), &tmVt,
+                        j * BKV + 64 * sl, bh * D, kvfull(s));
+          bulk_load(sbase + SMEM_SK + s * SK_BYTES, sk + row_base + j * BKV, SK_BYTES,
+                    kvfull(s));
+        }
+      }
+    } else if (warp == 1) {
+      // -------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        auto issue_s = [&](int t, int j) -> bool {  // S_t = Q_t K_j^T (int32)
+          const int s = j & 1;
+          if (!mbar_wait(tbar(t, 1), (j & 1) ^ 1u, err)) return false;  // S_t read
+          tc_fence_after();
+          const uint32_t a = sbase + SMEM_Q + t * Q_BYTES, b = sbase + SMEM_K + s * K_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_i8(tmem_base + (uint32_t)(t * BQ), sw128_kmajor_desc(a + 32 * kk),
+                   sw128_kmajor_desc(b + 32 * kk), kIdescS, kk);
+          mma_commit(tbar(t, 0));
+          return true;
+        };
+        bool ok = mbar_wait(qfull, 0, err) && mbar_wait(kvfull(0), 0, err);
+        for (int t = 0; t < kTiles && ok; ++t) ok = issue_s(t, 0);
+        for (int j = 0; j < nkb && ok; ++j) {
+          const int s = j & 1;
+          const bool next = j + 1 < nkb;
+          if (next && !mbar_wait(kvfull(s ^ 1), ((j + 1) >> 1) & 1, err)) break;
+          for (int t = 0; t < kTiles && ok; ++t) {
+            // O_t = P_t V_j once tile t's softmax wrote P_t and folded the last O_t
+            if (!mbar_wait(tbar(t, 2), j & 1, err) || !mbar_wait(tbar(t, 5), (j & 1) ^ 1u, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a = sbase + SMEM_P + t * P_BYTES, b = sbase + SMEM_VT + s * VT_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BKV / 16; ++kk)  // K = 16 keys per step: slab kk / 4
+              mma_bf16(tmem_base + (uint32_t)(256 + t * D),
+                       sw128_kmajor_desc(a + (kk >> 2) * (P_BYTES / 2) + 32 * (kk & 3)),
+                       sw128_kmajor_desc(b + (kk >> 2) * (VT_BYTES / 2) + 32 * (kk & 3)),
+                       kIdescPV, kk);
+            mma_commit(tbar(t, 4));  // O_t ready
+            mma_commit(tbar(t, 3));  // P_t read
+            // the next scores of this tile (its S buffer was read before P_t was written)
+            if (next && !issue_s(t, j + 1)) ok = false;
+          }
+          mma_commit(kvempty(s));  // K_j and v^T_j read by every tile
+        }
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T (int32)
-        const int s = j & 1;
-        if (!mbar_wait(kvfull(s), (j >> 1) & 1, err)) return false;
-        if (!mbar_wait(sfree(s), ((j >> 1) & 1) ^ 1u, err)) return false;
-        tc_fence_after();
-        const uint32_t a = sbase + SMEM_Q, b = sbase + SMEM_K + s * K_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8(tmem_base + (uint32_t)(s * BKV), sw128_kmajor_desc(a + 32 * kk),
-                 sw128_kmajor_desc(b + 32 * kk), kIdescS, kk);
-        mma_commit(sfull(s));
-        return true;
-      };
-      bool ok = mbar_wait(qfull, 0, err) && issue_s(0);
-      for (int j = 0; j < nkb && ok; ++j) {
-        if (j + 1 < nkb && !issue_s(j + 1)) break;  // the next scores overlap this softmax
-        const int s = j & 1;
-        if (!mbar_wait(pfull(s), (j >> 1) & 1, err)) break;
-        if (!mbar_wait(ofree(s), ((j >> 1) & 1) ^ 1u, err)) break;
-        tc_fence_after();
-        const uint32_t a = sbase + SMEM_P + s * P_BYTES, b = sbase + SMEM_VT + s * VT_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)  // K = 16 keys per step: slab kk / 4, 32 B in
-          mma_bf16(tmem_base + (uint32_t)(256 + s * D),
-                   sw128_kmajor_desc(a + (kk >> 2) * (P_BYTES / 2) + 32 * (kk & 3)),
-                   sw128_kmajor_desc(b + (kk >> 2) * (VT_BYTES / 2) + 32 * (kk & 3)), kIdescPV,
-                   kk);
-        mma_commit(ofull(s));    // O_j ready
-        mma_commit(pfree(s));    // P_j read
-        mma_commit(kvempty(s));  // K_j and v^T_j read
-      }
-    }
-  } else if (warp >= 8 - kSoftWarps) {
+  } else {
     // ------------------------------------------------- softmax and output
+    regs_inc<kRegsSoft>();
+    const int t = (warp >> 2) - 1;           // query tile of this warpgroup
     const int q = warp & 3;                  // TMEM lane quarter
-    const int row = q * 32 + lane;           // query row of the block (TMEM lane)
-    const int qi = q0 + row;
+    const int row = q * 32 + lane;           // query row of the tile (TMEM lane)
+    const int qi = q0 + t * BQ + row;
     const bool live = qi < L;
     const float cq = live ? __ldg(sq + row_base + qi) * scale_log2e : 0.0f;
     const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16);
+    const uint32_t t_s = t_lane + (uint32_t)(t * BQ);
+    const uint32_t t_o = t_lane + (uint32_t)(256 + t * D);
+    uint8_t* prow = smem + SMEM_P + t * P_BYTES + row * 128;
     float o[D];
 #pragma unroll
     for (int d = 0; d < D; ++d) o[d] = 0.0f;
     float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
     bool ok = true;
-    // o = alpha o + O_jo (the PV product of block jo), then hand the buffer back
+    // o = alpha o + O_t of block jo, then hand the O buffer back
     auto fold_o = [&](int jo, float alpha) -> bool {
-      const int sp = jo & 1;
-      if (!mbar_wait(ofull(sp), (jo >> 1) & 1, err)) return false;
+      if (!mbar_wait(tbar(t, 4), jo & 1, err)) return false;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(t_lane + (uint32_t)(256 + sp * D + 32 * c), v);
+        tmem_ld32(t_o + (uint32_t)(32 * c), v);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(alpha, o[32 * c + i], __uint_as_float(v[i]));
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ofree(sp));
+      if (lane == 0) mbar_arrive(tbar(t, 5));
       return true;
     };
     for (int j = 0; j < nkb; ++j) {
       const int s = j & 1;
-      if (!mbar_wait(sfull(s), (j >> 1) & 1, err)) {
+      if (!mbar_wait(tbar(t, 0), j & 1, err)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const float* skb = reinterpret_cast<const float*>(smem + SMEM_SK + s * SK_BYTES);
       const int kvalid = min(BKV, L - j * BKV);  // keys of this block inside the head
-      const uint32_t t_s = t_lane + (uint32_t)(s * BKV);
       // pass 1: the block's maximum of y = acc * sk (scores are cq * y, cq >= 0)
       const float my = kvalid == BKV ? block_max<false>(t_s, skb, kvalid)
                                      : block_max<true>(t_s, skb, kvalid);
       const float m_new = fmaxf(m, cq * my);
       const float alpha = ex2(m - m_new);  // 0 on the first block (m = -inf)
-      // pass 2: p = 2^(cq y - m_new) rounded to bf16, its row sum, P_j to shared
-      // memory (K-major, 128-byte swizzle; keys 64 sl .. 64 sl + 63 in slab sl)
-      if (!mbar_wait(pfree(s), ((j >> 1) & 1) ^ 1u, err)) {
+      // pass 2: P_t of this block (the buffer is free once P V of the last block ran)
+      if (!mbar_wait(tbar(t, 3), (j & 1) ^ 1u, err)) {
         ok = false;
         break;
       }
-      uint8_t* prow = smem + SMEM_P + s * P_BYTES + row * 128;
       const float rs = kvalid == BKV ? block_p<false>(t_s, skb, kvalid, cq, -m_new, prow, row)
                                      : block_p<true>(t_s, skb, kvalid, cq, -m_new, prow, row);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sfree(s));  // S_j read
-      fence_proxy_async_smem();              // P_j stores before the tensor cores read them
+      if (lane == 0) mbar_arrive(tbar(t, 1));  // S_t read
+      fence_proxy_async_smem();                // P_t stores before the tensor cores read them
       __syncwarp();
-      if (lane == 0) mbar_arrive(pfull(s));
+      if (lane == 0) mbar_arrive(tbar(t, 2));
       l = alpha * l + rs;
       if (j >= 1 && !fold_o(j - 1, alpha_prev)) {  // one block behind
         ok = false;
@@ -405,12 +428,17 @@ cudaError_t launch_sage_attention(const int8_t* qc, const float* sq, const int8_
     cudaError_t e = cudaFuncSetAttribute(sage_attn_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
     if (e != cudaSuccess) return e;
+    // the softmax warpgroups' register increase is only satisfiable with the
+    // launch allocation the split was computed for
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, sage_attn_kernel)) != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
     g_attr_done[dev] = true;
   }
   int* err = device_error_word();
   if (err == nullptr) return cudaErrorUnknown;
   const float scale_log2e = scale * 1.4426950408889634f;
-  dim3 grid((unsigned)((L + BQ - 1) / BQ), (unsigned)BH);
+  dim3 grid((unsigned)((L + kTiles * BQ - 1) / (kTiles * BQ)), (unsigned)BH);
   sage_attn_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tQ, tK, tV, sq, sk, out, (int)L, scale_log2e,
                                                       err);
   return cudaGetLastError();
