@@ -105,10 +105,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// Pass 1 over a block's scores: max over the keys (those < kvalid when masked)
-// of y = acc * sk, with acc the int32 dot products in TMEM.
+// One pass over a block's scores: y[key] = acc * sk for the 128 keys (acc the
+// int32 dot products in TMEM); returns the maximum over the keys below kvalid
+// (all of them unless masked).
 template <bool kMasked>
-__device__ __forceinline__ float block_max(uint32_t t_s, const float* skb, int kvalid) {
+__device__ __forceinline__ float load_scores(uint32_t t_s, const float* skb, int kvalid,
+                                             float (&y)[BKV]) {
   float my = -INFINITY;
 #pragma unroll
   for (int c = 0; c < BKV / 32; ++c) {
@@ -118,50 +120,36 @@ __device__ __forceinline__ float block_max(uint32_t t_s, const float* skb, int k
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {
       const float4 s4 = reinterpret_cast<const float4*>(skb)[(32 * c + i) >> 2];
-      const float y0 = __int2float_rn((int)v[i]) * s4.x;
-      const float y1 = __int2float_rn((int)v[i + 1]) * s4.y;
-      const float y2 = __int2float_rn((int)v[i + 2]) * s4.z;
-      const float y3 = __int2float_rn((int)v[i + 3]) * s4.w;
-      const int key = 32 * c + i;
-      if (!kMasked || key < kvalid) my = fmaxf(my, y0);
-      if (!kMasked || key + 1 < kvalid) my = fmaxf(my, y1);
-      if (!kMasked || key + 2 < kvalid) my = fmaxf(my, y2);
-      if (!kMasked || key + 3 < kvalid) my = fmaxf(my, y3);
+      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = 32 * c + i + e;
+        y[key] = __int2float_rn((int)v[i + e]) * sv[e];
+        if (!kMasked || key < kvalid) my = fmaxf(my, y[key]);
+      }
     }
   }
   return my;
 }
 
-// Pass 2: p = 2^(cq y + neg_m) rounded to bf16 (0 for masked keys), written as
-// this row of P (K-major, 128-byte swizzle, two slabs of 64 keys); returns the
-// sum of the rounded weights, the ones P V uses.
+// p = 2^(cq y + neg_m) rounded to bf16 (0 for keys past kvalid when masked),
+// written as this row of P (K-major, 128-byte swizzle, two slabs of 64 keys);
+// returns the sum of the rounded weights, the ones P V uses.
 template <bool kMasked>
-__device__ __forceinline__ float block_p(uint32_t t_s, const float* skb, int kvalid, float cq,
-                                         float neg_m, uint8_t* prow, int row) {
+__device__ __forceinline__ float write_p(const float (&y)[BKV], int kvalid, float cq, float neg_m,
+                                         uint8_t* prow, int row) {
   float rs = 0.0f;
 #pragma unroll
   for (int c = 0; c < BKV / 32; ++c) {
-    uint32_t v[32];
-    tmem_ld32(t_s + (uint32_t)(32 * c), v);
-    tmem_ld_wait();
     uint32_t pk[16];
 #pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-      const float4 s4 = reinterpret_cast<const float4*>(skb)[(32 * c + i) >> 2];
+    for (int i = 0; i < 32; i += 2) {
       const int key = 32 * c + i;
-      float p[4];
-      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float y = __int2float_rn((int)v[i + e]) * sv[e];
-        p[e] = (!kMasked || key + e < kvalid) ? ex2(fmaf(cq, y, neg_m)) : 0.0f;
-      }
-      const uint32_t w0 = pack_bf16x2(p[0], p[1]);
-      const uint32_t w1 = pack_bf16x2(p[2], p[3]);
-      rs += (__uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xFFFF0000u)) +
-            (__uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xFFFF0000u));
-      pk[i >> 1] = w0;
-      pk[(i >> 1) + 1] = w1;
+      const float p0 = (!kMasked || key < kvalid) ? ex2(fmaf(cq, y[key], neg_m)) : 0.0f;
+      const float p1 = (!kMasked || key + 1 < kvalid) ? ex2(fmaf(cq, y[key + 1], neg_m)) : 0.0f;
+      const uint32_t w = pack_bf16x2(p0, p1);
+      rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+      pk[i >> 1] = w;
     }
     uint8_t* srow = prow + (c >> 1) * (P_BYTES / 2);
 #pragma unroll
@@ -233,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(tbar(t, 1), kSoftWarps);  // S read
       mbar_init(tbar(t, 2), kSoftWarps);  // P written
       mbar_init(tbar(t, 3), 1);           // P read (MMA commit)
-      mbar_init(tbar(t, 4), 1);           // O ready (MMA commit)
-      mbar_init(tbar(t, 5), kSoftWarps);  // O read
+      mbar_init(tbar(t, 4), 1);           // O updated (MMA commit)
+      mbar_init(tbar(t, 5), kSoftWarps);  // (unused)
     }
     fence_mbar_init();
   }
@@ -295,8 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool next = j + 1 < nkb;
           if (next && !mbar_wait(kvfull(s ^ 1), ((j + 1) >> 1) & 1, err)) break;
           for (int t = 0; t < kTiles && ok; ++t) {
-            // O_t = P_t V_j once tile t's softmax wrote P_t and folded the last O_t
-            if (!mbar_wait(tbar(t, 2), j & 1, err) || !mbar_wait(tbar(t, 5), (j & 1) ^ 1u, err)) {
+            // O_t += P_t V_j once tile t's softmax wrote P_t (and rescaled O_t if
+            // its reference maximum moved)
+            if (!mbar_wait(tbar(t, 2), j & 1, err)) {
               ok = false;
               break;
             }
@@ -307,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_bf16(tmem_base + (uint32_t)(256 + t * D),
                        sw128_kmajor_desc(a + (kk >> 2) * (P_BYTES / 2) + 32 * (kk & 3)),
                        sw128_kmajor_desc(b + (kk >> 2) * (VT_BYTES / 2) + 32 * (kk & 3)),
-                       kIdescPV, kk);
-            mma_commit(tbar(t, 4));  // O_t ready
+                       kIdescPV, (j | kk) != 0 ? 1u : 0u);
+            mma_commit(tbar(t, 4));  // O_t updated
             mma_commit(tbar(t, 3));  // P_t read
             // the next scores of this tile (its S buffer was read before P_t was written)
             if (next && !issue_s(t, j + 1)) ok = false;
@@ -330,28 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_s = t_lane + (uint32_t)(t * BQ);
     const uint32_t t_o = t_lane + (uint32_t)(256 + t * D);
     uint8_t* prow = smem + SMEM_P + t * P_BYTES + row * 128;
-    float o[D];
-#pragma unroll
-    for (int d = 0; d < D; ++d) o[d] = 0.0f;
-    float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+    // reference maximum m (log2 units) and sum l; the output accumulates in
+    // TMEM (O_t += P V), rescaled only when a row's reference maximum moves
+    float m = -INFINITY, l = 0.0f;
     bool ok = true;
-    // o = alpha o + O_t of block jo, then hand the O buffer back
-    auto fold_o = [&](int jo, float alpha) -> bool {
-      if (!mbar_wait(tbar(t, 4), jo & 1, err)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(t_o + (uint32_t)(32 * c), v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(alpha, o[32 * c + i], __uint_as_float(v[i]));
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tbar(t, 5));
-      return true;
-    };
     for (int j = 0; j < nkb; ++j) {
       const int s = j & 1;
       if (!mbar_wait(tbar(t, 0), j & 1, err)) {
@@ -361,42 +332,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float* skb = reinterpret_cast<const float*>(smem + SMEM_SK + s * SK_BYTES);
       const int kvalid = min(BKV, L - j * BKV);  // keys of this block inside the head
-      // pass 1: the block's maximum of y = acc * sk (scores are cq * y, cq >= 0)
-      const float my = kvalid == BKV ? block_max<false>(t_s, skb, kvalid)
-                                     : block_max<true>(t_s, skb, kvalid);
-      const float m_new = fmaxf(m, cq * my);
-      const float alpha = ex2(m - m_new);  // 0 on the first block (m = -inf)
-      // pass 2: P_t of this block (the buffer is free once P V of the last block ran)
+      float y[BKV];
+      const float my = kvalid == BKV ? load_scores<false>(t_s, skb, kvalid, y)
+                                     : load_scores<true>(t_s, skb, kvalid, y);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tbar(t, 1));  // S_t read: the next scores may start
+      // keep the reference unless the block's maximum exceeds it by more than
+      // 2^8 (weights then stay below 256); a new reference rescales O and l
+      const float mb = cq * my;
+      const float m_new = mb > m + 8.0f ? mb : m;
+      const float alpha = ex2(m - m_new);  // 1 when kept; 0 on the first block
+      if (j >= 1 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+        // O_t holds P V up to block j - 1: wait for it, scale this warp's rows
+        if (!mbar_wait(tbar(t, 4), (j - 1) & 1, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_o + (uint32_t)(32 * c), v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tmem_st32(t_o + (uint32_t)(32 * c), v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      // P_t of this block (the buffer is free once P V of the last block ran)
       if (!mbar_wait(tbar(t, 3), (j & 1) ^ 1u, err)) {
         ok = false;
         break;
       }
-      const float rs = kvalid == BKV ? block_p<false>(t_s, skb, kvalid, cq, -m_new, prow, row)
-                                     : block_p<true>(t_s, skb, kvalid, cq, -m_new, prow, row);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tbar(t, 1));  // S_t read
-      fence_proxy_async_smem();                // P_t stores before the tensor cores read them
+      const float rs = kvalid == BKV ? write_p<false>(y, kvalid, cq, -m_new, prow, row)
+                                     : write_p<true>(y, kvalid, cq, -m_new, prow, row);
+      fence_proxy_async_smem();  // P_t stores before the tensor cores read them
       __syncwarp();
       if (lane == 0) mbar_arrive(tbar(t, 2));
       l = alpha * l + rs;
-      if (j >= 1 && !fold_o(j - 1, alpha_prev)) {  // one block behind
-        ok = false;
-        break;
-      }
-      alpha_prev = alpha;
       m = m_new;
     }
-    if (ok && nkb >= 1) ok = fold_o(nkb - 1, alpha_prev);
-    if (ok && live) {
+    // the output: O_t after the last block's P V, divided by l
+    if (ok && nkb >= 1 && mbar_wait(tbar(t, 4), (nkb - 1) & 1, err)) {
+      tc_fence_after();
       const float inv = 1.0f / l;
       uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(row_base + qi) * D);
 #pragma unroll
-      for (int u = 0; u < D / 8; ++u)
-        dst[u] = make_uint4(pack_bf16x2(o[8 * u] * inv, o[8 * u + 1] * inv),
-                            pack_bf16x2(o[8 * u + 2] * inv, o[8 * u + 3] * inv),
-                            pack_bf16x2(o[8 * u + 4] * inv, o[8 * u + 5] * inv),
-                            pack_bf16x2(o[8 * u + 6] * inv, o[8 * u + 7] * inv));
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(t_o + (uint32_t)(32 * c), v);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            dst[4 * c + u] = make_uint4(
+                pack_bf16x2(__uint_as_float(v[8 * u]) * inv, __uint_as_float(v[8 * u + 1]) * inv),
+                pack_bf16x2(__uint_as_float(v[8 * u + 2]) * inv, __uint_as_float(v[8 * u + 3]) * inv),
+                pack_bf16x2(__uint_as_float(v[8 * u + 4]) * inv, __uint_as_float(v[8 * u + 5]) * inv),
+                pack_bf16x2(__uint_as_float(v[8 * u + 6]) * inv, __uint_as_float(v[8 * u + 7]) * inv));
+        }
+      }
     }
   }
 
