@@ -81,7 +81,9 @@ def test_gemv_deterministic(qk, orc):
 
 
 GEMM_SHAPES = [(17, 64, 8), (129, 192, 72), (300, 1024, 264), (64, 4096, 136), (257, 320, 64),
-               (16, 256, 128)]
+               (16, 256, 128),
+               # K = 65536, the contract's maximum: 1024 groups folded per output
+               (40, 65536, 72)]
 
 
 @pytest.mark.parametrize("MKN", GEMM_SHAPES, ids=lambda s: "x".join(map(str, s)))

@@ -149,3 +149,29 @@ def test_w8a8_zero_rows_and_integer_closed_form(qk, orc):
     exact = (x.astype(np.int64) @ W.astype(np.int64).T + b.astype(np.int64)).astype(np.float32)
     want = torch.from_numpy(exact).to(torch.bfloat16)
     assert torch.equal(y.cpu().view(torch.int16), want.view(torch.int16))
+
+
+@pytest.mark.parametrize("MKN", [(130, 65536, 264), (8, 65536, 16)], ids=["tiles", "splitk"])
+def test_w8a8_max_k_saturated_codes(qk, orc, MKN):
+    """K = 65536, the contract's maximum, with every code at +-127 (x rows and W
+    rows of +-1): the int32 accumulators reach +-127^2 * 65536 = 1 057 030 144,
+    just below 2^31, exactly, and the outputs match the oracle."""
+    M, K, N = MKN
+    xs = np.where(np.arange(M)[:, None] % 2 == 0, 1.0, -1.0) * np.ones((M, K))
+    ws = np.where(np.arange(N)[:, None] % 3 == 0, -1.0, 1.0) * np.ones((N, K))
+    xb = synthetic.f32_to_bf16_bits(xs.astype(np.float32))
+    W = ws.astype(np.float32)
+    Wq_o, sw_o = orc.quant_w8(W)
+    Wq, sw = qk.qk_quantize_weights_int8(to_dev(W))
+    assert np.array_equal(host(Wq), Wq_o)
+    x = to_dev_bf16(xb)
+    y = qk.qk_w8a8_linear(x, Wq, sw)
+    xq, sx, _ = qk.qk_quantize_activations(x)
+    acc = qk.qk_debug_w8a8_acc(xq, Wq)
+    torch.cuda.synchronize()
+    want = (np.sign(xs[:, :1]) * np.sign(ws[:, 0])[None, :]) * 127 * 127 * K
+    assert np.array_equal(host(acc).astype(np.int64), want.astype(np.int64))
+    xq_o, sx_o = orc.quant_act(xb)
+    y_o = orc.w8a8_dequant(orc.w8a8_acc(xq_o, Wq_o), sx_o, sw_o, None)
+    assert bf16_ulp_distance(t2bits(y), y_o).max() <= TOL_ULP
+    qk.qk_check_device_error()
