@@ -56,8 +56,8 @@ constexpr int SMEM_VT = SMEM_K + kStages * K_BYTES;
 constexpr int SMEM_P = SMEM_VT + kStages * VT_BYTES;  // one P buffer per tile
 constexpr int SMEM_SK = SMEM_P + kTiles * P_BYTES;
 constexpr int SMEM_BAR = SMEM_SK + kStages * SK_BYTES;
-// qfull, kvfull[2], kvempty[2], then per tile sfull, sfree, pfull, pfree, ofull, ofree
-constexpr int kNumBars = 1 + 2 * kStages + 6 * kTiles;
+// qfull, kvfull[2], kvempty[2], then per tile sfull, sfree, pfull, pfree, ofull
+constexpr int kNumBars = 1 + 2 * kStages + 5 * kTiles;
 constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
 constexpr int SMEM_ALLOC = SMEM_SLOT + 16 + 1024;
 constexpr int kThreads = 128 * (1 + kTiles);  // warpgroup 0: producer, MMA, 2 idle
@@ -196,8 +196,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t qfull = bar0;
   auto kvfull = [&](int s) { return bar0 + 8u * (1 + s); };
   auto kvempty = [&](int s) { return bar0 + 8u * (3 + s); };
-  // per query tile t: 0 sfull, 1 sfree, 2 pfull, 3 pfree, 4 ofull, 5 ofree
-  auto tbar = [&](int t, int which) { return bar0 + 8u * (5 + 6 * t + which); };
+  // per query tile t: 0 sfull, 1 sfree, 2 pfull, 3 pfree, 4 ofull
+  auto tbar = [&](int t, int which) { return bar0 + 8u * (5 + 5 * t + which); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SMEM_SLOT);
 
   const int warp = threadIdx.x >> 5;
@@ -222,7 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(tbar(t, 2), kSoftWarps);  // P written
       mbar_init(tbar(t, 3), 1);           // P read (MMA commit)
       mbar_init(tbar(t, 4), 1);           // O updated (MMA commit)
-      mbar_init(tbar(t, 5), kSoftWarps);  // (unused)
     }
     fence_mbar_init();
   }
