@@ -246,6 +246,10 @@ def graph_runner(fn, steps):
             for i in range(steps):
                 fn(i)
     torch.cuda.current_stream().wait_stream(side)
+    # The first replay of a graph also uploads it to the device; replay once
+    # here (untimed, as warm-up) so the timed replay measures the kernels only.
+    g.replay()
+    torch.cuda.synchronize()
     return g.replay
 
 

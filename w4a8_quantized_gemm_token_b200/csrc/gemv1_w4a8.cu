@@ -12,18 +12,21 @@
 // lane busy:
 //  * a CTA owns 32 weight rows (4 per warp); before the programmatic-dependency
 //    wait one thread bulk-copies each warp's rows (contiguous, 4 x K/2 bytes)
-//    and the CTA's fp16 scales / offsets into shared memory, and the scales
-//    become an fp64 {s, o} table -- all off the critical path;
-//  * lane l owns the 16-byte chunks l, l + 32, l + 64, ... of a packed row
-//    (one 512-byte, conflict-free shared load per chunk index for the warp);
-//    after the wait every lane holds the matching activation codes in
-//    registers -- read straight from xq, or quantized by the CTA from bf16 x
-//    (the rule of the stand-alone kernel);
-//    nibbles split into even / odd codes feed dp4a against xq permuted the same
-//    way; the two halves of a group (lanes 2m, 2m + 1) add by one shuffle;
-//  * even lanes fold s * acc, odd lanes o * xsum, in fp64; a fixed-order
-//    butterfly over the warp gives the row, which lane 0 rounds once and
-//    stores -- no shared-memory reduction, no block barrier at the end.
+//    and the CTA's fp16 scales / offsets into shared memory, the scales become
+//    an fp64 {s, o} table, every warp waits for its rows and the activations
+//    are prefetched into L2 -- all off the critical path;
+//  * after the wait the CTA stages the activation codes in shared memory
+//    (quantizing bf16 x with the rule of the stand-alone kernel, or permuting
+//    xq), one block barrier, and lane l picks up the codes of the 16-byte
+//    packed chunks l, l + 32, l + 64, ... of a row (one 512-byte, conflict-free
+//    shared load per chunk index for the warp) with the sum of those 32 codes;
+//  * the low nibbles (even k) and the masked high nibbles (odd k, 16 times
+//    too large, one exact shift) feed dp4a against codes permuted the same
+//    way, and each lane folds s * acc + o * (its code sum) for its half-group
+//    in fp64;
+//  * a fixed-order reduction over the warp (two row-halving steps, then a
+//    butterfly) gives the four rows, each rounded once and stored -- no
+//    shared-memory reduction, no block barrier at the end.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -55,9 +58,9 @@ struct Gemv1Layout {
     w = off;    off += (size_t)kRows * KB;           // packed rows, contiguous
     s16 = off;  off += (size_t)kRows * G * 2 * 2;    // fp16 scales [row][g], then offsets
     so = off;   off += (size_t)kRows * G * 16;       // {s, o} in fp64 [row][g]
-    xq = off;   off += (size_t)K;                    // codes (in-kernel quantization only)
-    xs = off;   off += (size_t)G * 8;                // group sums in fp64 (ditto)
-    amx = off;  off += kWarps * 4;                   // per-warp absmax (ditto)
+    xq = off;   off += (size_t)K;                    // codes, even / odd permuted per 8
+    xs = off;   off += (size_t)(K / 32) * 8;         // half-group sums of the codes in fp64
+    amx = off;  off += kWarps * 4;                   // per-warp absmax (in-kernel quantization)
     bias = off; off += kRows * 4;
     off = (off + 15) & ~size_t(15);
     bars = off; off += (kWarps + 1) * 8;             // one per warp's rows, one for the scales
@@ -98,10 +101,55 @@ __device__ __forceinline__ uint2 even_odd(uint32_t lo, uint32_t hi) {
   return make_uint2(__byte_perm(lo, hi, 0x6420), __byte_perm(lo, hi, 0x7531));
 }
 
-// dot of the 8 codes of one packed word with their 8 activation codes
-__device__ __forceinline__ int dot8(uint32_t w, uint32_t x_even, uint32_t x_odd, int acc) {
-  acc = __dp4a((int)(w & 0x0F0F0F0Fu), (int)x_even, acc);
-  return __dp4a((int)((w >> 4) & 0x0F0F0F0Fu), (int)x_odd, acc);
+// The activation rule on 8 bf16 values (one 16-byte chunk), codes returned in
+// the even / odd order of `even_odd`: q = rint(fl(v * r)) with ties to even.
+// Adding 1.5 * 2^23 to the rounded product leaves rint(product) in the low
+// bits (the sum lies in [2^23, 2^24), where the fp32 spacing is 1, and rounds
+// to nearest-even); the product is rounded first, as the rule says, because
+// the multiply and the add are separate roundings (no contraction).  No clamp
+// is needed: with a finite absmax, |v| <= absmax makes |fl(v * r)| < 127.5.
+// (A row holding an inf or a NaN takes the general conversion instead.)
+__device__ __forceinline__ uint32_t rint_bits(float v, float r) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(v, r), 12582912.0f));
+}
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+__device__ __forceinline__ uint2 quant_chunk_even_odd(uint4 c, float r) {
+  // bf16 pairs: the low half of each word is the even k, the high half the odd
+  const uint32_t e0 = rint_bits(__uint_as_float(c.x << 16), r);
+  const uint32_t e1 = rint_bits(__uint_as_float(c.y << 16), r);
+  const uint32_t e2 = rint_bits(__uint_as_float(c.z << 16), r);
+  const uint32_t e3 = rint_bits(__uint_as_float(c.w << 16), r);
+  const uint32_t o0 = rint_bits(__uint_as_float(c.x & 0xFFFF0000u), r);
+  const uint32_t o1 = rint_bits(__uint_as_float(c.y & 0xFFFF0000u), r);
+  const uint32_t o2 = rint_bits(__uint_as_float(c.z & 0xFFFF0000u), r);
+  const uint32_t o3 = rint_bits(__uint_as_float(c.w & 0xFFFF0000u), r);
+  return make_uint2(pack4_low_bytes(e0, e1, e2, e3), pack4_low_bytes(o0, o1, o2, o3));
+}
+
+// dp4a with unsigned bytes in a and signed bytes in b
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Sum of the 32 codes of one packed 16-byte weight chunk times their
+// activation codes.  The low nibbles (even k) go through dp4a as they are; the
+// high nibbles (odd k) are only masked, so each byte holds 16 q and their dot
+// product is 16 times the wanted one -- exact, removed by one shift at the end.
+__device__ __forceinline__ int dot32(uint4 w, const uint32_t (&xe)[8]) {
+  int lo = 0, hi = 0;
+  lo = __dp4a((int)(w.x & 0x0F0F0F0Fu), (int)xe[0], lo);
+  hi = dp4a_us(w.x & 0xF0F0F0F0u, xe[1], hi);
+  lo = __dp4a((int)(w.y & 0x0F0F0F0Fu), (int)xe[2], lo);
+  hi = dp4a_us(w.y & 0xF0F0F0F0u, xe[3], hi);
+  lo = __dp4a((int)(w.z & 0x0F0F0F0Fu), (int)xe[4], lo);
+  hi = dp4a_us(w.z & 0xF0F0F0F0u, xe[5], hi);
+  lo = __dp4a((int)(w.w & 0x0F0F0F0Fu), (int)xe[6], lo);
+  hi = dp4a_us(w.w & 0xF0F0F0F0u, xe[7], hi);
+  return lo + (hi >> 4);
 }
 
 // NJ = K / 1024: 16-byte chunks of a packed row per lane.  kQuantX: x arrives
@@ -134,7 +182,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t bars = smem_u32(smem + L.bars);
   const uint32_t sbar = bars + 8u * kWarps;
 
-  // ---- before the dependency wait: weights, scales / offsets, bias
+  // ---- before the dependency wait: weights, scales / offsets, bias, and an
+  // L2 prefetch of the activations (a hint only: the loads that use them come
+  // after the wait, and L2 is coherent for every SM)
   if (threadIdx.x == 0) {
     for (int i = 0; i <= kWarps; ++i) mbar_init(bars + 8u * i, 1);
     fence_mbar_init();
@@ -152,6 +202,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       bulk_load(smem_u32(smem + L.w) + (uint32_t)(r0 * KB), Wp + (size_t)(n0 + r0) * KB,
                 (uint32_t)(nr * KB), bars + 8u * w);
     }
+    if constexpr (kQuantX) bulk_prefetch_l2(x, (uint32_t)K * 2u);
+    else bulk_prefetch_l2(xq, (uint32_t)K);
   }
   if (!kDump && threadIdx.x < kRows)
     bias_sm[threadIdx.x] =
@@ -162,27 +214,35 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = threadIdx.x; i < rows * G; i += kThreads)
       so_sm[i] = make_double2(h2d(s16[i]), h2d(o16[i]));
   }
+  __syncthreads();  // the {s, o} table is complete (read by every warp)
+  // A warp's four rows are all valid or all past N (rows is a multiple of 8).
+  // Its rows have landed long before the previous kernel releases this one,
+  // so the wait costs nothing there and none is left after the release.
+  const int r0 = warp * kRowsPerWarp;
+  if (r0 < rows) mbar_wait(bars + 8u * warp, 0, err);
 
-  // ---- activations (they come from the previous kernel).  Lane l owns chunks
-  // c = l + 32 j, i.e. codes 32 c .. 32 c + 31, of group 16 j + l / 2, and
-  // keeps their codes in registers.  Quantized activations are read by every
-  // warp straight from global memory (no warp waits on another); bf16 x is
-  // quantized by the whole CTA (one absmax) through shared memory.
+  // ---- activations (they come from the previous kernel).  The CTA stages
+  // the codes in shared memory (quantizing bf16 x with one absmax, or
+  // permuting xq) with the sum of every 32 codes; then lane l picks up the
+  // codes of its 16-byte packed chunks c = l + 32 j, i.e. codes 32 c .. 32 c +
+  // 31 (half of group c / 2), into registers with the sum of those codes as a
+  // double (the offset term of each half-group is folded by its own lane).
   pdl_wait();
   if (!early_trigger) pdl_launch_dependents();
   uint32_t xr[NJ][8];  // codes, even / odd permuted per 8 (the nibble-split order)
-  double xsj[NJ];      // xsum of the lane's group of chunk j
+  double xh[NJ];       // sum of the lane's 32 codes of chunk j
   float sxv = 1.0f;
   if constexpr (kQuantX) {
-    // cooperative: every thread quantizes two 16-byte chunks of x (absmax by a
+    // cooperative: every thread quantizes 16-byte chunks of x (absmax by a
     // block reduction), the codes go to shared memory in the even / odd order,
     // then each lane picks up its own
+    constexpr int kPer = (128 * NJ + kThreads - 1) / kThreads;  // 8-value chunks per thread
     const int nch = K >> 3;
     const uint4* src = reinterpret_cast<const uint4*>(x);
-    uint4 v[2];
+    uint4 v[kPer];
     uint32_t mb = 0u;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPer; ++i) {
       const int c = threadIdx.x + kThreads * i;
       v[i] = c < nch ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
       mb = bf16x2_absmax_bits(mb, v[i].x);
@@ -198,49 +258,58 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int w = 1; w < kWarps; ++w) amax_bits = max(amax_bits, amx_sm[w]);
     const float amax = __uint_as_float(amax_bits << 16);
     const float r = act_multiplier(amax);
+    const bool finite = amax_bits < 0x7F80u;  // block-uniform
     sxv = act_scale(amax);
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPer; ++i) {
       if (kThreads * i >= nch) break;  // block-uniform
       const int c = threadIdx.x + kThreads * i;
       int sum = 0;
       if (c < nch) {
-        const uint2 qc = quant_chunk(v[i], r, &sum);
-        *reinterpret_cast<uint2*>(xq_sm + 8 * c) = even_odd(qc.x, qc.y);
+        uint2 qc;
+        if (finite) {
+          qc = quant_chunk_even_odd(v[i], r);
+          sum = __dp4a((int)qc.x, 0x01010101, __dp4a((int)qc.y, 0x01010101, 0));
+        } else {  // an inf or NaN in the row: the general conversion
+          const uint2 qn = quant_chunk(v[i], r, &sum);
+          qc = even_odd(qn.x, qn.y);
+        }
+        *reinterpret_cast<uint2*>(xq_sm + 8 * c) = qc;
       }
-      // the 8 chunks of a group sit in 8 consecutive lanes (nch % 8 == 0)
-      sum = group8_sum(sum);
-      if ((lane & 7) == 0 && c < nch) xs_sm[c >> 3] = i32_to_f64(sum);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const uint4* p = reinterpret_cast<const uint4*>(xq_sm + 32 * (lane + 32 * j));
-      const uint4 a = p[0], b = p[1];
-      xr[j][0] = a.x; xr[j][1] = a.y; xr[j][2] = a.z; xr[j][3] = a.w;
-      xr[j][4] = b.x; xr[j][5] = b.y; xr[j][6] = b.z; xr[j][7] = b.w;
-      xsj[j] = xs_sm[16 * j + (lane >> 1)];
+      // the 4 chunks of a 32-code half-group sit in 4 consecutive lanes
+      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+      if ((lane & 3) == 0 && c < nch) xs_sm[c >> 2] = (double)sum;
     }
   } else {
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const uint4* p = reinterpret_cast<const uint4*>(xq) + 2 * (lane + 32 * j);
-      const uint4 a = __ldg(p), b = __ldg(p + 1);
-      const uint2 e0 = even_odd(a.x, a.y), e1 = even_odd(a.z, a.w);
-      const uint2 e2 = even_odd(b.x, b.y), e3 = even_odd(b.z, b.w);
-      xr[j][0] = e0.x; xr[j][1] = e0.y; xr[j][2] = e1.x; xr[j][3] = e1.y;
-      xr[j][4] = e2.x; xr[j][5] = e2.y; xr[j][6] = e3.x; xr[j][7] = e3.y;
-      xsj[j] = kDump ? 0.0 : i32_to_f64(__ldg(xsum + 16 * j + (lane >> 1)));
-    }
+    // cooperative: every thread permutes one 16-byte piece of xq into shared
+    // memory and sums its codes; the two pieces of a half-group are in
+    // consecutive lanes
+    const int nc = K >> 4;  // <= kThreads
+    const int c = threadIdx.x;
     if (!kDump) sxv = __ldg(sx);
+    const uint4 a = c < nc ? __ldg(reinterpret_cast<const uint4*>(xq) + c) : make_uint4(0u, 0u, 0u, 0u);
+    const uint2 e0 = even_odd(a.x, a.y), e1 = even_odd(a.z, a.w);
+    if (c < nc) *reinterpret_cast<uint4*>(xq_sm + 16 * c) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+    if constexpr (!kDump) {
+      int hs = __dp4a((int)a.x, 0x01010101, __dp4a((int)a.y, 0x01010101, 0));
+      hs = __dp4a((int)a.z, 0x01010101, __dp4a((int)a.w, 0x01010101, hs));
+      hs += __shfl_xor_sync(0xFFFFFFFFu, hs, 1);
+      if ((lane & 1) == 0 && c < nc) xs_sm[c >> 1] = (double)hs;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const uint4* p = reinterpret_cast<const uint4*>(xq_sm + 32 * (lane + 32 * j));
+    const uint4 a = p[0], b = p[1];
+    xr[j][0] = a.x; xr[j][1] = a.y; xr[j][2] = a.z; xr[j][3] = a.w;
+    xr[j][4] = b.x; xr[j][5] = b.y; xr[j][6] = b.z; xr[j][7] = b.w;
+    xh[j] = kDump ? 0.0 : xs_sm[lane + 32 * j];
   }
 
-  // A warp's four rows are all valid or all past N (rows is a multiple of 8),
-  // so they run as one straight-line block and their chains interleave.
-  const int r0 = warp * kRowsPerWarp;
+  // The four rows run as one straight-line block and their chains interleave.
   if (r0 < rows) {
-    mbar_wait(bars + 8u * warp, 0, err);  // this warp's rows landed
-    const bool odd = (lane & 1) != 0;
     double f[kRowsPerWarp];
 #pragma unroll
     for (int rr = 0; rr < kRowsPerWarp; ++rr) {
@@ -250,32 +319,35 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
         const uint4 wv = *reinterpret_cast<const uint4*>(wrow + 16 * (lane + 32 * j));
-        int acc = dot8(wv.x, xr[j][0], xr[j][1], 0);
-        acc = dot8(wv.y, xr[j][2], xr[j][3], acc);
-        acc = dot8(wv.z, xr[j][4], xr[j][5], acc);
-        acc = dot8(wv.w, xr[j][6], xr[j][7], acc);
-        const int accg = acc + __shfl_xor_sync(0xFFFFFFFFu, acc, 1);  // both halves of the group
-        const int g = 16 * j + (lane >> 1);
+        const int acc = dot32(wv, xr[j]);
         if constexpr (kDump) {
-          if (!odd) acc_out[(size_t)(n0 + r) * G + g] = accg;
+          const int accg = acc + __shfl_xor_sync(0xFFFFFFFFu, acc, 1);  // both halves of the group
+          if ((lane & 1) == 0) acc_out[(size_t)(n0 + r) * G + 16 * j + (lane >> 1)] = accg;
         } else {
-          // even lanes the scale term, odd lanes the offset term of group g
-          const double2 so = so_sm[r * G + g];
-          f[rr] = fma(odd ? so.y : so.x, odd ? xsj[j] : i32_to_f64(accg), f[rr]);
+          // each lane folds its half-group: s * acc + o * (sum of its codes)
+          const double2 so = so_sm[r * G + 16 * j + (lane >> 1)];
+          f[rr] = fma(so.x, i32_to_f64(acc), f[rr]);
+          f[rr] = fma(so.y, xh[j], f[rr]);
         }
       }
     }
     if constexpr (!kDump) {
-      // fixed-order butterflies, the four rows interleaved
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1)
-#pragma unroll
-        for (int rr = 0; rr < kRowsPerWarp; ++rr) f[rr] += __shfl_xor_sync(0xFFFFFFFFu, f[rr], o);
-      if (lane < kRowsPerWarp) {
-        double fr = f[0];
-#pragma unroll
-        for (int rr = 1; rr < kRowsPerWarp; ++rr) fr = lane == rr ? f[rr] : fr;
-        y[n0 + r0 + lane] = f64_to_bf16_bits(fma((double)sxv, fr, (double)bias_sm[r0 + lane]));
+      // fixed-order reduction of the four rows over the warp: halve the rows
+      // held per lane at the first two steps, then a butterfly; lane 8 q ends
+      // with row q
+      const bool up16 = (lane & 16) != 0, up8 = (lane & 8) != 0;
+      double a0 = up16 ? f[2] : f[0], a1 = up16 ? f[3] : f[1];
+      const double b0 = up16 ? f[0] : f[2], b1 = up16 ? f[1] : f[3];
+      a0 += __shfl_xor_sync(0xFFFFFFFFu, b0, 16);
+      a1 += __shfl_xor_sync(0xFFFFFFFFu, b1, 16);
+      double c = up8 ? a1 : a0;
+      c += __shfl_xor_sync(0xFFFFFFFFu, up8 ? a0 : a1, 8);
+      c += __shfl_xor_sync(0xFFFFFFFFu, c, 4);
+      c += __shfl_xor_sync(0xFFFFFFFFu, c, 2);
+      c += __shfl_xor_sync(0xFFFFFFFFu, c, 1);
+      if ((lane & 7) == 0) {
+        const int rr = lane >> 3;
+        y[n0 + r0 + rr] = f64_to_bf16_bits(fma((double)sxv, c, (double)bias_sm[r0 + rr]));
       }
     }
   }
