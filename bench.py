@@ -174,9 +174,10 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def traffic_from_profile(kernel_tag: str, src_path: str):
+def traffic_from_profile(kernel_tag: str, src_path: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current source of the kernel (matched by a hash of the .cu file)."""
+    the current source of the kernel (matched by a hash of the .cu file) and
+    on this workload (the summary's `workload:` line)."""
     import hashlib
 
     prof = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
@@ -187,7 +188,7 @@ def traffic_from_profile(kernel_tag: str, src_path: str):
             if ":" in line:
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
-        if fields.get("source_sha256_16") != digest:
+        if fields.get("source_sha256_16") != digest or fields.get("workload") != workload:
             return None
         return float(fields["dram_bytes_per_launch_full_workload"])
     except (OSError, KeyError, ValueError):
@@ -478,7 +479,7 @@ def run_ours(args, world, rank, local):
                            "gemv1_w4a8.cu" if one else "gemv_w4a8.cu")
         roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
-                "kernel": tag, "traffic": traffic_from_profile(tag, src)}
+                "kernel": tag, "traffic": traffic_from_profile(tag, src, args.workload)}
     elif not w4 and N <= 64 and M <= 8192:
         # thin W8A8 outputs run the split-K cluster kernel, bound by reading xq
         kbytes = M * K + N * K + 2 * M * N + 4 * (M + 2 * N)
@@ -486,7 +487,7 @@ def run_ours(args, world, rank, local):
         roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
                 "kernel": "w8a8_skinny_kernel",
-                "traffic": traffic_from_profile("w8a8_skinny_kernel", src)}
+                "traffic": traffic_from_profile("w8a8_skinny_kernel", src, args.workload)}
     else:
         peak = peaks["bf16"] * 2.0
         src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc",
@@ -496,7 +497,7 @@ def run_ours(args, world, rank, local):
                 "unit": "TFLOP/s",
                 "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2, the nominal int8/bf16 "
                                "ratio (4.5 / 2.25 POPS); int8 ops counted as 2*M*N*K",
-                "kernel": tag, "traffic": traffic_from_profile(tag, src)}
+                "kernel": tag, "traffic": traffic_from_profile(tag, src, args.workload)}
         if gated:
             roof["kernel"] = "w8a8_gemm_kernel (gated) with its activation quant: the timed call"
             roof["traffic"] = None  # the committed summary covers the plain epilogue

@@ -92,11 +92,15 @@ def test_every_workload_resolves_to_a_case():
 
 def test_traffic_lookup_follows_the_source_hash(tmp_path):
     csrc = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc")
-    for tag, src in [("w8a8_gemm_kernel", "gemm_w8a8.cu"), ("w4a8_gemm_kernel", "gemm_w4a8.cu")]:
+    cases = [("w8a8_gemm_kernel", "gemm_w8a8.cu", "dit_mlp"), ("w4a8_gemm_kernel", "gemm_w4a8.cu", "w4a8_m4096"),
+             ("w4a8_gemv1_kernel", "gemv1_w4a8.cu", "w4a8_m1")]
+    for tag, src, workload in cases:
         path = os.path.join(csrc, src)
-        t = bench.traffic_from_profile(tag, path)
+        t = bench.traffic_from_profile(tag, path, workload)
         assert t is None or t > 0  # a number only while the summary matches the source
+        # another workload of the same kernel never takes the summary's bytes
+        assert bench.traffic_from_profile(tag, path, "tiny") is None
         # any other file never matches the committed hash
         other = tmp_path / src
         other.write_bytes(open(path, "rb").read() + b"\n// edited\n")
-        assert bench.traffic_from_profile(tag, str(other)) is None
+        assert bench.traffic_from_profile(tag, str(other), workload) is None
