@@ -282,6 +282,9 @@ int qk_w4a8_linear_plan(int64_t M, int64_t K, int64_t N);
 /*
  * The product half of qk_w4a8_linear on quantized activations (xq, sx and
  * xsum from qk_quantize_activations), with an explicit route (qk_route).
+ * xsum must be the group sums of xq (as that call writes them): the one-token
+ * GEMV (M = 1, K a multiple of 1024 up to 4096) recomputes them from xq and
+ * does not read xsum, the other routes read it.
  * QK_ROUTE_GEMV with M > 16 returns QK_ERR_INVALID_ARG; with a shape whose
  * GEMV working set does not fit shared memory, QK_ERR_UNSUPPORTED_SHAPE.
  */
