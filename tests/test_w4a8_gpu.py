@@ -59,6 +59,36 @@ def test_gemv_group_acc_and_output(qk, orc, MKN):
     qk.qk_check_device_error()
 
 
+@pytest.mark.parametrize("K", [1024, 4096])
+def test_one_token_quantization_ties(qk, orc, K):
+    """The one-token GEMV quantizes bf16 x itself.  A row whose absmax is 127
+    has the multiplier 1, so values k + 1/2 sit exactly on rounding ties: its
+    output must equal, bit for bit, the product on the codes of the stand-alone
+    quantization kernel (which match the oracle), and the oracle within 2 ulp."""
+    N = 264
+    case = synthetic.LinearCase("ties", M=1, K=K, N=N, bias=True, seed=K + 5)
+    _, dev_w, ora_w, b = prepare(qk, orc, case)
+    rng = np.random.default_rng(K)
+    halves = np.arange(127, dtype=np.float32) + np.float32(0.5)            # 0.5 .. 126.5
+    vals = np.concatenate([halves, -halves, np.arange(-127, 128, dtype=np.float32)])
+    row = rng.choice(vals, size=K).astype(np.float32)
+    row[rng.integers(0, K)] = 127.0
+    xb = synthetic.f32_to_bf16_bits(row[None, :])
+    assert np.array_equal((xb.astype(np.uint32) << 16).view(np.float32), row[None, :])  # exact in bf16
+    x = to_dev_bf16(xb)
+    xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
+    bias = to_dev(b)
+    y = qk.qk_w4a8_linear(x, *dev_w, bias)
+    y2 = qk.qk_w4a8_gemm(xq, sx, xsum, *dev_w, bias, route=GEMV)
+    torch.cuda.synchronize()
+    y_o, xq_o, sx_o, _, _ = orc.w4a8_linear(xb, *ora_w, b)
+    assert float(sx_o[0]) == 1.0
+    assert np.array_equal(host(xq), xq_o)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    assert bf16_ulp_distance(t2bits(y), y_o).max() <= TOL_ULP
+    qk.qk_check_device_error()
+
+
 @pytest.mark.parametrize("case", synthetic.W4A8[:3], ids=lambda c: c.name)
 def test_w4a8_gemv_configs(qk, orc, case):
     xb, dev_w, ora_w, b = prepare(qk, orc, case)
