@@ -31,6 +31,11 @@ MUTANTS = [
     ("gated_residual_dropped", "t = t + (double)oracle_bf16_to_f32(r[m * N + n]);", "t = t;"),
     ("gated_gate_skips_bias", "double t = (double)gate[n] * v;",
      "double t = (double)gate[n] * (v - (bias ? (double)bias[n] : 0.0)) + (bias ? (double)bias[n] : 0.0);"),
+    ("act_divide_by_scale", "float t = v[k] * r;", "float t = v[k] / s;"),
+    ("w4_divide_by_scale", "float t = (w[i] - o) * r;", "float t = (w[i] - o) / s;"),
+    ("w4_codes_from_unrounded_scale", "float s = oracle_f16_to_f32(sb);",
+     "float s = (hi - lo) / 15.0f;"),
+    ("w4_codes_from_unrounded_offset", "float o = oracle_f16_to_f32(ob);", "float o = lo;"),
     ("group_sum_window", "for (int64_t k = 64 * g; k < 64 * g + 64; ++k)\n                s += xq[m * K + k];",
      "for (int64_t k = 64 * g; k < 64 * g + 63; ++k)\n                s += xq[m * K + k];"),
     ("sage_scale_dropped", "s[j] = (double)dot * (double)sq[i] * (double)sk[j] * scale;",

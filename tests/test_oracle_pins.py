@@ -187,20 +187,37 @@ def unpack_codes(Wp):
     return np.stack([lo, hi], axis=-1).reshape(Wp.shape[0], -1)
 
 
-def test_w4_affine_grid_golden(orc):
-    """Groups built on an fp16 affine grid come back with the same s, o and codes."""
+def w4_golden_groups():
+    """The hand-derived W4 groups of ``tests/golden/w4_affine_groups.json`` as
+    (64 fp32 inputs, scale fp16 bits, offset fp16 bits, codes): the fp16 affine
+    grids, and the groups given by their inputs that tell the reading R5 (codes
+    from the fp16-rounded scale and offset, times the reciprocal of the scale)
+    from the alternatives."""
     with open(os.path.join(GOLDEN, "w4_affine_groups.json")) as fh:
         fx = json.load(fh)
-    rows = []
+    out = []
     for grp in fx["groups"]:
         codes = np.array(grp["codes"], np.float32)
-        rows.append(np.float32(grp["offset"]) + codes * np.float32(grp["scale"]))
-    W = np.concatenate(rows)[None, :]              # one row, two groups
+        w = np.float32(grp["offset"]) + codes * np.float32(grp["scale"])
+        out.append((w, int(grp["scale_f16"], 16), int(grp["offset_f16"], 16), grp["codes"]))
+    for grp in fx["groups_w"]:
+        w = np.array(grp["w"], np.float32)
+        assert np.array_equal(w.astype(np.float64), np.array(grp["w"], np.float64))  # exact in fp32
+        out.append((w, int(grp["scale_f16"], 16), int(grp["offset_f16"], 16), grp["codes"]))
+    return out
+
+
+def test_w4_affine_grid_golden(orc):
+    """Groups built on an fp16 affine grid come back with the same s, o and
+    codes; the groups built to separate R5 from its alternatives (division by
+    the scale, codes from the unrounded scale or offset) give R5's codes."""
+    groups = w4_golden_groups()
+    W = np.concatenate([g[0] for g in groups])[None, :]    # one row, one group each
     Wp, s, o = orc.quant_w4(W)
-    for g, grp in enumerate(fx["groups"]):
-        assert s[0, g] == int(grp["scale_f16"], 16)
-        assert o[0, g] == int(grp["offset_f16"], 16)
-        assert unpack_codes(Wp)[0, 64 * g:64 * g + 64].tolist() == grp["codes"]
+    for g, (_, s16, o16, codes) in enumerate(groups):
+        assert s[0, g] == s16
+        assert o[0, g] == o16
+        assert unpack_codes(Wp)[0, 64 * g:64 * g + 64].tolist() == codes
 
 
 def test_w4_pack_nibble_order(orc):

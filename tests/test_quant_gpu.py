@@ -93,15 +93,13 @@ def test_w4_weight_quant_bit_exact(qk, orc, NK):
 
 
 def test_w4_golden_groups(qk):
-    from tests.test_oracle_pins import GOLDEN, unpack_codes
+    from tests.test_oracle_pins import unpack_codes, w4_golden_groups
 
-    with open(os.path.join(GOLDEN, "w4_affine_groups.json")) as fh:
-        groups = json.load(fh)["groups"]
-    W = np.concatenate([np.float32(g["offset"]) + np.array(g["codes"], np.float32) *
-                        np.float32(g["scale"]) for g in groups])[None, :]
+    groups = w4_golden_groups()
+    W = np.concatenate([g[0] for g in groups])[None, :]
     Wp, s, o = qk.qk_quantize_weights_int4(to_dev(W.astype(np.float32)))
     codes = unpack_codes(host(Wp))
-    for i, g in enumerate(groups):
-        assert t2bits(s)[0, i] == int(g["scale_f16"], 16)
-        assert t2bits(o)[0, i] == int(g["offset_f16"], 16)
-        assert codes[0, 64 * i: 64 * i + 64].tolist() == g["codes"]
+    for i, (_, s16, o16, want) in enumerate(groups):
+        assert t2bits(s)[0, i] == s16
+        assert t2bits(o)[0, i] == o16
+        assert codes[0, 64 * i: 64 * i + 64].tolist() == want
