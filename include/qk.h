@@ -79,7 +79,7 @@ int qk_version(void);
 int qk_is_available(int device);
 
 /*
- * Shape contract (qk_w8a8_*): 1 <= K <= 65536 with K % 32 == 0; N >= 8 with
+ * Shape contract (qk_w8a8_*): 32 <= K <= 65536 with K % 32 == 0; N >= 8 with
  * N % 8 == 0; M >= 0 (M == 0 returns QK_OK and launches nothing).
  * W4A8 (qk_w4a8_*, qk_quantize_weights_int4): additionally K % 64 == 0.
  * A shape outside the contract returns QK_ERR_UNSUPPORTED_SHAPE.
@@ -153,7 +153,12 @@ qk_status qk_quantize_activations(const uint16_t *x, int64_t M, int64_t K,
  *   y[m, n] = bf16( acc[m, n] * sx[m] * sw[n] + bias[n] ),
  *   acc[m, n] = sum_k xq[m, k] * Wq[n, k]  (exact int32),
  * where xq, sx are the per-token quantization of x (qk_quantize_activations).
- * The dequant is evaluated in fp64 and rounded once to bf16 (nearest even).
+ * The dequant is evaluated in fp32, fma(fp32(acc) * sx, sw, bias), wherever
+ * a per-element guard (|that value| >= 2^-12 |bias|, and no fp32 underflow)
+ * proves it within 1/8 bf16 ulp of the exact value; every other element
+ * (cancellation against the bias) takes the exact fp64 evaluation.  Each
+ * element is rounded once to bf16 (nearest even) and lies within 1 bf16 ulp
+ * of the exact value rounded once (0 ulp on most elements).
  *   x         : bf16 bits [M, K]   (in)
  *   Wq, sw    : from qk_quantize_weights_int8 (in)
  *   bias      : fp32 [N] (in, nullable: no bias)
@@ -174,8 +179,11 @@ qk_status qk_w8a8_linear(const uint16_t *x, int64_t M, int64_t K,
  * list: a quantized matmul with a gated residual epilogue, each element held
  * within 2 ulp), the update of a DiT block's residual stream:
  *   y[m, n] = bf16( residual[m, n] + gate[n] * (acc[m, n] * sx[m] * sw[n] + bias[n]) )
- * evaluated in fp64 and rounded once to bf16 (nearest even); the bracket is
- * the value qk_w8a8_linear rounds.
+ * rounded once to bf16 (nearest even); the bracket is the value qk_w8a8_linear
+ * rounds.  As there, fp32 evaluates every element a guard proves within half
+ * a bf16 ulp of the exact value, and the exact fp64 evaluation takes the rest
+ * (cancellation against the residual or the bias): within 1 bf16 ulp of the
+ * exact value rounded once.
  *   x, Wq, sw, bias, workspace : as for qk_w8a8_linear
  *   gate      : fp32 [N], one gate per output channel (in)
  *   residual  : bf16 bits [M, N] (in); y may be the residual itself (an
@@ -225,6 +233,9 @@ qk_status qk_w8a8_gemm(const int8_t *xq, const float *sx, int64_t M, int64_t K,
  *     overwrites the part it reads).  Calls whose executions overlap on the GPU
  *     (for example on two streams without ordering between them) race on the
  *     scratch and give wrong results: order them on one stream or with events.
+ *   - The scratch address is resolved once per device and kept; after
+ *     cudaDeviceReset (which unloads the module and its array) this entry
+ *     point must not be called again in the same process.
  * Arguments, layouts and the other errors are those of qk_w8a8_linear.
  */
 #define QK_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)

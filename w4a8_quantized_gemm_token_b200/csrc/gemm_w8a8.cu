@@ -3,7 +3,8 @@
 // Computes ("qlip-mlx" README, "w8a8_linear / W8A8Linear": INT8 x INT8 ->
 // INT32 matmul with dequant + bias fused behind it)
 //     acc[m, n] = sum_k xq[m, k] * Wq[n, k]                  (exact int32)
-//     y[m, n]   = bf16( acc * sx[m] * sw[n] + bias[n] )      (fp64, one rounding)
+//     y[m, n]   = bf16( acc * sx[m] * sw[n] + bias[n] )      (one rounding)
+// within 1 bf16 ulp of the exact value rounded once (see the epilogue below).
 //
 // Design (sm_100a):
 //  * CTA pairs (clusters of 2) run one tcgen05.mma.cta_group::2 kind::i8 over
@@ -18,13 +19,18 @@
 //  * warp 1 of the leader issues the MMAs (M = 256, N = 256, K = 32 each) into
 //    one of two 256-column accumulators and commits each stage and each
 //    finished accumulator to the barriers of both CTAs;
-//  * warps 2-5 (4 per CTA): epilogue.  tcgen05.ld, then exact int32 -> fp64
-//    (2^52 magic number), acc * sx exact in fp64, one fused multiply-add with
-//    sw and bias (pre-converted to fp64 once per tile in shared memory), and
-//    the fp64 -> bf16 round-to-nearest-even done with integer operations on the
-//    double's bits; rows staged in a swizzled shared buffer and written with TMA
-//    stores that clip the M and N edges.  Conversions avoid the XU pipe, whose
-//    throughput made the epilogue the bottleneck.
+//  * warps 2-5 (4 per CTA): epilogue.  tcgen05.ld of 32 columns at a time,
+//    then a guarded fp32 fast path: v32 = fma(fp32(acc) * sx, sw, bias) with
+//    per-column {sw, bias, guard, gate} built once per tile in shared memory.
+//    Where |v32| >= 2^-12 |bias| (and v32 is far from fp32 underflow) its error
+//    is below 1/8 bf16 ulp, so its rounding is within 1 ulp of the exact value
+//    rounded once; the few elements that fail the guard (cancellation against
+//    the bias) take the exact path: int32 -> fp64 by the 2^52 magic number,
+//    acc * sx exact in fp64, one fused multiply-add with sw and bias, and the
+//    fp64 -> bf16 round-to-nearest-even done with integer operations on the
+//    double's bits.  Rows are staged in a swizzled shared buffer and written
+//    with TMA stores that clip the M and N edges.  Conversions avoid the XU
+//    pipe, whose throughput had made the epilogue the bottleneck.
 // Every mbarrier wait is bounded (sm100.cuh); no load uses cluster multicast.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>

@@ -34,7 +34,10 @@ uint8_t* g_scratch_addr[kMaxDevices];
 std::mutex g_scratch_mu;
 
 // Device address of this device's copy of the scratch; resolved on the first
-// call made with that device current.  Null if the lookup fails.
+// call made with that device current and kept for the life of the process
+// (cudaDeviceReset unloads the module, after which the kept address is stale:
+// the header says not to call this entry point after a reset).  Null if the
+// lookup fails.
 uint8_t* scratch_address(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
@@ -64,8 +67,9 @@ extern "C" qk_status qk_w8a8_linear_noalloc(const uint16_t* x, int64_t M, int64_
     return QK_ERR_MISALIGNED;
   // codes [M, K] and scales [M] must fit the built-in scratch
   if (qk_w8a8_workspace_size(M, K) > (size_t)QK_NOALLOC_SCRATCH_BYTES) return QK_ERR_WORKSPACE;
+  if (qk::check_device() != QK_OK) return QK_ERR_NO_DEVICE;
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || !qk_is_available(dev)) return QK_ERR_NO_DEVICE;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QK_ERR_NO_DEVICE;
   uint8_t* scratch = scratch_address(dev);
   if (scratch == nullptr) return QK_ERR_CUDA;
 

@@ -57,13 +57,6 @@ qk_status check_shape(int64_t M, int64_t K, int64_t N, bool w4) {
   return QK_OK;
 }
 
-qk_status check_device() {
-  const int d = current_device();
-  if (d < 0 || d >= kMaxDevices) return QK_ERR_NO_DEVICE;
-  if (g_cc_ok[d] == 0) g_cc_ok[d] = qk_is_available(d) ? 1 : -1;
-  return g_cc_ok[d] == 1 ? QK_OK : QK_ERR_NO_DEVICE;
-}
-
 qk_status from_cuda(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return QK_OK;
   if (log_enabled()) std::fprintf(stderr, "[qk] %s: %s\n", what, cudaGetErrorString(e));
@@ -102,6 +95,13 @@ struct Workspace {
 };
 
 }  // namespace
+
+qk_status check_device() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return QK_ERR_NO_DEVICE;
+  if (g_cc_ok[d] == 0) g_cc_ok[d] = qk_is_available(d) ? 1 : -1;
+  return g_cc_ok[d] == 1 ? QK_OK : QK_ERR_NO_DEVICE;
+}
 
 int* device_error_word() {
   const int d = current_device();

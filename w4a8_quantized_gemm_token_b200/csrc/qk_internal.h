@@ -94,6 +94,10 @@ cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* x
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
                              int64_t m0, int64_t m1, bool pdl, cudaStream_t s);
 
+// QK_OK if the current device is an sm_100 device (the answer is cached per
+// device after the first query), else QK_ERR_NO_DEVICE.
+qk_status check_device();
+
 // Address of this device's error word (a __device__ int of the library),
 // resolved once per device with cudaGetSymbolAddress; null on failure.
 int* device_error_word();
