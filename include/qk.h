@@ -372,6 +372,20 @@ qk_status qk_debug_w4a8_group_acc(const int8_t *xq, int64_t M, int64_t K,
                                   int route, qk_stream_t stream);
 
 /*
+ * A probe of the device's INT8 tensor-pipe throughput (the denominator of the
+ * W8A8 GEMM's roofline fraction; the pages have no counterpart).  One CTA pair
+ * per two SMs issues `iters` x 8 tcgen05.mma.cta_group::2.kind::i8 of
+ * M = 256, N = 256, K = 32 -- the instruction stream of the W8A8 GEMM's
+ * mainloop -- on operands resident in shared memory (no global loads, no
+ * epilogue).  If `ops` is not NULL it receives (on the host, at return) the
+ * int8 operations the launch performs, 2 * 256 * 256 * 32 per MMA; the caller
+ * times the launch on `stream`.  1 <= iters <= 2^24 (one iteration takes about
+ * half a microsecond at full clock), else QK_ERR_INVALID_ARG.  The one wait
+ * (for the issued MMAs to drain) is bounded as in every kernel here.
+ */
+qk_status qk_debug_int8_peak(int64_t iters, double *ops, qk_stream_t stream);
+
+/*
  * The timeout path of the library's bounded waits, for tests: launches one
  * single-thread kernel that waits on an mbarrier no thread arrives at and on
  * a device word no thread sets.  Each wait gives up after limit_cycles SM

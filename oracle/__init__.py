@@ -22,7 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "qk_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared"]
+CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared"]
 
 
 def build(force: bool = False) -> str:
@@ -45,6 +45,7 @@ def _bind(path: str):
         "oracle_f32_to_f16": (ctypes.c_uint16, [ctypes.c_float]),
         "oracle_f16_to_f32": (ctypes.c_float, [ctypes.c_uint16]),
         "oracle_f64_to_bf16": (ctypes.c_uint16, [ctypes.c_double]),
+        "oracle_set_threads": (ctypes.c_int, [ctypes.c_int]),
         "oracle_quant_act_bf16": (None, [P, I64, I64, P, P]),
         "oracle_quant_w8": (None, [P, I64, I64, P, P]),
         "oracle_group_sums": (None, [P, I64, I64, P]),
@@ -71,7 +72,15 @@ def _load():
     global _lib
     if _lib is None:
         _lib = _bind(build())
+        _lib.oracle_set_threads(int(os.environ.get("QK_ORACLE_THREADS", "1")))
     return _lib
+
+
+def set_threads(n: int) -> int:
+    """Let the oracle's row loops use `n` OpenMP threads (each output is still
+    computed by one thread in the same order, so results do not change);
+    returns the count in effect."""
+    return int(_load().oracle_set_threads(int(n)))
 
 
 @contextlib.contextmanager
@@ -81,6 +90,7 @@ def using_library(path: str):
     global _lib
     saved = _load()
     _lib = _bind(path)
+    _lib.oracle_set_threads(int(os.environ.get("QK_ORACLE_THREADS", "1")))
     try:
         yield
     finally:

@@ -7,9 +7,15 @@
  * header, table or helper with the CUDA library: the library never links it and
  * it never includes anything from the library.
  *
- * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fPIC -shared
+ * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fopenmp -fPIC -shared
  * (x86-64 SSE arithmetic, so every float operation below is one IEEE binary32
  * operation in round-to-nearest-even, and no multiply-add is fused).
+ *
+ * Threads: the outer loop over independent rows (tokens, or output channels
+ * for the weight quantization) may be split over OpenMP threads.  Each output
+ * is still computed by one thread in the order written here, so the results
+ * are the same bits at any thread count.  oracle_set_threads picks the count
+ * (the Python loader sets 1 unless asked otherwise).
  *
  * Sources (by page and section):
  *   [qlip] "qlip-mlx" README, intro bullet "w8a8_linear / W8A8Linear":
@@ -56,6 +62,23 @@
 #include <stdlib.h>
 #include <string.h>
 #include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Number of threads the row loops below may use; returns the count in effect
+ * (1 when the library is built without OpenMP). */
+int oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 /* ---------------------------------------------------------------- encodings */
 
@@ -167,20 +190,25 @@ static void quant_row_sym(const float *v, int64_t K, int8_t *q, float *scale)
 void oracle_quant_act_bf16(const uint16_t *x, int64_t M, int64_t K,
                            int8_t *xq, float *sx)
 {
-    float *row = (float *)malloc((size_t)K * sizeof(float));
-    if (!row)
-        return;
-    for (int64_t m = 0; m < M; ++m) {
-        for (int64_t k = 0; k < K; ++k)
-            row[k] = oracle_bf16_to_f32(x[m * K + k]);
-        quant_row_sym(row, K, xq + m * K, sx + m);
+#pragma omp parallel
+    {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+#pragma omp for schedule(static)
+        for (int64_t m = 0; m < M; ++m) {
+            if (!row)
+                continue;
+            for (int64_t k = 0; k < K; ++k)
+                row[k] = oracle_bf16_to_f32(x[m * K + k]);
+            quant_row_sym(row, K, xq + m * K, sx + m);
+        }
+        free(row);
     }
-    free(row);
 }
 
 /* W8 weight quantization (R4): W fp32 [N, K] -> Wq int8 [N, K], sw fp32 [N]. */
 void oracle_quant_w8(const float *W, int64_t N, int64_t K, int8_t *Wq, float *sw)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n)
         quant_row_sym(W + n * K, K, Wq + n * K, sw + n);
 }
@@ -211,6 +239,7 @@ void oracle_quant_w4(const float *W, int64_t N, int64_t K,
                      uint8_t *Wp, uint16_t *s16, uint16_t *o16)
 {
     int64_t G = K / 64;
+#pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n)
         for (int64_t g = 0; g < G; ++g) {
             const float *w = W + n * K + 64 * g;
@@ -261,6 +290,7 @@ static int w4_code(const uint8_t *Wp, int64_t K, int64_t n, int64_t k)
 void oracle_w8a8_acc(const int8_t *xq, int64_t M, int64_t K,
                      const int8_t *Wq, int64_t N, int64_t *acc)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             int64_t s = 0;
@@ -278,6 +308,7 @@ void oracle_w4a8_group_acc(const int8_t *xq, int64_t M, int64_t K,
                            const uint8_t *Wp, int64_t N, int64_t *acc)
 {
     int64_t G = K / 64;
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
             for (int64_t g = 0; g < G; ++g) {
@@ -298,6 +329,7 @@ void oracle_w8a8_dequant_f64(const int64_t *acc, int64_t M, int64_t N,
                              const float *sx, const float *sw, const float *bias,
                              double *v)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             double t = ((double)acc[m * N + n] * (double)sx[m]) * (double)sw[n];
@@ -312,6 +344,7 @@ void oracle_w8a8_dequant(const int64_t *acc, int64_t M, int64_t N,
                          const float *sx, const float *sw, const float *bias,
                          uint16_t *y)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
         double v;
         for (int64_t n = 0; n < N; ++n) {
@@ -333,6 +366,7 @@ void oracle_w8a8_gated(const int64_t *acc, int64_t M, int64_t N,
                        const float *sx, const float *sw, const float *bias,
                        const float *gate, const uint16_t *r, uint16_t *out)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             double v;
@@ -355,6 +389,7 @@ void oracle_w4a8_dequant_f64(const int64_t *acc, const int32_t *xsum,
                              const float *sx, const uint16_t *s16, const uint16_t *o16,
                              const float *bias, double *v)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             double f = 0.0;
@@ -378,6 +413,7 @@ void oracle_w4a8_dequant(const int64_t *acc, const int32_t *xsum,
                          const float *sx, const uint16_t *s16, const uint16_t *o16,
                          const float *bias, uint16_t *y)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             double v;
@@ -402,37 +438,41 @@ void oracle_sage_attention_rows(const int8_t *qc, const float *sq, const int8_t 
                                 double scale, const int64_t *rows, int64_t nrows,
                                 double *out_f64, uint16_t *out)
 {
-    double *s = (double *)malloc((size_t)L * sizeof(double));
-    double *o = (double *)malloc((size_t)D * sizeof(double));
-    for (int64_t r = 0; r < nrows; ++r) {
-        const int64_t i = rows[r];
-        double mx = -INFINITY;
-        for (int64_t j = 0; j < L; ++j) {
-            int64_t dot = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc((size_t)L * sizeof(double));
+        double *o = (double *)malloc((size_t)D * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            const int64_t i = rows[r];
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < L; ++j) {
+                int64_t dot = 0;
+                for (int64_t d = 0; d < D; ++d)
+                    dot += (int64_t)qc[i * D + d] * (int64_t)kc[j * D + d];
+                s[j] = (double)dot * (double)sq[i] * (double)sk[j] * scale;
+                if (s[j] > mx)
+                    mx = s[j];
+            }
+            double l = 0.0;
             for (int64_t d = 0; d < D; ++d)
-                dot += (int64_t)qc[i * D + d] * (int64_t)kc[j * D + d];
-            s[j] = (double)dot * (double)sq[i] * (double)sk[j] * scale;
-            if (s[j] > mx)
-                mx = s[j];
+                o[d] = 0.0;
+            for (int64_t j = 0; j < L; ++j) {
+                double p = exp(s[j] - mx);
+                l += p;
+                for (int64_t d = 0; d < D; ++d)
+                    o[d] += p * (double)oracle_bf16_to_f32(v[j * D + d]);
+            }
+            for (int64_t d = 0; d < D; ++d) {
+                double res = o[d] / l;
+                if (out_f64)
+                    out_f64[r * D + d] = res;
+                out[r * D + d] = oracle_f64_to_bf16(res);
+            }
         }
-        double l = 0.0;
-        for (int64_t d = 0; d < D; ++d)
-            o[d] = 0.0;
-        for (int64_t j = 0; j < L; ++j) {
-            double p = exp(s[j] - mx);
-            l += p;
-            for (int64_t d = 0; d < D; ++d)
-                o[d] += p * (double)oracle_bf16_to_f32(v[j * D + d]);
-        }
-        for (int64_t d = 0; d < D; ++d) {
-            double res = o[d] / l;
-            if (out_f64)
-                out_f64[r * D + d] = res;
-            out[r * D + d] = oracle_f64_to_bf16(res);
-        }
+        free(s);
+        free(o);
     }
-    free(s);
-    free(o);
 }
 
 /* The same for every query row 0 .. L - 1 (outputs [L, D]). */

@@ -517,3 +517,28 @@ def test_sage_close_to_unquantized_attention(orc):
     p2 = np.exp(s2 - s2.max(axis=1, keepdims=True))
     wrong = (p2 @ vf) / p2.sum(axis=1, keepdims=True)
     assert np.abs(o64 - wrong).max() / np.abs(ref).max() > 10 * err
+
+
+# ------------------------------------------------------------ threading
+
+def test_thread_count_does_not_change_results(orc):
+    """The row loops may run on several OpenMP threads (the CPU baseline's
+    multi-core leg); every output is still computed by one thread in the same
+    order, so 1 and 4 threads give the same bits."""
+    case = synthetic.LinearCase("thr", M=37, K=256, N=40, outlier_frac=0.02, seed=31)
+    xb, W, b, _ = case.draw()
+    outs = []
+    try:
+        for n in (1, 4):
+            orc.set_threads(n)
+            Wq, sw = orc.quant_w8(W)
+            Wp, s16, o16 = orc.quant_w4(W)
+            y8 = orc.w8a8_linear(xb, Wq, sw, b)
+            y4 = orc.w4a8_linear(xb, Wp, s16, o16, b)
+            q, k, v = (xb[:32, :128], xb[1:33, :128], xb[2:34, :128])
+            att = orc.sage_attention_head(q, k, v, 128 ** -0.5)
+            outs.append([Wq, sw, Wp, s16, o16, *y8, *y4, att])
+    finally:
+        orc.set_threads(1)
+    for a, c in zip(*outs):
+        assert np.array_equal(a, c)

@@ -42,6 +42,7 @@ _SIGS = {
     "qk_debug_w8a8_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P]),
     "qk_debug_w4a8_group_acc": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I, _P]),
     "qk_debug_wait_timeout": (_I, [_I64, _P]),
+    "qk_debug_int8_peak": (_I, [_I64, _P, _P]),
     "qk_sage_attention_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "qk_sage_attention": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]),
 }
@@ -290,6 +291,15 @@ def qk_debug_wait_timeout(limit_cycles: int, stream=None) -> None:
     after `limit_cycles` SM cycles and records QK_ERR_TIMEOUT for
     qk_check_device_error."""
     _check(lib.qk_debug_wait_timeout(int(limit_cycles), _stream(stream)), "qk_debug_wait_timeout")
+
+
+def qk_debug_int8_peak(iters: int, stream=None) -> float:
+    """Launch the INT8 tensor-pipe probe (`iters` x 8 kind::i8 MMAs of
+    256 x 256 x 32 per CTA pair); returns the int8 operations it performs."""
+    ops = ctypes.c_double(0.0)
+    _check(lib.qk_debug_int8_peak(int(iters), ctypes.byref(ops), _stream(stream)),
+           "qk_debug_int8_peak")
+    return float(ops.value)
 
 
 def qk_sage_attention_workspace_size(B: int, H: int, L: int) -> int:

@@ -467,6 +467,18 @@ qk_status qk_debug_wait_timeout(int64_t limit_cycles, qk_stream_t stream) {
   return from_cuda(launch_wait_timeout_probe((long long)limit_cycles, stream), "wait_timeout_probe");
 }
 
+qk_status qk_debug_int8_peak(int64_t iters, double* ops, qk_stream_t stream) {
+  if (iters < 1 || iters > (int64_t(1) << 24)) return QK_ERR_INVALID_ARG;
+  qk_status st = check_device();
+  if (st != QK_OK) return st;
+  int* err = device_error_word();
+  if (err == nullptr) return QK_ERR_CUDA;
+  int pairs = 0;
+  st = from_cuda(launch_int8_peak((long long)iters, err, &pairs, stream), "int8_peak");
+  if (st == QK_OK && ops != nullptr) *ops = int8_peak_ops_per_iter(pairs) * (double)iters;
+  return st;
+}
+
 qk_status qk_debug_w8a8_acc(const int8_t* xq, int64_t M, int64_t K, const int8_t* Wq, int64_t N,
                             int32_t* acc, qk_stream_t stream) {
   qk_status st = check_shape(M, K, N, false);

@@ -98,6 +98,12 @@ cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* x
 // device after the first query), else QK_ERR_NO_DEVICE.
 qk_status check_device();
 
+// The INT8 tensor-pipe probe (peak_i8.cu): one pair of CTAs per two SMs,
+// each pair issuing `iters` x 8 tcgen05 kind::i8 MMAs of 256 x 256 x 32.
+// *pairs_out receives the number of pairs launched.
+cudaError_t launch_int8_peak(long long iters, int* err, int* pairs_out, cudaStream_t s);
+double int8_peak_ops_per_iter(int num_pairs);
+
 // Address of this device's error word (a __device__ int of the library),
 // resolved once per device with cudaGetSymbolAddress; null on failure.
 int* device_error_word();
