@@ -8,9 +8,20 @@ One step = one call of the linear (activation quant + tcgen05 GEMM with the
 fused dequant epilogue) on one batch of synthetic input already resident in
 HBM.  The default workload is the DiT MLP projection W8A8 linear,
 x [16384, 3072] bf16 -> y [16384, 12288] bf16 (1% outlier channels x20, bias).
-Rank 0 prints one JSON line.  Under torchrun each rank is an independent
-replica (the path needs no collective): per-GPU work is fixed, the value is the
-sum over ranks divided by the slowest rank's time ("scaling": "weak").
+Rank 0 prints one JSON line.  On one GPU the default run also carries
+  - `int8_peak_probe`: the INT8 tensor-pipe rate measured on the device by the
+    library's probe (the GEMM's tcgen05 kind::i8 MMA stream on shared-memory
+    operands), burst and sustained, with clocks -- the roofline denominator;
+  - `sustained`: the headline call back to back for two seconds, with clocks;
+  - `workloads`: every other configuration (tiny, the DiT attention
+    projection, the M = 2048 sweep, W4A8 at M = 1 / 8 / 16 / 4096, the
+    quick-start matmul, the gated epilogue, the INT8 attention), each with its
+    per-call time, throughput, the dominant kernel alone and its roofline
+    fraction;
+  - `cpu_baseline`: the oracle on the host cores, one thread and all cores.
+Under torchrun each rank is an independent replica (the path needs no
+collective): per-GPU work is fixed, the value is the sum over ranks divided by
+the slowest rank's time ("scaling": "weak").
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and torch.cuda.synchronize(), CUDA events on the launching stream, max over
@@ -19,8 +30,9 @@ its operands from HBM (x 100.7 MB + Wq 37.7 MB per set, y 402.7 MB written per
 step; more than the 126 MB L2).  SM clocks and throttle reasons are sampled
 with NVML during the timed region.
 
-`--impl reference` times the CPU oracle (oracle/, plain C) on the host cores
-for the same metric, one bounded sample of the workload per step.
+`--impl reference` times the CPU oracle (oracle/, plain C, OpenMP over rows)
+on all host cores for the same metric, one bounded sample of the workload per
+step.
 """
 from __future__ import annotations
 
@@ -254,15 +266,284 @@ def graph_runner(fn, steps):
     return g.replay
 
 
-def run_attention(args, world, rank, local):
+def event_ms(run, stream):
+    """Milliseconds of run() between two CUDA events on `stream` (synchronized
+    on both sides)."""
+    import torch
+
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def csrc(name):
+    return os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc", name)
+
+
+class LinearRun:
+    """One W8A8 / W4A8 linear workload resident on the device: rotating input
+    sets (enough that one pass over them exceeds twice the L2), quantized
+    weights, a workspace and the output."""
+
+    def __init__(self, name, dev, sets=0):
+        import torch
+
+        from w4a8_quantized_gemm_token_b200 import binding as qk
+        from w4a8_quantized_gemm_token_b200 import synthetic
+
+        self.qk, self.name, self.dev = qk, name, dev
+        self.case = case = get_case(name)
+        M, K, N = self.M, self.K, self.N = case.M, case.K, case.N
+        self.w4, self.gated = is_w4(name), is_gated(name)
+        xb, W, b, _ = case.draw()
+        self.x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
+        del xb
+        if self.gated:
+            gate_np, res_bits = synthetic.gated_inputs(case)
+            self.gate = torch.from_numpy(gate_np).to(dev)
+            self.res_host = torch.from_numpy(res_bits.view(np.int16)).view(torch.bfloat16)
+            self.res = self.res_host.to(dev)
+            del res_bits
+        W_dev = torch.from_numpy(W).to(dev)
+        del W
+        self.bias = torch.from_numpy(b).to(dev) if b is not None else None
+        w4 = self.w4
+        self.per_set = M * K * 2 + (N * K // 2 + N * (K // 64) * 4 if w4 else N * K + 4 * N)
+        self.nsets = sets or int(min(32, max(2, -(-2 * L2_BYTES // self.per_set))))
+        self.xs = [self.x_host.to(dev) for _ in range(self.nsets)]
+        if w4:
+            self.weights = [qk.qk_quantize_weights_int4(W_dev) for _ in range(self.nsets)]
+            wsz = qk.qk_w4a8_workspace_size(M, K)
+        else:
+            self.weights = [qk.qk_quantize_weights_int8(W_dev) for _ in range(self.nsets)]
+            wsz = qk.qk_w8a8_workspace_size(M, K)
+        del W_dev
+        self.ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        self.y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.ops = 2.0 * M * N * K
+        self.xq_sets = None
+
+    def step(self, i):
+        qk, wt, x = self.qk, self.weights[i % self.nsets], self.xs[i % self.nsets]
+        if self.w4:
+            qk.qk_w4a8_linear(x, *wt, self.bias, y=self.y, workspace=self.ws)
+        elif self.gated:
+            qk.qk_w8a8_linear_gated(x, *wt, self.bias, self.gate, self.res, y=self.y,
+                                    workspace=self.ws)
+        else:
+            qk.qk_w8a8_linear(x, *wt, self.bias, y=self.y, workspace=self.ws)
+
+    def kstep(self, i):
+        """The dominant kernel alone: the product on pre-quantized activations
+        (the gated linear has no such entry: its call is timed)."""
+        qk = self.qk
+        if self.gated:
+            return self.step(i)
+        if self.xq_sets is None:
+            self.xq_sets = [qk.qk_quantize_activations(x, with_xsum=self.w4) for x in self.xs]
+        xq, sx, xsum = self.xq_sets[i % self.nsets]
+        wt = self.weights[i % self.nsets]
+        if self.w4:
+            route = qk.QK_ROUTE_GEMV if self.M <= 16 else qk.QK_ROUTE_GEMM
+            qk.qk_w4a8_gemm(xq, sx, xsum, *wt, self.bias, y=self.y, route=route)
+        else:
+            qk.qk_w8a8_gemm(xq, sx, *wt, self.bias, y=self.y)
+
+    def kernel(self):
+        """(kernel tag, source file, bound, algorithmic bytes per launch)."""
+        M, K, N = self.M, self.K, self.N
+        if self.w4 and M <= 16:
+            G = K // 64
+            kbytes = N * K / 2 + 4 * N * G + M * K + 4 * M + 4 * M * G + 2 * M * N
+            one = M == 1 and K % 1024 == 0 and K <= 4096   # the dp4a one-token kernel
+            return (("w4a8_gemv1_kernel", "gemv1_w4a8.cu") if one else
+                    ("w4a8_gemv_kernel", "gemv_w4a8.cu")) + ("hbm", kbytes)
+        if not self.w4 and N <= 64 and M <= 8192:           # thin outputs: split-K route
+            return ("w8a8_skinny_kernel", "gemm_w8a8_skinny.cu", "hbm",
+                    M * K + N * K + 2 * M * N + 4 * (M + 2 * N))
+        if self.w4:
+            return ("w4a8_gemm_kernel", "gemm_w4a8.cu", "tensor", None)
+        return ("w8a8_gemm_kernel", "gemm_w8a8.cu", "tensor", None)
+
+
+def int8_peak_source(peaks, int8):
+    if int8 is not None:
+        return int8["burst"]["tops"], ("measured in this run: the tcgen05 kind::i8 probe "
+                                       "(qk_debug_int8_peak, the GEMM's MMA stream on "
+                                       "shared-memory operands), burst")
+    return peaks["bf16"] * 2.0, (f"{peaks['source']} bf16_tflops (burst) x 2, the nominal "
+                                 "int8/bf16 ratio (4.5 / 2.25 POPS)")
+
+
+def roofline(run, k_ms, peaks, int8, workload):
+    tag, src, bound, kbytes = run.kernel()
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
+                "algorithmic_bytes": kbytes}
+    else:
+        peak, psrc = int8_peak_source(peaks, int8)
+        roof = {"bound": "tensor", "achieved": run.ops / (k_ms / 1e3) / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "peak_source": psrc + "; int8 ops counted as 2*M*N*K",
+                "algorithmic_ops": run.ops}
+    roof["kernel"] = tag
+    roof["traffic"] = traffic_from_profile(tag, csrc(src), workload)
+    if run.gated:
+        roof["kernel"] = "w8a8_gemm_kernel (gated) with its activation quant: the timed call"
+        roof["traffic"] = None  # the committed summary covers the plain epilogue
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel_ms"] = k_ms
+    return roof
+
+
+def time_linear(run, steps, warmup, local, graph="auto"):
+    """Time `steps` calls (after `warmup`), then the dominant kernel alone.
+    Returns (ms per call, kernel ms, clock summary, timing label)."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        run.step(i)
+    torch.cuda.synchronize()
+    run.qk.qk_check_device_error()
+    use_graph = graph == "on" or (graph == "auto" and run.M <= 256)
+    run_steps = graph_runner(run.step, steps) if use_graph else \
+        (lambda: [run.step(i) for i in range(steps)])
+    sampler = ClockSampler(local)
+    barrier(run.dev)
+    torch.cuda.synchronize()
+    with sampler:
+        ms = event_ms(run_steps, stream)
+    barrier(run.dev)
+    run.qk.qk_check_device_error()
+    for i in range(warmup):
+        run.kstep(i)
+    torch.cuda.synchronize()
+    run_k = graph_runner(run.kstep, steps) if use_graph else \
+        (lambda: [run.kstep(i) for i in range(steps)])
+    k_ms = event_ms(run_k, stream) / steps
+    run.qk.qk_check_device_error()
+    return ms, k_ms, sampler.summary(), \
+        ("CUDA graph of the timed calls" if use_graph else "eager launches")
+
+
+def measure_int8_peak(local, burst_ms=20.0, sustained_s=2.0):
+    """INT8 tensor-pipe rate of the device from qk_debug_int8_peak: a burst
+    (one ~20 ms launch, best of 3) and a sustained run (~50 ms launches back to
+    back for `sustained_s`), with the SM clocks sampled during each."""
+    import torch
+
+    from w4a8_quantized_gemm_token_b200 import binding as qk
+
+    stream = torch.cuda.current_stream()
+    qk.qk_debug_int8_peak(256)
+    torch.cuda.synchronize()
+    cal = 4096
+    ops_cal = [0.0]
+    ms = event_ms(lambda: ops_cal.__setitem__(0, qk.qk_debug_int8_peak(cal)), stream)
+    iters = int(max(256, min(1 << 22, cal * burst_ms / max(ms, 1e-3))))
+    best = None
+    sampler = ClockSampler(local, period=0.005)
+    with sampler:
+        for _ in range(3):
+            ops = [0.0]
+            ms = event_ms(lambda: ops.__setitem__(0, qk.qk_debug_int8_peak(iters)), stream)
+            tops = ops[0] / (ms / 1e3) / 1e12
+            best = tops if best is None else max(best, tops)
+    burst = {"tops": best, "iters_per_launch": iters, "clocks": sampler.summary()}
+    per = int(max(256, min(1 << 22, iters * 50.0 / burst_ms)))
+    n = int(max(1, sustained_s * 1e3 / 50.0))
+    total = [0.0]
+
+    def chain():
+        for _ in range(n):
+            total[0] += qk.qk_debug_int8_peak(per)
+
+    sampler = ClockSampler(local)
+    with sampler:
+        ms = event_ms(chain, stream)
+    qk.qk_check_device_error()
+    sustained = {"tops": total[0] / (ms / 1e3) / 1e12, "seconds": ms / 1e3, "launches": n,
+                 "clocks": sampler.summary()}
+    return {"burst": burst, "sustained": sustained,
+            "shape": "tcgen05.mma.cta_group::2.kind::i8 256x256x32, one CTA pair per two SMs"}
+
+
+def measure_sustained(run, local, seconds, int8, peaks):
+    """The call back to back for `seconds` (thermal / power steady state)."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    ms1 = event_ms(lambda: [run.step(i) for i in range(10)], stream) / 10
+    steps = int(max(20, seconds * 1e3 / max(ms1, 1e-3)))
+    sampler = ClockSampler(local)
+    with sampler:
+        ms = event_ms(lambda: [run.step(i) for i in range(steps)], stream)
+    run.qk.qk_check_device_error()
+    value = run.ops * steps / (ms / 1e3) / 1e12
+    out = {"seconds": ms / 1e3, "steps": steps, "ms_per_step": ms / steps, "value": value,
+           "unit": "TOPS", "clocks": sampler.summary(),
+           "frac_of_bf16_sustained_x2": value / (2.0 * peaks["bf16_sustained"])}
+    if int8 is not None:
+        out["frac_of_int8_probe_sustained"] = value / int8["sustained"]["tops"]
+    return out
+
+
+# Workloads of the `workloads` record of the default run: every configuration
+# of the target (tiny, DiT attention projection, the M = 2048 sweep, the DiT
+# MLP, W4A8 at M = 1 / 8 / 16 / 4096), the README's quick-start matmul, the
+# gated residual epilogue and the INT8 attention.
+TABLE = ["tiny", "dit_attn", "sweep_4096x4096", "sweep_4096x12288", "sweep_12288x4096",
+         "sweep_thin_5120x48", "w4a8_m1", "w4a8_m8", "w4a8_m16", "w4a8_m4096",
+         "quickstart_w8a8", "quickstart_w4a8", "dit_mlp_gated", "sage_attn"]
+
+
+def table_entry(name, local, dev, peaks, int8):
+    """One workload of the `workloads` record: per-call time and throughput,
+    the dominant kernel alone and its roofline fraction."""
+    import torch
+
+    if is_attention(name):
+        rec = attention_entry(name, local, dev, peaks, steps=5, warmup=3)
+        torch.cuda.empty_cache()
+        return rec
+    run = LinearRun(name, dev)
+    # size the timed region: graph-replayed small calls 200, else ~25 ms
+    if run.M <= 256:
+        steps = 200
+    else:
+        for i in range(3):
+            run.step(i)
+        est = event_ms(lambda: [run.step(i) for i in range(3)],
+                       torch.cuda.current_stream()) / 3
+        steps = int(max(10, min(400, 25.0 / max(est, 1e-3))))
+    ms, k_ms, clocks, timing = time_linear(run, steps, 3, local)
+    roof = roofline(run, k_ms, peaks, int8, name)
+    per = ms / steps
+    rec = {"config": run.case.name + ("_gated_residual" if run.gated else ""),
+           "M": run.M, "K": run.K, "N": run.N, "steps": steps, "timing": timing,
+           "ms_per_call": per, "value": run.ops / (per / 1e3) / 1e12, "unit": "TOPS",
+           "pct_of_int8_spec": 100.0 * run.ops / (per / 1e3) / 1e12 / INT8_SPEC_TOPS,
+           "kernel": roof["kernel"], "kernel_ms": k_ms,
+           "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                             "traffic")},
+           "sm_mhz": clocks["sm_mhz"], "reasons": clocks["reasons"]}
+    del run
+    torch.cuda.empty_cache()
+    return rec
+
+
+def attention_entry(name, local, dev, peaks, steps, warmup, e2e_steps=0):
     """The INT8 attention (qk_sage_attention) on the quick-start shape."""
     import torch
 
     from w4a8_quantized_gemm_token_b200 import binding as qk
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    case = get_case(args.workload)
+    case = get_case(name)
     B, H, L, D = case.B, case.H, case.L, case.D
     qb, kb, vb = case.draw()
     hosts = [torch.from_numpy(t.view(np.int16)).view(torch.bfloat16) for t in (qb, kb, vb)]
@@ -271,46 +552,43 @@ def run_attention(args, world, rank, local):
     out = torch.empty_like(q)
     ws = torch.empty(qk.qk_sage_attention_workspace_size(B, H, L), dtype=torch.uint8, device=dev)
     flops = 4.0 * B * H * L * L * D
+    stream = torch.cuda.current_stream()
 
     def step(i):
         qk.qk_sage_attention(q, k, v, out=out, workspace=ws)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
     qk.qk_check_device_error()
-    stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     barrier(dev)
     torch.cuda.synchronize()
     with sampler:
-        e0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        ms = event_ms(lambda: [step(i) for i in range(steps)], stream)
     barrier(dev)
-    ms = e0.elapsed_time(e1)
     qk.qk_check_device_error()
-    max_ms = reduce_max(ms, dev)
-    value = whole_job_value(flops, args.steps, world, max_ms / 1e3)
     # Roofline: Q K^T at the INT8 rate, P V at the bf16 rate (measured bf16 x 2 and
     # measured bf16); the bound is the sum of the two times.
-    peaks = load_peaks()
     t_bound = (flops / 2) / (2 * peaks["bf16"] * 1e12) + (flops / 2) / (peaks["bf16"] * 1e12)
-    achieved = flops / (max_ms / args.steps / 1e3) / 1e12
+    per = ms / steps
+    achieved = flops / (per / 1e3) / 1e12
     roof = {"bound": "tensor", "achieved": achieved, "peak": flops / t_bound / 1e12,
             "unit": "TFLOP/s",
             "peak_source": f"{peaks['source']} bf16_tflops (burst): Q K^T at x2 (INT8), P V at x1",
             "kernel": "sage_attn_kernel with its q/k quantization and v transpose (the call)",
-            "traffic": None, "frac": None, "kernel_ms": max_ms / args.steps}
+            "traffic": None, "kernel_ms": per}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    e2e = None
-    if not args.no_e2e:
+    rec = {"config": case.name, "B": B, "H": H, "L": L, "D": D, "steps": steps,
+           "timing": "eager launches", "ms_per_call": per, "value": achieved,
+           "unit": "TFLOP/s", "kernel": roof["kernel"], "kernel_ms": per,
+           "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                             "traffic")},
+           "sm_mhz": sampler.summary()["sm_mhz"], "reasons": sampler.summary()["reasons"],
+           "_roof": roof, "_clocks": sampler.summary(), "_ms": ms}
+    if e2e_steps:
         pins = [t.pin_memory() for t in hosts]
         o_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        n_e2e = max(3, min(args.steps, 5))
 
         def e2e_step():
             for dst, src in zip((q, k, v), pins):
@@ -319,258 +597,171 @@ def run_attention(args, world, rank, local):
             o_pin.copy_(out, non_blocking=True)
 
         e2e_step()
-        torch.cuda.synchronize()
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        a1.record(stream)
-        torch.cuda.synchronize()
-        e_ms = reduce_max(a0.elapsed_time(a1), dev)
+        e_ms = event_ms(lambda: [e2e_step() for _ in range(e2e_steps)], stream)
+        rec["_e2e_ms"] = e_ms
+        rec["_e2e"] = {"h2d_bytes_per_step": 3 * q.numel() * 2,
+                       "d2h_bytes_per_step": out.numel() * 2}
+    return rec
+
+
+def run_attention(args, world, rank, local):
+    """`--workload sage_attn`: the INT8 attention as the bench line."""
+    import torch
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    n_e2e = 0 if args.no_e2e else max(3, min(args.steps, 5))
+    rec = attention_entry(args.workload, local, dev, peaks, args.steps, args.warmup,
+                          e2e_steps=n_e2e)
+    case = get_case(args.workload)
+    flops = 4.0 * case.B * case.H * case.L * case.L * case.D
+    max_ms = reduce_max(rec["_ms"], dev)
+    value = whole_job_value(flops, args.steps, world, max_ms / 1e3)
+    e2e = None
+    if n_e2e:
+        e_ms = reduce_max(rec["_e2e_ms"], dev)
         e2e = {"value": whole_job_value(flops, n_e2e, world, e_ms / 1e3), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
-               "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
+               **rec["_e2e"], "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = attention_cpu_baseline(case, args.cpu_seconds)
-    clocks = sampler.summary()
     if rank == 0:
         line = {
             "metric": ATTN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8 scores, bf16 P V", "data": "synthetic",
-            "config": {"workload": case.name, "B": B, "H": H, "L": L, "D": D,
+            "config": {"workload": case.name, "B": case.B, "H": case.H, "L": case.L,
+                       "D": case.D,
                        "l2": "q, k, v of 144 MB each: every step reads more than the L2",
                        "timing": "eager launches",
                        "parallelism": f"replicas x{world} (no collective)"},
-            "roofline": roof, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
+            "roofline": rec["_roof"], "e2e": e2e, "cpu_baseline": cpu, "clocks": rec["_clocks"],
             "gpu_launches": 4 * args.steps,
         }
         print(json.dumps(line), flush=True)
 
 
-def attention_cpu_baseline(case, seconds=10.0):
-    """The oracle on the host cores: sampled query rows of head 0 against every key."""
-    import oracle
-
-    qb, kb, vb = case.draw(heads=1)
-    q, k, v = qb[0, 0], kb[0, 0], vb[0, 0]
-    t0 = time.perf_counter()
-    oracle.sage_attention_rows(q, k, v, case.D ** -0.5, np.arange(2))
-    dt = max(time.perf_counter() - t0, 1e-6)
-    rows = int(max(2, min(case.L, 2 * seconds / dt)))
-    t0 = time.perf_counter()
-    oracle.sage_attention_rows(q, k, v, case.D ** -0.5, np.arange(rows))
-    dt = time.perf_counter() - t0
-    ops = 4.0 * rows * case.L * case.D
-    return {"value": ops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} query rows of head 0 x all {case.L} keys (quantization of the "
-                      f"head's q and k included), single thread, {dt:.1f} s"}
-
-
 def run_ours(args, world, rank, local):
     import torch
 
-    from w4a8_quantized_gemm_token_b200 import binding as qk
-
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    case = get_case(args.workload)
-    M, K, N = case.M, case.K, case.N
-    w4 = is_w4(args.workload)
-    gated = is_gated(args.workload)
-    xb, W, b, _ = case.draw()
-    x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
-    if gated:
-        from w4a8_quantized_gemm_token_b200 import synthetic
-
-        gate_np, res_bits = synthetic.gated_inputs(case)
-        gate = torch.from_numpy(gate_np).to(dev)
-        res_host = torch.from_numpy(res_bits.view(np.int16)).view(torch.bfloat16)
-        res = res_host.to(dev)
-        del res_bits
-    W_dev = torch.from_numpy(W).to(dev)
-    bias = torch.from_numpy(b).to(dev) if b is not None else None
-
-    # enough rotating input sets that one pass over them exceeds the L2 twice
-    per_set = M * K * 2 + (N * K // 2 + N * (K // 64) * 4 if w4 else N * K + 4 * N)
-    nsets = args.sets or int(min(32, max(2, -(-2 * L2_BYTES // per_set))))
-    xs = [x_host.to(dev) for _ in range(nsets)]
-    if w4:
-        weights = [qk.qk_quantize_weights_int4(W_dev) for _ in range(nsets)]
-        ws = torch.empty(qk.qk_w4a8_workspace_size(M, K), dtype=torch.uint8, device=dev)
-    else:
-        weights = [qk.qk_quantize_weights_int8(W_dev) for _ in range(nsets)]
-        ws = torch.empty(qk.qk_w8a8_workspace_size(M, K), dtype=torch.uint8, device=dev)
-    del W_dev
-    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-
-    def step(i):
-        wt = weights[i % nsets]
-        if w4:
-            qk.qk_w4a8_linear(xs[i % nsets], *wt, bias, y=y, workspace=ws)
-        elif gated:
-            qk.qk_w8a8_linear_gated(xs[i % nsets], *wt, bias, gate, res, y=y, workspace=ws)
-        else:
-            qk.qk_w8a8_linear(xs[i % nsets], *wt, bias, y=y, workspace=ws)
-
-    ops = 2.0 * M * N * K
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    qk.qk_check_device_error()
-
-    stream = torch.cuda.current_stream()
-    use_graph = args.graph == "on" or (args.graph == "auto" and M <= 256)
-    run_steps = graph_runner(step, args.steps) if use_graph else \
-        (lambda: [step(i) for i in range(args.steps)])
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    barrier(dev)
-    torch.cuda.synchronize()
-    with sampler:
-        e0.record(stream)
-        run_steps()
-        e1.record(stream)
-        torch.cuda.synchronize()
-    barrier(dev)
-    ms = e0.elapsed_time(e1)
-    qk.qk_check_device_error()
-    max_ms = reduce_max(ms, dev)
-    value = whole_job_value(ops, args.steps, world, max_ms / 1e3)
-
-    # ---- dominant kernel alone (the GEMM on pre-quantized activations)
+    run = LinearRun(args.workload, dev, args.sets)
+    M, K, N, w4, gated = run.M, run.K, run.N, run.w4, run.gated
     peaks = load_peaks()
-    if w4:
-        xq_sets = [qk.qk_quantize_activations(x, with_xsum=True) for x in xs]
-        route = qk.QK_ROUTE_GEMV if M <= 16 else qk.QK_ROUTE_GEMM
 
-        def kstep(i):
-            xq, sx, xsum = xq_sets[i % nsets]
-            qk.qk_w4a8_gemm(xq, sx, xsum, *weights[i % nsets], bias, y=y, route=route)
-    elif gated:
-        kstep = step  # no gated entry on pre-quantized activations: the call (quant + GEMM)
-    else:
-        xq_sets = [qk.qk_quantize_activations(x) for x in xs]
+    # ---- the headline: `steps` calls, max over ranks
+    ms, k_ms, clocks, timing = time_linear(run, args.steps, args.warmup, local, args.graph)
+    max_ms = reduce_max(ms, dev)
+    value = whole_job_value(run.ops, args.steps, world, max_ms / 1e3)
 
-        def kstep(i):
-            xq, sx, _ = xq_sets[i % nsets]
-            qk.qk_w8a8_gemm(xq, sx, *weights[i % nsets], bias, y=y)
-    for i in range(args.warmup):
-        kstep(i)
-    torch.cuda.synchronize()
-    run_k = graph_runner(kstep, args.steps) if use_graph else \
-        (lambda: [kstep(i) for i in range(args.steps)])
-    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    k0.record(stream)
-    run_k()
-    k1.record(stream)
-    torch.cuda.synchronize()
-    k_ms = k0.elapsed_time(k1) / args.steps
-    if w4 and M <= 16:
-        # weight-streaming GEMV: bound by HBM; algorithmic bytes per launch
-        G = K // 64
-        kbytes = N * K / 2 + 4 * N * G + M * K + 4 * M + 4 * M * G + 2 * M * N
-        # one token with K a multiple of 1024 (up to 4096) runs the dp4a kernel
-        one = M == 1 and K % 1024 == 0 and K <= 4096
-        tag = "w4a8_gemv1_kernel" if one else "w4a8_gemv_kernel"
-        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc",
-                           "gemv1_w4a8.cu" if one else "gemv_w4a8.cu")
-        roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
-                "kernel": tag, "traffic": traffic_from_profile(tag, src, args.workload)}
-    elif not w4 and N <= 64 and M <= 8192:
-        # thin W8A8 outputs run the split-K cluster kernel, bound by reading xq
-        kbytes = M * K + N * K + 2 * M * N + 4 * (M + 2 * N)
-        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc", "gemm_w8a8_skinny.cu")
-        roof = {"bound": "hbm", "achieved": kbytes / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "peak_source": f"{peaks['source']} hbm_gbs (copy)",
-                "kernel": "w8a8_skinny_kernel",
-                "traffic": traffic_from_profile("w8a8_skinny_kernel", src, args.workload)}
-    else:
-        peak = peaks["bf16"] * 2.0
-        src = os.path.join(ROOT, "w4a8_quantized_gemm_token_b200", "csrc",
-                           "gemm_w4a8.cu" if w4 else "gemm_w8a8.cu")
-        tag = "w4a8_gemm_kernel" if w4 else "w8a8_gemm_kernel"
-        roof = {"bound": "tensor", "achieved": ops / (k_ms / 1e3) / 1e12, "peak": peak,
-                "unit": "TFLOP/s",
-                "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2, the nominal int8/bf16 "
-                               "ratio (4.5 / 2.25 POPS); int8 ops counted as 2*M*N*K",
-                "kernel": tag, "traffic": traffic_from_profile(tag, src, args.workload)}
-        if gated:
-            roof["kernel"] = "w8a8_gemm_kernel (gated) with its activation quant: the timed call"
-            roof["traffic"] = None  # the committed summary covers the plain epilogue
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel_ms"] = k_ms
+    # ---- the INT8 tensor-pipe probe (roofline denominator), burst right after;
+    # the probe, the sustained record and the per-configuration record are
+    # one-GPU measurements: replicas under torchrun skip them
+    single = world == 1
+    int8 = None
+    if single and not args.no_peak_probe and not (w4 and M <= 16):
+        int8 = measure_int8_peak(local, sustained_s=0.0 if args.no_sustained else 2.0)
+    roof = roofline(run, k_ms, peaks, int8, args.workload)
 
     # ---- end to end through the public call, host buffers in and out
     e2e = None
+    e2e_step = None
     if not args.no_e2e:
-        x_pin = x_host.pin_memory()
+        stream = torch.cuda.current_stream()
+        x_pin = run.x_host.pin_memory()
         y_pin = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
         x_dev = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
         n_e2e = max(3, min(args.steps, args.e2e_steps))
-
-        if gated:
-            r_pin = res_host.pin_memory()
+        r_pin = run.res_host.pin_memory() if gated else None
 
         def e2e_step(i):
             x_dev.copy_(x_pin, non_blocking=True)
-            wt = weights[i % nsets]
+            wt = run.weights[i % run.nsets]
             if w4:
-                qk.qk_w4a8_linear(x_dev, *wt, bias, y=y, workspace=ws)
+                run.qk.qk_w4a8_linear(x_dev, *wt, run.bias, y=run.y, workspace=run.ws)
             elif gated:
-                res.copy_(r_pin, non_blocking=True)
-                qk.qk_w8a8_linear_gated(x_dev, *wt, bias, gate, res, y=y, workspace=ws)
+                run.res.copy_(r_pin, non_blocking=True)
+                run.qk.qk_w8a8_linear_gated(x_dev, *wt, run.bias, run.gate, run.res, y=run.y,
+                                            workspace=run.ws)
             else:
-                qk.qk_w8a8_linear(x_dev, *wt, bias, y=y, workspace=ws)
-            y_pin.copy_(y, non_blocking=True)
+                run.qk.qk_w8a8_linear(x_dev, *wt, run.bias, y=run.y, workspace=run.ws)
+            y_pin.copy_(run.y, non_blocking=True)
 
         for i in range(2):
             e2e_step(i)
         torch.cuda.synchronize()
         barrier(dev)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for i in range(n_e2e):
-            e2e_step(i)
-        a1.record(stream)
-        torch.cuda.synchronize()
-        e_ms = reduce_max(a0.elapsed_time(a1), dev)
-        e2e = {"value": whole_job_value(ops, n_e2e, world, e_ms / 1e3), "unit": "TOPS",
+        e_ms = reduce_max(event_ms(lambda: [e2e_step(i) for i in range(n_e2e)], stream), dev)
+        e2e = {"value": whole_job_value(run.ops, n_e2e, world, e_ms / 1e3), "unit": "TOPS",
                "h2d_bytes_per_step": M * K * 2 + (M * N * 2 if gated else 0),
                "d2h_bytes_per_step": M * N * 2,
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
 
+    # ---- the same call back to back for seconds (power-capped steady state)
+    sustained = None
+    if single and not args.no_sustained and not w4 and M > 256:
+        sustained = measure_sustained(run, local, 2.0, int8, peaks)
+    config = {"workload": run.case.name + ("_gated_residual" if gated else ""),
+              "M": M, "K": K, "N": N,
+              "weights": "W4 affine g64" if w4 else "W8 per-channel",
+              "bias": run.bias is not None,
+              "activations": "bf16 N(0,1)" + (", 1% channels x20" if run.case.outlier_frac else ""),
+              "l2": f"{run.nsets} rotating input sets of {run.per_set / 1e6:.1f} MB; "
+                    "one pass over them exceeds twice the 126 MB L2",
+              "timing": timing, "parallelism": f"replicas x{world} (no collective)"}
+    del run, e2e_step
+    torch.cuda.empty_cache()
+
+    # ---- every other configuration, each with its dominant kernel alone
+    workloads = None
+    if single and args.workload == "dit_mlp" and not args.no_workloads:
+        workloads = {}
+        for name in TABLE:
+            workloads[name] = table_entry(name, local, dev, peaks, int8)
+            for k in [k for k in workloads[name] if k.startswith("_")]:
+                del workloads[name][k]
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(case, seconds=args.cpu_seconds, gated=gated)
+        cpu = cpu_baseline(get_case(args.workload), seconds=args.cpu_seconds, gated=gated)
 
-    clocks = sampler.summary()
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8", "data": "synthetic",
-            "config": {"workload": case.name + ("_gated_residual" if gated else ""),
-                       "M": M, "K": K, "N": N,
-                       "weights": "W4 affine g64" if w4 else "W8 per-channel",
-                       "bias": bias is not None,
-                       "activations": "bf16 N(0,1)" + (", 1% channels x20" if case.outlier_frac else ""),
-                       "l2": f"{nsets} rotating input sets of {per_set / 1e6:.1f} MB; "
-                             "one pass over them exceeds twice the 126 MB L2",
-                       "timing": "CUDA graph of the timed steps" if use_graph else "eager launches",
-                       "parallelism": f"replicas x{world} (no collective)"},
+            "dtype": "int8", "data": "synthetic", "config": config,
             "pct_of_int8_spec": 100.0 * value / world / INT8_SPEC_TOPS,
             "roofline": roof, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
             "gpu_launches": 2 * args.steps,
+            "int8_peak_probe": int8, "sustained": sustained, "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------ oracle legs
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
 
 class OracleSample:
     """Inputs for bounded oracle samples of a workload (same recipe as the GPU
@@ -591,6 +782,10 @@ class OracleSample:
             self.Wp, self.s16, self.o16 = oracle.quant_w4(W)
         else:
             self.Wq, self.sw = oracle.quant_w8(W)
+
+    @property
+    def rows(self):
+        return self.xb.shape[0]
 
     def run(self, rows, ncols):
         """Quantize `rows` activation rows and compute their outputs for the first
@@ -614,38 +809,72 @@ class OracleSample:
         return time.perf_counter() - t0, 2.0 * rows * ncols * self.case.K
 
 
+def _oracle_leg(smp, seconds, threads):
+    """Time the oracle over about `seconds` of rows with `threads` OpenMP
+    threads (one row per thread to calibrate).  Returns (rows, s, ops, threads)."""
+    import oracle
+
+    got = oracle.set_threads(threads)
+    try:
+        probe = max(1, min(smp.rows, got))
+        dt, _ = smp.run(probe, smp.case.N)
+        rows = int(max(probe, min(smp.rows, probe * seconds / max(dt, 1e-6))))
+        dt, ops = smp.run(rows, smp.case.N)
+    finally:
+        oracle.set_threads(1)
+    return rows, dt, ops, min(got, rows)
+
+
 def cpu_baseline(case, seconds=10.0, gated=False):
-    """The oracle on the host cores over a bounded sample of the same workload."""
-    smp = OracleSample(case, "w4a8" in case.name, gated=gated)
-    dt, _ = smp.run(1, case.N)          # calibrate on one row
-    rows = int(max(1, min(smp.xb.shape[0], seconds / max(dt, 1e-6))))
-    dt, ops = smp.run(rows, case.N)
-    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} of {case.M} rows x all {case.N} output channels "
-                      f"(quant + exact int accumulate + fp64 dequant), single thread, "
-                      f"{dt:.1f} s"}
+    """The oracle on the GPU machine's host cores, over bounded samples of the same
+    workload: one thread, then every core (OpenMP over rows)."""
+    ncores = host_cores()
+    # enough rows that the all-core leg keeps every thread busy for its share
+    smp = OracleSample(case, "w4a8" in case.name, gated=gated,
+                       max_rows=int(min(case.M, max(1024, 64 * ncores))))
+    r1, t1, o1, _ = _oracle_leg(smp, seconds / 2, 1)
+    rn, tn, on, used = _oracle_leg(smp, seconds / 2, ncores)
+    what = (f"of {case.M} rows x all {case.N} output channels (quant + exact int accumulate "
+            f"+ fp64 dequant)")
+    return {"value": on / tn / 1e12, "unit": "TOPS", "cores": used, "kind": "oracle",
+            "sample": f"{rn} {what}, {used} OpenMP threads over rows, {tn:.1f} s",
+            "nproc": ncores, "cpu_model": cpu_model(),
+            "one_thread": {"value": o1 / t1 / 1e12, "unit": "TOPS", "cores": 1,
+                           "sample": f"{r1} {what}, single thread, {t1:.1f} s"}}
 
 
 def run_reference(args, world, rank, local):
     if rank != 0:
         return  # rank 0 alone runs the oracle
+    import oracle
+
     case = get_case(args.workload)
-    smp = OracleSample(case, is_w4(args.workload), max_rows=8, gated=is_gated(args.workload))
+    threads = oracle.set_threads(host_cores())
+    oracle.set_threads(1)
+    rows = max(1, min(case.M, threads))  # one row per thread in every step
+    smp = OracleSample(case, is_w4(args.workload), max_rows=rows, gated=is_gated(args.workload))
     # size each step so that warm-up + timed steps take about `budget` seconds
     budget = args.ref_seconds
-    dt1, _ = smp.run(1, case.N)
-    per_step = budget / max(1, args.steps + args.warmup)
-    ncols = int(max(8, min(case.N, case.N * per_step / max(dt1, 1e-6)))) // 8 * 8
-    for _ in range(args.warmup):
-        smp.run(1, ncols)
-    t_total, ops_total = 0.0, 0.0
-    for _ in range(args.steps):
-        dt, ops = smp.run(1, ncols)
-        t_total += dt
-        ops_total += ops
+    oracle.set_threads(threads)
+    try:
+        dt1, _ = smp.run(rows, 8)
+        dtn, _ = smp.run(rows, min(case.N, 64))
+        per_col = max((dtn - dt1) / max(1, min(case.N, 64) - 8), 1e-9)
+        per_step = budget / max(1, args.steps + args.warmup)
+        ncols = int(max(8, min(case.N, per_step / per_col))) // 8 * 8
+        for _ in range(args.warmup):
+            smp.run(rows, ncols)
+        t_total, ops_total = 0.0, 0.0
+        for _ in range(args.steps):
+            dt, ops = smp.run(rows, ncols)
+            t_total += dt
+            ops_total += ops
+    finally:
+        oracle.set_threads(1)
     value = ops_total / t_total / 1e12
-    sample = (f"per step: 1 of {case.M} rows x {ncols} of {case.N} output channels "
-              f"(quant + exact int accumulate + fp64 dequant), single thread")
+    threads = min(threads, rows)  # the row loops give each thread one row at most
+    sample = (f"per step: {rows} of {case.M} rows x {ncols} of {case.N} output channels "
+              f"(quant + exact int accumulate + fp64 dequant), {threads} OpenMP threads over rows")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
@@ -653,11 +882,37 @@ def run_reference(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": case.name + ("_gated_residual" if is_gated(args.workload) else ""),
                    "M": case.M, "K": case.K, "N": case.N},
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def attention_cpu_baseline(case, seconds=10.0, threads=None):
+    """The oracle on the host cores: sampled query rows of head 0 against every key."""
+    import oracle
+
+    threads = host_cores() if threads is None else threads
+    qb, kb, vb = case.draw(heads=1)
+    q, k, v = qb[0, 0], kb[0, 0], vb[0, 0]
+    used = oracle.set_threads(threads)
+    try:
+        probe = max(2, used)
+        t0 = time.perf_counter()
+        oracle.sage_attention_rows(q, k, v, case.D ** -0.5, np.arange(probe))
+        dt = max(time.perf_counter() - t0, 1e-6)
+        rows = int(max(probe, min(case.L, probe * seconds / dt)))
+        t0 = time.perf_counter()
+        oracle.sage_attention_rows(q, k, v, case.D ** -0.5, np.arange(rows))
+        dt = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(1)
+    ops = 4.0 * rows * case.L * case.D
+    return {"value": ops / dt / 1e12, "unit": "TFLOP/s", "cores": used, "kind": "oracle",
+            "sample": f"{rows} query rows of head 0 x all {case.L} keys (quantization of the "
+                      f"head's q and k included), {used} OpenMP threads over rows, {dt:.1f} s",
+            "cpu_model": cpu_model()}
 
 
 def run_attention_reference(args, world):
@@ -694,7 +949,13 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-configuration record of the default run")
+    ap.add_argument("--no-sustained", action="store_true",
+                    help="skip the seconds-long sustained records")
+    ap.add_argument("--no-peak-probe", action="store_true",
+                    help="skip the INT8 tensor-pipe probe (then bf16 x 2 is the denominator)")
+    ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
