@@ -955,6 +955,8 @@ def main(argv=None):
                     help="skip the seconds-long sustained records")
     ap.add_argument("--no-peak-probe", action="store_true",
                     help="skip the INT8 tensor-pipe probe (then bf16 x 2 is the denominator)")
+    ap.add_argument("--probe-only", action="store_true",
+                    help="run only the INT8 tensor-pipe probe and print its record")
     ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     args = ap.parse_args(argv)
@@ -978,6 +980,11 @@ def main(argv=None):
     import torch
     import torch.distributed as dist
 
+    if args.probe_only:
+        torch.cuda.set_device(local)
+        print(json.dumps({"int8_peak_probe": measure_int8_peak(
+            local, sustained_s=0.0 if args.no_sustained else 2.0)}), flush=True)
+        return
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

@@ -32,7 +32,7 @@ def assert_halo_intact(flat):
     assert not bool((flat[PAD:-PAD] == SENTINEL).any()), "an output element was not written"
 
 
-def w4_weights(K, N, seed):
+def w4_weights(qk, K, N, seed):
     rng = np.random.default_rng(seed)
     W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
     return qk.qk_quantize_weights_int4(to_dev(W))
@@ -55,7 +55,7 @@ GEMV_SHAPES = [(1, 64, 8), (1, 1024, 264), (1, 3072, 136), (1, 2048, 40), (3, 19
 @pytest.mark.parametrize("MKN", GEMV_SHAPES, ids=lambda s: "x".join(map(str, s)))
 def test_gemv_guard_bands(qk, MKN):
     M, K, N = MKN
-    Wp, s, o = w4_weights(K, N, seed=K + N)
+    Wp, s, o = w4_weights(qk, K, N, seed=K + N)
     bias = to_dev(np.linspace(-1, 1, N).astype(np.float32))
     x = x_dev(M, K, seed=M + K)
     flat, y = haloed((M, N))
@@ -74,7 +74,7 @@ def test_gemv_guard_bands(qk, MKN):
                          ids=lambda s: "x".join(map(str, s)))
 def test_w4a8_gemm_guard_bands(qk, MKN):
     M, K, N = MKN
-    Wp, s, o = w4_weights(K, N, seed=K * 3 + N)
+    Wp, s, o = w4_weights(qk, K, N, seed=K * 3 + N)
     bias = to_dev(np.linspace(-2, 2, N).astype(np.float32))
     x = x_dev(M, K, seed=M * 5 + K)
     xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
