@@ -257,9 +257,12 @@ qk_status qk_w8a8_linear_noalloc(const uint16_t *x, int64_t M, int64_t K,
  * M <= 16 takes the weight-streaming GEMV when its per-CTA working set fits
  * in shared memory (K <= 4096 at M = 16), otherwise the tensor-core GEMM; both
  * compute the same per-group integers and agree to the fp64 rounding order.
- * When also M * K <= 65536 the GEMV quantizes x itself (same rule and codes as
- * qk_quantize_activations) and the call is one kernel; the workspace is then
- * checked but not used (qk_w4a8_linear_plan tells which case applies).
+ * When also M <= 8 and each CTA's K slice of x fits its registers (M times
+ * the slice <= 16384 elements) the GEMV quantizes x itself (same rule and
+ * codes as qk_quantize_activations) and the call is one kernel; the workspace
+ * is then checked but not used (qk_w4a8_linear_plan tells which case
+ * applies).  From 9 tokens on, the quantization kernel followed by the GEMV
+ * on its codes is faster.
  *   x                  : bf16 bits [M, K]            (in)
  *   Wp, wscale, woffset: from qk_quantize_weights_int4 (in)
  *   bias               : fp32 [N] (nullable)

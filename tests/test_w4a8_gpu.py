@@ -27,9 +27,10 @@ def prepare(qk, orc, case):
 
 
 # 9 x 1024 x 2376: 32-row CTAs with a ragged last CTA.  qk_w4a8_linear
-# quantizes x inside the GEMV when one CTA's K slice of x fits its registers;
-# 16 x 3072 x 128 and 12 x 2112 x 136 do not and take the quantization kernel
-# + GEMV (2112 = 33 groups: a partial last group range).
+# quantizes x inside the GEMV for up to 8 tokens when one CTA's K slice of x
+# fits its registers; 9 tokens and more, 16 x 3072 x 128 and 12 x 2112 x 136
+# take the quantization kernel + GEMV (2112 = 33 groups: a partial last group
+# range).
 GEMV_SHAPES = [(1, 64, 8), (1, 4096, 4096), (8, 4096, 4096), (16, 4096, 4096), (3, 192, 40),
                (11, 1024, 264), (16, 3072, 128), (5, 640, 2056), (9, 1024, 2376),
                (12, 2112, 136),
