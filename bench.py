@@ -370,6 +370,18 @@ class LinearRun:
         return ("w8a8_gemm_kernel", "gemm_w8a8.cu", "tensor", None)
 
 
+def launches_per_call(M, K, N, w4, gated, qk):
+    """Kernels one call of the linear launches: the W8A8 linear is one kernel
+    (quantization fused into the GEMM) except for thin outputs (N <= 64, the
+    quantization kernel + the split-K kernel) and the gated epilogue (two);
+    the W4A8 linear follows its plan (qk_w4a8_linear_plan)."""
+    if w4:
+        return 1 if qk.qk_w4a8_linear_plan(M, K, N) == qk.QK_PLAN_GEMV_QUANT else 2
+    if gated or (N <= 64 and M <= 8192):
+        return 2
+    return 1
+
+
 def int8_peak_source(peaks, int8):
     if int8 is not None:
         return int8["burst"]["tops"], ("measured in this run: the tcgen05 kind::i8 probe "
@@ -704,6 +716,7 @@ def run_ours(args, world, rank, local):
     sustained = None
     if single and not args.no_sustained and not w4 and M > 256:
         sustained = measure_sustained(run, local, 2.0, int8, peaks)
+    launches = launches_per_call(M, K, N, w4, gated, run.qk)
     config = {"workload": run.case.name + ("_gated_residual" if gated else ""),
               "M": M, "K": K, "N": N,
               "weights": "W4 affine g64" if w4 else "W8 per-channel",
@@ -736,7 +749,7 @@ def run_ours(args, world, rank, local):
             "dtype": "int8", "data": "synthetic", "config": config,
             "pct_of_int8_spec": 100.0 * value / world / INT8_SPEC_TOPS,
             "roofline": roof, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": launches * args.steps,
             "int8_peak_probe": int8, "sustained": sustained, "workloads": workloads,
         }
         print(json.dumps(line), flush=True)

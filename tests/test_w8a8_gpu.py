@@ -17,6 +17,12 @@ pytestmark = pytest.mark.gpu
 TOL_ULP = 2
 
 SHAPES = [  # (M, K, N): tiles of 128 x 256 with K blocks of 128
+    # qk_w8a8_linear runs these in one kernel (the GEMM's epilogue warps
+    # quantize x); 8192 x 256 x 72: 64 row blocks behind one column of tiles;
+    # 600 x 8192: rows longer than 4096 elements (two passes per row)
+    (8192, 256, 72),
+    (600, 8192, 264),
+    (2, 4096, 4096),
     (64, 256, 128),
     (1, 32, 8),
     (3, 96, 24),
@@ -128,6 +134,26 @@ def test_w8a8_guard_bands(qk, orc, MKN):
     torch.cuda.synchronize()
     assert bool((flat[:pad] == 0x7FBF).all()) and bool((flat[-pad:] == 0x7FBF).all())
     assert not bool((flat[pad: pad + M * N] == 0x7FBF).any())
+
+
+def test_w8a8_fused_workspace_reuse_and_garbage(qk, orc):
+    """The one-kernel W8A8 linear keeps per-row-block readiness words in the
+    workspace, tagged with each launch's epoch: a workspace full of garbage, or
+    left by a call of another shape, gives the same bits as a fresh one."""
+    cases = [synthetic.LinearCase("wa", M=700, K=1024, N=520, seed=41),
+             synthetic.LinearCase("wb", M=1300, K=512, N=264, seed=42)]
+    prepared = [prepare(qk, orc, c) for c in cases]
+    need = max(qk.qk_w8a8_workspace_size(c.M, c.K) for c in cases)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    fresh = [qk.qk_w8a8_linear(to_dev_bf16(p[0]), p[1], p[2], to_dev(p[5])) for p in prepared]
+    for rep in range(2):
+        for p, want in zip(prepared, fresh):
+            y = qk.qk_w8a8_linear(to_dev_bf16(p[0]), p[1], p[2], to_dev(p[5]), workspace=ws)
+            torch.cuda.synchronize()
+            assert torch.equal(y.view(torch.int16), want.view(torch.int16))
+    y_o, _, _, _ = orc.w8a8_linear(prepared[0][0], prepared[0][3], prepared[0][4], prepared[0][5])
+    assert bf16_ulp_distance(t2bits(fresh[0]), y_o).max() <= TOL_ULP
+    qk.qk_check_device_error()
 
 
 def test_w8a8_zero_rows_and_integer_closed_form(qk, orc):

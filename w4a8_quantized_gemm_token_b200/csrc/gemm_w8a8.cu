@@ -35,8 +35,11 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <chrono>
 #include <cstdint>
 
+#include "act_quant.cuh"
 #include "qk_internal.h"
 #include "sm100.cuh"
 
@@ -140,16 +143,61 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
   return sign | bits;
 }
 
+// ---- readiness of the quantized rows (the fused-quantization kernel)
+//
+// Row block b (rows 128 b .. 128 b + 127 of x) is ready when the 64-bit word
+// ready[b] holds (epoch << 8) | (its number of rows): every warp that
+// quantized one of its rows adds 1, tagged with the launch's epoch (a value
+// the host never reuses), so the words need no clearing between launches and
+// a word left by an earlier launch never reads as ready.
+
+// Adds one finished row to a readiness word (lock-free; bounded retries).
+__device__ __forceinline__ void ready_add(unsigned long long* p, unsigned long long epoch,
+                                          int* err) {
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(p);
+  for (int i = 0; i < (1 << 20); ++i) {
+    const unsigned long long base = (old >> 8) == epoch ? old : (epoch << 8);
+    const unsigned long long prev = atomicCAS(p, old, base + 1ull);
+    if (prev == old) return;
+    old = prev;
+  }
+  record_timeout(err);
+}
+
+// Waits (bounded) until a readiness word holds `want`; then orders the TMA
+// (async proxy) reads that follow after the generic-proxy writes it observed.
+__device__ __forceinline__ bool ready_wait(const unsigned long long* p, unsigned long long want,
+                                           int* err) {
+  const long long t0 = clock64();
+  while (true) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    if (v == want) break;
+    if (clock64() - t0 > QK_WAIT_LIMIT_CYCLES) {
+      record_timeout(err);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
 // kAccOut: store the int32 sums instead of y.  kGated: the gated residual
 // epilogue ("mlx-kquant PR #89", commit list), y = bf16(residual + gate[n] *
 // (acc * sx * sw + bias)) in fp64 for every output.
-template <bool kAccOut, bool kGated>
+// kFused: the activations arrive as bf16 x and the epilogue warps quantize
+// them into xq / sx (the workspace the TMA loads read) while the tiles run;
+// the producers wait for each 128-row block's readiness word (see above).
+template <bool kAccOut, bool kGated, bool kFused>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const float* __restrict__ sx,
                      const float* __restrict__ sw, const float* __restrict__ bias,
                      const float* __restrict__ gate, const uint16_t* residual, int M, int N,
-                     int K, int group_m, int* err) {
+                     int K, int group_m, int* err, const uint16_t* __restrict__ x,
+                     int8_t* xq_out, float* sx_out, unsigned long long* ready,
+                     unsigned long long epoch) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -214,6 +262,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
         const int arow = mb * 2 * BM + (int)rank * BM;
         const int brow = nb * BN + (int)rank * (BN / 2);
+        if constexpr (kFused) {
+          // this CTA's 128 rows of xq must be quantized before the TMA reads them
+          const int nrows = min(BM, M - arow);
+          if (nrows > 0 &&
+              !ready_wait(ready + (arow / BM), (epoch << 8) | (unsigned long long)nrows, err)) {
+            ok = false;
+            break;
+          }
+        }
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, err)) {
             ok = false;
@@ -300,10 +357,120 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (prow < M && pcol < N)
         bulk_prefetch_l2(residual + (size_t)prow * N + pcol, (uint32_t)(min(BN, N - pcol) * 2));
     };
+    // ---- fused quantization: rows qw, qw + QW, qw + 2 QW, ... of x are this
+    // warp's (QW = all epilogue warps of the grid, so the first rows are spread
+    // over every SM).  Each row: absmax, multiplier and scale, codes (the rule
+    // of the stand-alone kernel, act_quant.cuh), then the row is published to
+    // its block's readiness word.  Rows of up to 4096 elements are held in
+    // registers two at a time; longer rows take two passes over 4096-element
+    // segments (the second from L2).
+    const int QW = (int)gridDim.x * kEpiWarps;
+    int qrow = (int)blockIdx.x * kEpiWarps + e;
+    const int nch = K >> 3;  // 16-byte chunks of bf16 per row
+    auto publish = [&](int r, float amax) {
+      if (lane == 0) sx_out[r] = act_scale(amax);
+      // every lane's codes (and the scale) before the row counts as done
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) ready_add(ready + (r >> 7), epoch, err);
+    };
+    auto quantize_until = [&](int limit) {
+      if constexpr (kFused) {
+        limit = min(limit, M);
+        while (qrow < limit) {
+          if (nch <= 512) {
+            const int r0 = qrow, r1 = qrow + QW;
+            const bool two = r1 < limit;
+            const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r0 * K);
+            const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)(two ? r1 : r0) * K);
+            uint4 v0[16], v1[16];
+            uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = i * 32 + lane;
+              v0[i] = make_uint4(0u, 0u, 0u, 0u);
+              v1[i] = make_uint4(0u, 0u, 0u, 0u);
+              if (c < nch) {
+                v0[i] = __ldcs(s0 + c);
+                if (two) v1[i] = __ldcs(s1 + c);
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              m0 = bf16x2_absmax_bits(m0, v0[i].x);
+              m0 = bf16x2_absmax_bits(m0, v0[i].y);
+              m0 = bf16x2_absmax_bits(m0, v0[i].z);
+              m0 = bf16x2_absmax_bits(m0, v0[i].w);
+              m1 = bf16x2_absmax_bits(m1, v1[i].x);
+              m1 = bf16x2_absmax_bits(m1, v1[i].y);
+              m1 = bf16x2_absmax_bits(m1, v1[i].z);
+              m1 = bf16x2_absmax_bits(m1, v1[i].w);
+            }
+            const float a0 = warp_max_bits_to_float(m0), a1 = warp_max_bits_to_float(m1);
+            const float q0 = act_multiplier(a0), q1 = act_multiplier(a1);
+            uint2* d0 = reinterpret_cast<uint2*>(xq_out + (size_t)r0 * K);
+            uint2* d1 = reinterpret_cast<uint2*>(xq_out + (size_t)r1 * K);
+            int dummy = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = i * 32 + lane;
+              if (c < nch) {
+                d0[c] = quant_chunk(v0[i], q0, &dummy);
+                if (two) d1[c] = quant_chunk(v1[i], q1, &dummy);
+              }
+            }
+            publish(r0, a0);
+            if (two) publish(r1, a1);
+            qrow += two ? 2 * QW : QW;
+          } else {
+            const int r0 = qrow;
+            const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r0 * K);
+            uint2* d0 = reinterpret_cast<uint2*>(xq_out + (size_t)r0 * K);
+            uint32_t m0 = 0;
+            for (int seg = 0; seg < nch; seg += 512) {  // warp-uniform
+              uint4 v[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int c = seg + i * 32 + lane;
+                v[i] = c < nch ? __ldcs(s0 + c) : make_uint4(0u, 0u, 0u, 0u);
+              }
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                m0 = bf16x2_absmax_bits(m0, v[i].x);
+                m0 = bf16x2_absmax_bits(m0, v[i].y);
+                m0 = bf16x2_absmax_bits(m0, v[i].z);
+                m0 = bf16x2_absmax_bits(m0, v[i].w);
+              }
+            }
+            const float a0 = warp_max_bits_to_float(m0);
+            const float q0 = act_multiplier(a0);
+            int dummy = 0;
+            for (int seg = 0; seg < nch; seg += 512) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int c = seg + i * 32 + lane;
+                if (c < nch) d0[c] = quant_chunk(__ldcg(s0 + c), q0, &dummy);
+              }
+            }
+            publish(r0, a0);
+            qrow += QW;
+          }
+        }
+      }
+    };
+    // rows that the tiles before index T need (whole raster groups)
+    auto rows_before = [&](int T) {
+      const int last = min(T, num_tiles) - 1;
+      const int gid = last / (group_m * tiles_n);
+      return min(M, (gid + 1) * group_m * 2 * BM);
+    };
     if constexpr (kGated) prefetch_residual(pair);
     for (int t = pair; t < num_tiles; t += num_pairs, ++iter) {
       int mb, nb;
       tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
+      // keep this warp's share of the rows two waves ahead of the tiles
+      if constexpr (kFused) quantize_until(rows_before(t + 2 * num_pairs + 1));
       if constexpr (kGated) prefetch_residual(t + num_pairs);
       const int ncol0 = nb * BN;
       float4* tcol = tab + (iter & 1) * BN;
@@ -328,7 +495,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;  // this warp's 32-row slab
       const int row = row0 + lane;
-      const float sxf = (!kAccOut && row < M) ? __ldg(sx + row) : 0.0f;
+      float sxf = 0.0f;
+      if constexpr (kFused) {
+        // the scales were written in this launch by other warps: acquire the
+        // block's readiness word, then read past L1
+        const int nrows = min(BM, M - (row0 - q * 32));
+        if (lane == 0 && nrows > 0)
+          ready_wait(ready + ((row0 - q * 32) / BM), (epoch << 8) | (unsigned long long)nrows, err);
+        __syncwarp();
+        if (row < M) sxf = __ldcg(sx + row);
+      } else {
+        sxf = (!kAccOut && row < M) ? __ldg(sx + row) : 0.0f;
+      }
       const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       constexpr int kChunk = kAccOut ? 32 : 64;  // columns per 128-byte staged row
       constexpr int kChunks = BN / kChunk;
@@ -481,6 +659,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         aphase ^= 1u;
       }
     }
+    // the rest of this warp's rows (tiles of other CTAs may still need them)
+    if constexpr (kFused) quantize_until(M);
     if (lane == 0) bulk_wait<0>();
   }
 
@@ -491,7 +671,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
-bool g_attr_done[3][64];  // plain, accumulator dump, gated
+bool g_attr_done[4][64];  // plain, accumulator dump, gated, fused quantization
+
+// Epochs of the fused-quantization launches: distinct for every launch of the
+// process (56 bits, never zero), so a readiness word left by an earlier launch
+// in the same workspace never equals this launch's target.
+std::atomic<unsigned long long> g_epoch{0};
+
+unsigned long long next_epoch() {
+  static const unsigned long long seed = [] {
+    const unsigned long long t =
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    return (t * 0x9E3779B97F4A7C15ull) >> 9;
+  }();
+  unsigned long long e = (seed + g_epoch.fetch_add(1, std::memory_order_relaxed)) & ((1ull << 56) - 1);
+  return e == 0 ? 1 : e;
+}
+
+// Pairs of CTAs that can be resident at once (the fused kernel's producers wait
+// for rows that other CTAs quantize, so its whole grid must be resident).
+int resident_pairs(const void* kernel) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int cached[64];
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = num_sms() / 2;
+  }
+  n = n < num_sms() / 2 ? n : num_sms() / 2;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
 
 }  // namespace
 
@@ -520,8 +743,9 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   int dev = 0;
   cudaGetDevice(&dev);
   const bool gated = gate != nullptr;
-  auto kernel = acc_mode ? w8a8_gemm_kernel<true, false>
-                         : (gated ? w8a8_gemm_kernel<false, true> : w8a8_gemm_kernel<false, false>);
+  auto kernel = acc_mode ? w8a8_gemm_kernel<true, false, false>
+                         : (gated ? w8a8_gemm_kernel<false, true, false>
+                                  : w8a8_gemm_kernel<false, false, false>);
   const int variant = acc_mode ? 1 : (gated ? 2 : 0);
   if (dev < 64 && !g_attr_done[variant][dev]) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -551,7 +775,58 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, tA, tB, tC, sx, sw, bias, gate, residual, (int)M,
-                            (int)N, (int)K, (int)group_m, err);
+                            (int)N, (int)K, (int)group_m, err, (const uint16_t*)nullptr,
+                            (int8_t*)nullptr, (float*)nullptr, (unsigned long long*)nullptr,
+                            0ull);
+}
+
+bool w8a8_use_fused(int64_t M, int64_t K, int64_t N) { return !w8a8_use_skinny(M, K, N); }
+
+cudaError_t launch_w8a8_fused(const uint16_t* x, int64_t M, int64_t K, const int8_t* Wq,
+                              const float* sw, const float* bias, int64_t N, uint16_t* y,
+                              int8_t* xq, float* sx, unsigned long long* ready, bool pdl,
+                              cudaStream_t s) {
+  CUtensorMap tA, tB, tC;
+  if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
+                      (uint64_t)K, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, (uint64_t)K, (uint64_t)N,
+                      (uint64_t)K, 128, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
+                      (uint64_t)N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kernel = w8a8_gemm_kernel<false, false, true>;
+  if (dev < 64 && !g_attr_done[3][dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    g_attr_done[3][dev] = true;
+  }
+  int* err = device_error_word();
+  if (err == nullptr) return cudaErrorUnknown;
+  const long long tiles_m = (M + 2 * BM - 1) / (2 * BM);
+  const long long tiles_n = (N + BN - 1) / BN;
+  const long long tiles = tiles_m * tiles_n;
+  const long long pairs = resident_pairs((const void*)kernel);
+  const long long used = tiles < pairs ? tiles : pairs;
+  // Raster groups just large enough that one wave of tiles stays inside one
+  // group: the first wave then needs only the rows of its group's M tiles.
+  long long group_m = (used + tiles_n - 1) / tiles_n;
+  group_m = group_m < 1 ? 1 : (group_m > tiles_m ? tiles_m : group_m);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (int)used);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, tA, tB, tC, (const float*)sx, sw, bias,
+                            (const float*)nullptr, (const uint16_t*)nullptr, (int)M, (int)N,
+                            (int)K, (int)group_m, err, x, xq, sx, ready, next_epoch());
 }
 
 }  // namespace qk

@@ -69,6 +69,7 @@ struct Workspace {
   int8_t* xq = nullptr;
   float* sx = nullptr;
   int32_t* xsum = nullptr;
+  unsigned long long* ready = nullptr;  // W8A8: readiness words of the fused quantization
   void* owned = nullptr;
   cudaStream_t stream = nullptr;
 
@@ -85,8 +86,12 @@ struct Workspace {
     }
     xq = reinterpret_cast<int8_t*>(base);
     sx = reinterpret_cast<float*>(base + round256((size_t)M * (size_t)K));
-    if (w4) xsum = reinterpret_cast<int32_t*>(base + round256((size_t)M * (size_t)K) +
-                                               round256((size_t)M * 4u));
+    if (w4)
+      xsum = reinterpret_cast<int32_t*>(base + round256((size_t)M * (size_t)K) +
+                                        round256((size_t)M * 4u));
+    else
+      ready = reinterpret_cast<unsigned long long*>(base + round256((size_t)M * (size_t)K) +
+                                                    round256((size_t)M * 4u));
     return QK_OK;
   }
   ~Workspace() {
@@ -188,12 +193,15 @@ int qk_is_available(int device) {
 
 size_t qk_w8a8_workspace_size(int64_t M, int64_t K) {
   if (M < 0 || K < 0) return 0;
-  return round256((size_t)M * (size_t)K) + round256((size_t)M * 4u);
+  // codes, scales, and one 8-byte readiness word per 128 rows
+  return round256((size_t)M * (size_t)K) + round256((size_t)M * 4u) +
+         round256((size_t)((M + 127) / 128) * 8u);
 }
 
 size_t qk_w4a8_workspace_size(int64_t M, int64_t K) {
   if (M < 0 || K < 0) return 0;
-  return qk_w8a8_workspace_size(M, K) + round256((size_t)M * (size_t)(K / 64) * 4u);
+  return round256((size_t)M * (size_t)K) + round256((size_t)M * 4u) +
+         round256((size_t)M * (size_t)(K / 64) * 4u);
 }
 
 qk_status qk_quantize_weights_int8(const float* W, int64_t N, int64_t K, int8_t* Wq, float* sw,
@@ -261,11 +269,20 @@ qk_status qk_w8a8_linear(const uint16_t* x, int64_t M, int64_t K, const int8_t* 
   if ((st = check_device()) != QK_OK) return st;
   Workspace ws;
   if ((st = ws.init(workspace, ws_bytes, M, K, false, stream)) != QK_OK) return st;
+  if (w8a8_use_fused(M, K, N)) {
+    // one kernel: the GEMM's epilogue warps quantize x into the workspace
+    if (log_enabled())
+      std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> fused quant + tcgen05 GEMM\n",
+                   (long long)M, (long long)K, (long long)N);
+    return from_cuda(launch_w8a8_fused(x, M, K, Wq, sw, bias, N, y, ws.xq, ws.sx, ws.ready, true,
+                                       stream),
+                     "w8a8_fused");
+  }
   if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, nullptr, stream, true),
                       "quant_act")) != QK_OK)
     return st;
   if (log_enabled())
-    std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> quant_act + tcgen05 GEMM\n",
+    std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> quant_act + split-K GEMM\n",
                  (long long)M, (long long)K, (long long)N);
   return from_cuda(launch_w8a8_gemm(ws.xq, ws.sx, M, K, Wq, sw, bias, N, y, nullptr, true, stream),
                    "w8a8_gemm");

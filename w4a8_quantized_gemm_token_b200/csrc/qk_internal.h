@@ -37,6 +37,17 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
                              uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s,
                              const float* gate = nullptr, const uint16_t* residual = nullptr);
 
+// The W8A8 linear in one kernel: the GEMM's epilogue warps quantize bf16 x
+// (per token, the rule of act_quant.cuh) into xq / sx while the tiles run;
+// the producers wait for each 128-row block through `ready` (ceil(M / 128)
+// 8-byte words, epoch-tagged: no clearing needed).  For the shapes
+// w8a8_use_fused accepts (every shape not routed to the split-K kernel).
+bool w8a8_use_fused(int64_t M, int64_t K, int64_t N);
+cudaError_t launch_w8a8_fused(const uint16_t* x, int64_t M, int64_t K, const int8_t* Wq,
+                              const float* sw, const float* bias, int64_t N, uint16_t* y,
+                              int8_t* xq, float* sx, unsigned long long* ready, bool pdl,
+                              cudaStream_t s);
+
 // The same product for thin outputs (N <= 64, see w8a8_use_skinny): 128-row
 // tiles split along K over a cluster, exact int32 partial sums reduced through
 // distributed shared memory.  launch_w8a8_gemm routes such shapes here.
