@@ -56,6 +56,9 @@ L2_BYTES = 126 * 1024 * 1024
 WORKLOADS = {
     "dit_mlp": ("DIT_MLP", None),
     "dit_mlp_gated": ("DIT_MLP", None),
+    "dit_mlp_fused": ("DIT_MLP", None),
+    "dit_attn_fused": ("DIT_ATTN", None),
+    "quickstart_w8a8_fused": ("QUICKSTART", 0),
     "dit_attn": ("DIT_ATTN", None),
     "sweep_4096x4096": ("SWEEP", 0),
     "sweep_4096x12288": ("SWEEP", 1),
@@ -87,6 +90,11 @@ def is_w4(name):
 
 def is_attention(name):
     return name.startswith("sage")
+
+
+def is_fused(name):
+    """The W8A8 linear as one kernel (qk_w8a8_linear_fused)."""
+    return name.endswith("_fused")
 
 
 def is_gated(name):
@@ -335,14 +343,15 @@ class LinearRun:
             qk.qk_w8a8_linear_gated(x, *wt, self.bias, self.gate, self.res, y=self.y,
                                     workspace=self.ws)
         else:
-            qk.qk_w8a8_linear(x, *wt, self.bias, y=self.y, workspace=self.ws)
+            qk.qk_w8a8_linear(x, *wt, self.bias, y=self.y, workspace=self.ws,
+                              fused=is_fused(self.name))
 
     def kstep(self, i):
         """The dominant kernel alone: the product on pre-quantized activations
         (the gated linear has no such entry: its call is timed)."""
         qk = self.qk
-        if self.gated:
-            return self.step(i)
+        if self.gated or (is_fused(self.name) and self.N > 64):
+            return self.step(i)  # the call is the kernel (gated: no split entry)
         if self.xq_sets is None:
             self.xq_sets = [qk.qk_quantize_activations(x, with_xsum=self.w4) for x in self.xs]
         xq, sx, xsum = self.xq_sets[i % self.nsets]
@@ -370,14 +379,14 @@ class LinearRun:
         return ("w8a8_gemm_kernel", "gemm_w8a8.cu", "tensor", None)
 
 
-def launches_per_call(M, K, N, w4, gated, qk):
-    """Kernels one call of the linear launches: the W8A8 linear is one kernel
-    (quantization fused into the GEMM) except for thin outputs (N <= 64, the
-    quantization kernel + the split-K kernel) and the gated epilogue (two);
-    the W4A8 linear follows its plan (qk_w4a8_linear_plan)."""
+def launches_per_call(M, K, N, w4, gated, qk, fused=False):
+    """Kernels one call of the linear launches: the W8A8 linear is the
+    quantization kernel + the GEMM (qk_w8a8_linear_fused: one kernel, except
+    for thin outputs, N <= 64); the W4A8 linear follows its plan
+    (qk_w4a8_linear_plan)."""
     if w4:
         return 1 if qk.qk_w4a8_linear_plan(M, K, N) == qk.QK_PLAN_GEMV_QUANT else 2
-    if gated or (N <= 64 and M <= 8192):
+    if gated or not fused or (N <= 64 and M <= 8192):
         return 2
     return 1
 
@@ -407,6 +416,9 @@ def roofline(run, k_ms, peaks, int8, workload):
     if run.gated:
         roof["kernel"] = "w8a8_gemm_kernel (gated) with its activation quant: the timed call"
         roof["traffic"] = None  # the committed summary covers the plain epilogue
+    elif is_fused(workload) and run.N > 64:
+        roof["kernel"] = "w8a8_gemm_kernel with fused activation quantization: the timed call"
+        roof["traffic"] = None
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel_ms"] = k_ms
     return roof
@@ -511,7 +523,8 @@ def measure_sustained(run, local, seconds, int8, peaks):
 # gated residual epilogue and the INT8 attention.
 TABLE = ["tiny", "dit_attn", "sweep_4096x4096", "sweep_4096x12288", "sweep_12288x4096",
          "sweep_thin_5120x48", "w4a8_m1", "w4a8_m8", "w4a8_m16", "w4a8_m4096",
-         "quickstart_w8a8", "quickstart_w4a8", "dit_mlp_gated", "sage_attn"]
+         "quickstart_w8a8", "quickstart_w4a8", "dit_mlp_gated", "sage_attn",
+         "dit_mlp_fused", "dit_attn_fused", "quickstart_w8a8_fused"]
 
 
 def table_entry(name, local, dev, peaks, int8):
@@ -536,7 +549,8 @@ def table_entry(name, local, dev, peaks, int8):
     ms, k_ms, clocks, timing = time_linear(run, steps, 3, local)
     roof = roofline(run, k_ms, peaks, int8, name)
     per = ms / steps
-    rec = {"config": run.case.name + ("_gated_residual" if run.gated else ""),
+    rec = {"config": run.case.name + ("_gated_residual" if run.gated else "")
+                     + ("_one_kernel" if is_fused(name) else ""),
            "M": run.M, "K": run.K, "N": run.N, "steps": steps, "timing": timing,
            "ms_per_call": per, "value": run.ops / (per / 1e3) / 1e12, "unit": "TOPS",
            "pct_of_int8_spec": 100.0 * run.ops / (per / 1e3) / 1e12 / INT8_SPEC_TOPS,
@@ -716,7 +730,7 @@ def run_ours(args, world, rank, local):
     sustained = None
     if single and not args.no_sustained and not w4 and M > 256:
         sustained = measure_sustained(run, local, 2.0, int8, peaks)
-    launches = launches_per_call(M, K, N, w4, gated, run.qk)
+    launches = launches_per_call(M, K, N, w4, gated, run.qk, is_fused(args.workload))
     config = {"workload": run.case.name + ("_gated_residual" if gated else ""),
               "M": M, "K": K, "N": N,
               "weights": "W4 affine g64" if w4 else "W8 per-channel",

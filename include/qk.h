@@ -87,8 +87,9 @@ int qk_is_available(int device);
 
 /* ------------------------------------------------------------- workspace */
 
-/* Bytes of workspace qk_w8a8_linear needs: int8 codes [M, K] and fp32 scales
- * [M], each 256-byte aligned inside the block. */
+/* Bytes of workspace qk_w8a8_linear (and qk_w8a8_linear_fused) needs: int8
+ * codes [M, K], fp32 scales [M] and one 8-byte readiness word per row (used
+ * by qk_w8a8_linear_fused), each 256-byte aligned inside the block. */
 size_t qk_w8a8_workspace_size(int64_t M, int64_t K);
 
 /* Bytes of workspace qk_w4a8_linear needs: codes [M, K], scales [M] and int32
@@ -173,6 +174,28 @@ qk_status qk_w8a8_linear(const uint16_t *x, int64_t M, int64_t K,
                          const int8_t *Wq, const float *sw, const float *bias, int64_t N,
                          uint16_t *y, void *workspace, size_t ws_bytes,
                          qk_stream_t stream);
+
+/*
+ * The W8A8 linear as ONE kernel ("qlip-mlx" README, "w8a8_linear /
+ * W8A8Linear": the activations quantized dynamically inside the op, the
+ * whole linear a single graph node).  Same inputs, outputs, workspace and
+ * errors as qk_w8a8_linear, and the same result (the codes and scales left in
+ * the workspace are the same bits): the tcgen05 GEMM's epilogue warps
+ * quantize the rows of x into the workspace while the tiles run (rows spread
+ * over every warp of the grid, kept two waves of tiles ahead), and the loads
+ * of each tile wait until its rows are ready (one readiness word per row,
+ * set to a per-launch value, so the workspace needs no clearing).  Thin
+ * outputs (N <= 64) take the split-K route behind the quantization kernel,
+ * as qk_w8a8_linear does.
+ * On B200 this is slower than the two kernels of qk_w8a8_linear at the DiT
+ * shapes measured (the quantization's memory traffic and latency inside the
+ * GEMM cost more than the kernel boundary saves), so qk_w8a8_linear does not
+ * use it.
+ */
+qk_status qk_w8a8_linear_fused(const uint16_t *x, int64_t M, int64_t K,
+                               const int8_t *Wq, const float *sw, const float *bias, int64_t N,
+                               uint16_t *y, void *workspace, size_t ws_bytes,
+                               qk_stream_t stream);
 
 /*
  * The W8A8 linear with a gated residual epilogue ("mlx-kquant PR #89", commit

@@ -46,9 +46,9 @@ def test_status_strings(qk):
 
 def test_workspace_sizes(qk):
     r = lambda b: (b + 255) // 256 * 256
-    # codes, scales and one 8-byte readiness word per 128 rows (fused quantization)
-    assert qk.qk_w8a8_workspace_size(16384, 3072) == r(16384 * 3072) + r(16384 * 4) + r(128 * 8)
-    assert qk.qk_w8a8_workspace_size(300, 64) == r(300 * 64) + r(300 * 4) + r(3 * 8)
+    # codes, scales and one 8-byte readiness word per row (fused quantization)
+    assert qk.qk_w8a8_workspace_size(16384, 3072) == r(16384 * 3072) + r(16384 * 4) + r(16384 * 8)
+    assert qk.qk_w8a8_workspace_size(300, 64) == r(300 * 64) + r(300 * 4) + r(300 * 8)
     assert qk.qk_w4a8_workspace_size(17, 4096) == r(17 * 4096) + r(17 * 4) + r(17 * 64 * 4)
     assert qk.qk_w8a8_workspace_size(0, 256) == 0
 

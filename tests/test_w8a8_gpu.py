@@ -17,9 +17,9 @@ pytestmark = pytest.mark.gpu
 TOL_ULP = 2
 
 SHAPES = [  # (M, K, N): tiles of 128 x 256 with K blocks of 128
-    # qk_w8a8_linear runs these in one kernel (the GEMM's epilogue warps
-    # quantize x); 8192 x 256 x 72: 64 row blocks behind one column of tiles;
-    # 600 x 8192: rows longer than 4096 elements (two passes per row)
+    # the one-kernel form (qk_w8a8_linear_fused: the GEMM's epilogue warps
+    # quantize x): 8192 x 256 x 72 has 64 row blocks behind one column of
+    # tiles; 600 x 8192 has rows longer than 4096 elements (two passes per row)
     (8192, 256, 72),
     (600, 8192, 264),
     (2, 4096, 4096),
@@ -57,6 +57,8 @@ def test_w8a8_small_full_parity(qk, orc, MKN, with_bias):
     x = to_dev_bf16(xb)
     bias = to_dev(b) if with_bias else None
     y = qk.qk_w8a8_linear(x, Wq, sw, bias)
+    ws = torch.empty(qk.qk_w8a8_workspace_size(M, K), dtype=torch.uint8, device="cuda")
+    yf = qk.qk_w8a8_linear(x, Wq, sw, bias, workspace=ws, fused=True)
     xq, sx, _ = qk.qk_quantize_activations(x)
     acc = qk.qk_debug_w8a8_acc(xq, Wq)
     torch.cuda.synchronize()
@@ -65,6 +67,12 @@ def test_w8a8_small_full_parity(qk, orc, MKN, with_bias):
     assert np.array_equal(host(acc).astype(np.int64), acc_o)
     d = bf16_ulp_distance(t2bits(y), y_o)
     assert d.max() <= TOL_ULP, f"worst {d.max()} ulp"
+    # the one-kernel form: the same bits, and the same codes and scales left
+    # in the workspace
+    assert torch.equal(yf.view(torch.int16), y.view(torch.int16))
+    off = (M * K + 255) // 256 * 256
+    assert np.array_equal(host(ws[: M * K].view(torch.int8).view(M, K)), xq_o)
+    assert np.array_equal(host(ws[off: off + 4 * M].view(torch.float32)), sx_o)
     qk.qk_check_device_error()
 
 
@@ -79,9 +87,11 @@ def test_w8a8_configs(qk, orc, case):
     bias = to_dev(b) if b is not None else None
     ws = torch.empty(qk.qk_w8a8_workspace_size(case.M, case.K), dtype=torch.uint8, device="cuda")
     y = qk.qk_w8a8_linear(x, Wq, sw, bias, workspace=ws)
+    yf = qk.qk_w8a8_linear(x, Wq, sw, bias, workspace=ws, fused=True)  # one-kernel form
     xq, sx, _ = qk.qk_quantize_activations(x)
     acc = qk.qk_debug_w8a8_acc(xq, Wq)
     torch.cuda.synchronize()
+    assert torch.equal(yf.view(torch.int16), y.view(torch.int16))
     rows = np.arange(case.M) if case.M <= 256 else sample_rows(case.M, extra=6, seed=case.M)
     xq_all, sx_all = orc.quant_act(xb)
     assert np.array_equal(host(xq), xq_all) and np.array_equal(host(sx), sx_all)
@@ -137,9 +147,10 @@ def test_w8a8_guard_bands(qk, orc, MKN):
 
 
 def test_w8a8_fused_workspace_reuse_and_garbage(qk, orc):
-    """The one-kernel W8A8 linear keeps per-row-block readiness words in the
-    workspace, tagged with each launch's epoch: a workspace full of garbage, or
-    left by a call of another shape, gives the same bits as a fresh one."""
+    """The one-kernel W8A8 linear keeps a readiness word per row in the
+    workspace, set to each launch's own value: a workspace full of garbage, or
+    left by a call of another shape, gives the same bits as the two-kernel
+    linear."""
     cases = [synthetic.LinearCase("wa", M=700, K=1024, N=520, seed=41),
              synthetic.LinearCase("wb", M=1300, K=512, N=264, seed=42)]
     prepared = [prepare(qk, orc, c) for c in cases]
@@ -148,7 +159,8 @@ def test_w8a8_fused_workspace_reuse_and_garbage(qk, orc):
     fresh = [qk.qk_w8a8_linear(to_dev_bf16(p[0]), p[1], p[2], to_dev(p[5])) for p in prepared]
     for rep in range(2):
         for p, want in zip(prepared, fresh):
-            y = qk.qk_w8a8_linear(to_dev_bf16(p[0]), p[1], p[2], to_dev(p[5]), workspace=ws)
+            y = qk.qk_w8a8_linear(to_dev_bf16(p[0]), p[1], p[2], to_dev(p[5]), workspace=ws,
+                                  fused=True)
             torch.cuda.synchronize()
             assert torch.equal(y.view(torch.int16), want.view(torch.int16))
     y_o, _, _, _ = orc.w8a8_linear(prepared[0][0], prepared[0][3], prepared[0][4], prepared[0][5])

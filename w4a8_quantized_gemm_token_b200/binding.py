@@ -33,6 +33,7 @@ _SIGS = {
     "qk_quantize_weights_int4": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "qk_quantize_activations": (_I, [_P, _I64, _I64, _P, _P, _P, _P]),
     "qk_w8a8_linear": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "qk_w8a8_linear_fused": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w8a8_gemm": (_I, [_P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P]),
     "qk_w8a8_linear_gated": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w4a8_linear": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
@@ -171,8 +172,9 @@ def qk_quantize_activations(x, xq=None, sx=None, xsum=None, with_xsum=False, str
     return xq, sx, xsum
 
 
-def qk_w8a8_linear(x, Wq, sw, bias=None, y=None, workspace=None, stream=None):
-    """y bf16 [M, N] = bf16(quant(x) . Wq^T * sx * sw + bias)."""
+def qk_w8a8_linear(x, Wq, sw, bias=None, y=None, workspace=None, stream=None, fused=False):
+    """y bf16 [M, N] = bf16(quant(x) . Wq^T * sx * sw + bias).  fused=True calls
+    qk_w8a8_linear_fused (the same result from one kernel)."""
     _need(x, torch.bfloat16, 2, "x")
     _need(Wq, torch.int8, 2, "Wq")
     _need(sw, torch.float32, 1, "sw")
@@ -182,8 +184,9 @@ def qk_w8a8_linear(x, Wq, sw, bias=None, y=None, workspace=None, stream=None):
     N = Wq.shape[0]
     y = _out(y, (M, N), torch.bfloat16, x.device, "y")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.qk_w8a8_linear(_ptr(x), M, K, _ptr(Wq), _ptr(sw), _ptr(bias), N, _ptr(y),
-                              _ptr(workspace), ws_bytes, _stream(stream)), "qk_w8a8_linear")
+    fn = lib.qk_w8a8_linear_fused if fused else lib.qk_w8a8_linear
+    _check(fn(_ptr(x), M, K, _ptr(Wq), _ptr(sw), _ptr(bias), N, _ptr(y), _ptr(workspace),
+              ws_bytes, _stream(stream)), "qk_w8a8_linear_fused" if fused else "qk_w8a8_linear")
     return y
 
 

@@ -145,42 +145,119 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
 
 // ---- readiness of the quantized rows (the fused-quantization kernel)
 //
-// Row block b (rows 128 b .. 128 b + 127 of x) is ready when the 64-bit word
-// ready[b] holds (epoch << 8) | (its number of rows): every warp that
-// quantized one of its rows adds 1, tagged with the launch's epoch (a value
-// the host never reuses), so the words need no clearing between launches and
-// a word left by an earlier launch never reads as ready.
+// Row r of xq / sx is ready when the 64-bit word ready[r] holds the launch's
+// epoch (a value the host never reuses): the warp that quantized the row
+// stores it with release semantics after its codes and scale.  No word is
+// ever incremented, so none needs clearing between launches, and a word left
+// by an earlier launch (or any garbage) never reads as ready.
 
-// Adds one finished row to a readiness word (lock-free; bounded retries).
-__device__ __forceinline__ void ready_add(unsigned long long* p, unsigned long long epoch,
-                                          int* err) {
-  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(p);
-  for (int i = 0; i < (1 << 20); ++i) {
-    const unsigned long long base = (old >> 8) == epoch ? old : (epoch << 8);
-    const unsigned long long prev = atomicCAS(p, old, base + 1ull);
-    if (prev == old) return;
-    old = prev;
-  }
-  record_timeout(err);
+__device__ __forceinline__ void ready_publish(unsigned long long* p, unsigned long long epoch) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(epoch) : "memory");
 }
 
-// Waits (bounded) until a readiness word holds `want`; then orders the TMA
-// (async proxy) reads that follow after the generic-proxy writes it observed.
-__device__ __forceinline__ bool ready_wait(const unsigned long long* p, unsigned long long want,
-                                           int* err) {
+__device__ __forceinline__ unsigned long long ready_load(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Warp-collective: waits (bounded) until rows [r0, r0 + nrows) (nrows <= 128)
+// are ready, each lane watching four of them.  Returns the same value in
+// every lane; afterwards the TMA (async proxy) reads of lane 0 are ordered
+// after the generic-proxy writes the warp observed.
+__device__ __forceinline__ bool ready_wait_rows(const unsigned long long* ready, int r0, int nrows,
+                                                unsigned long long epoch, int lane, int* err) {
   const long long t0 = clock64();
+  bool ok = true;
   while (true) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    if (v == want) break;
+    bool mine = true;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = lane + 32 * i;
+      if (r < nrows && ready_load(ready + r0 + r) != epoch) mine = false;
+    }
+    if (__all_sync(0xFFFFFFFFu, mine)) break;
     if (clock64() - t0 > QK_WAIT_LIMIT_CYCLES) {
-      record_timeout(err);
-      return false;
+      if (lane == 0) record_timeout(err);
+      ok = false;
+      break;
     }
     __nanosleep(32);
   }
+  __syncwarp();
   asm volatile("fence.proxy.async.global;" ::: "memory");
-  return true;
+  return ok;
+}
+
+// One lane's row: waits (bounded) until it is ready.
+__device__ __forceinline__ void ready_wait_row(const unsigned long long* p,
+                                               unsigned long long epoch, int* err) {
+  const long long t0 = clock64();
+  while (ready_load(p) != epoch) {
+    if (clock64() - t0 > QK_WAIT_LIMIT_CYCLES) {
+      record_timeout(err);
+      return;
+    }
+    __nanosleep(32);
+  }
+}
+
+// Quantizes RB = min(16, 32 / CPL) rows of x held in registers at once (rows r0,
+// r0 + stride, ...; the first nrows of them), each row <= 32 CPL 16-byte
+// chunks (the rule of act_quant.cuh); writes their codes, then their scales
+// and readiness words (all lanes' writes fenced before the release).
+template <int CPL>
+__device__ __forceinline__ void quant_rows(const uint16_t* __restrict__ x, int K, int nch, int r0,
+                                           int stride, int nrows, int8_t* xq, float* sxo,
+                                           unsigned long long* ready, unsigned long long epoch,
+                                           int lane) {
+  constexpr int RB = 32 / CPL < 16 ? 32 / CPL : 16;
+  uint4 v[RB][CPL];
+#pragma unroll
+  for (int i = 0; i < RB; ++i) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(r0 + i * stride) * K);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const int cc = c * 32 + lane;
+      v[i][c] = (i < nrows && cc < nch) ? __ldcs(src + cc) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  float amax[RB];
+#pragma unroll
+  for (int i = 0; i < RB; ++i) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      m = bf16x2_absmax_bits(m, v[i][c].x);
+      m = bf16x2_absmax_bits(m, v[i][c].y);
+      m = bf16x2_absmax_bits(m, v[i][c].z);
+      m = bf16x2_absmax_bits(m, v[i][c].w);
+    }
+    amax[i] = warp_max_bits_to_float(m);
+  }
+  int dummy = 0;
+#pragma unroll
+  for (int i = 0; i < RB; ++i) {
+    if (i < nrows) {
+      const float q = act_multiplier(amax[i]);
+      uint2* dst = reinterpret_cast<uint2*>(xq + (size_t)(r0 + i * stride) * K);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const int cc = c * 32 + lane;
+        if (cc < nch) dst[cc] = quant_chunk(v[i][c], q, &dummy);
+      }
+      if (lane == 0) sxo[r0 + i * stride] = act_scale(amax[i]);
+    }
+  }
+  // every lane's codes (and the scales) before any of the rows counts as done
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < RB; ++i)
+      if (i < nrows) ready_publish(ready + r0 + i * stride, epoch);
+  }
 }
 
 // kAccOut: store the int32 sums instead of y.  kGated: the gated residual
@@ -253,24 +330,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-        int mb, nb;
-        tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
-        const int arow = mb * 2 * BM + (int)rank * BM;
-        const int brow = nb * BN + (int)rank * (BN / 2);
-        if constexpr (kFused) {
-          // this CTA's 128 rows of xq must be quantized before the TMA reads them
-          const int nrows = min(BM, M - arow);
-          if (nrows > 0 &&
-              !ready_wait(ready + (arow / BM), (epoch << 8) | (unsigned long long)nrows, err)) {
-            ok = false;
-            break;
-          }
-        }
+    // (lane 0 issues the loads; with fused quantization the whole warp first
+    // checks that the CTA's 128 rows of the tile are quantized)
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+      int mb, nb;
+      tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
+      const int arow = mb * 2 * BM + (int)rank * BM;
+      const int brow = nb * BN + (int)rank * (BN / 2);
+      if constexpr (kFused) {
+        const int nrows = min(BM, M - arow);
+        if (nrows > 0 && !ready_wait_rows(ready, arow, nrows, epoch, lane, err)) break;
+      }
+      if (lane == 0) {
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, err)) {
             ok = false;
@@ -291,6 +365,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
       }
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
     }
   } else if (warp == 1) {
     // ------------------------------------------- MMA issuer (pair leader)
@@ -359,70 +434,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
     // ---- fused quantization: rows qw, qw + QW, qw + 2 QW, ... of x are this
     // warp's (QW = all epilogue warps of the grid, so the first rows are spread
-    // over every SM).  Each row: absmax, multiplier and scale, codes (the rule
-    // of the stand-alone kernel, act_quant.cuh), then the row is published to
-    // its block's readiness word.  Rows of up to 4096 elements are held in
-    // registers two at a time; longer rows take two passes over 4096-element
-    // segments (the second from L2).
+    // over every SM).  Rows of up to 4096 elements are quantized in batches held
+    // in registers (min(16, 32 / CPL) rows of up to 32 CPL chunks each); longer rows take
+    // two passes over 4096-element segments (the second from L2).
     const int QW = (int)gridDim.x * kEpiWarps;
     int qrow = (int)blockIdx.x * kEpiWarps + e;
     const int nch = K >> 3;  // 16-byte chunks of bf16 per row
-    auto publish = [&](int r, float amax) {
-      if (lane == 0) sx_out[r] = act_scale(amax);
-      // every lane's codes (and the scale) before the row counts as done
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) ready_add(ready + (r >> 7), epoch, err);
-    };
+    const int cpl = nch <= 32 ? 1 : nch <= 64 ? 2 : nch <= 128 ? 4 : nch <= 256 ? 8 : 16;
     auto quantize_until = [&](int limit) {
       if constexpr (kFused) {
         limit = min(limit, M);
         while (qrow < limit) {
           if (nch <= 512) {
-            const int r0 = qrow, r1 = qrow + QW;
-            const bool two = r1 < limit;
-            const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r0 * K);
-            const uint4* s1 = reinterpret_cast<const uint4*>(x + (size_t)(two ? r1 : r0) * K);
-            uint4 v0[16], v1[16];
-            uint32_t m0 = 0, m1 = 0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = i * 32 + lane;
-              v0[i] = make_uint4(0u, 0u, 0u, 0u);
-              v1[i] = make_uint4(0u, 0u, 0u, 0u);
-              if (c < nch) {
-                v0[i] = __ldcs(s0 + c);
-                if (two) v1[i] = __ldcs(s1 + c);
-              }
+            const int rb = min(16, 32 / cpl);
+            const int n = min(rb, (limit - qrow + QW - 1) / QW);
+            switch (cpl) {
+              case 1: quant_rows<1>(x, K, nch, qrow, QW, n, xq_out, sx_out, ready, epoch, lane); break;
+              case 2: quant_rows<2>(x, K, nch, qrow, QW, n, xq_out, sx_out, ready, epoch, lane); break;
+              case 4: quant_rows<4>(x, K, nch, qrow, QW, n, xq_out, sx_out, ready, epoch, lane); break;
+              case 8: quant_rows<8>(x, K, nch, qrow, QW, n, xq_out, sx_out, ready, epoch, lane); break;
+              default: quant_rows<16>(x, K, nch, qrow, QW, n, xq_out, sx_out, ready, epoch, lane); break;
             }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              m0 = bf16x2_absmax_bits(m0, v0[i].x);
-              m0 = bf16x2_absmax_bits(m0, v0[i].y);
-              m0 = bf16x2_absmax_bits(m0, v0[i].z);
-              m0 = bf16x2_absmax_bits(m0, v0[i].w);
-              m1 = bf16x2_absmax_bits(m1, v1[i].x);
-              m1 = bf16x2_absmax_bits(m1, v1[i].y);
-              m1 = bf16x2_absmax_bits(m1, v1[i].z);
-              m1 = bf16x2_absmax_bits(m1, v1[i].w);
-            }
-            const float a0 = warp_max_bits_to_float(m0), a1 = warp_max_bits_to_float(m1);
-            const float q0 = act_multiplier(a0), q1 = act_multiplier(a1);
-            uint2* d0 = reinterpret_cast<uint2*>(xq_out + (size_t)r0 * K);
-            uint2* d1 = reinterpret_cast<uint2*>(xq_out + (size_t)r1 * K);
-            int dummy = 0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = i * 32 + lane;
-              if (c < nch) {
-                d0[c] = quant_chunk(v0[i], q0, &dummy);
-                if (two) d1[c] = quant_chunk(v1[i], q1, &dummy);
-              }
-            }
-            publish(r0, a0);
-            if (two) publish(r1, a1);
-            qrow += two ? 2 * QW : QW;
+            qrow += n * QW;
           } else {
             const int r0 = qrow;
             const uint4* s0 = reinterpret_cast<const uint4*>(x + (size_t)r0 * K);
@@ -453,7 +486,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (c < nch) d0[c] = quant_chunk(__ldcg(s0 + c), q0, &dummy);
               }
             }
-            publish(r0, a0);
+            if (lane == 0) sx_out[r0] = act_scale(a0);
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) ready_publish(ready + r0, epoch);
             qrow += QW;
           }
         }
@@ -497,13 +534,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row = row0 + lane;
       float sxf = 0.0f;
       if constexpr (kFused) {
-        // the scales were written in this launch by other warps: acquire the
-        // block's readiness word, then read past L1
-        const int nrows = min(BM, M - (row0 - q * 32));
-        if (lane == 0 && nrows > 0)
-          ready_wait(ready + ((row0 - q * 32) / BM), (epoch << 8) | (unsigned long long)nrows, err);
-        __syncwarp();
-        if (row < M) sxf = __ldcg(sx + row);
+        // the scale was written in this launch by another warp: acquire the
+        // row's readiness word, then read past L1
+        if (row < M) {
+          ready_wait_row(ready + row, epoch, err);
+          sxf = __ldcg(sx + row);
+        }
       } else {
         sxf = (!kAccOut && row < M) ? __ldg(sx + row) : 0.0f;
       }

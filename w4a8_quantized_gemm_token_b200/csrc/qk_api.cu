@@ -193,9 +193,8 @@ int qk_is_available(int device) {
 
 size_t qk_w8a8_workspace_size(int64_t M, int64_t K) {
   if (M < 0 || K < 0) return 0;
-  // codes, scales, and one 8-byte readiness word per 128 rows
-  return round256((size_t)M * (size_t)K) + round256((size_t)M * 4u) +
-         round256((size_t)((M + 127) / 128) * 8u);
+  // codes, scales, and one 8-byte readiness word per row
+  return round256((size_t)M * (size_t)K) + round256((size_t)M * 4u) + round256((size_t)M * 8u);
 }
 
 size_t qk_w4a8_workspace_size(int64_t M, int64_t K) {
@@ -269,23 +268,43 @@ qk_status qk_w8a8_linear(const uint16_t* x, int64_t M, int64_t K, const int8_t* 
   if ((st = check_device()) != QK_OK) return st;
   Workspace ws;
   if ((st = ws.init(workspace, ws_bytes, M, K, false, stream)) != QK_OK) return st;
-  if (w8a8_use_fused(M, K, N)) {
-    // one kernel: the GEMM's epilogue warps quantize x into the workspace
-    if (log_enabled())
-      std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> fused quant + tcgen05 GEMM\n",
-                   (long long)M, (long long)K, (long long)N);
-    return from_cuda(launch_w8a8_fused(x, M, K, Wq, sw, bias, N, y, ws.xq, ws.sx, ws.ready, true,
-                                       stream),
-                     "w8a8_fused");
-  }
   if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, nullptr, stream, true),
                       "quant_act")) != QK_OK)
     return st;
   if (log_enabled())
-    std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> quant_act + split-K GEMM\n",
+    std::fprintf(stderr, "[qk] w8a8_linear M=%lld K=%lld N=%lld -> quant_act + tcgen05 GEMM\n",
                  (long long)M, (long long)K, (long long)N);
   return from_cuda(launch_w8a8_gemm(ws.xq, ws.sx, M, K, Wq, sw, bias, N, y, nullptr, true, stream),
                    "w8a8_gemm");
+}
+
+qk_status qk_w8a8_linear_fused(const uint16_t* x, int64_t M, int64_t K, const int8_t* Wq,
+                               const float* sw, const float* bias, int64_t N, uint16_t* y,
+                               void* workspace, size_t ws_bytes, qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, false);
+  if (st != QK_OK || M == 0) return st;
+  if (!x || !Wq || !sw || !y) return QK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(sw) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return QK_ERR_MISALIGNED;
+  if ((st = check_device()) != QK_OK) return st;
+  Workspace ws;
+  if ((st = ws.init(workspace, ws_bytes, M, K, false, stream)) != QK_OK) return st;
+  if (!w8a8_use_fused(M, K, N)) {
+    // thin outputs: the split-K route, behind the quantization kernel
+    if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, nullptr, stream, true),
+                        "quant_act")) != QK_OK)
+      return st;
+    return from_cuda(
+        launch_w8a8_gemm(ws.xq, ws.sx, M, K, Wq, sw, bias, N, y, nullptr, true, stream),
+        "w8a8_gemm");
+  }
+  if (log_enabled())
+    std::fprintf(stderr, "[qk] w8a8_linear_fused M=%lld K=%lld N=%lld -> one kernel\n",
+                 (long long)M, (long long)K, (long long)N);
+  return from_cuda(
+      launch_w8a8_fused(x, M, K, Wq, sw, bias, N, y, ws.xq, ws.sx, ws.ready, true, stream),
+      "w8a8_fused");
 }
 
 qk_status qk_w8a8_linear_gated(const uint16_t* x, int64_t M, int64_t K, const int8_t* Wq,

@@ -39,8 +39,8 @@ cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64
 
 // The W8A8 linear in one kernel: the GEMM's epilogue warps quantize bf16 x
 // (per token, the rule of act_quant.cuh) into xq / sx while the tiles run;
-// the producers wait for each 128-row block through `ready` (ceil(M / 128)
-// 8-byte words, epoch-tagged: no clearing needed).  For the shapes
+// the producers wait for each row through `ready` (M 8-byte words, each set
+// to the launch's epoch when its row is quantized: no clearing needed).  For the shapes
 // w8a8_use_fused accepts (every shape not routed to the split-K kernel).
 bool w8a8_use_fused(int64_t M, int64_t K, int64_t N);
 cudaError_t launch_w8a8_fused(const uint16_t* x, int64_t M, int64_t K, const int8_t* Wq,
