@@ -375,7 +375,8 @@ class LinearRun:
             return ("w8a8_skinny_kernel", "gemm_w8a8_skinny.cu", "hbm",
                     M * K + N * K + 2 * M * N + 4 * (M + 2 * N))
         if self.w4:
-            return ("w4a8_gemm_kernel", "gemm_w4a8.cu", "tensor", None)
+            # the GEMM route: plane count, plane build, gated fold, byte-plane GEMM
+            return ("w4a8_planes_kernel", "gemm_w4a8_planes.cu", "tensor", None)
         return ("w8a8_gemm_kernel", "gemm_w8a8.cu", "tensor", None)
 
 
@@ -383,9 +384,12 @@ def launches_per_call(M, K, N, w4, gated, qk, fused=False):
     """Kernels one call of the linear launches: the W8A8 linear is the
     quantization kernel + the GEMM (qk_w8a8_linear_fused: one kernel, except
     for thin outputs, N <= 64); the W4A8 linear follows its plan
-    (qk_w4a8_linear_plan)."""
+    (qk_w4a8_linear_plan); its GEMM route is four kernels (the plane count,
+    the plane build, the per-group fold that computes only when the byte
+    planes cannot, and the byte-plane GEMM)."""
     if w4:
-        return 1 if qk.qk_w4a8_linear_plan(M, K, N) == qk.QK_PLAN_GEMV_QUANT else 2
+        plan = qk.qk_w4a8_linear_plan(M, K, N)
+        return {qk.QK_PLAN_GEMV_QUANT: 1, qk.QK_PLAN_QUANT_GEMV: 2}.get(plan, 5)
     if gated or not fused or (N <= 64 and M <= 8192):
         return 2
     return 1

@@ -62,9 +62,11 @@ typedef enum {
 
 /* Routes of the W4A8 product. */
 typedef enum {
-    QK_ROUTE_AUTO = 0, /* GEMV when M <= 16 and it fits, else GEMM             */
-    QK_ROUTE_GEMM = 1, /* tensor-core GEMM (tcgen05), any M                   */
-    QK_ROUTE_GEMV = 2  /* weight-streaming GEMV, M <= 16 only                 */
+    QK_ROUTE_AUTO = 0,     /* GEMV when M <= 16 and it fits, else GEMM          */
+    QK_ROUTE_GEMM = 1,     /* tensor-core GEMM (tcgen05), any M: byte planes,   */
+                           /* or the per-group fold where planes cannot serve   */
+    QK_ROUTE_GEMV = 2,     /* weight-streaming GEMV, M <= 16 only              */
+    QK_ROUTE_GEMM_FOLD = 3 /* tensor-core GEMM with the per-group fold, any M  */
 } qk_route;
 
 /* Static string for a status code (never NULL). */
@@ -93,7 +95,9 @@ int qk_is_available(int device);
 size_t qk_w8a8_workspace_size(int64_t M, int64_t K);
 
 /* Bytes of workspace qk_w4a8_linear needs: codes [M, K], scales [M] and int32
- * group sums [M, K/64]. */
+ * group sums [M, K/64], each 256-byte aligned inside the block.  (The GEMM
+ * route's byte planes of the weight, up to 3 N K bytes, are allocated
+ * stream-ordered by the call itself: see qk_w4a8_linear.) */
 size_t qk_w4a8_workspace_size(int64_t M, int64_t K);
 
 /* ------------------------------------------------------ offline weights */
@@ -280,6 +284,16 @@ qk_status qk_w8a8_linear_noalloc(const uint16_t *x, int64_t M, int64_t K,
  * M <= 16 takes the weight-streaming GEMV when its per-CTA working set fits
  * in shared memory (K <= 4096 at M = 16), otherwise the tensor-core GEMM; both
  * compute the same per-group integers and agree to the fp64 rounding order.
+ * The GEMM route computes the same value through byte planes of the
+ * dequantized weight: every scale and offset of weight row n is an integer
+ * multiple of 2^e_n (e_n the smallest exponent of their lowest set bits), so
+ * every dequantized weight is 2^e_n times an integer W; when W + 0x80..80 fits
+ * P <= 3 bytes for every weight (Gaussian weights need 2 or 3), the product is
+ * P exact int8 GEMMs on those bytes, rounded once -- the fold's exact value,
+ * the same bits as the per-group fold wherever that fold is exact in fp64;
+ * otherwise the per-group fold kernel computes it.  The route allocates its
+ * scratch (the planes, up to 3 N K bytes) stream-ordered from a memory pool of
+ * the library that keeps freed blocks for reuse.
  * When also M <= 8 and each CTA's K slice of x fits its registers (M times
  * the slice <= 16384 elements) the GEMV quantizes x itself (same rule and
  * codes as qk_quantize_activations) and the call is one kernel; the workspace
@@ -324,6 +338,8 @@ int qk_w4a8_linear_plan(int64_t M, int64_t K, int64_t N);
  * does not read xsum, the other routes read it.
  * QK_ROUTE_GEMV with M > 16 returns QK_ERR_INVALID_ARG; with a shape whose
  * GEMV working set does not fit shared memory, QK_ERR_UNSUPPORTED_SHAPE.
+ * QK_ROUTE_GEMM takes the byte planes (or the fold where they cannot serve);
+ * QK_ROUTE_GEMM_FOLD always takes the per-group fold kernel (any M).
  */
 qk_status qk_w4a8_gemm(const int8_t *xq, const float *sx, const int32_t *xsum,
                        int64_t M, int64_t K,
@@ -396,6 +412,21 @@ qk_status qk_debug_w4a8_group_acc(const int8_t *xq, int64_t M, int64_t K,
                                   const uint8_t *Wp, int64_t N,
                                   int64_t m0, int64_t m1, int32_t *acc,
                                   int route, qk_stream_t stream);
+
+/*
+ * The plane count the W4A8 GEMM route computes for a weight (the byte-plane
+ * reformulation of the fold: with e_n the smallest exponent of the lowest set
+ * bit over the nonzero scales and offsets of weight row n, every dequantized
+ * weight of the row is 2^e_n times the integer S q + O; the count is the
+ * fewest bytes P <= 3 holding S q + O + 0x80..80 for every code q of every row,
+ * else 255, or 255 for a non-finite scale or offset).  Writes it to *planes
+ * (host) after synchronizing `stream`.  The route uses the byte-plane GEMM
+ * for P <= 3, the per-group fold kernel otherwise.  Shapes as for the W4A8
+ * calls; N >= 8.
+ */
+qk_status qk_debug_w4a8_plane_count(const uint16_t *wscale, const uint16_t *woffset,
+                                    int64_t N, int64_t K, int *planes,
+                                    qk_stream_t stream);
 
 /*
  * A probe of the device's INT8 tensor-pipe throughput (the denominator of the

@@ -44,6 +44,7 @@ _SIGS = {
     "qk_debug_w4a8_group_acc": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I, _P]),
     "qk_debug_wait_timeout": (_I, [_I64, _P]),
     "qk_debug_int8_peak": (_I, [_I64, _P, _P]),
+    "qk_debug_w4a8_plane_count": (_I, [_P, _P, _I64, _I64, _P, _P]),
     "qk_sage_attention_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "qk_sage_attention": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]),
 }
@@ -53,7 +54,7 @@ for _name, (_res, _args) in _SIGS.items():
     _fn.argtypes = _args
 
 QK_OK = 0
-QK_ROUTE_AUTO, QK_ROUTE_GEMM, QK_ROUTE_GEMV = 0, 1, 2
+QK_ROUTE_AUTO, QK_ROUTE_GEMM, QK_ROUTE_GEMV, QK_ROUTE_GEMM_FOLD = 0, 1, 2, 3
 QK_PLAN_NONE, QK_PLAN_GEMV_QUANT, QK_PLAN_QUANT_GEMV, QK_PLAN_QUANT_GEMM = 0, 1, 2, 3
 
 
@@ -287,6 +288,19 @@ def qk_debug_w4a8_group_acc(xq, Wp, m0, m1, route, acc=None, stream=None):
     _check(lib.qk_debug_w4a8_group_acc(_ptr(xq), M, K, _ptr(Wp), N, m0, m1, _ptr(acc), int(route),
                                        _stream(stream)), "qk_debug_w4a8_group_acc")
     return acc
+
+
+def qk_debug_w4a8_plane_count(wscale, woffset, K: int, stream=None) -> int:
+    """Byte planes the W4A8 GEMM route needs for these scales and offsets
+    (1..4), or 255 when it takes the per-group fold kernel."""
+    _need(wscale, torch.float16, 2, "wscale")
+    _need(woffset, torch.float16, 2, "woffset")
+    N = wscale.shape[0]
+    planes = ctypes.c_int(0)
+    _check(lib.qk_debug_w4a8_plane_count(_ptr(wscale), _ptr(woffset), N, int(K),
+                                         ctypes.byref(planes), _stream(stream)),
+           "qk_debug_w4a8_plane_count")
+    return int(planes.value)
 
 
 def qk_debug_wait_timeout(limit_cycles: int, stream=None) -> None:

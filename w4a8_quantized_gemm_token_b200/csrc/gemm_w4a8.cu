@@ -1,4 +1,4 @@
-// gemm_w4a8.cu -- the W4A8 tensor-core GEMM (M > 16 rows).
+// gemm_w4a8.cu -- the W4A8 tensor-core GEMM with the per-group fold.
 //
 // Computes ("qlip-mlx" README, "w4a8_linear / W4A8Linear": packed 4-bit
 // weights, the same int8 compute; "MLX PR #4722": affine 4-bit weights with
@@ -7,20 +7,26 @@
 //   y[m, n] = bf16( sx[m] * sum_g (s[n,g] * acc + o[n,g] * xsum[m,g]) + bias[n] )
 // with the fold in fp64 and one rounding to bf16.
 //
+// The byte-plane GEMM (gemm_w4a8_planes.cu) computes the same value several
+// times faster whenever the scales and offsets of every weight row fit a common
+// integer grid within three bytes; this kernel runs beside it for the products
+// that do not (it then does the work, gated by the same plane-count word), when
+// the per-group fold is asked for explicitly, and for the per-group int32 dump.
+//
 // The per-group rescaling makes this kernel bound by the fp64 fold (M N G
 // multiply-add pairs on the CUDA cores), not by the tensor cores, so the tile is
-// chosen for the fold: 128 x 64 outputs per CTA (one CTA per SM, persistent).
+// chosen for the fold: 128 x 128 outputs per CTA (one CTA per SM, persistent).
 //  * warp 0: TMA producer -- per K block of 128 (two groups) the 128 x 128 int8
-//    tile of xq (128-byte swizzle) and the 64 x 64-byte packed-nibble tile of
+//    tile of xq (128-byte swizzle) and the 128 x 64-byte packed-nibble tile of
 //    Wp, into a 4-stage ring;
-//  * warps 2-3: unpack -- expand the nibbles into a 64 x 128 u8 code tile in the
-//    swizzled K-major layout the MMA reads (then fence.proxy.async), and convert
-//    the block's fp16 scales and offsets to fp64 into a table ring;
+//  * warps 2-3: unpack -- expand the nibbles into a 128 x 128 u8 code tile in
+//    the swizzled K-major layout the MMA reads (then fence.proxy.async), and
+//    convert the block's fp16 scales, offsets and xsum to fp64 into a table ring;
 //  * warp 1: per group, two tcgen05.mma kind::i8 (A signed, B unsigned, M = 128,
-//    N = 64, K = 32) into one of four 64-column TMEM buffers;
-//  * warps 4-19: fold -- tcgen05.ld a group's int32 sums, f += s * acc + o * xsum
-//    in fp64 (exact int -> fp64 by the 2^52 magic number), one row and 16
-//    columns per thread (16 warps hide the fp64 and TMEM latencies);
+//    N = 128, K = 32) into one of four 128-column TMEM buffers;
+//  * warps 4-11: fold -- tcgen05.ld a group's int32 sums, f += s * acc + o * xsum
+//    in fp64 (exact int -> fp64 by the 2^52 magic number), one row and 64
+//    columns per thread (two warps per TMEM lane quarter);
 //    at the end of the tile y = sx * f + bias is rounded once to bf16 (integer
 //    operations on the double's bits) and written with a TMA store.
 // A debug mode stores the per-group int32 sums of rows [m0, m1) instead.
@@ -124,7 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmY, const float* __restrict__ sx,
                      const int32_t* __restrict__ xsum, const uint16_t* __restrict__ wscale,
                      const uint16_t* __restrict__ woffset, const float* __restrict__ bias, int M,
-                     int N, int K, int32_t* __restrict__ acc_out, int m0, int m1, int* err) {
+                     int N, int K, int32_t* __restrict__ acc_out, int m0, int m1, int* err,
+                     const unsigned long long* pword, unsigned long long epoch) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -186,8 +193,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   pdl_wait();  // xq, sx and xsum come from the activation-quant kernel
 
+  // Beside the byte-plane GEMM (gemm_w4a8_planes.cu) this kernel computes only
+  // the products that one cannot: a plane-count word of this launch's epoch
+  // holding 1..3 planes means the plane kernel takes the product.
+  bool skip = false;
+  if (pword != nullptr) {
+    const unsigned long long pw = *reinterpret_cast<const volatile unsigned long long*>(pword);
+    const unsigned long long p = pw & 0xFFull;
+    skip = (pw >> 8) == epoch && p >= 1 && p <= 3;
+  }
 
-  if (warp < 4) {
+  if (skip) {
+    // nothing to compute
+  } else if (warp < 4) {
     // warpgroup 0: warp 0 loads, warp 1 issues the MMAs, warps 2-3 unpack;
     // most of its registers go to the fold warpgroups
     regs_dec<kRegsCtl>();
@@ -455,10 +473,11 @@ bool g_attr_done[2][64];
 
 }  // namespace
 
-cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+cudaError_t launch_w4a8_fold(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                              int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
-                             int64_t m0, int64_t m1, bool pdl, cudaStream_t s) {
+                             int64_t m0, int64_t m1, bool pdl, cudaStream_t s,
+                             const unsigned long long* pword, unsigned long long epoch) {
   const bool acc_mode = acc_out != nullptr;
   CUtensorMap tA, tP, tY;
   if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
@@ -500,7 +519,7 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, tA, tP, tY, sx, xsum, ws, wo, bias, (int)M, (int)N,
-                            (int)K, acc_out, (int)m0, (int)m1, err);
+                            (int)K, acc_out, (int)m0, (int)m1, err, pword, epoch);
 }
 
 }  // namespace qk

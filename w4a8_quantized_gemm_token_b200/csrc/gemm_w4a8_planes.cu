@@ -1,0 +1,719 @@
+// gemm_w4a8_planes.cu -- the W4A8 tensor-core GEMM (M > 16 rows) as int8 GEMMs
+// on the bytes of the dequantized weight.
+//
+// Computes what the per-group fold of gemm_w4a8.cu computes ("qlip-mlx"
+// README, "w4a8_linear / W4A8Linear": packed 4-bit weights, the same INT8
+// compute; "MLX PR #4722": affine 4-bit weights of group size 64 staged as int8
+// for the matmul), with G = K / 64:
+//   y[m, n] = bf16( sx[m] * sum_g (s[n,g] * acc[m,n,g] + o[n,g] * xsum[m,g]) + bias[n] ).
+//
+// The exact reformulation.  A nonzero fp16 value is an odd integer times a
+// power of two.  For weight row n let e_n be the smallest such exponent over
+// the row's nonzero scales and offsets; then S_g = s[n,g] / 2^e_n and
+// O_g = o[n,g] / 2^e_n are integers, every dequantized weight s q + o of the
+// row is 2^e_n W with the integer W = S_g q + O_g, and
+//   sum_g (s acc + o xsum) = 2^e_n sum_k xq[m,k] W[n,k]            (exactly).
+// With c_P = 0x80..80 (P bytes) and U = W + c_P: when every U of the matrix lies
+// in [0, 2^(8P)) for some P <= 3 (Gaussian or trained weights need 2, or 3 when
+// a row holds a group of unusually small range), the integer sum is P int8
+// GEMMs on the bytes U_p of U (unsigned), less c_P times the row sum of xq:
+//   Y[m,n] = sum_p 256^p sum_k xq[m,k] U_p[n,k] - c_P sum_k xq[m,k].
+// Each byte GEMM is exact in int32 (|xq| <= 127, U_p <= 255, K <= 65536) and Y is
+// exact in fp64, so
+//   y = bf16( sx[m] 2^e_n Y + bias[n] )
+// is the exact value of the fold rounded once (with one fused multiply-add,
+// as the fold kernel rounds it).  The per-group fp64 fold is itself exact under
+// the same bound on the integers, so both kernels give the same bits.
+//
+// Kernels (one call of the GEMM route runs them in this order, each a
+// programmatic dependent of the one before):
+//  * w4a8_plane_count_kernel: one warp per weight row finds e_n (written to
+//    the call's scratch) and the bytes its integers need; the launch's P (the
+//    maximum, or 255 when some row needs more than 3 bytes or holds a
+//    non-finite value) goes into a 64-bit word as (epoch << 8) | P, with the
+//    launch's epoch (a value never reused): a word of another epoch is
+//    replaced, one of this epoch raised, so the word needs no clearing;
+//  * w4a8_plane_build_kernel: memory-bound; writes the P byte planes of every
+//    weight row to the scratch as rows n P + p of [P N, K] bytes (one thread per
+//    16 codes: 8 packed bytes in, P 16-byte stores out);
+//  * (the per-group fold kernel of gemm_w4a8.cu, gated by the same word: it
+//    computes only when P > 3);
+//  * w4a8_planes_kernel: the W8A8 GEMM's structure on those planes -- CTA pairs
+//    (clusters of 2) run tcgen05.mma.cta_group::2 kind::i8 with M = 256 rows of
+//    xq and N = P R plane rows (R = 256 / P weight rows; 64 for P = 3), both
+//    operands loaded by TMA into a 6-stage ring, one MMA covering every plane
+//    so that a row's P sums sit in adjacent accumulator columns; the epilogue
+//    tcgen05.ld's the P sums of 16 outputs at a time, forms Y in fp64 (exact),
+//    y = fma(sx, 2^e_n Y, bias) rounded once to bf16 by integer operations, and
+//    writes it by TMA stores that clip the edges.
+//    The plane GEMM does nothing unless the word holds 1..3 planes of this
+//    launch's epoch.
+// (Building the planes inside the GEMM was measured and not kept: a transform
+// split over the pair needs a cluster-scope handoff per stage, about a
+// microsecond of release and acquire, and one done by the issuing CTA alone
+// runs at a third of the tensor pipe's pace.)
+// Every mbarrier wait is bounded (sm100.cuh); no load uses cluster multicast.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "qk_internal.h"
+#include "sm100.cuh"
+
+namespace qk {
+namespace {
+
+constexpr int BM = 128;                 // rows of xq per CTA (the pair covers 256)
+constexpr int BK = 128;                 // K per stage: two groups of 64
+constexpr int STAGES = 6;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 32 * (2 + kEpiWarps);  // 192
+constexpr int A_BYTES = BM * BK;        // 16 KiB of xq per stage
+constexpr int B_BYTES = 128 * BK;       // 16 KiB: up to 128 plane rows per CTA
+constexpr int STG_BYTES = 32 * 128;     // 32 output rows x 64 bf16
+constexpr int SMEM_A = 0;
+constexpr int SMEM_B = SMEM_A + STAGES * A_BYTES;
+constexpr int SMEM_STG = SMEM_B + STAGES * B_BYTES;
+constexpr int SMEM_BAR = SMEM_STG + kEpiWarps * STG_BYTES;
+constexpr int kNumBars = 2 * STAGES + 4;  // full, empty per stage; tfull, tempty per accumulator
+constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
+constexpr int SMEM_USED = SMEM_SLOT + 16;
+constexpr int SMEM_ALLOC = SMEM_USED + 1024;
+constexpr int kTmemCols = 512;          // two accumulators of up to 256 columns
+constexpr int kMaxPlanes = 3;
+
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(SMEM_B % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled operand tiles");
+static_assert(SMEM_STG % 1024 == 0, "swizzled output stages");
+
+constexpr int kNoExp = 1 << 20;         // "no nonzero value" in a minimum of exponents
+
+__host__ __device__ constexpr int tile_rows_of(int P) { return P == 3 ? 64 : 256 / P; }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  return __byte_perm(a, b, sel);
+}
+
+// Exponent of the lowest set bit of a nonzero finite fp16 value (its value is
+// an odd integer times 2^this), or kNoExp for +-0.
+__device__ __forceinline__ int f16_low_exp(uint32_t h) {
+  const uint32_t E = (h >> 10) & 31u;
+  const uint32_t m = h & 1023u;
+  const uint32_t mant = E != 0u ? (m | 1024u) : m;
+  if (mant == 0u) return kNoExp;
+  return (E != 0u ? (int)E - 25 : -24) + (__ffs((int)mant) - 1);
+}
+
+// Left shift that puts the 11-bit significand of fp16 h on the grid 2^eb
+// (negative: a right shift of trailing zero bits).
+__device__ __forceinline__ int f16_grid_shift(uint32_t h, int eb) {
+  const uint32_t E = (h >> 10) & 31u;
+  return (E != 0u ? (int)E - 25 : -24) - eb;
+}
+
+// fp16 value / 2^eb as an integer (exact when eb <= f16_low_exp(h)); 64-bit so
+// that the plane count below sees every value, however far from the grid.
+__device__ __forceinline__ long long f16_on_grid64(uint32_t h, int eb) {
+  const uint32_t E = (h >> 10) & 31u;
+  const uint32_t m = h & 1023u;
+  const long long mant = E != 0u ? (long long)(m | 1024u) : (long long)m;
+  if (mant == 0) return 0;
+  const int sh = (E != 0u ? (int)E - 25 : -24) - eb;
+  const long long v = sh >= 0 ? (mant << sh) : (mant >> -sh);
+  return (h & 0x8000u) ? -v : v;
+}
+
+// Same, as 32 bits (the plane count guarantees the value fits when P <= 4).
+__device__ __forceinline__ uint32_t f16_on_grid32(uint32_t h, int eb) {
+  const uint32_t E = (h >> 10) & 31u;
+  const uint32_t m = h & 1023u;
+  const uint32_t mant = E != 0u ? (m | 1024u) : m;
+  if (mant == 0u) return 0u;
+  const int sh = (E != 0u ? (int)E - 25 : -24) - eb;
+  const uint32_t v = sh >= 0 ? (mant << sh) : (mant >> -sh);
+  return (h & 0x8000u) ? (0u - v) : v;
+}
+
+__host__ __device__ constexpr uint32_t plane_bias(int P) {
+  return P == 1 ? 0x80u : P == 2 ? 0x8080u : P == 3 ? 0x808080u : 0x80808080u;
+}
+
+// ------------------------------------------------------------ plane count
+
+constexpr int kCountRowsPerBlock = 8;
+
+__global__ void __launch_bounds__(32 * kCountRowsPerBlock)
+    w4a8_plane_count_kernel(const uint16_t* __restrict__ wscale,
+                            const uint16_t* __restrict__ woffset, int N, int K, int* ebase,
+                            unsigned long long* pword, unsigned long long epoch) {
+  __shared__ int s_p[kCountRowsPerBlock];
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * kCountRowsPerBlock + warp;
+  const int G = K >> 6;
+  int prow = 0;
+  if (n < N) {
+    const uint16_t* s = wscale + (size_t)n * G;
+    const uint16_t* o = woffset + (size_t)n * G;
+    int eb = kNoExp;
+    bool bad = false;
+    for (int g = lane; g < G; g += 32) {
+      const uint32_t hs = s[g], ho = o[g];
+      bad |= ((hs >> 10) & 31u) == 31u || ((ho >> 10) & 31u) == 31u;
+      eb = min(eb, min(f16_low_exp(hs), f16_low_exp(ho)));
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) eb = min(eb, __shfl_xor_sync(0xFFFFFFFFu, eb, d));
+    bad = __any_sync(0xFFFFFFFFu, bad);
+    if (eb == kNoExp) eb = 0;
+    if (lane == 0) ebase[n] = eb;
+    long long lo = 0, hi = 0;
+    for (int g = lane; g < G && !bad; g += 32) {
+      const uint32_t hs = s[g], ho = o[g];
+      // 11 significant bits shifted by more than 40 would leave the int64 range
+      // of 15 S + O; such a row is far outside the four planes anyway
+      if (f16_grid_shift(hs, eb) > 40 || f16_grid_shift(ho, eb) > 40) {
+        bad = true;
+        break;
+      }
+      const long long S = f16_on_grid64(hs, eb), O = f16_on_grid64(ho, eb);
+      const long long a = O, b = O + 15 * S;
+      lo = min(lo, min(a, b));
+      hi = max(hi, max(a, b));
+    }
+    bad = __any_sync(0xFFFFFFFFu, bad);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+      lo = min(lo, (long long)__shfl_xor_sync(0xFFFFFFFFu, lo, d));
+      hi = max(hi, (long long)__shfl_xor_sync(0xFFFFFFFFu, hi, d));
+    }
+    prow = 255;
+    if (!bad) {
+      for (int p = kMaxPlanes; p >= 1; --p) {
+        const long long c = (long long)plane_bias(p);
+        if (lo + c >= 0 && hi + c < (1ll << (8 * p))) prow = p;
+      }
+    }
+  }
+  if (lane == 0) s_p[warp] = prow;
+  __syncthreads();
+  // an earlier kernel of the stream may still read the word until the
+  // dependency wait returns
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    int pmax = 0;
+    for (int w = 0; w < kCountRowsPerBlock; ++w) pmax = max(pmax, s_p[w]);
+    // The word holds (epoch << 8) | P.  A word of another epoch (an earlier
+    // launch, or whatever the scratch held) is replaced, one of this epoch is
+    // raised to pmax if below it: a compare-and-swap loop that most blocks
+    // leave after one read, since the first block already wrote their P.
+    const unsigned long long want = (epoch << 8) | (unsigned long long)pmax;
+    unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(pword);
+    while (pmax > 0 && ((old >> 8) != epoch || (old & 0xFFull) < (unsigned long long)pmax)) {
+      const unsigned long long prev = atomicCAS(pword, old, want);
+      if (prev == old) break;
+      old = prev;
+    }
+  }
+}
+
+// ------------------------------------------------------------ plane build
+
+constexpr int kBuildThreads = 256;
+
+// 8 packed bytes (16 codes) of one weight row -> the 16 bytes of each of the P
+// planes at the same K offset.  S and Op = O + c_P are the row's integers for
+// the codes' group.
+template <int P>
+__device__ __forceinline__ void planes_of16(const uint2 w2, uint32_t S, uint32_t Op,
+                                            uint4 (&out)[P]) {
+  const uint32_t w[2] = {w2.x, w2.y};
+  uint32_t pl[P][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t even = w[i] & 0x0F0F0F0Fu, odd = (w[i] >> 4) & 0x0F0F0F0Fu;
+    if constexpr (P == 1) {
+      // four codes per word: bytes S q + O + 128, no carries between them
+      const uint32_t O4 = Op * 0x01010101u;
+      pl[0][2 * i] = S * prmt(even, odd, 0x5140) + O4;      // codes 8i .. 8i + 3
+      pl[0][2 * i + 1] = S * prmt(even, odd, 0x7362) + O4;  // codes 8i + 4 .. 8i + 7
+    } else if constexpr (P == 2) {
+      // two codes per word (16-bit halves): U0 + 2^16 U2 = S (q0 + 2^16 q2) + O (1 + 2^16)
+      const uint32_t O2 = Op * 0x00010001u;
+      const uint32_t ya = S * prmt(even, 0u, 0x4140) + O2;  // codes 0, 2 of the word
+      const uint32_t yb = S * prmt(odd, 0u, 0x4140) + O2;   // codes 1, 3
+      const uint32_t yc = S * prmt(even, 0u, 0x4342) + O2;  // codes 4, 6
+      const uint32_t yd = S * prmt(odd, 0u, 0x4342) + O2;   // codes 5, 7
+      pl[0][2 * i] = prmt(ya, yb, 0x6240);
+      pl[1][2 * i] = prmt(ya, yb, 0x7351);
+      pl[0][2 * i + 1] = prmt(yc, yd, 0x6240);
+      pl[1][2 * i + 1] = prmt(yc, yd, 0x7351);
+    } else {
+      // one code per word, then a 4 x 4 byte transpose into the planes
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t q4 = h == 0 ? prmt(even, odd, 0x5140) : prmt(even, odd, 0x7362);
+        const uint32_t u0 = S * prmt(q4, 0u, 0x4440) + Op;
+        const uint32_t u1 = S * prmt(q4, 0u, 0x4441) + Op;
+        const uint32_t u2 = S * prmt(q4, 0u, 0x4442) + Op;
+        const uint32_t u3 = S * prmt(q4, 0u, 0x4443) + Op;
+        const uint32_t a_lo = prmt(u0, u1, 0x5140), a_hi = prmt(u0, u1, 0x7362);
+        const uint32_t b_lo = prmt(u2, u3, 0x5140), b_hi = prmt(u2, u3, 0x7362);
+        pl[0][2 * i + h] = prmt(a_lo, b_lo, 0x5410);
+        pl[1][2 * i + h] = prmt(a_lo, b_lo, 0x7632);
+        pl[2][2 * i + h] = prmt(a_hi, b_hi, 0x5410);
+      }
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < P; ++p) out[p] = make_uint4(pl[p][0], pl[p][1], pl[p][2], pl[p][3]);
+}
+
+template <int P>
+__device__ __forceinline__ void build_rows(const uint8_t* __restrict__ Wp,
+                                           const uint16_t* __restrict__ wscale,
+                                           const uint16_t* __restrict__ woffset,
+                                           const int* __restrict__ ebase, int N, int K,
+                                           uint8_t* __restrict__ planes) {
+  const int G = K >> 6;
+  const int units_per_row = K >> 4;  // 16 codes each
+  const long long total = (long long)N * units_per_row;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(u / units_per_row);
+    const int c = (int)(u - (long long)n * units_per_row);  // codes 16c .. 16c + 15
+    const int g = c >> 2;
+    const int eb = __ldg(ebase + n);
+    const uint32_t S = f16_on_grid32(__ldg(wscale + (size_t)n * G + g), eb);
+    const uint32_t Op = f16_on_grid32(__ldg(woffset + (size_t)n * G + g), eb) + plane_bias(P);
+    const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(Wp + (size_t)n * (K / 2)) + c);
+    uint4 out[P];
+    planes_of16<P>(w2, S, Op, out);
+#pragma unroll
+    for (int p = 0; p < P; ++p)
+      __stcg(reinterpret_cast<uint4*>(planes + ((size_t)n * P + p) * K) + c, out[p]);
+  }
+}
+
+__global__ void __launch_bounds__(kBuildThreads)
+    w4a8_plane_build_kernel(const uint8_t* __restrict__ Wp, const uint16_t* __restrict__ wscale,
+                            const uint16_t* __restrict__ woffset, const int* ebase, int N,
+                            int K, uint8_t* planes, const unsigned long long* pword,
+                            unsigned long long epoch) {
+  pdl_launch_dependents();
+  pdl_wait();  // e_n and the plane count come from the kernel before
+  const unsigned long long pw = *reinterpret_cast<const volatile unsigned long long*>(pword);
+  const int P = (pw >> 8) == epoch ? (int)(pw & 0xFFull) : 0;
+  switch (P) {
+    case 1: build_rows<1>(Wp, wscale, woffset, ebase, N, K, planes); break;
+    case 2: build_rows<2>(Wp, wscale, woffset, ebase, N, K, planes); break;
+    case 3: build_rows<3>(Wp, wscale, woffset, ebase, N, K, planes); break;
+    default: break;  // the fold kernel computes the product
+  }
+}
+
+// -------------------------------------------------------- the plane GEMM
+
+// Raster: groups of group_m M tiles walked down M first (as the W8A8 GEMM).
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int group_m, int& mb,
+                                            int& nb) {
+  const int per_group = group_m * tiles_n;
+  const int gid = t / per_group;
+  const int first_m = gid * group_m;
+  const int gm = min(tiles_m - first_m, group_m);
+  const int r = t - gid * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ double i32_to_f64(uint32_t a) {
+  return __hiloint2double(0x43300000, (int)(a ^ 0x80000000u)) - 4503601774854144.0;
+}
+
+// fp64 -> bf16 bits, one rounding to nearest-even (as in gemm_w8a8.cu).
+__device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
+  const uint32_t hi = (uint32_t)__double2hiint(v);
+  const uint32_t lo = (uint32_t)__double2loint(v);
+  const uint32_t sign = (hi >> 16) & 0x8000u;
+  const uint32_t mag = hi & 0x7FFFFFFFu;
+  if (mag < 0x38100000u) {
+    if ((mag | lo) == 0u) return sign;
+    float f = __double2float_rz(v);
+    if ((double)f != v) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+  }
+  const uint32_t keep = mag >> 13;
+  const uint32_t low13 = (mag & 0x1FFFu) | min(lo, 1u);
+  const uint32_t up = (low13 + 0x0FFFu + (keep & 1u)) >> 13;
+  return sign | min(keep + up - (896u << 7), 0x7F80u);
+}
+
+// The epilogue of one tile for a fixed P: 16 outputs per TMEM load group,
+// 64 outputs per staged 128-byte row and TMA store.
+template <int P>
+__device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __restrict__ ebase,
+                                              const float* __restrict__ bias, double sxd,
+                                              double xb, uint8_t* stg_ptr, uint32_t stg,
+                                              const CUtensorMap* tmY, int ncol0, int row0, int M,
+                                              int N, int lane, uint32_t lead_tempty, bool& used) {
+  constexpr int TR = tile_rows_of(P);
+  constexpr int kChunks = TR / 64;
+#pragma unroll 1
+  for (int ch = 0; ch < kChunks; ++ch) {
+    uint32_t out[32];
+#pragma unroll
+    for (int sub = 0; sub < 4; ++sub) {
+      const int r0 = ch * 64 + sub * 16;  // first weight row of this load group
+      // the group's 2^e_n and bias (the same for every lane: broadcast loads)
+      double p2[16], bv[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int n = ncol0 + r0 + j;
+        p2[j] = n < N ? __hiloint2double((1023 + __ldg(ebase + n)) << 20, 0) : 0.0;
+        bv[j] = (bias != nullptr && n < N) ? (double)__ldg(bias + n) : 0.0;
+      }
+      uint32_t v[16 * P];
+      const uint32_t a = t_lane + (uint32_t)(r0 * P);
+      if constexpr (P == 1) {
+        uint32_t (&vv)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
+        tmem_ld16(a, vv);
+      } else if constexpr (P == 2) {
+        uint32_t (&vv)[32] = *reinterpret_cast<uint32_t(*)[32]>(v);
+        tmem_ld32(a, vv);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          uint32_t (&vv)[16] = *reinterpret_cast<uint32_t(*)[16]>(v + 16 * j);
+          tmem_ld16(a + 16u * j, vv);
+        }
+      }
+      tmem_ld_wait();
+      if (ch == kChunks - 1 && sub == 3) {
+        // every TMEM read of this accumulator is done: hand it back to the leader
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_tempty);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        uint32_t hb[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int j = i + h;
+          double Y = i32_to_f64(v[j * P + P - 1]);
+#pragma unroll
+          for (int p = P - 2; p >= 0; --p) Y = fma(Y, 256.0, i32_to_f64(v[j * P + p]));
+          hb[h] = f64_to_bf16_bits(fma(sxd, (Y + xb) * p2[j], bv[j]));
+        }
+        out[sub * 8 + (i >> 1)] = hb[0] | (hb[1] << 16);
+      }
+    }
+    const int n0 = ncol0 + ch * 64;
+    if (n0 >= N || row0 >= M) continue;  // whole box outside y
+    if (lane == 0 && used) bulk_wait_read<0>();
+    __syncwarp();
+    uint8_t* rowp = stg_ptr + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+          make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmY, stg, n0, row0);
+      bulk_commit();
+    }
+    used = true;
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    w4a8_planes_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmY, const float* __restrict__ sx,
+                       const int32_t* __restrict__ xsum, const int* __restrict__ ebase,
+                       const float* __restrict__ bias, int M, int N, int K, int group_m,
+                       const unsigned long long* pword, unsigned long long epoch, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_smem<1024>(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + SMEM_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SMEM_SLOT);
+
+  const uint32_t rank = cluster_ctarank();
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmY);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * kEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  pdl_launch_dependents();
+  pdl_wait();  // xq, sx, xsum, e_n, the planes and the plane-count word come from earlier kernels
+
+  const unsigned long long pw = *reinterpret_cast<const volatile unsigned long long*>(pword);
+  const int P = (pw >> 8) == epoch ? (int)(pw & 0xFFull) : 0;
+  if (P >= 1 && P <= kMaxPlanes) {
+    const int TR = tile_rows_of(P);
+    const int RC = TR / 2;                 // weight rows of each CTA's half
+    const int tiles_m = (M + 2 * BM - 1) / (2 * BM);
+    const int tiles_n = (N + TR - 1) / TR;
+    const int num_tiles = tiles_m * tiles_n;
+    const int num_kb = (K + BK - 1) / BK;
+    const int G = K >> 6;
+
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      // each CTA loads its 128 rows of xq and its P RC plane rows (32-row
+      // boxes), completing on the leader's barrier
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        const uint32_t tx = 2u * (uint32_t)(A_BYTES + P * RC * BK);
+        for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+          int mb, nb;
+          tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
+          const int arow = mb * 2 * BM + (int)rank * BM;
+          const int brow = (nb * TR + (int)rank * RC) * P;
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, err)) {
+              ok = false;
+              break;
+            }
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), tx);
+            const uint32_t lead_full = mapa_shared(full_bar(stage), 0);
+            tma_load_2d_pair(sbase + SMEM_A + stage * A_BYTES, &tmA, kb * BK, arow, lead_full);
+            for (int i = 0; i < P * RC / 32; ++i)
+              tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES + i * 32 * BK, &tmB, kb * BK,
+                               brow + 32 * i, lead_full);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------- MMA issuer (pair leader)
+      if (rank == 0 && lane == 0) {
+        const uint32_t idesc = i8_idesc(2 * BM, P * TR, true, false);
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t aphase = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+          if (!mbar_wait(tempty_bar(acc), aphase ^ 1u, err)) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(full_bar(stage), phase, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = sbase + SMEM_A + stage * A_BYTES;
+            const uint32_t b_addr = sbase + SMEM_B + stage * B_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)
+              mma_i8_pair(d_tmem, sw128_kmajor_desc(a_addr + 32 * kk),
+                          sw128_kmajor_desc(b_addr + 32 * kk), idesc, (kb | kk) != 0 ? 1u : 0u);
+            mma_commit_pair(empty_bar(stage), 0x3);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          mma_commit_pair(tfull_bar(acc), 0x3);
+          if (++acc == 2) {
+            acc = 0;
+            aphase ^= 1u;
+          }
+        }
+      }
+    } else {
+      // ---------------------------------------------------------- epilogue
+      const int e = warp - 2;
+      const int q = warp & 3;
+      uint8_t* stg_ptr = smem + SMEM_STG + e * STG_BYTES;
+      const uint32_t stg = sbase + SMEM_STG + (uint32_t)(e * STG_BYTES);
+      const double xbias = -(double)plane_bias(P);
+      int acc = 0;
+      uint32_t aphase = 0;
+      bool used = false;
+      for (int t = pair; t < num_tiles; t += num_pairs) {
+        int mb, nb;
+        tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
+        const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;
+        const int row = row0 + lane;
+        double sxd = 0.0, xb = 0.0;
+        if (row < M) {
+          // sx and c_P times the row sum of xq (the sum of its group sums)
+          sxd = (double)__ldg(sx + row);
+          const int32_t* xs = xsum + (size_t)row * G;
+          int tot = 0;
+          if ((G & 3) == 0) {
+            const int4* x4 = reinterpret_cast<const int4*>(xs);
+            for (int g = 0; g < G / 4; ++g) {
+              const int4 v = __ldg(x4 + g);
+              tot += (v.x + v.y) + (v.z + v.w);
+            }
+          } else {
+            for (int g = 0; g < G; ++g) tot += __ldg(xs + g);
+          }
+          xb = xbias * (double)tot;
+        }
+        if (!mbar_wait(tfull_bar(acc), aphase, err)) break;
+        tc_fence_after();
+        const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+        const uint32_t lead_tempty = mapa_shared(tempty_bar(acc), 0);
+        switch (P) {
+          case 1: epilogue_tile<1>(t_lane, ebase, bias, sxd, xb, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          case 2: epilogue_tile<2>(t_lane, ebase, bias, sxd, xb, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          default: epilogue_tile<3>(t_lane, ebase, bias, sxd, xb, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+        }
+        if (++acc == 2) {
+          acc = 0;
+          aphase ^= 1u;
+        }
+      }
+      if (lane == 0) bulk_wait<0>();
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();  // every remote arrival and MMA of the pair is done
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
+bool g_attr_done[64];
+
+}  // namespace
+
+size_t w4a8_plane_scratch_bytes(int64_t N, int64_t K) {
+  auto r = [](size_t b) { return (b + 255u) & ~size_t(255u); };
+  return r(8) + r((size_t)N * 4u) + (size_t)kMaxPlanes * (size_t)N * (size_t)K;
+}
+
+cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                             const float* bias, int64_t N, uint16_t* y, void* scratch, bool pdl,
+                             cudaStream_t s) {
+  auto r = [](size_t b) { return (b + 255u) & ~size_t(255u); };
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  auto* pword = reinterpret_cast<unsigned long long*>(base);
+  auto* ebase = reinterpret_cast<int*>(base + r(8));
+  uint8_t* planes = base + r(8) + r((size_t)N * 4u);
+  const unsigned long long epoch = next_epoch();
+  auto launch = [&](auto kernel, dim3 grid, dim3 block, size_t smem, bool dep, auto... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dep ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+  };
+  // 1. plane count and e_n
+  cudaError_t e = launch(w4a8_plane_count_kernel,
+                         dim3((unsigned)((N + kCountRowsPerBlock - 1) / kCountRowsPerBlock)),
+                         dim3(32 * kCountRowsPerBlock), 0, pdl, ws, wo, (int)N, (int)K, ebase,
+                         pword, epoch);
+  if (e != cudaSuccess) return e;
+  // 2. the planes (a few waves of the SMs; each thread loops over 16-code units)
+  const long long units = N * (K / 16);
+  long long blocks = (units + kBuildThreads - 1) / kBuildThreads;
+  const long long cap = 8ll * num_sms();
+  e = launch(w4a8_plane_build_kernel, dim3((unsigned)(blocks < cap ? blocks : cap)),
+             dim3(kBuildThreads), 0, true, Wp, ws, wo, (const int*)ebase, (int)N, (int)K, planes,
+             (const unsigned long long*)pword, epoch);
+  if (e != cudaSuccess) return e;
+  // 3. the per-group fold, which computes only when the planes cannot
+  e = launch_w4a8_fold(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, true, s, pword,
+                       epoch);
+  if (e != cudaSuccess) return e;
+  // 4. the plane GEMM
+  CUtensorMap tA, tB, tY;
+  if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
+                      (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes, (uint64_t)K,
+                      (uint64_t)(kMaxPlanes * N), (uint64_t)K, BK, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
+                      (uint64_t)N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !g_attr_done[dev]) {
+    e = cudaFuncSetAttribute(w4a8_planes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    g_attr_done[dev] = true;
+  }
+  int* err = device_error_word();
+  if (err == nullptr) return cudaErrorUnknown;
+  // the tile count depends on the plane count, which only the device knows:
+  // size the grid for the smallest tiles (64 weight rows, P = 3); pairs
+  // without a tile at the actual P exit at once
+  const long long tiles_m = (M + 2 * BM - 1) / (2 * BM);
+  const long long max_tiles = tiles_m * ((N + 63) / 64);
+  const long long pairs = num_sms() / 2;
+  const int grid = 2 * (int)(max_tiles < pairs ? max_tiles : pairs);
+  // a raster group's rows of xq (256 rows x K bytes per M tile) stay in L2
+  long long group_m = (40ll << 20) / (2 * BM * K);
+  group_m = group_m < 1 ? 1 : (group_m > tiles_m ? tiles_m : group_m);
+  return launch(w4a8_planes_kernel, dim3(grid), dim3(kThreads), (size_t)SMEM_ALLOC, true, tA, tB,
+                tY, sx, xsum, (const int*)ebase, bias, (int)M, (int)N, (int)K, (int)group_m,
+                (const unsigned long long*)pword, epoch, err);
+}
+
+cudaError_t launch_w4a8_plane_count(const uint16_t* ws, const uint16_t* wo, int64_t N, int64_t K,
+                                    int* ebase, unsigned long long* pword,
+                                    unsigned long long epoch, bool pdl, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((N + kCountRowsPerBlock - 1) / kCountRowsPerBlock));
+  cfg.blockDim = dim3(32 * kCountRowsPerBlock);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, w4a8_plane_count_kernel, ws, wo, (int)N, (int)K, ebase, pword,
+                            epoch);
+}
+
+}  // namespace qk

@@ -709,20 +709,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 bool g_attr_done[4][64];  // plain, accumulator dump, gated, fused quantization
 
-// Epochs of the fused-quantization launches: distinct for every launch of the
-// process (56 bits, never zero), so a readiness word left by an earlier launch
-// in the same workspace never equals this launch's target.
 std::atomic<unsigned long long> g_epoch{0};
-
-unsigned long long next_epoch() {
-  static const unsigned long long seed = [] {
-    const unsigned long long t =
-        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
-    return (t * 0x9E3779B97F4A7C15ull) >> 9;
-  }();
-  unsigned long long e = (seed + g_epoch.fetch_add(1, std::memory_order_relaxed)) & ((1ull << 56) - 1);
-  return e == 0 ? 1 : e;
-}
 
 // Pairs of CTAs that can be resident at once (the fused kernel's producers wait
 // for rows that other CTAs quantize, so its whole grid must be resident).
@@ -753,6 +740,16 @@ int resident_pairs(const void* kernel) {
 }
 
 }  // namespace
+
+unsigned long long next_epoch() {
+  static const unsigned long long seed = [] {
+    const unsigned long long t =
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    return (t * 0x9E3779B97F4A7C15ull) >> 9;
+  }();
+  unsigned long long e = (seed + g_epoch.fetch_add(1, std::memory_order_relaxed)) & ((1ull << 56) - 1);
+  return e == 0 ? 1 : e;
+}
 
 cudaError_t launch_w8a8_gemm(const int8_t* xq, const float* sx, int64_t M, int64_t K,
                              const int8_t* Wq, const float* sw, const float* bias, int64_t N,

@@ -122,6 +122,41 @@ int* device_error_word() {
   return g_err_ptr[d];
 }
 
+// The library's stream-ordered memory pool on the current device (created on
+// first use): it keeps freed blocks reserved instead of returning them to the
+// driver at each synchronization, so the large per-call scratch of the W4A8
+// GEMM route (the weight's byte planes) is recycled, not mapped again on every
+// call.  Null if the pool cannot be made (callers then use the default pool).
+cudaMemPool_t scratch_pool() {
+  static cudaMemPool_t pools[kMaxDevices];
+  static bool tried[kMaxDevices];
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!tried[d]) {
+    tried[d] = true;
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = d;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) == cudaSuccess) {
+      unsigned long long keep = ~0ull;
+      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+      pools[d] = pool;
+    } else {
+      cudaGetLastError();
+    }
+  }
+  return pools[d];
+}
+
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t s) {
+  cudaMemPool_t pool = scratch_pool();
+  return pool != nullptr ? cudaMallocFromPoolAsync(p, bytes, pool, s) : cudaMallocAsync(p, bytes, s);
+}
+
 int num_sms() {
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return 1;
@@ -340,17 +375,33 @@ static qk_status check_w4_product(const uint8_t* Wp, const uint16_t* wscale,
   return QK_OK;
 }
 
+static bool w4a8_takes_gemv(int route, int64_t M, int64_t K, int64_t N) {
+  return route == QK_ROUTE_GEMV || (route == QK_ROUTE_AUTO && gemv_fits(M, K, N));
+}
+
+// The GEMM route allocates its plane scratch (w4a8_plane_scratch_bytes)
+// stream-ordered for the call, from the library's pool (scratch_pool).
 static cudaError_t run_w4a8(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                             const float* bias, int64_t N, uint16_t* y, int route, bool pdl,
                             cudaStream_t s) {
-  const bool gemv = route == QK_ROUTE_GEMV || (route == QK_ROUTE_AUTO && gemv_fits(M, K, N));
+  const bool gemv = w4a8_takes_gemv(route, M, K, N);
   if (log_enabled())
     std::fprintf(stderr, "[qk] w4a8 M=%lld K=%lld N=%lld -> %s\n", (long long)M, (long long)K,
-                 (long long)N, gemv ? "GEMV" : "tcgen05 GEMM");
+                 (long long)N,
+                 gemv ? "GEMV"
+                      : route == QK_ROUTE_GEMM_FOLD ? "tcgen05 GEMM, per-group fold"
+                                                    : "tcgen05 GEMM, byte planes (fold if needed)");
   if (gemv)
     return launch_w4a8_gemv(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, pdl, s);
-  return launch_w4a8_gemm(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, pdl, s);
+  if (route == QK_ROUTE_GEMM_FOLD)
+    return launch_w4a8_fold(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, pdl, s);
+  void* scratch = nullptr;
+  cudaError_t e = scratch_alloc(&scratch, w4a8_plane_scratch_bytes(N, K), s);
+  if (e != cudaSuccess) return e;
+  e = launch_w4a8_gemm(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, scratch, pdl, s);
+  const cudaError_t f = cudaFreeAsync(scratch, s);
+  return e != cudaSuccess ? e : f;
 }
 
 int qk_w4a8_linear_plan(int64_t M, int64_t K, int64_t N) {
@@ -368,7 +419,8 @@ qk_status qk_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, i
                        int route, qk_stream_t stream) {
   qk_status st = check_shape(M, K, N, true);
   if (st != QK_OK) return st;
-  if (route != QK_ROUTE_AUTO && route != QK_ROUTE_GEMM && route != QK_ROUTE_GEMV)
+  if (route != QK_ROUTE_AUTO && route != QK_ROUTE_GEMM && route != QK_ROUTE_GEMV &&
+      route != QK_ROUTE_GEMM_FOLD)
     return QK_ERR_INVALID_ARG;
   if (route == QK_ROUTE_GEMV && M > 16) return QK_ERR_INVALID_ARG;
   if (route == QK_ROUTE_GEMV && M > 0 && !gemv_fits(M, K, N)) return QK_ERR_UNSUPPORTED_SHAPE;
@@ -527,6 +579,32 @@ qk_status qk_debug_w8a8_acc(const int8_t* xq, int64_t M, int64_t K, const int8_t
       "w8a8_acc");
 }
 
+qk_status qk_debug_w4a8_plane_count(const uint16_t* wscale, const uint16_t* woffset, int64_t N,
+                                    int64_t K, int* planes, qk_stream_t stream) {
+  qk_status st = check_shape(1, K, N, true);
+  if (st != QK_OK) return st;
+  if (!wscale || !woffset || !planes) return QK_ERR_INVALID_ARG;
+  if (!aligned16(wscale) || !aligned16(woffset)) return QK_ERR_MISALIGNED;
+  if ((st = check_device()) != QK_OK) return st;
+  void* scratch = nullptr;
+  const size_t bytes = 256 + round256((size_t)N * 4u);
+  if ((st = from_cuda(cudaMallocAsync(&scratch, bytes, stream), "cudaMallocAsync(plane count)")) !=
+      QK_OK)
+    return st;
+  const unsigned long long epoch = next_epoch();
+  unsigned long long word = 0;
+  cudaError_t e = launch_w4a8_plane_count(
+      wscale, woffset, N, K, reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) + 256),
+      static_cast<unsigned long long*>(scratch), epoch, false, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, stream);
+  cudaFreeAsync(scratch, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if ((st = from_cuda(e, "w4a8_plane_count")) != QK_OK) return st;
+  *planes = (word >> 8) == epoch ? (int)(word & 0xFFull) : 0;
+  return QK_OK;
+}
+
 qk_status qk_debug_w4a8_group_acc(const int8_t* xq, int64_t M, int64_t K, const uint8_t* Wp,
                                   int64_t N, int64_t m0, int64_t m1, int32_t* acc, int route,
                                   qk_stream_t stream) {
@@ -544,7 +622,7 @@ qk_status qk_debug_w4a8_group_acc(const int8_t* xq, int64_t M, int64_t K, const 
       route == QK_ROUTE_GEMV
           ? launch_w4a8_gemv(xq, nullptr, nullptr, M, K, Wp, nullptr, nullptr, nullptr, N,
                              nullptr, acc, m0, m1, false, stream)
-          : launch_w4a8_gemm(xq, nullptr, nullptr, M, K, Wp, nullptr, nullptr, nullptr, N,
+          : launch_w4a8_fold(xq, nullptr, nullptr, M, K, Wp, nullptr, nullptr, nullptr, N,
                              nullptr, acc, m0, m1, false, stream);
   return from_cuda(e, "w4a8_group_acc");
 }

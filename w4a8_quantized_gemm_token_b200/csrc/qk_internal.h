@@ -71,12 +71,43 @@ cudaError_t launch_w8a8_skinny(const int8_t* xq, const float* sx, int64_t M, int
                                uint16_t* y, int32_t* acc_out, bool pdl, cudaStream_t s,
                                const float* gate = nullptr, const uint16_t* residual = nullptr);
 
-// W4A8 tensor-core GEMM (any M).  When `acc_out` is not null it stores the
-// per-group int32 accumulators of rows [m0, m1) instead of y.
-cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+// A value never returned before in this process (56 bits, never zero): the
+// epoch of a launch whose device words (readiness, plane count) are tagged
+// with it, so that words left by earlier launches never match.
+unsigned long long next_epoch();
+
+// W4A8 tensor-core GEMM with the per-group fp64 fold (gemm_w4a8.cu).  When
+// `acc_out` is not null it stores the per-group int32 accumulators of rows
+// [m0, m1) instead of y.  With `pword`, the kernel computes only when that
+// plane-count word (written by launch_w4a8_plane_count with `epoch`) does not
+// hold 1..3 planes of this epoch: the fallback beside the byte-plane GEMM.
+cudaError_t launch_w4a8_fold(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                              int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                              const float* bias, int64_t N, uint16_t* y, int32_t* acc_out,
-                             int64_t m0, int64_t m1, bool pdl, cudaStream_t s);
+                             int64_t m0, int64_t m1, bool pdl, cudaStream_t s,
+                             const unsigned long long* pword = nullptr,
+                             unsigned long long epoch = 0);
+
+// The byte-plane W4A8 GEMM (gemm_w4a8_planes.cu).  The plane-count kernel
+// writes e_n of every weight row to ebase and (epoch << 8) | P to *pword
+// (raised within an epoch, replacing any other epoch's word; no clearing
+// needed).
+cudaError_t launch_w4a8_plane_count(const uint16_t* ws, const uint16_t* wo, int64_t N, int64_t K,
+                                    int* ebase, unsigned long long* pword,
+                                    unsigned long long epoch, bool pdl, cudaStream_t s);
+
+// Device scratch the W4A8 GEMM route needs: the plane-count word, e_n of every
+// weight row and the byte planes of the dequantized weight (up to 3 N K bytes).
+size_t w4a8_plane_scratch_bytes(int64_t N, int64_t K);
+
+// The W4A8 GEMM route (any M): the plane count, the plane build, the gated
+// per-group fold and the plane GEMM -- four launches, one of the two GEMMs
+// computing.  `scratch`: w4a8_plane_scratch_bytes(N, K) bytes of device memory
+// owned by the call (256-byte aligned).
+cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                             const float* bias, int64_t N, uint16_t* y, void* scratch, bool pdl,
+                             cudaStream_t s);
 
 // W4A8 weight-streaming GEMV (M <= 16; its per-CTA working set -- the weight
 // slice of R rows x one K slice, xq, scales -- must fit shared memory, see
