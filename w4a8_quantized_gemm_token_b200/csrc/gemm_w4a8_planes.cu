@@ -15,11 +15,12 @@
 //   sum_g (s acc + o xsum) = 2^e_n sum_k xq[m,k] W[n,k]            (exactly).
 // With c_P = 0x80..80 (P bytes) and U = W + c_P: when every U of the matrix lies
 // in [0, 2^(8P)) for some P <= 3 (Gaussian or trained weights need 2, or 3 when
-// a row holds a group of unusually small range), the integer sum is P int8
-// GEMMs on the bytes U_p of U (unsigned), less c_P times the row sum of xq:
-//   Y[m,n] = sum_p 256^p sum_k xq[m,k] U_p[n,k] - c_P sum_k xq[m,k].
-// Each byte GEMM is exact in int32 (|xq| <= 127, U_p <= 255, K <= 65536) and Y is
-// exact in fp64, so
+// a row holds a group of unusually small range), W has the signed base-256
+// digits d_p = U_p - 128 in [-128, 127] (U_p the bytes of U), W = sum_p 256^p d_p,
+// and the integer sum is P int8 GEMMs on those digits:
+//   Y[m,n] = sum_p 256^p sum_k xq[m,k] d_p[n,k].
+// Each digit GEMM is exact in int32 (|xq| <= 127, |d_p| <= 128, K <= 65536) and Y
+// is exact in fp64, so
 //   y = bf16( sx[m] 2^e_n Y + bias[n] )
 // is the exact value of the fold rounded once (with one fused multiply-add,
 // as the fold kernel rounds it).  The per-group fp64 fold is itself exact under
@@ -33,8 +34,8 @@
 //    non-finite value) goes into a 64-bit word as (epoch << 8) | P, with the
 //    launch's epoch (a value never reused): a word of another epoch is
 //    replaced, one of this epoch raised, so the word needs no clearing;
-//  * w4a8_plane_build_kernel: memory-bound; writes the P byte planes of every
-//    weight row to the scratch as rows n P + p of [P N, K] bytes (one thread per
+//  * w4a8_plane_build_kernel: memory-bound; writes the P digit planes of every
+//    weight row to the scratch as rows n P + p of [P N, K] int8 (one thread per
 //    16 codes: 8 packed bytes in, P 16-byte stores out);
 //  * (the per-group fold kernel of gemm_w4a8.cu, gated by the same word: it
 //    computes only when P > 3);
@@ -42,10 +43,11 @@
 //    (clusters of 2) run tcgen05.mma.cta_group::2 kind::i8 with M = 256 rows of
 //    xq and N = P R plane rows (R = 256 / P weight rows; 64 for P = 3), both
 //    operands loaded by TMA into a 6-stage ring, one MMA covering every plane
-//    so that a row's P sums sit in adjacent accumulator columns; the epilogue
-//    tcgen05.ld's the P sums of 16 outputs at a time, forms Y in fp64 (exact),
-//    y = fma(sx, 2^e_n Y, bias) rounded once to bf16 by integer operations, and
-//    writes it by TMA stores that clip the edges.
+//    so that a row's P sums sit in adjacent accumulator columns; two epilogue
+//    warpgroups, one per TMEM accumulator (so consecutive tiles drain in
+//    parallel), tcgen05.ld the P sums of 16 outputs at a time, form Y in fp64
+//    (exact), y = fma(sx 2^e_n, Y, bias) rounded once to bf16 by integer
+//    operations, and write it by TMA stores that clip the edges.
 //    The plane GEMM does nothing unless the word holds 1..3 planes of this
 //    launch's epoch.
 // (Building the planes inside the GEMM was measured and not kept: a transform
@@ -67,8 +69,8 @@ namespace {
 constexpr int BM = 128;                 // rows of xq per CTA (the pair covers 256)
 constexpr int BK = 128;                 // K per stage: two groups of 64
 constexpr int STAGES = 6;
-constexpr int kEpiWarps = 4;
-constexpr int kThreads = 32 * (2 + kEpiWarps);  // 192
+constexpr int kEpiWarps = 8;            // two warpgroups, one per TMEM accumulator
+constexpr int kThreads = 32 * (2 + kEpiWarps);  // 320
 constexpr int A_BYTES = BM * BK;        // 16 KiB of xq per stage
 constexpr int B_BYTES = 128 * BK;       // 16 KiB: up to 128 plane rows per CTA
 constexpr int STG_BYTES = 32 * 128;     // 32 output rows x 64 bf16
@@ -222,8 +224,8 @@ __global__ void __launch_bounds__(32 * kCountRowsPerBlock)
 
 constexpr int kBuildThreads = 256;
 
-// 8 packed bytes (16 codes) of one weight row -> the 16 bytes of each of the P
-// planes at the same K offset.  S and Op = O + c_P are the row's integers for
+// 8 packed bytes (16 codes) of one weight row -> the 16 signed digits of each
+// of the P planes at the same K offset.  S and Op = O + c_P are the row's integers for
 // the codes' group.
 template <int P>
 __device__ __forceinline__ void planes_of16(const uint2 w2, uint32_t S, uint32_t Op,
@@ -267,7 +269,10 @@ __device__ __forceinline__ void planes_of16(const uint2 w2, uint32_t S, uint32_t
     }
   }
 #pragma unroll
-  for (int p = 0; p < P; ++p) out[p] = make_uint4(pl[p][0], pl[p][1], pl[p][2], pl[p][3]);
+  // signed digits d_p = U_p - 128: flip the top bit of every byte
+  for (int p = 0; p < P; ++p)
+    out[p] = make_uint4(pl[p][0] ^ 0x80808080u, pl[p][1] ^ 0x80808080u, pl[p][2] ^ 0x80808080u,
+                        pl[p][3] ^ 0x80808080u);
 }
 
 template <int P>
@@ -354,7 +359,7 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
 template <int P>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __restrict__ ebase,
                                               const float* __restrict__ bias, double sxd,
-                                              double xb, uint8_t* stg_ptr, uint32_t stg,
+                                              uint8_t* stg_ptr, uint32_t stg,
                                               const CUtensorMap* tmY, int ncol0, int row0, int M,
                                               int N, int lane, uint32_t lead_tempty, bool& used) {
   constexpr int TR = tile_rows_of(P);
@@ -365,12 +370,13 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __rest
 #pragma unroll
     for (int sub = 0; sub < 4; ++sub) {
       const int r0 = ch * 64 + sub * 16;  // first weight row of this load group
-      // the group's 2^e_n and bias (the same for every lane: broadcast loads)
-      double p2[16], bv[16];
+      // sx 2^e_n (exact: a power-of-two scaling) and the bias of the group's
+      // columns (the same for every lane: broadcast loads)
+      double sc[16], bv[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int n = ncol0 + r0 + j;
-        p2[j] = n < N ? __hiloint2double((1023 + __ldg(ebase + n)) << 20, 0) : 0.0;
+        sc[j] = n < N ? sxd * __hiloint2double((1023 + __ldg(ebase + n)) << 20, 0) : 0.0;
         bv[j] = (bias != nullptr && n < N) ? (double)__ldg(bias + n) : 0.0;
       }
       uint32_t v[16 * P];
@@ -404,7 +410,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __rest
           double Y = i32_to_f64(v[j * P + P - 1]);
 #pragma unroll
           for (int p = P - 2; p >= 0; --p) Y = fma(Y, 256.0, i32_to_f64(v[j * P + p]));
-          hb[h] = f64_to_bf16_bits(fma(sxd, (Y + xb) * p2[j], bv[j]));
+          hb[h] = f64_to_bf16_bits(fma(sc[j], Y, bv[j]));
         }
         out[sub * 8 + (i >> 1)] = hb[0] | (hb[1] << 16);
       }
@@ -431,7 +437,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __rest
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w4a8_planes_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmY, const float* __restrict__ sx,
-                       const int32_t* __restrict__ xsum, const int* __restrict__ ebase,
+                       const int* __restrict__ ebase,
                        const float* __restrict__ bias, int M, int N, int K, int group_m,
                        const unsigned long long* pword, unsigned long long epoch, int* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -460,7 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 2 * kEpiWarps);
+      mbar_init(tempty_bar(a), 2 * (kEpiWarps / 2));  // one warpgroup in each CTA
     }
     fence_mbar_init();
   }
@@ -475,7 +481,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   pdl_launch_dependents();
-  pdl_wait();  // xq, sx, xsum, e_n, the planes and the plane-count word come from earlier kernels
+  pdl_wait();  // xq, sx, e_n, the planes and the plane-count word come from earlier kernels
 
   const unsigned long long pw = *reinterpret_cast<const volatile unsigned long long*>(pword);
   const int P = (pw >> 8) == epoch ? (int)(pw & 0xFFull) : 0;
@@ -486,7 +492,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int tiles_n = (N + TR - 1) / TR;
     const int num_tiles = tiles_m * tiles_n;
     const int num_kb = (K + BK - 1) / BK;
-    const int G = K >> 6;
 
     if (warp == 0) {
       // ---------------------------------------------------------- producer
@@ -523,7 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ------------------------------------------- MMA issuer (pair leader)
       if (rank == 0 && lane == 0) {
-        const uint32_t idesc = i8_idesc(2 * BM, P * TR, true, false);
+        const uint32_t idesc = i8_idesc(2 * BM, P * TR, true, true);
         int stage = 0;
         uint32_t phase = 0;
         int acc = 0;
@@ -561,49 +566,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     } else {
       // ---------------------------------------------------------- epilogue
-      const int e = warp - 2;
-      const int q = warp & 3;
+      // warpgroup eg drains accumulator eg: the pair's tiles 2i + eg
+      const int e = warp - 2;             // 0..7
+      const int eg = e >> 2;              // warpgroup = accumulator
+      const int q = warp & 3;             // TMEM lane quarter
       uint8_t* stg_ptr = smem + SMEM_STG + e * STG_BYTES;
       const uint32_t stg = sbase + SMEM_STG + (uint32_t)(e * STG_BYTES);
-      const double xbias = -(double)plane_bias(P);
-      int acc = 0;
       uint32_t aphase = 0;
       bool used = false;
-      for (int t = pair; t < num_tiles; t += num_pairs) {
+      for (int t = pair + eg * num_pairs; t < num_tiles; t += 2 * num_pairs) {
         int mb, nb;
         tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
         const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;
         const int row = row0 + lane;
-        double sxd = 0.0, xb = 0.0;
-        if (row < M) {
-          // sx and c_P times the row sum of xq (the sum of its group sums)
-          sxd = (double)__ldg(sx + row);
-          const int32_t* xs = xsum + (size_t)row * G;
-          int tot = 0;
-          if ((G & 3) == 0) {
-            const int4* x4 = reinterpret_cast<const int4*>(xs);
-            for (int g = 0; g < G / 4; ++g) {
-              const int4 v = __ldg(x4 + g);
-              tot += (v.x + v.y) + (v.z + v.w);
-            }
-          } else {
-            for (int g = 0; g < G; ++g) tot += __ldg(xs + g);
-          }
-          xb = xbias * (double)tot;
-        }
-        if (!mbar_wait(tfull_bar(acc), aphase, err)) break;
+        const double sxd = row < M ? (double)__ldg(sx + row) : 0.0;
+        if (!mbar_wait(tfull_bar(eg), aphase, err)) break;
         tc_fence_after();
-        const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
-        const uint32_t lead_tempty = mapa_shared(tempty_bar(acc), 0);
+        const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(eg * 256);
+        const uint32_t lead_tempty = mapa_shared(tempty_bar(eg), 0);
         switch (P) {
-          case 1: epilogue_tile<1>(t_lane, ebase, bias, sxd, xb, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
-          case 2: epilogue_tile<2>(t_lane, ebase, bias, sxd, xb, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
-          default: epilogue_tile<3>(t_lane, ebase, bias, sxd, xb, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          case 1: epilogue_tile<1>(t_lane, ebase, bias, sxd, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          case 2: epilogue_tile<2>(t_lane, ebase, bias, sxd, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          default: epilogue_tile<3>(t_lane, ebase, bias, sxd, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
         }
-        if (++acc == 2) {
-          acc = 0;
-          aphase ^= 1u;
-        }
+        aphase ^= 1u;
       }
       if (lane == 0) bulk_wait<0>();
     }
@@ -696,7 +682,7 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
   long long group_m = (40ll << 20) / (2 * BM * K);
   group_m = group_m < 1 ? 1 : (group_m > tiles_m ? tiles_m : group_m);
   return launch(w4a8_planes_kernel, dim3(grid), dim3(kThreads), (size_t)SMEM_ALLOC, true, tA, tB,
-                tY, sx, xsum, (const int*)ebase, bias, (int)M, (int)N, (int)K, (int)group_m,
+                tY, sx, (const int*)ebase, bias, (int)M, (int)N, (int)K, (int)group_m,
                 (const unsigned long long*)pword, epoch, err);
 }
 
