@@ -562,6 +562,17 @@ def table_entry(name, local, dev, peaks, int8):
            "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac",
                                              "traffic")},
            "sm_mhz": clocks["sm_mhz"], "reasons": clocks["reasons"]}
+    if run.w4 and run.M > 16 and roof["bound"] == "tensor":
+        # the GEMM route runs P int8 GEMMs (the byte planes of the weight): the
+        # tensor pipe does P times the product's 2 M N K operations
+        from w4a8_quantized_gemm_token_b200 import binding as qk
+
+        _, s16, o16 = run.weights[0]
+        planes = qk.qk_debug_w4a8_plane_count(s16, o16, run.K)
+        rec["planes"] = planes
+        if 1 <= planes <= 3:
+            rec["tensor_ops_per_call"] = planes * run.ops
+            rec["tensor_frac"] = planes * roof["achieved"] / roof["peak"]
     del run
     torch.cuda.empty_cache()
     return rec
