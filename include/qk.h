@@ -421,11 +421,14 @@ qk_status qk_debug_w4a8_group_acc(const int8_t *xq, int64_t M, int64_t K,
  * fewest bytes P <= 3 holding S q + O + 0x80..80 for every code q of every row,
  * else 255, or 255 for a non-finite scale or offset).  Writes it to *planes
  * (host) after synchronizing `stream`.  The route uses the byte-plane GEMM
- * for P <= 3, the per-group fold kernel otherwise.  Shapes as for the W4A8
- * calls; N >= 8.
+ * for P <= 3, the per-group fold kernel otherwise.  When P = 3 the GEMM takes
+ * the mixed layout (two digit planes for every row, the third digit only for
+ * the rows that need one, at most 8 in each aligned block of 60 rows) if every
+ * block fits; *mixed (host, nullable) receives 1 then, else 0.  Shapes as for
+ * the W4A8 calls; N >= 8.
  */
 qk_status qk_debug_w4a8_plane_count(const uint16_t *wscale, const uint16_t *woffset,
-                                    int64_t N, int64_t K, int *planes,
+                                    int64_t N, int64_t K, int *planes, int *mixed,
                                     qk_stream_t stream);
 
 /*

@@ -91,9 +91,9 @@ def test_routes_are_checked(qk):
     assert qk.lib.qk_w4a8_gemm(*args, 7, None) == 1        # unknown route
     assert qk.lib.qk_w4a8_gemm(*args, 4, None) == 1
     # the plane-count hook: shape contract, null output, alignment
-    assert qk.lib.qk_debug_w4a8_plane_count(FAKE, FAKE, 64, 96, ctypes.byref(ctypes.c_int()), None) == 2
-    assert qk.lib.qk_debug_w4a8_plane_count(FAKE, FAKE, 64, 256, None, None) == 1
-    assert qk.lib.qk_debug_w4a8_plane_count(FAKE + 2, FAKE, 64, 256, ctypes.byref(ctypes.c_int()), None) == 3
+    assert qk.lib.qk_debug_w4a8_plane_count(FAKE, FAKE, 64, 96, ctypes.byref(ctypes.c_int()), None, None) == 2
+    assert qk.lib.qk_debug_w4a8_plane_count(FAKE, FAKE, 64, 256, None, None, None) == 1
+    assert qk.lib.qk_debug_w4a8_plane_count(FAKE + 2, FAKE, 64, 256, ctypes.byref(ctypes.c_int()), None, None) == 3
     assert qk.lib.qk_debug_w4a8_group_acc(FAKE, 8, 256, FAKE, 64, 4, 2, FAKE, 1, None) == 1
     # the timeout test hook checks its limit on the host
     assert qk.lib.qk_debug_wait_timeout(0, None) == 1
@@ -114,7 +114,7 @@ def test_no_device_here(qk):
     for route in (0, 1, 3):
         assert qk.lib.qk_w4a8_gemm(FAKE, FAKE, FAKE, 32, 256, FAKE, FAKE, FAKE, None, 64, FAKE,
                                    route, None) == 4
-    assert qk.lib.qk_debug_w4a8_plane_count(FAKE, FAKE, 64, 256, ctypes.byref(ctypes.c_int()), None) == 4
+    assert qk.lib.qk_debug_w4a8_plane_count(FAKE, FAKE, 64, 256, ctypes.byref(ctypes.c_int()), None, None) == 4
 
 
 def test_binding_rejects_cpu_tensors(qk):

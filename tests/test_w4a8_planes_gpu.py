@@ -26,6 +26,25 @@ TOL_ULP = 2
 GEMM, FOLD = 1, 3
 
 
+def host_row_planes(s16, o16):
+    """Digits each weight row needs (1..3, or 255), from the fp16 bits (numpy,
+    int64; a shift past 40 bits or a non-finite value gives 255)."""
+    out = []
+    for n in range(np.asarray(s16).shape[0]):
+        out.append(host_plane_count(np.asarray(s16)[n:n + 1], np.asarray(o16)[n:n + 1], 0))
+    return np.array(out)
+
+
+def host_mixed(s16, o16, K):
+    """Whether a three-digit weight takes the mixed layout: at most 8 rows
+    needing a third digit in every aligned block of 60 rows."""
+    if host_plane_count(s16, o16, K) != 3:
+        return False
+    wide = host_row_planes(s16, o16) == 3
+    n = len(wide)
+    return all(wide[b:b + 60].sum() <= 8 for b in range(0, n, 60))
+
+
 def host_plane_count(s16, o16, K):
     """The plane count from the fp16 bits (numpy, int64; a shift past 40 bits
     or a non-finite value gives 255)."""
@@ -159,7 +178,8 @@ def test_gemm_route_parity(qk, orc, kind, MKN):
     Wp, s16, o16, allowed = make_weights(orc, kind, N, K, seed=M + K + N)
     expect = host_plane_count(s16, o16, K)
     assert expect in allowed
-    assert qk.qk_debug_w4a8_plane_count(dev_fp16(s16), dev_fp16(o16), K) == expect
+    assert qk.qk_debug_w4a8_plane_count(dev_fp16(s16), dev_fp16(o16), K, with_mixed=True) == \
+        (expect, host_mixed(s16, o16, K))
     case = synthetic.LinearCase("pl", M=M, K=K, N=N, bias=True, outlier_frac=0.01, seed=M * 3 + N)
     xb, _, b, _ = case.draw()
     _, _, _, y_g, y_f, y_o = run_both_routes(qk, orc, xb, Wp, s16, o16, b, M, K, N)
@@ -167,6 +187,41 @@ def test_gemm_route_parity(qk, orc, kind, MKN):
     assert d.max() <= TOL_ULP, f"{kind}: worst {d.max()} ulp"
     assert bf16_ulp_distance(t2bits(y_f), y_o).max() <= TOL_ULP
     assert torch.equal(y_g.view(torch.int16), y_f.view(torch.int16)), kind
+    qk.qk_check_device_error()
+
+
+def test_mixed_layout_boundaries(qk, orc):
+    """The mixed layout at its edges: a 60-row block with exactly 8 rows needing
+    a third digit (mixed) and one with 9 (uniform three planes), ragged N, and
+    the rows needing it at the first and last positions of a block."""
+    M, K = 300, 1024
+    G = K // 64
+    rng = np.random.default_rng(7)
+    for N, wide_rows, mixed in [(136, [0, 7, 20, 33, 41, 50, 58, 59], True),
+                                (136, [0, 7, 20, 33, 41, 50, 58, 59, 30], False),
+                                (264, [60, 119, 120, 179, 263], True)]:
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        Wp, s16, o16 = orc.quant_w4(W)
+        s = s16.view(np.float16).astype(np.float32)
+        o = o16.view(np.float16).astype(np.float32)
+        narrow = host_row_planes(s16, o16) <= 2
+        # keep only rows that need two digits, then give the chosen rows one
+        # group of a small range (subnormal fp16 scale and offset): a third digit
+        for n in range(N):
+            if not narrow[n]:
+                s[n], o[n] = s[n - 1], o[n - 1]
+        for n in wide_rows:
+            s[n, 1], o[n, 1] = 3e-6, -2e-5
+        s16, o16 = fp16_bits(s), fp16_bits(o)
+        rows = host_row_planes(s16, o16)
+        assert set(np.flatnonzero(rows == 3)) == set(wide_rows)
+        assert host_mixed(s16, o16, K) == mixed
+        assert qk.qk_debug_w4a8_plane_count(dev_fp16(s16), dev_fp16(o16), K, with_mixed=True) == (3, mixed)
+        case = synthetic.LinearCase("mx", M=M, K=K, N=N, bias=True, seed=N + len(wide_rows))
+        xb, _, b, _ = case.draw()
+        _, _, _, y_g, y_f, y_o = run_both_routes(qk, orc, xb, Wp, s16, o16, b, M, K, N)
+        assert bf16_ulp_distance(t2bits(y_g), y_o).max() <= TOL_ULP
+        assert torch.equal(y_g.view(torch.int16), y_f.view(torch.int16))
     qk.qk_check_device_error()
 
 
@@ -210,4 +265,57 @@ def test_workspace_reuse_across_plane_counts(qk, orc):
     torch.cuda.synchronize()
     y_o, _, _, _, _ = orc.w4a8_linear(xb, Wp, s16, o16, b)
     assert bf16_ulp_distance(t2bits(y), y_o).max() <= TOL_ULP
+    qk.qk_check_device_error()
+
+
+@pytest.mark.parametrize("kind", ["gauss", "unit", "p3"])
+@pytest.mark.parametrize("scene", ["tiny_x", "huge_x", "cancel"])
+def test_epilogue_exact_path(qk, orc, kind, scene):
+    """Outputs the epilogue's fp32 fast path must hand to its exact fp64 path:
+    activations so small that sx 2^e_n could underflow fp32 (every output takes
+    the exact path), so large that outputs overflow, and a bias that cancels
+    the product of most rows to a small remainder (the fp32 error bound then
+    exceeds the distance to the bf16 rounding midpoint).  The result must equal
+    the per-group fold route bit for bit either way."""
+    M, K, N = 300, 1024, 264
+    Wp, s16, o16, allowed = make_weights(orc, kind, N, K, seed=41 + len(kind))
+    assert host_plane_count(s16, o16, K) in allowed
+    rng = np.random.default_rng(len(scene) * 7 + len(kind))
+    xf = rng.standard_normal((M, K)).astype(np.float32)
+    b = (rng.standard_normal(N) * 0.1).astype(np.float32)
+    if scene == "tiny_x":
+        xf *= np.float32(1e-33)
+    elif scene == "huge_x":
+        xf = np.clip(xf, -1, 1) * np.float32(3.3e38)
+    else:
+        # rows 0..239 repeat one activation row; the bias is minus that row's
+        # output (computed by the oracle without bias), rounded to fp32
+        xf[:240] = xf[0]
+        y0, _, _, _, _ = orc.w4a8_linear(synthetic.f32_to_bf16_bits(xf[:1]), Wp, s16, o16, None)
+        b = -(y0[0].astype(np.uint32) << 16).view(np.float32)
+        b = b + (rng.standard_normal(N) * 1e-3 * np.abs(b)).astype(np.float32)
+    xb = synthetic.f32_to_bf16_bits(xf)
+    _, _, _, y_g, y_f, y_o = run_both_routes(qk, orc, xb, Wp, s16, o16, b, M, K, N)
+    assert torch.equal(y_g.view(torch.int16), y_f.view(torch.int16)), (kind, scene)
+    if scene == "huge_x":
+        assert bool(torch.isinf(y_g.float()).any()), "no output overflowed"
+    assert bf16_ulp_distance(t2bits(y_g), y_o).max() <= TOL_ULP
+    qk.qk_check_device_error()
+
+
+def test_epilogue_fast_path_many_outputs(qk, orc):
+    """4M outputs of Gaussian weights (two and three digit planes) with a bias:
+    about one output in ten thousand lies near enough to a bf16 rounding
+    midpoint to take the exact path; every output must equal the fold route's
+    bits."""
+    M, K, N = 2048, 1024, 2048
+    Wp, s16, o16, _ = make_weights(orc, "gauss", N, K, seed=77)
+    case = synthetic.LinearCase("fp", M=M, K=K, N=N, bias=True, outlier_frac=0.01, seed=78)
+    xb, _, b, _ = case.draw()
+    x = to_dev_bf16(xb)
+    dw = (to_dev(Wp), dev_fp16(s16), dev_fp16(o16))
+    xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
+    y_g = qk.qk_w4a8_gemm(xq, sx, xsum, *dw, to_dev(b), route=GEMM)
+    y_f = qk.qk_w4a8_gemm(xq, sx, xsum, *dw, to_dev(b), route=FOLD)
+    assert torch.equal(y_g.view(torch.int16), y_f.view(torch.int16))
     qk.qk_check_device_error()

@@ -44,7 +44,7 @@ _SIGS = {
     "qk_debug_w4a8_group_acc": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I, _P]),
     "qk_debug_wait_timeout": (_I, [_I64, _P]),
     "qk_debug_int8_peak": (_I, [_I64, _P, _P]),
-    "qk_debug_w4a8_plane_count": (_I, [_P, _P, _I64, _I64, _P, _P]),
+    "qk_debug_w4a8_plane_count": (_I, [_P, _P, _I64, _I64, _P, _P, _P]),
     "qk_sage_attention_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "qk_sage_attention": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]),
 }
@@ -290,17 +290,20 @@ def qk_debug_w4a8_group_acc(xq, Wp, m0, m1, route, acc=None, stream=None):
     return acc
 
 
-def qk_debug_w4a8_plane_count(wscale, woffset, K: int, stream=None) -> int:
-    """Byte planes the W4A8 GEMM route needs for these scales and offsets
-    (1..4), or 255 when it takes the per-group fold kernel."""
+def qk_debug_w4a8_plane_count(wscale, woffset, K: int, stream=None, with_mixed=False):
+    """Digit planes the W4A8 GEMM route needs for these scales and offsets
+    (1..3), or 255 when it takes the per-group fold kernel; with
+    `with_mixed`, also whether a three-plane weight takes the mixed layout."""
     _need(wscale, torch.float16, 2, "wscale")
     _need(woffset, torch.float16, 2, "woffset")
     N = wscale.shape[0]
     planes = ctypes.c_int(0)
+    mixed = ctypes.c_int(0)
     _check(lib.qk_debug_w4a8_plane_count(_ptr(wscale), _ptr(woffset), N, int(K),
-                                         ctypes.byref(planes), _stream(stream)),
+                                         ctypes.byref(planes), ctypes.byref(mixed),
+                                         _stream(stream)),
            "qk_debug_w4a8_plane_count")
-    return int(planes.value)
+    return (int(planes.value), bool(mixed.value)) if with_mixed else int(planes.value)
 
 
 def qk_debug_wait_timeout(limit_cycles: int, stream=None) -> None:

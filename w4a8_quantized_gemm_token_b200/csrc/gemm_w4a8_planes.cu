@@ -45,9 +45,11 @@
 //    operands loaded by TMA into a 6-stage ring, one MMA covering every plane
 //    so that a row's P sums sit in adjacent accumulator columns; two epilogue
 //    warpgroups, one per TMEM accumulator (so consecutive tiles drain in
-//    parallel), tcgen05.ld the P sums of 16 outputs at a time, form Y in fp64
-//    (exact), y = fma(sx 2^e_n, Y, bias) rounded once to bf16 by integer
-//    operations, and write it by TMA stores that clip the edges.
+//    parallel), tcgen05.ld the P sums of 16 outputs at a time, form Y exactly
+//    (int64), and round y = sx 2^e_n Y + bias once to bf16: in fp32 where a
+//    bound proves the result on the same side of the bf16 rounding midpoint as
+//    the exact value (so the bits are the exact value's), in fp64 otherwise;
+//    TMA stores that clip the edges write y.
 //    The plane GEMM does nothing unless the word holds 1..3 planes of this
 //    launch's epoch.
 // (Building the planes inside the GEMM was measured and not kept: a transform
@@ -68,7 +70,7 @@ namespace {
 
 constexpr int BM = 128;                 // rows of xq per CTA (the pair covers 256)
 constexpr int BK = 128;                 // K per stage: two groups of 64
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int kEpiWarps = 8;            // two warpgroups, one per TMEM accumulator
 constexpr int kThreads = 32 * (2 + kEpiWarps);  // 320
 constexpr int A_BYTES = BM * BK;        // 16 KiB of xq per stage
@@ -77,13 +79,44 @@ constexpr int STG_BYTES = 32 * 128;     // 32 output rows x 64 bf16
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_BYTES;
 constexpr int SMEM_STG = SMEM_B + STAGES * B_BYTES;
-constexpr int SMEM_BAR = SMEM_STG + kEpiWarps * STG_BYTES;
+// per epilogue warp, the current tile's column constants: {2^e_n, bias} for
+// the up to 256 weight rows of a uniform tile, or {2^e_n, bias, top-digit
+// offset} for the kMixRows rows of a mixed one (the same 2 KiB)
+struct ColInfo {
+  float p2;    // 2^e_n
+  float bias;
+};
+struct MixInfo {
+  float p2;
+  float bias;
+  uint32_t exoff;  // byte offset of the row's top-digit sum in a lane's ex row (8: none)
+  uint32_t pad;
+};
+constexpr int COL_BYTES = 256 * (int)sizeof(ColInfo);  // 2 KiB
+// per epilogue warp, each lane's top-digit sums of the current mixed half:
+// kMixExtra words and a zero, one 9-word row per lane (an odd stride: no bank
+// conflicts when every lane reads its own row)
+constexpr int kExStride = 9;
+constexpr int EX_BYTES = 32 * kExStride * 4;
+constexpr int SMEM_COL = SMEM_STG + kEpiWarps * STG_BYTES;
+constexpr int SMEM_EX = SMEM_COL + kEpiWarps * COL_BYTES;
+constexpr int SMEM_BAR = SMEM_EX + kEpiWarps * EX_BYTES;
 constexpr int kNumBars = 2 * STAGES + 4;  // full, empty per stage; tfull, tempty per accumulator
 constexpr int SMEM_SLOT = SMEM_BAR + kNumBars * 8;
 constexpr int SMEM_USED = SMEM_SLOT + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;
 constexpr int kTmemCols = 512;          // two accumulators of up to 256 columns
 constexpr int kMaxPlanes = 3;
+// Mixed mode (the matrix needs three digits but few rows do): tiles of
+// kMixRows weight rows, each CTA's half (kMixHalf rows) holding the two low
+// digit planes of its rows (2 kMixHalf plane rows) and the top digit of up to
+// kMixExtra of them that need it, 2 kMixHalf + kMixExtra = 128 plane rows.
+constexpr int kMixHalf = 60;
+constexpr int kMixRows = 2 * kMixHalf;
+constexpr int kMixExtra = 8;
+constexpr int kMixBox = 40;             // TMA box rows of the two low planes (three per half)
+static_assert(2 * kMixHalf + kMixExtra == 128, "mixed half = 128 plane rows");
+static_assert((2 * kMixHalf) % kMixBox == 0 && kMixBox % 8 == 0, "whole swizzle atoms per box");
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert(SMEM_B % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled operand tiles");
@@ -148,7 +181,8 @@ constexpr int kCountRowsPerBlock = 8;
 __global__ void __launch_bounds__(32 * kCountRowsPerBlock)
     w4a8_plane_count_kernel(const uint16_t* __restrict__ wscale,
                             const uint16_t* __restrict__ woffset, int N, int K, int* ebase,
-                            unsigned long long* pword, unsigned long long epoch) {
+                            int* slot, unsigned long long* hcount, unsigned long long* pword,
+                            unsigned long long* oword, unsigned long long epoch) {
   __shared__ int s_p[kCountRowsPerBlock];
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,9 +234,39 @@ __global__ void __launch_bounds__(32 * kCountRowsPerBlock)
   }
   if (lane == 0) s_p[warp] = prow;
   __syncthreads();
-  // an earlier kernel of the stream may still read the word until the
+  // an earlier kernel of the stream may still read the words until the
   // dependency wait returns
   pdl_wait();
+  if (n < N && lane == 0) {
+    // a row that needs a third digit takes one of its mixed-mode half tile's
+    // kMixExtra top-digit slots (counters tagged with the epoch, as the word
+    // below); a half tile with more such rows sets the overflow word
+    int sl = -1;
+    if (prow == 3) {
+      unsigned long long* c = hcount + n / kMixHalf;
+      unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(c);
+      while (true) {
+        const bool same = (old >> 8) == epoch;
+        const unsigned long long want = same ? old + 1 : ((epoch << 8) | 1ull);
+        const unsigned long long prev = atomicCAS(c, old, want);
+        if (prev == old) {
+          sl = same ? (int)(old & 0xFFull) : 0;
+          break;
+        }
+        old = prev;
+      }
+      if (sl >= kMixExtra) {
+        const unsigned long long want = (epoch << 8) | 1ull;
+        unsigned long long o = *reinterpret_cast<volatile unsigned long long*>(oword);
+        while (o != want) {
+          const unsigned long long prev = atomicCAS(oword, o, want);
+          if (prev == o) break;
+          o = prev;
+        }
+      }
+    }
+    slot[n] = sl;
+  }
   if (threadIdx.x == 0) {
     int pmax = 0;
     for (int w = 0; w < kCountRowsPerBlock; ++w) pmax = max(pmax, s_p[w]);
@@ -275,11 +339,15 @@ __device__ __forceinline__ void planes_of16(const uint2 w2, uint32_t S, uint32_t
                         pl[p][3] ^ 0x80808080u);
 }
 
-template <int P>
+// kMixed: the matrix needs three digits; the two low digit planes of every row
+// go to rows 2 n + p, the top digit of a row holding a slot to row
+// 2 N + kMixExtra (n / kMixHalf) + slot.
+template <int P, bool kMixed>
 __device__ __forceinline__ void build_rows(const uint8_t* __restrict__ Wp,
                                            const uint16_t* __restrict__ wscale,
                                            const uint16_t* __restrict__ woffset,
-                                           const int* __restrict__ ebase, int N, int K,
+                                           const int* __restrict__ ebase,
+                                           const int* __restrict__ slot, int N, int K,
                                            uint8_t* __restrict__ planes) {
   const int G = K >> 6;
   const int units_per_row = K >> 4;  // 16 codes each
@@ -295,25 +363,49 @@ __device__ __forceinline__ void build_rows(const uint8_t* __restrict__ Wp,
     const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(Wp + (size_t)n * (K / 2)) + c);
     uint4 out[P];
     planes_of16<P>(w2, S, Op, out);
+    if constexpr (kMixed) {
+      __stcg(reinterpret_cast<uint4*>(planes + ((size_t)n * 2) * K) + c, out[0]);
+      __stcg(reinterpret_cast<uint4*>(planes + ((size_t)n * 2 + 1) * K) + c, out[1]);
+      const int sl = __ldg(slot + n);
+      if (sl >= 0)
+        __stcg(reinterpret_cast<uint4*>(planes + ((size_t)2 * N + (size_t)kMixExtra * (n / kMixHalf) +
+                                                  sl) * K) + c,
+               out[2]);
+    } else {
 #pragma unroll
-    for (int p = 0; p < P; ++p)
-      __stcg(reinterpret_cast<uint4*>(planes + ((size_t)n * P + p) * K) + c, out[p]);
+      for (int p = 0; p < P; ++p)
+        __stcg(reinterpret_cast<uint4*>(planes + ((size_t)n * P + p) * K) + c, out[p]);
+    }
   }
+}
+
+// The launch's plane mode from the plane-count words: 1..3 uniform planes,
+// 4 = mixed (three digits needed, every half tile's top digits fit its
+// slots), 0 = nothing for the plane kernels (the fold computes).
+__device__ __forceinline__ int plane_mode(const unsigned long long* pword,
+                                          const unsigned long long* oword,
+                                          unsigned long long epoch) {
+  const unsigned long long pw = *reinterpret_cast<const volatile unsigned long long*>(pword);
+  const unsigned long long ow = *reinterpret_cast<const volatile unsigned long long*>(oword);
+  const int P = (pw >> 8) == epoch ? (int)(pw & 0xFFull) : 0;
+  const bool over = (ow >> 8) == epoch && (ow & 1ull) != 0;
+  if (P == 3) return over ? 3 : 4;
+  return (P >= 1 && P <= 2) ? P : 0;
 }
 
 __global__ void __launch_bounds__(kBuildThreads)
     w4a8_plane_build_kernel(const uint8_t* __restrict__ Wp, const uint16_t* __restrict__ wscale,
-                            const uint16_t* __restrict__ woffset, const int* ebase, int N,
-                            int K, uint8_t* planes, const unsigned long long* pword,
+                            const uint16_t* __restrict__ woffset, const int* ebase,
+                            const int* slot, int N, int K, uint8_t* planes,
+                            const unsigned long long* pword, const unsigned long long* oword,
                             unsigned long long epoch) {
   pdl_launch_dependents();
-  pdl_wait();  // e_n and the plane count come from the kernel before
-  const unsigned long long pw = *reinterpret_cast<const volatile unsigned long long*>(pword);
-  const int P = (pw >> 8) == epoch ? (int)(pw & 0xFFull) : 0;
-  switch (P) {
-    case 1: build_rows<1>(Wp, wscale, woffset, ebase, N, K, planes); break;
-    case 2: build_rows<2>(Wp, wscale, woffset, ebase, N, K, planes); break;
-    case 3: build_rows<3>(Wp, wscale, woffset, ebase, N, K, planes); break;
+  pdl_wait();  // e_n, the slots and the plane count come from the kernel before
+  switch (plane_mode(pword, oword, epoch)) {
+    case 1: build_rows<1, false>(Wp, wscale, woffset, ebase, slot, N, K, planes); break;
+    case 2: build_rows<2, false>(Wp, wscale, woffset, ebase, slot, N, K, planes); break;
+    case 3: build_rows<3, false>(Wp, wscale, woffset, ebase, slot, N, K, planes); break;
+    case 4: build_rows<3, true>(Wp, wscale, woffset, ebase, slot, N, K, planes); break;
     default: break;  // the fold kernel computes the product
   }
 }
@@ -354,12 +446,85 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
   return sign | min(keep + up - (896u << 7), 0x7F80u);
 }
 
-// The epilogue of one tile for a fixed P: 16 outputs per TMEM load group,
-// 64 outputs per staged 128-byte row and TMA store.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The fp32 fast path of one output.  With the digit sums A_p converted to
+// fp32 (one rounding each) and combined by fused multiply-adds, |yf - Y| is at
+// most 3 2^-24 T (1 + 2^-22), where T = sum_p 256^p |A_p| is formed the same way
+// (P = 3; fewer roundings for fewer planes); v = fma(sc, yf, bias) with
+// sc = sx 2^e_n exact in fp32 (sx a normal value in [2^-100, 2^100], or 0).
+// So |v - y| <= 3 2^-24 sc T (1 + 2^-22) + 2^-24 |v| for the exact
+// y = sc Y + bias while v is normal, and
+//   err = 2^-23 (1 + 2^-16) (1.5 sc T + |v|) + 2^-99
+// exceeds |v - y| + 2^-24 (|v| + err), the bound plus the roundings of v - err
+// and v + err, through every rounding of its own computation.  The absolute
+// term covers a subnormal v, whose rounding error is absolute: the interval
+// then straddles a bf16 midpoint whenever |v| is below about 2^-92.
+// Round-to-nearest-even to bf16 is monotone, so when v - err and v + err round
+// to the same bf16 value, y (and v) round to it too: those are the bits of the
+// exact path.  Returns the two roundings (low half: of v - err; high half: of
+// v + err).  A NaN v (from a NaN bias) must not reach here, since both halves
+// would agree; an infinite v gives a NaN and an infinity, which differ.
+__device__ __forceinline__ uint32_t fast_pair(float yf, float T, float sc, float bias) {
+  const float v = __fmaf_rn(sc, yf, bias);
+  const float err = __fmaf_rn(__fmaf_rn(1.5f * sc, T, fabsf(v)),
+                              1.192111085401848e-07f,   // 2^-23 (1 + 2^-16)
+                              1.5777218104420236e-30f); // 2^-99
+  return pack_bf16x2(v - err, v + err);
+}
+
+// Two outputs of the fast path, packed: the bf16 of outputs j (low half) and
+// j + 1 (high half), and in `dp` the halves where the two roundings differ.
+__device__ __forceinline__ uint32_t pack_pair(uint32_t hl0, uint32_t hl1, uint32_t& dp) {
+  const uint32_t lo = __byte_perm(hl0, hl1, 0x5410);  // the roundings of v - err
+  dp = lo ^ __byte_perm(hl0, hl1, 0x7632);            // against those of v + err
+  return lo;
+}
+
+// yf and T of one output from its P digit sums (int32 bit patterns).
 template <int P>
-__device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __restrict__ ebase,
-                                              const float* __restrict__ bias, double sxd,
-                                              uint8_t* stg_ptr, uint32_t stg,
+__device__ __forceinline__ void digits_to_f32(const uint32_t* a, float& yf, float& T) {
+  const float a0 = __int2float_rn((int)a[0]);
+  yf = a0;
+  T = fabsf(a0);
+  if constexpr (P >= 2) {
+    const float a1 = __int2float_rn((int)a[1]);
+    yf = __fmaf_rn(a1, 256.0f, yf);
+    T = __fmaf_rn(fabsf(a1), 256.0f, T);
+  }
+  if constexpr (P >= 3) {
+    const float a2 = __int2float_rn((int)a[2]);
+    yf = __fmaf_rn(a2, 65536.0f, yf);
+    T = __fmaf_rn(fabsf(a2), 65536.0f, T);
+  }
+}
+
+// 0xFFFFFFFF (every output of the lane takes the exact path) when sx is
+// outside the fast path's range: nonzero below 2^-100, where sx 2^e_n could lose
+// bits to fp32 underflow, or above 2^100, where it could overflow.
+__device__ __forceinline__ uint32_t sx_force_exact(float sxf) {
+  const float a = fabsf(sxf);
+  return ((a != 0.0f && a < 7.888609052210118e-31f) || a > 1.2676506002282294e30f) ? 0xFFFFFFFFu
+                                                                                     : 0u;
+}
+
+// The exact path of one output: Y in fp64 (exact, |Y| < 2^53), one fused
+// multiply-add with sx 2^e_n and the bias, one rounding to bf16.
+__device__ __forceinline__ uint32_t exact_value(long long Y, double sxd, float p2, float bias) {
+  return f64_to_bf16_bits(fma(sxd * (double)p2, __ll2double_rn(Y), (double)bias));
+}
+
+// The epilogue of one tile for a fixed P: 16 outputs per TMEM load group,
+// 64 outputs per staged 128-byte row and TMA store.  `force` is the lane's
+// sx_force_exact, or'ed with all-ones when a column of the tile has a
+// non-finite bias.
+template <int P>
+__device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const ColInfo* col, float sxf,
+                                              uint32_t force, uint8_t* stg_ptr, uint32_t stg,
                                               const CUtensorMap* tmY, int ncol0, int row0, int M,
                                               int N, int lane, uint32_t lead_tempty, bool& used) {
   constexpr int TR = tile_rows_of(P);
@@ -370,15 +535,6 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __rest
 #pragma unroll
     for (int sub = 0; sub < 4; ++sub) {
       const int r0 = ch * 64 + sub * 16;  // first weight row of this load group
-      // sx 2^e_n (exact: a power-of-two scaling) and the bias of the group's
-      // columns (the same for every lane: broadcast loads)
-      double sc[16], bv[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int n = ncol0 + r0 + j;
-        sc[j] = n < N ? sxd * __hiloint2double((1023 + __ldg(ebase + n)) << 20, 0) : 0.0;
-        bv[j] = (bias != nullptr && n < N) ? (double)__ldg(bias + n) : 0.0;
-      }
       uint32_t v[16 * P];
       const uint32_t a = t_lane + (uint32_t)(r0 * P);
       if constexpr (P == 1) {
@@ -401,18 +557,39 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __rest
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lead_tempty);
       }
+      uint32_t dp[8];
+      uint32_t differs = force;
 #pragma unroll
-      for (int i = 0; i < 16; i += 2) {
-        uint32_t hb[2];
+      for (int j = 0; j < 16; j += 2) {
+        uint32_t hl[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int j = i + h;
-          double Y = i32_to_f64(v[j * P + P - 1]);
-#pragma unroll
-          for (int p = P - 2; p >= 0; --p) Y = fma(Y, 256.0, i32_to_f64(v[j * P + p]));
-          hb[h] = f64_to_bf16_bits(fma(sc[j], Y, bv[j]));
+          const ColInfo ci = col[r0 + j + h];  // the same for every lane
+          float yf, T;
+          digits_to_f32<P>(v + (j + h) * P, yf, T);
+          hl[h] = fast_pair(yf, T, sxf * ci.p2, ci.bias);
         }
-        out[sub * 8 + (i >> 1)] = hb[0] | (hb[1] << 16);
+        out[sub * 8 + (j >> 1)] = pack_pair(hl[0], hl[1], dp[j >> 1]);
+        differs |= dp[j >> 1];
+      }
+      if (__any_sync(0xFFFFFFFFu, differs != 0u)) {
+        // the exact path, for each pair of outputs that some lane needs it for
+        const double sxd = (double)sxf;
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          if (__any_sync(0xFFFFFFFFu, (dp[j >> 1] | force) != 0u)) {
+            uint32_t hb[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              long long y = (long long)(int)v[(j + h) * P + P - 1];
+#pragma unroll
+              for (int p = P - 2; p >= 0; --p) y = y * 256 + (long long)(int)v[(j + h) * P + p];
+              const volatile ColInfo* cv = col + r0 + j + h;  // not merged with the fast path's reads
+              hb[h] = exact_value(y, sxd, cv->p2, cv->bias);
+            }
+            out[sub * 8 + (j >> 1)] = hb[0] | (hb[1] << 16);
+          }
+        }
       }
     }
     const int n0 = ncol0 + ch * 64;
@@ -434,12 +611,130 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_lane, const int* __rest
   }
 }
 
+// The epilogue of one mixed-mode tile (kMixRows weight rows): per half h, the
+// two low digit sums of row lr in columns h 128 + 2 lr + {0, 1} and the top
+// digit sums of the half's slots in columns h 128 + 2 kMixHalf + slot, which
+// each lane parks in its row of `ex` so that a row's top digit is one shared
+// load at the offset its column entry holds.  The kMixRows outputs of the
+// thread's row are assembled in registers and written as a 64-column TMA box
+// (once its outputs are final) and a 56-column one.
+__device__ __forceinline__ void epilogue_mixed(uint32_t t_lane, const MixInfo* col, float sxf,
+                                               uint32_t force, uint8_t* ex_ptr, uint8_t* stg_ptr,
+                                               uint32_t stg, const CUtensorMap* tmY,
+                                               const CUtensorMap* tmY56, int ncol0, int row0,
+                                               int M, int N, int lane, uint32_t lead_tempty,
+                                               bool& used) {
+  uint32_t out[kMixRows / 2];
+  uint8_t* exrow = ex_ptr + lane * (kExStride * 4);
+  // box 0 holds outputs 0..63, box 1 outputs 64..119 (56 columns, 112 bytes)
+  auto store_box = [&](int ch) {
+    const int n0 = ncol0 + 64 * ch;
+    if (n0 >= N || row0 >= M) return;  // whole box outside y
+    if (lane == 0 && used) bulk_wait_read<0>();
+    __syncwarp();
+    uint8_t* rowp = stg_ptr + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (ch == 1 && j == 7) break;
+      *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+          make_uint4(out[32 * ch + 4 * j], out[32 * ch + 4 * j + 1], out[32 * ch + 4 * j + 2],
+                     out[32 * ch + 4 * j + 3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(ch == 0 ? tmY : tmY56, stg, n0, row0);
+      bulk_commit();
+    }
+    used = true;
+  };
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t hb = t_lane + (uint32_t)(h * 128);
+    {
+      uint32_t ex[8];
+      tmem_ld8(hb + 2 * kMixHalf, ex);  // the half's top-digit sums
+      tmem_ld_wait();
+      // (each lane reads only its own row: no synchronisation between lanes)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) reinterpret_cast<uint32_t*>(exrow)[k] = ex[k];
+      reinterpret_cast<uint32_t*>(exrow)[8] = 0u;
+    }
+#pragma unroll
+    for (int sub = 0; sub < 4; ++sub) {
+      constexpr int kSub[4] = {16, 16, 16, kMixHalf - 48};
+      const int lr0 = 16 * sub;
+      const int cnt = kSub[sub];
+      uint32_t v[32];
+      if (sub < 3) {
+        tmem_ld32(hb + (uint32_t)(2 * lr0), v);
+      } else {
+        uint32_t (&v16)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
+        uint32_t (&v8)[8] = *reinterpret_cast<uint32_t(*)[8]>(v + 16);
+        tmem_ld16(hb + (uint32_t)(2 * lr0), v16);
+        tmem_ld8(hb + (uint32_t)(2 * lr0 + 16), v8);
+      }
+      tmem_ld_wait();
+      if (h == 1 && sub == 3) {
+        // every TMEM read of this accumulator is done: hand it back to the leader
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_tempty);
+      }
+      uint32_t dp[8];
+      uint32_t differs = force;
+#pragma unroll
+      for (int j = 0; j < 16; j += 2) {
+        if (j < cnt) {
+          uint32_t hl[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const MixInfo ci = col[h * kMixHalf + lr0 + j + e];  // the same for every lane
+            uint32_t d[3] = {v[2 * (j + e)], v[2 * (j + e) + 1],
+                             *reinterpret_cast<const uint32_t*>(exrow + ci.exoff)};
+            float yf, T;
+            digits_to_f32<3>(d, yf, T);
+            hl[e] = fast_pair(yf, T, sxf * ci.p2, ci.bias);
+          }
+          out[(h * kMixHalf + lr0 + j) >> 1] = pack_pair(hl[0], hl[1], dp[j >> 1]);
+          differs |= dp[j >> 1];
+        }
+      }
+      if (__any_sync(0xFFFFFFFFu, differs != 0u)) {
+        // the exact path, for each pair of outputs that some lane needs it for
+        const double sxd = (double)sxf;
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          if (j < cnt && __any_sync(0xFFFFFFFFu, (dp[j >> 1] | force) != 0u)) {
+            uint32_t hv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const volatile MixInfo* cv = col + h * kMixHalf + lr0 + j + e;
+              const long long top =
+                  (long long)*reinterpret_cast<const volatile int*>(exrow + cv->exoff);
+              const long long y = (top * 256 + (long long)(int)v[2 * (j + e) + 1]) * 256 +
+                                  (long long)(int)v[2 * (j + e)];
+              hv[e] = exact_value(y, sxd, cv->p2, cv->bias);
+            }
+            out[(h * kMixHalf + lr0 + j) >> 1] = hv[0] | (hv[1] << 16);
+          }
+        }
+      }
+      if (h == 1 && sub == 0) store_box(0);  // outputs 0..63 are final: free their registers
+    }
+  }
+  store_box(1);
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w4a8_planes_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const __grid_constant__ CUtensorMap tmY, const float* __restrict__ sx,
-                       const int* __restrict__ ebase,
+                       const __grid_constant__ CUtensorMap tmB40, const __grid_constant__ CUtensorMap tmB8,
+                       const __grid_constant__ CUtensorMap tmY,
+                       const __grid_constant__ CUtensorMap tmY56, const float* __restrict__ sx,
+                       const int* __restrict__ ebase, const int* __restrict__ slot,
                        const float* __restrict__ bias, int M, int N, int K, int group_m,
-                       const unsigned long long* pword, unsigned long long epoch, int* err) {
+                       const unsigned long long* pword, const unsigned long long* oword,
+                       unsigned long long epoch, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -459,7 +754,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmB40);
+    prefetch_tmap(&tmB8);
     prefetch_tmap(&tmY);
+    prefetch_tmap(&tmY56);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
@@ -483,11 +781,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   pdl_wait();  // xq, sx, e_n, the planes and the plane-count word come from earlier kernels
 
-  const unsigned long long pw = *reinterpret_cast<const volatile unsigned long long*>(pword);
-  const int P = (pw >> 8) == epoch ? (int)(pw & 0xFFull) : 0;
-  if (P >= 1 && P <= kMaxPlanes) {
-    const int TR = tile_rows_of(P);
+  const int mode = plane_mode(pword, oword, epoch);
+  if (mode != 0) {
+    const bool mixed = mode == 4;
+    const int P = mixed ? 3 : mode;        // digits per weight
+    const int TR = mixed ? kMixRows : tile_rows_of(P);
     const int RC = TR / 2;                 // weight rows of each CTA's half
+    const int nplane = mixed ? 128 : P * RC;  // plane rows of each CTA's half
     const int tiles_m = (M + 2 * BM - 1) / (2 * BM);
     const int tiles_n = (N + TR - 1) / TR;
     const int num_tiles = tiles_m * tiles_n;
@@ -501,12 +801,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        const uint32_t tx = 2u * (uint32_t)(A_BYTES + P * RC * BK);
+        const uint32_t tx = 2u * (uint32_t)(A_BYTES + nplane * BK);
         for (int t = pair; t < num_tiles && ok; t += num_pairs) {
           int mb, nb;
           tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
           const int arow = mb * 2 * BM + (int)rank * BM;
-          const int brow = (nb * TR + (int)rank * RC) * P;
+          // uniform: rows (nb TR + rank RC) P ..; mixed: the two low planes of
+          // the half's rows and its kMixExtra top-digit rows after the 2 N
+          const int brow = mixed ? (nb * TR + (int)rank * RC) * 2 : (nb * TR + (int)rank * RC) * P;
+          const int xrow = 2 * N + kMixExtra * (2 * nb + (int)rank);
           for (int kb = 0; kb < num_kb; ++kb) {
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, err)) {
               ok = false;
@@ -515,9 +818,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), tx);
             const uint32_t lead_full = mapa_shared(full_bar(stage), 0);
             tma_load_2d_pair(sbase + SMEM_A + stage * A_BYTES, &tmA, kb * BK, arow, lead_full);
-            for (int i = 0; i < P * RC / 32; ++i)
-              tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES + i * 32 * BK, &tmB, kb * BK,
-                               brow + 32 * i, lead_full);
+            if (mixed) {
+              for (int i = 0; i < 2 * kMixHalf / kMixBox; ++i)
+                tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES + i * kMixBox * BK, &tmB40,
+                                 kb * BK, brow + kMixBox * i, lead_full);
+              tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES + 2 * kMixHalf * BK, &tmB8,
+                               kb * BK, xrow, lead_full);
+            } else {
+              for (int i = 0; i < P * RC / 32; ++i)
+                tma_load_2d_pair(sbase + SMEM_B + stage * B_BYTES + i * 32 * BK, &tmB, kb * BK,
+                                 brow + 32 * i, lead_full);
+            }
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -528,7 +839,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ------------------------------------------- MMA issuer (pair leader)
       if (rank == 0 && lane == 0) {
-        const uint32_t idesc = i8_idesc(2 * BM, P * TR, true, true);
+        const uint32_t idesc = i8_idesc(2 * BM, 2 * nplane, true, true);
         int stage = 0;
         uint32_t phase = 0;
         int acc = 0;
@@ -572,6 +883,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int q = warp & 3;             // TMEM lane quarter
       uint8_t* stg_ptr = smem + SMEM_STG + e * STG_BYTES;
       const uint32_t stg = sbase + SMEM_STG + (uint32_t)(e * STG_BYTES);
+      ColInfo* col = reinterpret_cast<ColInfo*>(smem + SMEM_COL + e * COL_BYTES);
+      MixInfo* mcol = reinterpret_cast<MixInfo*>(smem + SMEM_COL + e * COL_BYTES);
+      uint8_t* ex_ptr = smem + SMEM_EX + e * EX_BYTES;
       uint32_t aphase = 0;
       bool used = false;
       for (int t = pair + eg * num_pairs; t < num_tiles; t += 2 * num_pairs) {
@@ -579,15 +893,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tile_coords(t, tiles_m, tiles_n, group_m, mb, nb);
         const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;
         const int row = row0 + lane;
-        const double sxd = row < M ? (double)__ldg(sx + row) : 0.0;
+        const float sxf = row < M ? __ldg(sx + row) : 0.0f;
+        // this tile's column constants, one table per warp (columns past N:
+        // e_n 0, no bias, no slot -- their outputs are clipped by the stores);
+        // a non-finite bias sends the whole tile to the exact path
+        __syncwarp();  // every lane is done with the previous tile's table
+        bool bad_bias = false;
+        for (int r = lane; r < TR; r += 32) {
+          const int n = nb * TR + r;
+          const float p2 = __uint_as_float((uint32_t)(127 + (n < N ? __ldg(ebase + n) : 0)) << 23);
+          const float bv = (bias != nullptr && n < N) ? __ldg(bias + n) : 0.0f;
+          bad_bias |= !(fabsf(bv) <= 3.4028234663852886e38f);
+          if (mixed) {
+            const int sl = n < N ? __ldg(slot + n) : -1;
+            MixInfo mi;
+            mi.p2 = p2;
+            mi.bias = bv;
+            mi.exoff = (uint32_t)(sl >= 0 ? sl : kMixExtra) * 4u;
+            mi.pad = 0u;
+            mcol[r] = mi;
+          } else {
+            ColInfo ci;
+            ci.p2 = p2;
+            ci.bias = bv;
+            col[r] = ci;
+          }
+        }
+        const uint32_t force = sx_force_exact(sxf) |
+                               (__any_sync(0xFFFFFFFFu, bad_bias) ? 0xFFFFFFFFu : 0u);
+        __syncwarp();
         if (!mbar_wait(tfull_bar(eg), aphase, err)) break;
         tc_fence_after();
         const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(eg * 256);
         const uint32_t lead_tempty = mapa_shared(tempty_bar(eg), 0);
-        switch (P) {
-          case 1: epilogue_tile<1>(t_lane, ebase, bias, sxd, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
-          case 2: epilogue_tile<2>(t_lane, ebase, bias, sxd, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
-          default: epilogue_tile<3>(t_lane, ebase, bias, sxd, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+        switch (mode) {
+          case 1: epilogue_tile<1>(t_lane, col, sxf, force, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          case 2: epilogue_tile<2>(t_lane, col, sxf, force, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          case 3: epilogue_tile<3>(t_lane, col, sxf, force, stg_ptr, stg, &tmY, nb * TR, row0, M, N, lane, lead_tempty, used); break;
+          default: epilogue_mixed(t_lane, mcol, sxf, force, ex_ptr, stg_ptr, stg, &tmY, &tmY56, nb * TR, row0, M, N, lane, lead_tempty, used); break;
         }
         aphase ^= 1u;
       }
@@ -606,20 +949,36 @@ bool g_attr_done[64];
 
 }  // namespace
 
-size_t w4a8_plane_scratch_bytes(int64_t N, int64_t K) {
-  auto r = [](size_t b) { return (b + 255u) & ~size_t(255u); };
-  return r(8) + r((size_t)N * 4u) + (size_t)kMaxPlanes * (size_t)N * (size_t)K;
-}
+// Scratch of the GEMM route: the plane-count and overflow words, e_n and the
+// top-digit slot of every row, the mixed-mode half-tile counters, then the
+// planes ([3 N, K] int8: P N rows uniform, or 2 N rows + the top-digit rows).
+struct PlaneScratch {
+  size_t words, ebase, slot, hcount, planes, total;
+  PlaneScratch(int64_t N, int64_t K) {
+    auto r = [](size_t b) { return (b + 255u) & ~size_t(255u); };
+    words = 0;
+    ebase = words + r(16);
+    slot = ebase + r((size_t)N * 4u);
+    hcount = slot + r((size_t)N * 4u);
+    planes = hcount + r((size_t)((N + kMixHalf - 1) / kMixHalf) * 8u);
+    total = planes + (size_t)kMaxPlanes * (size_t)N * (size_t)K;
+  }
+};
+
+size_t w4a8_plane_scratch_bytes(int64_t N, int64_t K) { return PlaneScratch(N, K).total; }
 
 cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
                              int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
                              const float* bias, int64_t N, uint16_t* y, void* scratch, bool pdl,
                              cudaStream_t s) {
-  auto r = [](size_t b) { return (b + 255u) & ~size_t(255u); };
+  const PlaneScratch L(N, K);
   uint8_t* base = static_cast<uint8_t*>(scratch);
-  auto* pword = reinterpret_cast<unsigned long long*>(base);
-  auto* ebase = reinterpret_cast<int*>(base + r(8));
-  uint8_t* planes = base + r(8) + r((size_t)N * 4u);
+  auto* pword = reinterpret_cast<unsigned long long*>(base + L.words);
+  auto* oword = pword + 1;
+  auto* ebase = reinterpret_cast<int*>(base + L.ebase);
+  auto* slot = reinterpret_cast<int*>(base + L.slot);
+  auto* hcount = reinterpret_cast<unsigned long long*>(base + L.hcount);
+  uint8_t* planes = base + L.planes;
   const unsigned long long epoch = next_epoch();
   auto launch = [&](auto kernel, dim3 grid, dim3 block, size_t smem, bool dep, auto... args) {
     cudaLaunchConfig_t cfg = {};
@@ -638,28 +997,36 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
   cudaError_t e = launch(w4a8_plane_count_kernel,
                          dim3((unsigned)((N + kCountRowsPerBlock - 1) / kCountRowsPerBlock)),
                          dim3(32 * kCountRowsPerBlock), 0, pdl, ws, wo, (int)N, (int)K, ebase,
-                         pword, epoch);
+                         slot, hcount, pword, oword, epoch);
   if (e != cudaSuccess) return e;
   // 2. the planes (a few waves of the SMs; each thread loops over 16-code units)
   const long long units = N * (K / 16);
   long long blocks = (units + kBuildThreads - 1) / kBuildThreads;
   const long long cap = 8ll * num_sms();
   e = launch(w4a8_plane_build_kernel, dim3((unsigned)(blocks < cap ? blocks : cap)),
-             dim3(kBuildThreads), 0, true, Wp, ws, wo, (const int*)ebase, (int)N, (int)K, planes,
-             (const unsigned long long*)pword, epoch);
+             dim3(kBuildThreads), 0, true, Wp, ws, wo, (const int*)ebase, (const int*)slot,
+             (int)N, (int)K, planes, (const unsigned long long*)pword,
+             (const unsigned long long*)oword, epoch);
   if (e != cudaSuccess) return e;
   // 3. the per-group fold, which computes only when the planes cannot
   e = launch_w4a8_fold(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, true, s, pword,
                        epoch);
   if (e != cudaSuccess) return e;
   // 4. the plane GEMM
-  CUtensorMap tA, tB, tY;
+  CUtensorMap tA, tB, tB40, tB8, tY, tY56;
   if (!encode_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
                       (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes, (uint64_t)K,
                       (uint64_t)(kMaxPlanes * N), (uint64_t)K, BK, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tB40, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes, (uint64_t)K,
+                      (uint64_t)(kMaxPlanes * N), (uint64_t)K, BK, kMixBox,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tB8, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes, (uint64_t)K,
+                      (uint64_t)(kMaxPlanes * N), (uint64_t)K, BK, 8, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
-                      (uint64_t)N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+                      (uint64_t)N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&tY56, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
+                      (uint64_t)N * 2, 56, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -682,13 +1049,20 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
   long long group_m = (40ll << 20) / (2 * BM * K);
   group_m = group_m < 1 ? 1 : (group_m > tiles_m ? tiles_m : group_m);
   return launch(w4a8_planes_kernel, dim3(grid), dim3(kThreads), (size_t)SMEM_ALLOC, true, tA, tB,
-                tY, sx, (const int*)ebase, bias, (int)M, (int)N, (int)K, (int)group_m,
-                (const unsigned long long*)pword, epoch, err);
+                tB40, tB8, tY, tY56, sx, (const int*)ebase, (const int*)slot, bias, (int)M, (int)N,
+                (int)K, (int)group_m, (const unsigned long long*)pword,
+                (const unsigned long long*)oword, epoch, err);
 }
 
 cudaError_t launch_w4a8_plane_count(const uint16_t* ws, const uint16_t* wo, int64_t N, int64_t K,
-                                    int* ebase, unsigned long long* pword,
-                                    unsigned long long epoch, bool pdl, cudaStream_t s) {
+                                    void* scratch, unsigned long long epoch, bool pdl,
+                                    cudaStream_t s) {
+  const PlaneScratch L(N, K);
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  auto* pword = reinterpret_cast<unsigned long long*>(base + L.words);
+  auto* ebase = reinterpret_cast<int*>(base + L.ebase);
+  auto* slot = reinterpret_cast<int*>(base + L.slot);
+  auto* hcount = reinterpret_cast<unsigned long long*>(base + L.hcount);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((N + kCountRowsPerBlock - 1) / kCountRowsPerBlock));
   cfg.blockDim = dim3(32 * kCountRowsPerBlock);
@@ -698,8 +1072,8 @@ cudaError_t launch_w4a8_plane_count(const uint16_t* ws, const uint16_t* wo, int6
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, w4a8_plane_count_kernel, ws, wo, (int)N, (int)K, ebase, pword,
-                            epoch);
+  return cudaLaunchKernelEx(&cfg, w4a8_plane_count_kernel, ws, wo, (int)N, (int)K, ebase, slot,
+                            hcount, pword, pword + 1, epoch);
 }
 
 }  // namespace qk

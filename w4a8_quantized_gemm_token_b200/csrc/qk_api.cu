@@ -580,28 +580,27 @@ qk_status qk_debug_w8a8_acc(const int8_t* xq, int64_t M, int64_t K, const int8_t
 }
 
 qk_status qk_debug_w4a8_plane_count(const uint16_t* wscale, const uint16_t* woffset, int64_t N,
-                                    int64_t K, int* planes, qk_stream_t stream) {
+                                    int64_t K, int* planes, int* mixed, qk_stream_t stream) {
   qk_status st = check_shape(1, K, N, true);
   if (st != QK_OK) return st;
   if (!wscale || !woffset || !planes) return QK_ERR_INVALID_ARG;
   if (!aligned16(wscale) || !aligned16(woffset)) return QK_ERR_MISALIGNED;
   if ((st = check_device()) != QK_OK) return st;
   void* scratch = nullptr;
-  const size_t bytes = 256 + round256((size_t)N * 4u);
-  if ((st = from_cuda(cudaMallocAsync(&scratch, bytes, stream), "cudaMallocAsync(plane count)")) !=
-      QK_OK)
+  if ((st = from_cuda(cudaMallocAsync(&scratch, w4a8_plane_scratch_bytes(N, 0), stream),
+                      "cudaMallocAsync(plane count)")) != QK_OK)
     return st;
   const unsigned long long epoch = next_epoch();
-  unsigned long long word = 0;
-  cudaError_t e = launch_w4a8_plane_count(
-      wscale, woffset, N, K, reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) + 256),
-      static_cast<unsigned long long*>(scratch), epoch, false, stream);
+  unsigned long long words[2] = {0, 0};
+  cudaError_t e = launch_w4a8_plane_count(wscale, woffset, N, K, scratch, epoch, false, stream);
   if (e == cudaSuccess)
-    e = cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, stream);
+    e = cudaMemcpyAsync(words, scratch, sizeof(words), cudaMemcpyDeviceToHost, stream);
   cudaFreeAsync(scratch, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if ((st = from_cuda(e, "w4a8_plane_count")) != QK_OK) return st;
-  *planes = (word >> 8) == epoch ? (int)(word & 0xFFull) : 0;
+  *planes = (words[0] >> 8) == epoch ? (int)(words[0] & 0xFFull) : 0;
+  if (mixed != nullptr)
+    *mixed = (*planes == 3 && !((words[1] >> 8) == epoch && (words[1] & 1ull) != 0)) ? 1 : 0;
   return QK_OK;
 }
 

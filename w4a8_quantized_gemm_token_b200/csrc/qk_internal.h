@@ -89,15 +89,19 @@ cudaError_t launch_w4a8_fold(const int8_t* xq, const float* sx, const int32_t* x
                              unsigned long long epoch = 0);
 
 // The byte-plane W4A8 GEMM (gemm_w4a8_planes.cu).  The plane-count kernel
-// writes e_n of every weight row to ebase and (epoch << 8) | P to *pword
-// (raised within an epoch, replacing any other epoch's word; no clearing
-// needed).
+// writes, into the route's scratch (laid out by w4a8_plane_scratch_bytes),
+// e_n and the top-digit slot of every weight row and two words tagged with
+// `epoch` (raised within an epoch, replacing any other epoch's word; no
+// clearing needed): word 0 = (epoch << 8) | P, word 1 = (epoch << 8) | 1 when
+// some half tile has more rows needing a third digit than it has slots.
 cudaError_t launch_w4a8_plane_count(const uint16_t* ws, const uint16_t* wo, int64_t N, int64_t K,
-                                    int* ebase, unsigned long long* pword,
-                                    unsigned long long epoch, bool pdl, cudaStream_t s);
+                                    void* scratch, unsigned long long epoch, bool pdl,
+                                    cudaStream_t s);
 
-// Device scratch the W4A8 GEMM route needs: the plane-count word, e_n of every
-// weight row and the byte planes of the dequantized weight (up to 3 N K bytes).
+// Device scratch the W4A8 GEMM route needs: the plane-count words, e_n and
+// the top-digit slot of every weight row, the half-tile counters and the digit
+// planes of the dequantized weight (3 N K bytes; none for K = 0, which sizes
+// the scratch of the count alone).
 size_t w4a8_plane_scratch_bytes(int64_t N, int64_t K);
 
 // The W4A8 GEMM route (any M): the plane count, the plane build, the gated
