@@ -289,8 +289,10 @@ qk_status qk_w8a8_linear_noalloc(const uint16_t *x, int64_t M, int64_t K,
  * multiple of 2^e_n (e_n the smallest exponent of their lowest set bits), so
  * every dequantized weight is 2^e_n times an integer W; when W + 0x80..80 fits
  * P <= 3 bytes for every weight (Gaussian weights need 2 or 3), the product is
- * P exact int8 GEMMs on those bytes, rounded once -- the fold's exact value,
- * the same bits as the per-group fold wherever that fold is exact in fp64;
+ * P exact int8 GEMMs on those bytes, rounded once -- the fold's exact value
+ * (rounded in fp32 where an error bound proves the bf16 result equal to the
+ * exact value's, in fp64 otherwise), the same bits as the per-group fold
+ * wherever that fold is exact in fp64;
  * otherwise the per-group fold kernel computes it.  The route allocates its
  * scratch (the planes, up to 3 N K bytes) stream-ordered from a memory pool of
  * the library that keeps freed blocks for reuse.
