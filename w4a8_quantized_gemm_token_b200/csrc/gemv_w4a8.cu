@@ -31,9 +31,11 @@
 //    absmax is exchanged through distributed shared memory) or reads
 //    quantized xq / sx / xsum.
 //  * 8 warps = R/16 row tiles x KW group ranges.  Nibbles are split in
-//    registers straight into the A fragments of mma.sync m16n8k32 u8 x s8
-//    (weights as A, tokens as the N = 8 side); K is permuted identically in A
-//    and B so each lane uses 8 packed bytes and 16 activation bytes per group.
+//    registers and put back in K order (two byte permutes per packed word)
+//    as the A fragments of mma.sync m16n8k32 u8 x s8 (weights as A, tokens as
+//    the N = 8 side), so each lane pairs its 8 packed bytes of a group with 16
+//    consecutive activation bytes, and the activations stay in their natural
+//    order: the quantized rows arrive by bulk copies issued by one thread.
 //  * Per-group sums fold into fp64 (exact int -> fp64 by the 2^52 magic
 //    number).  With one token the lanes first gather one group each by
 //    shuffles, so no lane folds an all-zero token column.
@@ -102,7 +104,8 @@ struct GemvLayout {
     bias = off; off += (size_t)RO * 4;                // bias of the rows this CTA finalizes
     off = (off + 15) & ~size_t(15);
     part = off; off += (size_t)C * KW * M * RO * 8;   // fp64 partials [slot][token][row]
-    bars = off; off += (size_t)(nbox + 1) * 8;        // mbarriers: the boxes, the scales
+    bars = off; off += (size_t)(nbox + 2) * 8;        // mbarriers: the boxes, the scales,
+                                                      // the activation rows
     total = off + 1024;                               // base alignment slack
   }
 };
@@ -163,10 +166,16 @@ __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Bytes 0..7 of an 8-code group of xq reordered: the four even k, then the
-// four odd k (the order in which the nibble split delivers the weight codes).
-__device__ __forceinline__ uint2 even_odd(uint32_t lo, uint32_t hi) {
-  return make_uint2(__byte_perm(lo, hi, 0x6420), __byte_perm(lo, hi, 0x7531));
+// The A fragment of one m16n8k32 MMA from 4 packed bytes (8 codes, code 2i
+// in the low nibble of byte i) of each of the lane's two rows: the codes back
+// in K order, four per register.
+__device__ __forceinline__ void split_codes(uint32_t wa, uint32_t wb, uint32_t (&a)[4]) {
+  const uint32_t la = wa & 0x0F0F0F0Fu, ha = (wa >> 4) & 0x0F0F0F0Fu;  // even, odd codes
+  const uint32_t lb = wb & 0x0F0F0F0Fu, hb = (wb >> 4) & 0x0F0F0F0Fu;
+  a[0] = __byte_perm(la, ha, 0x5140);  // row ra:     codes 0..3
+  a[1] = __byte_perm(lb, hb, 0x5140);  // row ra + 8: codes 0..3
+  a[2] = __byte_perm(la, ha, 0x7362);  // row ra:     codes 4..7
+  a[3] = __byte_perm(lb, hb, 0x7362);  // row ra + 8: codes 4..7
 }
 
 
@@ -206,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint8_t* w_sm = smem + L.w;
   const uint32_t wbar0 = smem_u32(smem + L.bars);      // box j: wbar0 + 8 j
   const uint32_t sbar = wbar0 + 8u * (uint32_t)L.nbox;
+  const uint32_t abar = sbar + 8u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rt = warp % RT, kw = warp / RT;
   const int grp = lane >> 2, tq = lane & 3;
@@ -218,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // packed codes of this lane's two rows into registers, the bias.
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmW);
-    for (int q = 0; q <= L.nbox; ++q) mbar_init(wbar0 + 8u * q, 1);
+    for (int q = 0; q <= L.nbox + 1; ++q) mbar_init(wbar0 + 8u * q, 1);
     fence_mbar_init();
     if (kFold) {
       if (C > 1) {
@@ -258,16 +268,24 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (!early_trigger) pdl_launch_dependents();
   if constexpr (kQuantX) {
     const int nch = GC * 8;         // 16-byte chunks per row of the slice
-    const int total = M * nch;      // chunk c: row c / nch
+    const int total = M * nch;      // chunk c = threadIdx.x + kThreads i: row c / nch
+    // (row, chunk) of c for every i, by steps of kThreads (one division each)
+    const int dm = kThreads / nch, dr = kThreads - dm * nch;
+    const int m_first = (int)threadIdx.x / nch, r_first = (int)threadIdx.x - m_first * nch;
     const uint4* src = reinterpret_cast<const uint4*>(x);
     uint4 v[kQuantChunks];
+    {
+      int m = m_first, r = r_first;
 #pragma unroll
-    for (int i = 0; i < kQuantChunks; ++i) {
-      const int c = threadIdx.x + kThreads * i;
-      v[i] = make_uint4(0u, 0u, 0u, 0u);
-      if (c < total) {
-        const int m = c / nch;
-        v[i] = __ldg(src + (((size_t)m * K + (size_t)g0 * 64) >> 3) + (c - m * nch));
+      for (int i = 0; i < kQuantChunks; ++i) {
+        v[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (m < M) v[i] = __ldg(src + (((size_t)m * K + (size_t)g0 * 64) >> 3) + r);
+        m += dm;
+        r += dr;
+        if (r >= nch) {
+          r -= nch;
+          ++m;
+        }
       }
     }
     unsigned int* amx_local = amx_sm + C * 16;
@@ -324,67 +342,73 @@ __global__ void __launch_bounds__(kThreads, 2)
       sx_sm[threadIdx.x] = act_scale(amax);
     }
     __syncthreads();
+    {
+      int m = m_first, cc = r_first;
 #pragma unroll
-    for (int i = 0; i < kQuantChunks; ++i) {
-      if (kThreads * i >= total) break;  // warp-uniform
-      const int c = threadIdx.x + kThreads * i;
-      int sum = 0, m = 0, cc = 0;
-      if (c < total) {
-        m = c / nch;
-        cc = c - m * nch;
-        const uint2 qc = quant_chunk(v[i], rmul_sm[m], &sum);
-        *reinterpret_cast<uint2*>(xq_sm + (size_t)m * XS + 8 * cc) = even_odd(qc.x, qc.y);
+      for (int i = 0; i < kQuantChunks; ++i) {
+        if (kThreads * i >= total) break;  // warp-uniform
+        int sum = 0;
+        if (m < M) {
+          const uint2 qc = quant_chunk(v[i], rmul_sm[m], &sum);
+          *reinterpret_cast<uint2*>(xq_sm + (size_t)m * XS + 8 * cc) = qc;
+        }
+        // the 8 chunks of a group sit in 8 consecutive lanes (nch % 8 == 0)
+        sum = group8_sum(sum);
+        if ((lane & 7) == 0 && m < M) xs_sm[m * (GC + 1) + (cc >> 3)] = i32_to_f64(sum);
+        m += dm;
+        cc += dr;
+        if (cc >= nch) {
+          cc -= nch;
+          ++m;
+        }
       }
-      // the 8 chunks of a group sit in 8 consecutive lanes (nch % 8 == 0)
-      sum = group8_sum(sum);
-      if ((lane & 7) == 0 && c < total) xs_sm[m * (GC + 1) + (cc >> 3)] = i32_to_f64(sum);
     }
     __syncthreads();
   } else {
-    // quantized activations: the slice of xq, byte-permuted on the way in.
-    // Every global load of this stage (the group sums and sx too) is issued
-    // before any is used: one round trip to L2 instead of several.
-    const int nc16 = GC * 4;  // 16-byte chunks per row of the slice
-    const int total = M * nc16;
-    constexpr int kXs = 8;    // group sums per thread (M * GC <= 16 * 128 = 2048)
-    int xsv[kXs];
-#pragma unroll
-    for (int i = 0; i < kXs; ++i) {
-      const int idx = threadIdx.x + kThreads * i;
-      const int m = idx / GC, g = idx - (idx / GC) * GC;
-      xsv[i] = (kFold && idx < M * GC && g < gcount) ? __ldg(xsum + (size_t)m * G + g0 + g) : 0;
-    }
-    const float sxl = (kFold && (int)threadIdx.x < M) ? __ldg(sx + threadIdx.x) : 0.0f;
-    for (int base = 0; base < total; base += 8 * kThreads) {
-      uint4 v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int idx = base + threadIdx.x + kThreads * i;
-        if (idx < total) {
-          const int m = idx / nc16;
-          v[i] = __ldg(reinterpret_cast<const uint4*>(xq + (size_t)m * K + (size_t)g0 * 64) +
-                       (idx - m * nc16));
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int idx = base + threadIdx.x + kThreads * i;
-        if (idx < total) {
-          const int m = idx / nc16, cc = idx - m * nc16;
-          const uint2 a = even_odd(v[i].x, v[i].y), b = even_odd(v[i].z, v[i].w);
-          *reinterpret_cast<uint4*>(xq_sm + (size_t)m * XS + 16 * cc) =
-              make_uint4(a.x, a.y, b.x, b.y);
-        }
-      }
+    // quantized activations: the M rows of the slice by bulk copy (issued by
+    // one thread), the group sums and sx by plain loads meanwhile
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(abar, (uint32_t)(M * gcount * 64));
+      for (int m = 0; m < M; ++m)
+        bulk_load(smem_u32(xq_sm + (size_t)m * XS), xq + (size_t)m * K + (size_t)g0 * 64,
+                  (uint32_t)(gcount * 64), abar);
     }
     if (kFold) {
+      // (row, group) pairs by steps of kThreads (one division each)
+      const int dm = kThreads / GC, dg = kThreads - dm * GC;
+      int m = (int)threadIdx.x / GC, g = (int)threadIdx.x - m * GC;
+      constexpr int kXs = 8;    // M * GC <= kXs * kThreads in every plan with K <= 4096
+      int xv[kXs];
+      int mi[kXs], gi[kXs];
 #pragma unroll
       for (int i = 0; i < kXs; ++i) {
-        const int idx = threadIdx.x + kThreads * i;
-        if (idx < M * GC) xs_sm[(idx / GC) * (GC + 1) + idx % GC] = i32_to_f64(xsv[i]);
+        mi[i] = m;
+        gi[i] = g;
+        xv[i] = m < M ? __ldg(xsum + (size_t)m * G + g0 + g) : 0;
+        m += dm;
+        g += dg;
+        if (g >= GC) {
+          g -= GC;
+          ++m;
+        }
       }
-      if ((int)threadIdx.x < M) sx_sm[threadIdx.x] = sxl;
+      if ((int)threadIdx.x < M) sx_sm[threadIdx.x] = __ldg(sx + threadIdx.x);
+#pragma unroll
+      for (int i = 0; i < kXs; ++i)
+        if (mi[i] < M) xs_sm[mi[i] * (GC + 1) + gi[i]] = i32_to_f64(xv[i]);
+      // the rest (a larger K slice)
+      for (; m < M;) {
+        xs_sm[m * (GC + 1) + g] = i32_to_f64(__ldg(xsum + (size_t)m * G + g0 + g));
+        m += dm;
+        g += dg;
+        if (g >= GC) {
+          g -= GC;
+          ++m;
+        }
+      }
     }
+    // (if the rows never land the results are wrong and the error word is set)
+    __all_sync(0xFFFFFFFFu, mbar_wait(abar, 0, err));
     __syncthreads();
     if (C > 1) cluster_wait_acquire();  // the start barrier
   }
@@ -416,11 +440,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t offb = offa + 8u * 128u;
 
   // K map.  For group g, lane (grp, tq) handles the 16 consecutive codes
-  // k = 64 g + 16 tq + 0..15 (8 packed bytes).  Splitting a packed word into
-  // its low nibbles (codes 0, 2, 4, 6) and high nibbles (codes 1, 3, 5, 7)
-  // gives the A registers of one m16n8k32 MMA directly; xq was permuted to the
-  // same even / odd order, so each MMA sums the same 32 k on both sides, and
-  // the two MMAs of a group cover its 64 k once.
+  // k = 64 g + 16 tq + 0..15 (8 packed bytes, 16 bytes of xq).  The first MMA
+  // takes codes 0..7 of every lane's 16 (A: split_codes of the first packed
+  // word; B: xq bytes 0..7), the second codes 8..15, so each MMA sums the same
+  // 32 k on both sides and the two MMAs of a group cover its 64 k once.
   //
   // All kWarpGroups groups in straight-line code (no branch between them, so
   // the loads, MMAs and folds of different groups overlap); groups past gn
@@ -436,11 +459,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t sw = (uint32_t)(((2 * (gl & 3) + (tq >> 1)) ^ grp) << 4);
       const uint2 wa = *reinterpret_cast<const uint2*>(box + offa + sw);
       const uint2 wb = *reinterpret_cast<const uint2*>(box + offb + sw);
-      // A registers: {row grp, row grp + 8} x {even codes, odd codes}, per MMA
-      const uint32_t a0[4] = {wa.x & 0x0F0F0F0Fu, wb.x & 0x0F0F0F0Fu, (wa.x >> 4) & 0x0F0F0F0Fu,
-                              (wb.x >> 4) & 0x0F0F0F0Fu};
-      const uint32_t a1[4] = {wa.y & 0x0F0F0F0Fu, wb.y & 0x0F0F0F0Fu, (wa.y >> 4) & 0x0F0F0F0Fu,
-                              (wb.y >> 4) & 0x0F0F0F0Fu};
+      // A registers of the two MMAs: codes 0..7 and 8..15 of the lane's 16
+      uint32_t a0[4], a1[4];
+      split_codes(wa.x, wb.x, a0);
+      split_codes(wa.y, wb.y, a1);
       // two independent MMAs per token tile (half a group each), then one add
       int acc[TT][4];
 #pragma unroll
