@@ -296,11 +296,11 @@ qk_status qk_w8a8_linear_noalloc(const uint16_t *x, int64_t M, int64_t K,
  * otherwise the per-group fold kernel computes it.  The route allocates its
  * scratch (the planes, up to 3 N K bytes) stream-ordered from a memory pool of
  * the library that keeps freed blocks for reuse.
- * When also M <= 8 and each CTA's K slice of x fits its registers (M times
+ * When also M <= 6 and each CTA's K slice of x fits its registers (M times
  * the slice <= 16384 elements) the GEMV quantizes x itself (same rule and
  * codes as qk_quantize_activations) and the call is one kernel; the workspace
  * is then checked but not used (qk_w4a8_linear_plan tells which case
- * applies).  From 9 tokens on, the quantization kernel followed by the GEMV
+ * applies).  From 7 tokens on, the quantization kernel followed by the GEMV
  * on its codes is faster.
  *   x                  : bf16 bits [M, K]            (in)
  *   Wp, wscale, woffset: from qk_quantize_weights_int4 (in)

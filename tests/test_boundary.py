@@ -132,7 +132,9 @@ def test_w4a8_linear_plan(qk):
     for larger K at M <= 16, quantization + GEMM above M = 16."""
     assert qk.qk_w4a8_linear_plan(0, 64, 64) == qk.QK_PLAN_NONE
     assert qk.qk_w4a8_linear_plan(1, 4096, 4096) == qk.QK_PLAN_GEMV_QUANT
-    assert qk.qk_w4a8_linear_plan(8, 4096, 4096) == qk.QK_PLAN_GEMV_QUANT
+    assert qk.qk_w4a8_linear_plan(6, 4096, 4096) == qk.QK_PLAN_GEMV_QUANT
+    assert qk.qk_w4a8_linear_plan(7, 4096, 4096) == qk.QK_PLAN_QUANT_GEMV
+    assert qk.qk_w4a8_linear_plan(8, 4096, 4096) == qk.QK_PLAN_QUANT_GEMV
     assert qk.qk_w4a8_linear_plan(16, 4096, 4096) == qk.QK_PLAN_QUANT_GEMV
     assert qk.qk_w4a8_linear_plan(16, 3072, 128) == qk.QK_PLAN_QUANT_GEMV
     assert qk.qk_w4a8_linear_plan(12, 2112, 136) == qk.QK_PLAN_QUANT_GEMV

@@ -731,13 +731,13 @@ size_t gemv_smem_bytes(int64_t M, int64_t K, int64_t N) {
   return choose_plan(M, K, N, false, &p) ? p.smem : ~size_t(0);
 }
 
-// The in-kernel quantization pays off up to 8 tokens: at N = K = 4096 a
-// 16-token call takes 13.4 us quantizing in the kernel (clusters of four
-// exchanging the row maxima) against 12.1 us as the quantization kernel + the
-// GEMV on its codes; at 8 tokens 9.9 us against 10.6 us (graph-chained calls).
+// The in-kernel quantization pays off up to 6 tokens: at N = K = 4096
+// (graph-chained calls) 4 tokens take 8.4 us quantizing in the kernel against
+// 9.8 us as the quantization kernel + the GEMV on its codes, 6 tokens 9.5 us
+// both ways, and 8 tokens 9.6 us against 9.1 us.
 bool gemv_quant_fits(int64_t M, int64_t K, int64_t N) {
   GemvPlan p;
-  return M <= 8 && choose_plan(M, K, N, true, &p);
+  return M <= 6 && choose_plan(M, K, N, true, &p);
 }
 
 cudaError_t launch_w4a8_gemv(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,

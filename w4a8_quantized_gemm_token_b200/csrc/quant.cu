@@ -272,7 +272,16 @@ cudaError_t launch_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq
       default: return nullptr;
     }
   };
-  if (per_lane <= 1)
+  // Few rows (at most one block per SM either way): a whole block per row,
+  // so that each thread holds at most four chunks and the call's latency is
+  // one round of loads.
+  if (M <= 148 && nch >= 128 && nch <= 1024) {
+    const int cpt = (nch + 255) / 256;
+    kernel = cpt == 1 ? quant_act_split_kernel<8, 1>
+           : cpt == 2 ? quant_act_split_kernel<8, 2>
+           : cpt == 3 ? quant_act_split_kernel<8, 3> : quant_act_split_kernel<8, 4>;
+    rows_per_block = 1;
+  } else if (per_lane <= 1)
     kernel = quant_act_kernel<1>;
   else if (per_lane <= 2)
     kernel = quant_act_kernel<2>;
