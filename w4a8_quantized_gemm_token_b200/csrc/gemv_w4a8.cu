@@ -75,8 +75,9 @@ constexpr int kWarpGroups = 16;
 // M token rows.
 struct GemvLayout {
   int R, C, M, G, GC, RT, KW, GW, RO, Mp, XS, nbox;
-  size_t w, s16, xq, xs, sx, amx, bias, part, bars, total;
-  __host__ __device__ GemvLayout(int R_, int C_, int K, int M_) {
+  bool tab;                    // M <= 8 quantizing x in the kernel: fp64 scale table
+  size_t w, s16, xq, st, xs, sx, amx, bias, part, bars, total;
+  __host__ __device__ GemvLayout(int R_, int C_, int K, int M_, bool quant_x) {
     R = R_;
     C = C_;
     M = M_;
@@ -91,11 +92,22 @@ struct GemvLayout {
     // phase fall in opposite halves of the banks
     XS = (GC * 64 + 127) / 128 * 128 + 64;
     nbox = (GC + 3) / 4;       // 128-byte weight boxes per row of the slice
+    tab = quant_x && M <= 8;
     size_t off = 0;
     w = off;    off += (size_t)nbox * R * 128;        // packed codes, 128-byte-swizzled boxes
-    s16 = off;  off += (size_t)R * GC * 2 * 2;        // fp16 scales [R][GC], then offsets
-    off = (off + 127) & ~size_t(127);
-    xq = off;   off += (size_t)M * XS;                // xq rows of the slice (permuted)
+    s16 = off;                                        // fp16 scales [R][GC], then offsets
+    if (tab) {
+      // the fp16 scales are consumed into the table before the dependency
+      // wait; the xq rows land in the same bytes after it
+      xq = off; off += std::max((size_t)R * GC * 2 * 2, (size_t)M * XS);
+      off = (off + 15) & ~size_t(15);
+      st = off; off += (size_t)R * (GC + 1) * 8;      // {hi(s), hi(o)} [R][GC + 1]
+    } else {
+      off += (size_t)R * GC * 2 * 2;
+      off = (off + 127) & ~size_t(127);
+      xq = off; off += (size_t)M * XS;                // xq rows of the slice
+      st = off;
+    }
     off = (off + 15) & ~size_t(15);
     xs = off;   off += (size_t)Mp * (GC + 1) * 8;     // xsum as fp64, zero past M
     sx = off;   off += 16 * 4;                        // sx
@@ -128,6 +140,10 @@ __device__ __forceinline__ double i32_to_f64(int a) {
 __device__ __forceinline__ double h2d(uint16_t h) {
   return (double)__half2float(__ushort_as_half(h));
 }
+
+// An fp16 value widened to fp64 has a zero low word: the table keeps the
+// high words only.
+__device__ __forceinline__ double hi_to_f64(uint32_t hi) { return __hiloint2double((int)hi, 0); }
 
 // fp64 -> bf16 bits with one rounding to nearest-even (integer operations on
 // the bits for |v| >= 2^-126, round-to-odd into fp32 below).
@@ -196,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                      int early_trigger, int* err) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = align_smem<1024>(smem_raw);
-  const GemvLayout L(R, C, K, M);
+  const GemvLayout L(R, C, K, M, kQuantX);
   const int G = L.G, GC = L.GC, RT = L.RT, KW = L.KW, RO = L.RO, XS = L.XS;
   const int crank = (int)blockIdx.x;  // rank in the cluster = K slice
   const int n0 = (int)blockIdx.y * R;
@@ -258,8 +274,38 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int i = threadIdx.x; i < (L.Mp - M) * (GC + 1); i += kThreads)
     xs_sm[(size_t)M * (GC + 1) + i] = 0.0;
   if (threadIdx.x < 16) amx_sm[C * 16 + threadIdx.x] = 0u;
+  // M <= 8 quantizing x in the kernel: the scales and offsets widened to fp64
+  // (high words) in a table with rows padded to GC + 1 entries (the eight rows
+  // a warp reads at once fall in distinct banks), so the product loop
+  // converts nothing.  Built before the dependency wait (calls of this form
+  // follow one another, and the scales have long landed); the activation
+  // codes land on the fp16 scales after the wait.  (With xq from the
+  // quantization kernel in front, the GEMV starts too shortly before its
+  // release: waiting for the scales there, or building the table after the
+  // release, measured slower than converting in the loop.)
+  auto build_table = [&]() {
+    __all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, err));
+    uint2* stab = reinterpret_cast<uint2*>(smem + L.st);
+    const int dr = kThreads / GC, dg = kThreads - dr * GC;
+    int r = (int)threadIdx.x / GC, g = (int)threadIdx.x - r * GC;
+    while (r < R) {
+      stab[r * (GC + 1) + g] = make_uint2((uint32_t)__double2hiint(h2d(s16[r * GC + g])),
+                                          (uint32_t)__double2hiint(h2d(o16[r * GC + g])));
+      r += dr;
+      g += dg;
+      if (g >= GC) {
+        g -= GC;
+        ++r;
+      }
+    }
+  };
+  if constexpr (kFold && TT == 1 && kQuantX) {  // (exactly when L.tab)
+    __syncthreads();  // thread 0 has initialized the barriers
+    build_table();
+  }
   // peers write into this CTA's shared memory only after every CTA of the
-  // cluster has arrived here (it has started)
+  // cluster has arrived here (it has started); with the table, every thread
+  // is done with the fp16 scales before the activation rows overwrite them
   if (C > 1) cluster_arrive_relaxed();
   __syncthreads();
 
@@ -490,8 +536,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         A0[u] = acc[0][0];  // token 0 lives in the lanes with tq == 0
         A2[u] = acc[0][2];
       } else if (i < gn) {
-        const double sa = h2d(s16[ra * GC + gl]), sb = h2d(s16[(ra + 8) * GC + gl]);
-        const double oa = h2d(o16[ra * GC + gl]), ob = h2d(o16[(ra + 8) * GC + gl]);
+        double sa, sb, oa, ob;
+        if constexpr (TT == 1 && kQuantX) {
+          const uint2* stab = reinterpret_cast<const uint2*>(smem + L.st);
+          const uint2 ta = stab[ra * (GC + 1) + gl], tb = stab[(ra + 8) * (GC + 1) + gl];
+          sa = hi_to_f64(ta.x);
+          oa = hi_to_f64(ta.y);
+          sb = hi_to_f64(tb.x);
+          ob = hi_to_f64(tb.y);
+        } else {
+          sa = h2d(s16[ra * GC + gl]);
+          sb = h2d(s16[(ra + 8) * GC + gl]);
+          oa = h2d(o16[ra * GC + gl]);
+          ob = h2d(o16[(ra + 8) * GC + gl]);
+        }
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
           const double x0 = xs_sm[(tt * 8 + 2 * tq) * (GC + 1) + gl];
@@ -520,9 +578,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (ig < gn) {
         const int g = gbeg + ig;
         const double x0 = xs_sm[g];
-        fa = fma(h2d(o16[ra * GC + g]), x0, fma(h2d(s16[ra * GC + g]), i32_to_f64(s0), fa));
-        fb = fma(h2d(o16[(ra + 8) * GC + g]), x0,
-                 fma(h2d(s16[(ra + 8) * GC + g]), i32_to_f64(s2), fb));
+        if constexpr (kQuantX) {
+          const uint2* stab = reinterpret_cast<const uint2*>(smem + L.st);
+          const uint2 ta = stab[ra * (GC + 1) + g], tb = stab[(ra + 8) * (GC + 1) + g];
+          fa = fma(hi_to_f64(ta.y), x0, fma(hi_to_f64(ta.x), i32_to_f64(s0), fa));
+          fb = fma(hi_to_f64(tb.y), x0, fma(hi_to_f64(tb.x), i32_to_f64(s2), fb));
+        } else {
+          fa = fma(h2d(o16[ra * GC + g]), x0, fma(h2d(s16[ra * GC + g]), i32_to_f64(s0), fa));
+          fb = fma(h2d(o16[(ra + 8) * GC + g]), x0,
+                   fma(h2d(s16[(ra + 8) * GC + g]), i32_to_f64(s2), fb));
+        }
       }
     }
   }
@@ -601,7 +666,7 @@ bool choose_plan(int64_t M, int64_t K, int64_t N, bool quant_x, GemvPlan* out) {
     if (C > 1 && (G % C != 0 || (G / C) % 8 != 0)) continue;
     for (int R : {32, 64, 128}) {
       if (R / C < 16) continue;
-      const GemvLayout L(R, C, (int)K, (int)M);
+      const GemvLayout L(R, C, (int)K, (int)M, quant_x);
       if (L.total > (size_t)kSmemLimit || L.GW > kWarpGroups) continue;
       if (quant_x && M * L.GC * 64 > (int64_t)kQuantChunks * 8 * kThreads) continue;
       const long grid = (long)C * ((N + R - 1) / R);
