@@ -563,16 +563,22 @@ def table_entry(name, local, dev, peaks, int8):
                                              "traffic")},
            "sm_mhz": clocks["sm_mhz"], "reasons": clocks["reasons"]}
     if run.w4 and run.M > 16 and roof["bound"] == "tensor":
-        # the GEMM route runs P int8 GEMMs (the byte planes of the weight): the
-        # tensor pipe does P times the product's 2 M N K operations
+        # the GEMM route runs int8 GEMMs on the digit rows of the weight: P per
+        # weight row in tiles of 256 / P rows (64 for P = 3), or in the mixed
+        # layout 256 digit rows per tile of 120 weight rows; the tensor pipe
+        # does (digit rows / N) times the product's 2 M N K operations
         from w4a8_quantized_gemm_token_b200 import binding as qk
 
         _, s16, o16 = run.weights[0]
-        planes = qk.qk_debug_w4a8_plane_count(s16, o16, run.K)
+        planes, mixed = qk.qk_debug_w4a8_plane_count(s16, o16, run.K, with_mixed=True)
         rec["planes"] = planes
+        rec["mixed_layout"] = bool(mixed)
         if 1 <= planes <= 3:
-            rec["tensor_ops_per_call"] = planes * run.ops
-            rec["tensor_frac"] = planes * roof["achieved"] / roof["peak"]
+            tile = 120 if mixed else {1: 256, 2: 128, 3: 64}[planes]
+            rows = (256 if mixed else planes * tile) * (-(-run.N // tile))
+            rec["digit_rows"] = rows
+            rec["tensor_ops_per_call"] = rows / run.N * run.ops
+            rec["tensor_frac"] = rows / run.N * roof["achieved"] / roof["peak"]
     del run
     torch.cuda.empty_cache()
     return rec
