@@ -71,6 +71,8 @@ WORKLOADS = {
     "w4a8_m4096": ("W4A8", 3),
     "quickstart_w8a8": ("QUICKSTART", 0),
     "quickstart_w4a8": ("QUICKSTART", 1),
+    "w4a8_m4096_prepared": ("W4A8", 3),
+    "quickstart_w4a8_prepared": ("QUICKSTART", 1),
     "sage_attn": ("SAGE_QUICKSTART", None),
 }
 ATTN_METRIC = "INT8 attention TFLOP/s (4 B H L^2 D ops) at DiT shapes"
@@ -95,6 +97,12 @@ def is_attention(name):
 def is_fused(name):
     """The W8A8 linear as one kernel (qk_w8a8_linear_fused)."""
     return name.endswith("_fused")
+
+
+def is_prepared(name):
+    """The W4A8 linear on a prepared weight (qk_w4a8_prepare once, then
+    qk_w4a8_linear_prepared): the digit planes are not rebuilt per call."""
+    return name.endswith("_prepared")
 
 
 def is_gated(name):
@@ -307,6 +315,7 @@ class LinearRun:
         self.case = case = get_case(name)
         M, K, N = self.M, self.K, self.N = case.M, case.K, case.N
         self.w4, self.gated = is_w4(name), is_gated(name)
+        self.prepared = None
         xb, W, b, _ = case.draw()
         self.x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
         del xb
@@ -326,6 +335,8 @@ class LinearRun:
         if w4:
             self.weights = [qk.qk_quantize_weights_int4(W_dev) for _ in range(self.nsets)]
             wsz = qk.qk_w4a8_workspace_size(M, K)
+            self.prepared = ([qk.qk_w4a8_prepare(*wt)[0] for wt in self.weights]
+                             if is_prepared(name) else None)
         else:
             self.weights = [qk.qk_quantize_weights_int8(W_dev) for _ in range(self.nsets)]
             wsz = qk.qk_w8a8_workspace_size(M, K)
@@ -337,7 +348,10 @@ class LinearRun:
 
     def step(self, i):
         qk, wt, x = self.qk, self.weights[i % self.nsets], self.xs[i % self.nsets]
-        if self.w4:
+        if self.w4 and self.prepared is not None:
+            qk.qk_w4a8_linear_prepared(x, *wt, self.prepared[i % self.nsets], self.bias, y=self.y,
+                                       workspace=self.ws)
+        elif self.w4:
             qk.qk_w4a8_linear(x, *wt, self.bias, y=self.y, workspace=self.ws)
         elif self.gated:
             qk.qk_w8a8_linear_gated(x, *wt, self.bias, self.gate, self.res, y=self.y,
@@ -356,7 +370,10 @@ class LinearRun:
             self.xq_sets = [qk.qk_quantize_activations(x, with_xsum=self.w4) for x in self.xs]
         xq, sx, xsum = self.xq_sets[i % self.nsets]
         wt = self.weights[i % self.nsets]
-        if self.w4:
+        if self.w4 and self.prepared is not None:
+            qk.qk_w4a8_gemm_prepared(xq, sx, xsum, *wt, self.prepared[i % self.nsets], self.bias,
+                                     y=self.y)
+        elif self.w4:
             route = qk.QK_ROUTE_GEMV if self.M <= 16 else qk.QK_ROUTE_GEMM
             qk.qk_w4a8_gemm(xq, sx, xsum, *wt, self.bias, y=self.y, route=route)
         else:
@@ -380,16 +397,16 @@ class LinearRun:
         return ("w8a8_gemm_kernel", "gemm_w8a8.cu", "tensor", None)
 
 
-def launches_per_call(M, K, N, w4, gated, qk, fused=False):
+def launches_per_call(M, K, N, w4, gated, qk, fused=False, prepared=False):
     """Kernels one call of the linear launches: the W8A8 linear is the
     quantization kernel + the GEMM (qk_w8a8_linear_fused: one kernel, except
     for thin outputs, N <= 64); the W4A8 linear follows its plan
     (qk_w4a8_linear_plan); its GEMM route is four kernels (the plane count,
     the plane build, the per-group fold that computes only when the byte
-    planes cannot, and the byte-plane GEMM)."""
+    planes cannot, and the byte-plane GEMM), two on a prepared weight."""
     if w4:
         plan = qk.qk_w4a8_linear_plan(M, K, N)
-        return {qk.QK_PLAN_GEMV_QUANT: 1, qk.QK_PLAN_QUANT_GEMV: 2}.get(plan, 5)
+        return {qk.QK_PLAN_GEMV_QUANT: 1, qk.QK_PLAN_QUANT_GEMV: 2}.get(plan, 3 if prepared else 5)
     if gated or not fused or (N <= 64 and M <= 8192):
         return 2
     return 1
@@ -527,7 +544,8 @@ def measure_sustained(run, local, seconds, int8, peaks):
 # gated residual epilogue and the INT8 attention.
 TABLE = ["tiny", "dit_attn", "sweep_4096x4096", "sweep_4096x12288", "sweep_12288x4096",
          "sweep_thin_5120x48", "w4a8_m1", "w4a8_m8", "w4a8_m16", "w4a8_m4096",
-         "quickstart_w8a8", "quickstart_w4a8", "dit_mlp_gated", "sage_attn",
+         "quickstart_w8a8", "quickstart_w4a8", "w4a8_m4096_prepared", "quickstart_w4a8_prepared",
+         "dit_mlp_gated", "sage_attn",
          "dit_mlp_fused", "dit_attn_fused", "quickstart_w8a8_fused"]
 
 
@@ -554,7 +572,8 @@ def table_entry(name, local, dev, peaks, int8):
     roof = roofline(run, k_ms, peaks, int8, name)
     per = ms / steps
     rec = {"config": run.case.name + ("_gated_residual" if run.gated else "")
-                     + ("_one_kernel" if is_fused(name) else ""),
+                     + ("_one_kernel" if is_fused(name) else "")
+                     + ("_prepared_weight" if is_prepared(name) else ""),
            "M": run.M, "K": run.K, "N": run.N, "steps": steps, "timing": timing,
            "ms_per_call": per, "value": run.ops / (per / 1e3) / 1e12, "unit": "TOPS",
            "pct_of_int8_spec": 100.0 * run.ops / (per / 1e3) / 1e12 / INT8_SPEC_TOPS,
@@ -751,8 +770,10 @@ def run_ours(args, world, rank, local):
     sustained = None
     if single and not args.no_sustained and not w4 and M > 256:
         sustained = measure_sustained(run, local, 2.0, int8, peaks)
-    launches = launches_per_call(M, K, N, w4, gated, run.qk, is_fused(args.workload))
-    config = {"workload": run.case.name + ("_gated_residual" if gated else ""),
+    launches = launches_per_call(M, K, N, w4, gated, run.qk, is_fused(args.workload),
+                                 is_prepared(args.workload))
+    config = {"workload": run.case.name + ("_gated_residual" if gated else "")
+                          + ("_prepared_weight" if is_prepared(args.workload) else ""),
               "M": M, "K": K, "N": N,
               "weights": "W4 affine g64" if w4 else "W8 per-channel",
               "bias": run.bias is not None,
@@ -928,7 +949,8 @@ def run_reference(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": case.name + ("_gated_residual" if is_gated(args.workload) else ""),
+        "config": {"workload": case.name + ("_gated_residual" if is_gated(args.workload) else "")
+                               + ("_prepared_weight" if is_prepared(args.workload) else ""),
                    "M": case.M, "K": case.K, "N": case.N},
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
                          "sample": sample, "cpu_model": cpu_model()},

@@ -349,6 +349,59 @@ qk_status qk_w4a8_gemm(const int8_t *xq, const float *sx, const int32_t *xsum,
                        const float *bias, int64_t N, uint16_t *y, int route,
                        qk_stream_t stream);
 
+/*
+ * A prepared W4A8 weight, for weights that do not change between calls (the
+ * usual inference case).  The GEMM route of qk_w4a8_linear (M > 16) first
+ * counts the digit planes of the weight and writes them to a scratch (see
+ * qk_w4a8_linear); qk_w4a8_prepare does that once into caller-owned device
+ * memory, and the _prepared products below then launch only the activation
+ * quantization, the gated per-group fold and the plane GEMM, with the same
+ * results bit for bit as qk_w4a8_linear / qk_w4a8_gemm.  (The pages' W4 path
+ * unpacks the weight per call; this keeps the unpacked form instead.)
+ *
+ * qk_w4a8_prepared_size: bytes of the prepared form of an [N, K] weight (the
+ * plane-count words, e_n and the top-digit slot of every row, and up to
+ * 3 N K bytes of digit rows), or 0 for an unsupported shape (N % 8 != 0,
+ * K % 64 != 0, K outside [64, 65536]).
+ *
+ * qk_w4a8_prepare: writes the prepared form of (Wp, wscale, woffset) to
+ * `prepared` (device, 256-byte aligned, >= qk_w4a8_prepared_size(N, K)
+ * bytes, owned by the caller and read by every later _prepared call: it must
+ * not be written or freed while one is in flight, and must be prepared again
+ * after the weight changes).  `planes` (host, nullable): when given, the call
+ * synchronizes `stream` and writes the digit-plane count there (1..3; 255
+ * when the per-group fold computes the product).  Errors: QK_ERR_INVALID_ARG
+ * (NULL pointers), QK_ERR_UNSUPPORTED_SHAPE, QK_ERR_MISALIGNED (inputs not
+ * 16-byte or `prepared` not 256-byte aligned), QK_ERR_WORKSPACE (`bytes` too
+ * small).
+ *
+ * qk_w4a8_gemm_prepared / qk_w4a8_linear_prepared: as qk_w4a8_gemm with
+ * QK_ROUTE_AUTO / qk_w4a8_linear, with `prepared` (from qk_w4a8_prepare on
+ * the same Wp, wscale, woffset, N, K) serving the GEMM route; M <= 16 takes the
+ * same GEMV as there (`prepared` is then not read).  Same errors as those
+ * calls, plus QK_ERR_INVALID_ARG for a NULL `prepared` and QK_ERR_MISALIGNED
+ * for one not 256-byte aligned.
+ */
+size_t qk_w4a8_prepared_size(int64_t N, int64_t K);
+
+qk_status qk_w4a8_prepare(const uint8_t *Wp, const uint16_t *wscale, const uint16_t *woffset,
+                          int64_t N, int64_t K, void *prepared, size_t bytes, int *planes,
+                          qk_stream_t stream);
+
+qk_status qk_w4a8_gemm_prepared(const int8_t *xq, const float *sx, const int32_t *xsum,
+                                int64_t M, int64_t K,
+                                const uint8_t *Wp, const uint16_t *wscale,
+                                const uint16_t *woffset, const void *prepared,
+                                const float *bias, int64_t N, uint16_t *y,
+                                qk_stream_t stream);
+
+qk_status qk_w4a8_linear_prepared(const uint16_t *x, int64_t M, int64_t K,
+                                  const uint8_t *Wp, const uint16_t *wscale,
+                                  const uint16_t *woffset, const void *prepared,
+                                  const float *bias, int64_t N,
+                                  uint16_t *y, void *workspace, size_t ws_bytes,
+                                  qk_stream_t stream);
+
 /* ---------------------------------------------------------------- errors */
 
 /*

@@ -145,3 +145,38 @@ def test_w4a8_linear_plan(qk):
     with pytest.raises(qk.QKError) as e:
         qk.qk_w4a8_linear_plan(8, 96, 64)  # K % 64 != 0
     assert e.value.status == 2
+
+
+def test_prepared_w4a8_arguments(qk):
+    """The prepared-weight calls: the size follows the route's scratch layout,
+    and shapes, pointers, alignment (256 bytes for the prepared form) and the
+    buffer size are checked on the host; valid arguments stop at the device
+    check here."""
+    import torch
+
+    r = lambda b: (b + 255) // 256 * 256
+    N, K = 264, 1024
+    size = r(16) + r(N * 4) + r(N * 4) + r(-(-N // 60) * 8) + 3 * N * K
+    assert qk.qk_w4a8_prepared_size(N, K) == size
+    assert qk.qk_w4a8_prepared_size(N, 96) == 0        # K % 64 != 0
+    assert qk.qk_w4a8_prepared_size(12, K) == 0        # N % 8 != 0
+    planes = ctypes.byref(ctypes.c_int())
+    prep = qk.lib.qk_w4a8_prepare
+    assert prep(FAKE, FAKE, FAKE, N, 96, FAKE, size, planes, None) == 2
+    assert prep(None, FAKE, FAKE, N, K, FAKE, size, planes, None) == 1
+    assert prep(FAKE, FAKE, FAKE, N, K, None, size, planes, None) == 1
+    assert prep(FAKE, FAKE, FAKE, N, K, FAKE + 16, size, planes, None) == 3
+    assert prep(FAKE, FAKE + 2, FAKE, N, K, FAKE, size, planes, None) == 3
+    assert prep(FAKE, FAKE, FAKE, N, K, FAKE, size - 1, planes, None) == 5
+    gp = qk.lib.qk_w4a8_gemm_prepared
+    assert gp(FAKE, FAKE, FAKE, 32, K, FAKE, FAKE, FAKE, None, None, N, FAKE, None) == 1
+    assert gp(FAKE, FAKE, FAKE, 32, K, FAKE, FAKE, FAKE, FAKE + 16, None, N, FAKE, None) == 3
+    assert gp(None, None, None, 0, K, None, None, None, None, None, N, None, None) == 0  # M = 0
+    lp = qk.lib.qk_w4a8_linear_prepared
+    assert lp(FAKE, 32, K, FAKE, FAKE, FAKE, None, None, N, FAKE, None, 0, None) == 1
+    assert lp(FAKE, 32, K, FAKE, FAKE, FAKE, FAKE + 16, None, N, FAKE, None, 0, None) == 3
+    assert lp(FAKE, 32, 96, FAKE, FAKE, FAKE, FAKE, None, N, FAKE, None, 0, None) == 2
+    if not torch.cuda.is_available():
+        assert prep(FAKE, FAKE, FAKE, N, K, FAKE, size, planes, None) == 4
+        assert gp(FAKE, FAKE, FAKE, 32, K, FAKE, FAKE, FAKE, FAKE, None, N, FAKE, None) == 4
+        assert lp(FAKE, 32, K, FAKE, FAKE, FAKE, FAKE, None, N, FAKE, None, 0, None) == 4

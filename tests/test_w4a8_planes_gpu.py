@@ -319,3 +319,42 @@ def test_epilogue_fast_path_many_outputs(qk, orc):
     y_f = qk.qk_w4a8_gemm(xq, sx, xsum, *dw, to_dev(b), route=FOLD)
     assert torch.equal(y_g.view(torch.int16), y_f.view(torch.int16))
     qk.qk_check_device_error()
+
+
+@pytest.mark.parametrize("kind", ["gauss", "unit", "p3", "fold", "negscale"])
+def test_prepared_weight(qk, orc, kind):
+    """The prepared form (qk_w4a8_prepare once, then the _prepared products)
+    gives the same bits as the per-call route for every plane count and the
+    fold fallback, on quantized and on bf16 activations, for a small-M (GEMV)
+    call too; preparing a second weight into the same (garbage-filled) buffer
+    leaves nothing of the first."""
+    M, K, N = 300, 1024, 264
+    other = "p3" if kind != "p3" else "gauss"
+    Wp0, s0, o0, _ = make_weights(orc, other, N, K, seed=91)
+    Wp, s16, o16, allowed = make_weights(orc, kind, N, K, seed=90 + len(kind))
+    expect = host_plane_count(s16, o16, K)
+    dw0 = (to_dev(Wp0), dev_fp16(s0), dev_fp16(o0))
+    dw = (to_dev(Wp), dev_fp16(s16), dev_fp16(o16))
+    buf = torch.randint(0, 256, (qk.qk_w4a8_prepared_size(N, K),), dtype=torch.uint8,
+                        device="cuda")
+    qk.qk_w4a8_prepare(*dw0, prepared=buf)
+    prepared, planes = qk.qk_w4a8_prepare(*dw, prepared=buf)
+    assert planes == (expect if 1 <= expect <= 3 else 255)
+    case = synthetic.LinearCase("pr", M=M, K=K, N=N, bias=True, seed=M + N + len(kind))
+    xb, _, b, _ = case.draw()
+    x = to_dev_bf16(xb)
+    bias = to_dev(b)
+    y_lin = qk.qk_w4a8_linear(x, *dw, bias)
+    y_pre = qk.qk_w4a8_linear_prepared(x, *dw, prepared, bias)
+    xq, sx, xsum = qk.qk_quantize_activations(x, with_xsum=True)
+    y_gem = qk.qk_w4a8_gemm(xq, sx, xsum, *dw, bias, route=GEMM)
+    y_gpr = qk.qk_w4a8_gemm_prepared(xq, sx, xsum, *dw, prepared, bias)
+    x8 = x[:8].contiguous()
+    y8 = qk.qk_w4a8_linear_prepared(x8, *dw, prepared, bias)
+    y8_lin = qk.qk_w4a8_linear(x8, *dw, bias)
+    torch.cuda.synchronize()
+    for a, c in ((y_pre, y_lin), (y_gpr, y_gem), (y_pre, y_gem), (y8, y8_lin)):
+        assert torch.equal(a.view(torch.int16), c.view(torch.int16)), kind
+    y_o, _, _, _, _ = orc.w4a8_linear(xb, Wp, s16, o16, b)
+    assert bf16_ulp_distance(t2bits(y_pre), y_o).max() <= TOL_ULP
+    qk.qk_check_device_error()

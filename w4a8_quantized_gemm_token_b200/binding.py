@@ -39,6 +39,11 @@ _SIGS = {
     "qk_w4a8_linear": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w4a8_gemm": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I, _P]),
     "qk_w4a8_linear_plan": (_I, [_I64, _I64, _I64]),
+    "qk_w4a8_prepared_size": (_SZ, [_I64, _I64]),
+    "qk_w4a8_prepare": (_I, [_P, _P, _P, _I64, _I64, _P, _SZ, _P, _P]),
+    "qk_w4a8_gemm_prepared": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P]),
+    "qk_w4a8_linear_prepared": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ,
+                                     _P]),
     "qk_check_device_error": (_I, [_P]),
     "qk_debug_w8a8_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P]),
     "qk_debug_w4a8_group_acc": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I, _P]),
@@ -242,6 +247,71 @@ def qk_w4a8_linear(x, Wp, wscale, woffset, bias=None, y=None, workspace=None, st
     _check(lib.qk_w4a8_linear(_ptr(x), M, K, _ptr(Wp), _ptr(wscale), _ptr(woffset), _ptr(bias),
                               N, _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
            "qk_w4a8_linear")
+    return y
+
+
+def qk_w4a8_prepared_size(N: int, K: int) -> int:
+    return int(lib.qk_w4a8_prepared_size(int(N), int(K)))
+
+
+def qk_w4a8_prepare(Wp, wscale, woffset, prepared=None, stream=None):
+    """(prepared uint8 tensor, plane count): the GEMM route's digit planes of
+    the weight, built once for the _prepared calls (plane count 1..3, or 255
+    when the per-group fold computes the product)."""
+    _need(Wp, torch.uint8, 2, "Wp")
+    _need(wscale, torch.float16, 2, "wscale")
+    _need(woffset, torch.float16, 2, "woffset")
+    N, K = Wp.shape[0], Wp.shape[1] * 2
+    if prepared is None:
+        size = lib.qk_w4a8_prepared_size(N, K)
+        prepared = torch.empty(max(int(size), 1), dtype=torch.uint8, device=Wp.device)
+    else:
+        _need(prepared, torch.uint8, 1, "prepared")
+    planes = ctypes.c_int(0)
+    _check(lib.qk_w4a8_prepare(_ptr(Wp), _ptr(wscale), _ptr(woffset), N, K, _ptr(prepared),
+                               prepared.numel(), ctypes.byref(planes), _stream(stream)),
+           "qk_w4a8_prepare")
+    return prepared, int(planes.value)
+
+
+def qk_w4a8_linear_prepared(x, Wp, wscale, woffset, prepared, bias=None, y=None, workspace=None,
+                            stream=None):
+    _need(x, torch.bfloat16, 2, "x")
+    _need(Wp, torch.uint8, 2, "Wp")
+    _need(wscale, torch.float16, 2, "wscale")
+    _need(woffset, torch.float16, 2, "woffset")
+    _need(prepared, torch.uint8, 1, "prepared")
+    if bias is not None:
+        _need(bias, torch.float32, 1, "bias")
+    M, K = x.shape
+    N = Wp.shape[0]
+    y = _out(y, (M, N), torch.bfloat16, x.device, "y")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qk_w4a8_linear_prepared(_ptr(x), M, K, _ptr(Wp), _ptr(wscale), _ptr(woffset),
+                                       _ptr(prepared), _ptr(bias), N, _ptr(y), _ptr(workspace),
+                                       ws_bytes, _stream(stream)),
+           "qk_w4a8_linear_prepared")
+    return y
+
+
+def qk_w4a8_gemm_prepared(xq, sx, xsum, Wp, wscale, woffset, prepared, bias=None, y=None,
+                          stream=None):
+    _need(xq, torch.int8, 2, "xq")
+    _need(sx, torch.float32, 1, "sx")
+    _need(xsum, torch.int32, 2, "xsum")
+    _need(Wp, torch.uint8, 2, "Wp")
+    _need(wscale, torch.float16, 2, "wscale")
+    _need(woffset, torch.float16, 2, "woffset")
+    _need(prepared, torch.uint8, 1, "prepared")
+    if bias is not None:
+        _need(bias, torch.float32, 1, "bias")
+    M, K = xq.shape
+    N = Wp.shape[0]
+    y = _out(y, (M, N), torch.bfloat16, xq.device, "y")
+    _check(lib.qk_w4a8_gemm_prepared(_ptr(xq), _ptr(sx), _ptr(xsum), M, K, _ptr(Wp),
+                                     _ptr(wscale), _ptr(woffset), _ptr(prepared), _ptr(bias), N,
+                                     _ptr(y), _stream(stream)),
+           "qk_w4a8_gemm_prepared")
     return y
 
 

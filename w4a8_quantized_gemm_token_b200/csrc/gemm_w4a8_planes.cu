@@ -424,10 +424,6 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   nb = r / gm;
 }
 
-__device__ __forceinline__ double i32_to_f64(uint32_t a) {
-  return __hiloint2double(0x43300000, (int)(a ^ 0x80000000u)) - 4503601774854144.0;
-}
-
 // fp64 -> bf16 bits, one rounding to nearest-even (as in gemm_w8a8.cu).
 __device__ __forceinline__ uint32_t f64_to_bf16_bits(double v) {
   const uint32_t hi = (uint32_t)__double2hiint(v);
@@ -967,50 +963,88 @@ struct PlaneScratch {
 
 size_t w4a8_plane_scratch_bytes(int64_t N, int64_t K) { return PlaneScratch(N, K).total; }
 
-cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
-                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
-                             const float* bias, int64_t N, uint16_t* y, void* scratch, bool pdl,
-                             cudaStream_t s) {
-  const PlaneScratch L(N, K);
-  uint8_t* base = static_cast<uint8_t*>(scratch);
-  auto* pword = reinterpret_cast<unsigned long long*>(base + L.words);
-  auto* oword = pword + 1;
-  auto* ebase = reinterpret_cast<int*>(base + L.ebase);
-  auto* slot = reinterpret_cast<int*>(base + L.slot);
-  auto* hcount = reinterpret_cast<unsigned long long*>(base + L.hcount);
-  uint8_t* planes = base + L.planes;
-  const unsigned long long epoch = next_epoch();
-  auto launch = [&](auto kernel, dim3 grid, dim3 block, size_t smem, bool dep, auto... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = dep ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
-  };
+namespace {
+
+// The words of a prepared weight carry this fixed epoch: qk_w4a8_prepare
+// zeroes them before counting, so no word of an earlier preparation of the
+// same buffer survives, and every product with the prepared form passes it.
+constexpr unsigned long long kPreparedEpoch = 1;
+
+struct PlanePtrs {
+  unsigned long long* pword;
+  unsigned long long* oword;
+  int* ebase;
+  int* slot;
+  unsigned long long* hcount;
+  uint8_t* planes;
+  PlanePtrs(const void* scratch, int64_t N, int64_t K) {
+    const PlaneScratch L(N, K);
+    uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(scratch));
+    pword = reinterpret_cast<unsigned long long*>(base + L.words);
+    oword = pword + 1;
+    ebase = reinterpret_cast<int*>(base + L.ebase);
+    slot = reinterpret_cast<int*>(base + L.slot);
+    hcount = reinterpret_cast<unsigned long long*>(base + L.hcount);
+    planes = base + L.planes;
+  }
+};
+
+template <typename Kernel, typename... Args>
+cudaError_t launch_ex(Kernel kernel, dim3 grid, dim3 block, size_t smem, bool dep, cudaStream_t s,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dep ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// The plane count (e_n, the slots, the plane-count word) and the digit rows
+// of a weight, tagged with `epoch`.
+cudaError_t launch_count_build(const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                               int64_t N, int64_t K, void* scratch, unsigned long long epoch,
+                               bool pdl, cudaStream_t s) {
+  const PlanePtrs P(scratch, N, K);
   // 1. plane count and e_n
-  cudaError_t e = launch(w4a8_plane_count_kernel,
-                         dim3((unsigned)((N + kCountRowsPerBlock - 1) / kCountRowsPerBlock)),
-                         dim3(32 * kCountRowsPerBlock), 0, pdl, ws, wo, (int)N, (int)K, ebase,
-                         slot, hcount, pword, oword, epoch);
+  cudaError_t e = launch_ex(w4a8_plane_count_kernel,
+                            dim3((unsigned)((N + kCountRowsPerBlock - 1) / kCountRowsPerBlock)),
+                            dim3(32 * kCountRowsPerBlock), 0, pdl, s, ws, wo, (int)N, (int)K,
+                            P.ebase, P.slot, P.hcount, P.pword, P.oword, epoch);
   if (e != cudaSuccess) return e;
   // 2. the planes (a few waves of the SMs; each thread loops over 16-code units)
   const long long units = N * (K / 16);
   long long blocks = (units + kBuildThreads - 1) / kBuildThreads;
   const long long cap = 8ll * num_sms();
-  e = launch(w4a8_plane_build_kernel, dim3((unsigned)(blocks < cap ? blocks : cap)),
-             dim3(kBuildThreads), 0, true, Wp, ws, wo, (const int*)ebase, (const int*)slot,
-             (int)N, (int)K, planes, (const unsigned long long*)pword,
-             (const unsigned long long*)oword, epoch);
-  if (e != cudaSuccess) return e;
+  return launch_ex(w4a8_plane_build_kernel, dim3((unsigned)(blocks < cap ? blocks : cap)),
+                   dim3(kBuildThreads), 0, true, s, Wp, ws, wo, (const int*)P.ebase,
+                   (const int*)P.slot, (int)N, (int)K, P.planes,
+                   (const unsigned long long*)P.pword, (const unsigned long long*)P.oword,
+                   epoch);
+}
+
+// The product on counted and built planes: the per-group fold (it computes
+// only when the planes cannot serve; launched as a programmatic dependent when
+// fold_dep), then the plane GEMM.
+cudaError_t launch_plane_product(const int8_t* xq, const float* sx, const int32_t* xsum,
+                                 int64_t M, int64_t K, const uint8_t* Wp, const uint16_t* ws,
+                                 const uint16_t* wo, const float* bias, int64_t N, uint16_t* y,
+                                 const void* scratch, unsigned long long epoch, bool fold_dep,
+                                 cudaStream_t s) {
+  const PlanePtrs P(scratch, N, K);
+  const unsigned long long* pword = P.pword;
+  const unsigned long long* oword = P.oword;
+  const int* ebase = P.ebase;
+  const int* slot = P.slot;
+  const uint8_t* planes = P.planes;
   // 3. the per-group fold, which computes only when the planes cannot
-  e = launch_w4a8_fold(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, true, s, pword,
-                       epoch);
+  cudaError_t e = launch_w4a8_fold(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0,
+                                   fold_dep, s, pword, epoch);
   if (e != cudaSuccess) return e;
   // 4. the plane GEMM
   CUtensorMap tA, tB, tB40, tB8, tY, tY56;
@@ -1048,11 +1082,49 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
   // a raster group's rows of xq (256 rows x K bytes per M tile) stay in L2
   long long group_m = (40ll << 20) / (2 * BM * K);
   group_m = group_m < 1 ? 1 : (group_m > tiles_m ? tiles_m : group_m);
-  return launch(w4a8_planes_kernel, dim3(grid), dim3(kThreads), (size_t)SMEM_ALLOC, true, tA, tB,
-                tB40, tB8, tY, tY56, sx, (const int*)ebase, (const int*)slot, bias, (int)M, (int)N,
-                (int)K, (int)group_m, (const unsigned long long*)pword,
-                (const unsigned long long*)oword, epoch, err);
+  return launch_ex(w4a8_planes_kernel, dim3(grid), dim3(kThreads), (size_t)SMEM_ALLOC, true, s,
+                   tA, tB, tB40, tB8, tY, tY56, sx, ebase, slot, bias, (int)M, (int)N, (int)K,
+                   (int)group_m, pword, oword, epoch, err);
 }
+
+}  // namespace
+
+cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* xsum, int64_t M,
+                             int64_t K, const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                             const float* bias, int64_t N, uint16_t* y, void* scratch, bool pdl,
+                             cudaStream_t s) {
+  const unsigned long long epoch = next_epoch();
+  cudaError_t e = launch_count_build(Wp, ws, wo, N, K, scratch, epoch, pdl, s);
+  if (e != cudaSuccess) return e;
+  return launch_plane_product(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, scratch, epoch, true,
+                              s);
+}
+
+cudaError_t launch_w4a8_prepare(const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                                int64_t N, int64_t K, void* prepared, int* planes,
+                                cudaStream_t s) {
+  const PlaneScratch L(N, K);
+  // zero the words, e_n, the slots and the slot counters (not the planes)
+  cudaError_t e = cudaMemsetAsync(prepared, 0, L.planes, s);
+  if (e != cudaSuccess) return e;
+  e = launch_count_build(Wp, ws, wo, N, K, prepared, kPreparedEpoch, false, s);
+  if (e != cudaSuccess || planes == nullptr) return e;
+  unsigned long long word = 0;
+  e = cudaMemcpyAsync(&word, prepared, sizeof(word), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) *planes = (word >> 8) == kPreparedEpoch ? (int)(word & 0xFFull) : 0;
+  return e;
+}
+
+cudaError_t launch_w4a8_gemm_prepared(const int8_t* xq, const float* sx, const int32_t* xsum,
+                                      int64_t M, int64_t K, const uint8_t* Wp,
+                                      const uint16_t* ws, const uint16_t* wo,
+                                      const void* prepared, const float* bias, int64_t N,
+                                      uint16_t* y, bool pdl, cudaStream_t s) {
+  return launch_plane_product(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, prepared,
+                              kPreparedEpoch, pdl, s);
+}
+
 
 cudaError_t launch_w4a8_plane_count(const uint16_t* ws, const uint16_t* wo, int64_t N, int64_t K,
                                     void* scratch, unsigned long long epoch, bool pdl,

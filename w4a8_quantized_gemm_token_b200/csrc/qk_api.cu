@@ -472,6 +472,93 @@ qk_status qk_w4a8_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
                    "w4a8");
 }
 
+// ---- prepared W4A8 weights (the GEMM route's digit planes built once)
+
+static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+static cudaError_t run_w4a8_prepared(const int8_t* xq, const float* sx, const int32_t* xsum,
+                                     int64_t M, int64_t K, const uint8_t* Wp, const uint16_t* ws,
+                                     const uint16_t* wo, const void* prepared, const float* bias,
+                                     int64_t N, uint16_t* y, bool pdl, cudaStream_t s) {
+  const bool gemv = w4a8_takes_gemv(QK_ROUTE_AUTO, M, K, N);
+  if (log_enabled())
+    std::fprintf(stderr, "[qk] w4a8 M=%lld K=%lld N=%lld -> %s\n", (long long)M, (long long)K,
+                 (long long)N, gemv ? "GEMV" : "tcgen05 GEMM, prepared byte planes");
+  if (gemv)
+    return launch_w4a8_gemv(xq, sx, xsum, M, K, Wp, ws, wo, bias, N, y, nullptr, 0, 0, pdl, s);
+  return launch_w4a8_gemm_prepared(xq, sx, xsum, M, K, Wp, ws, wo, prepared, bias, N, y, pdl, s);
+}
+
+size_t qk_w4a8_prepared_size(int64_t N, int64_t K) {
+  if (check_shape(1, K, N, true) != QK_OK) return 0;
+  return w4a8_plane_scratch_bytes(N, K);
+}
+
+qk_status qk_w4a8_prepare(const uint8_t* Wp, const uint16_t* wscale, const uint16_t* woffset,
+                          int64_t N, int64_t K, void* prepared, size_t bytes, int* planes,
+                          qk_stream_t stream) {
+  qk_status st = check_shape(1, K, N, true);
+  if (st != QK_OK) return st;
+  if (!Wp || !wscale || !woffset || !prepared) return QK_ERR_INVALID_ARG;
+  if (!aligned16(Wp) || !aligned16(wscale) || !aligned16(woffset) || !aligned256(prepared))
+    return QK_ERR_MISALIGNED;
+  if (bytes < w4a8_plane_scratch_bytes(N, K)) return QK_ERR_WORKSPACE;
+  if ((st = check_device()) != QK_OK) return st;
+  int p = 0;
+  st = from_cuda(launch_w4a8_prepare(Wp, wscale, woffset, N, K, prepared,
+                                     planes != nullptr ? &p : nullptr, stream),
+                 "w4a8 prepare");
+  if (st == QK_OK && planes != nullptr) *planes = (p >= 1 && p <= 3) ? p : 255;
+  return st;
+}
+
+qk_status qk_w4a8_gemm_prepared(const int8_t* xq, const float* sx, const int32_t* xsum,
+                                int64_t M, int64_t K, const uint8_t* Wp, const uint16_t* wscale,
+                                const uint16_t* woffset, const void* prepared, const float* bias,
+                                int64_t N, uint16_t* y, qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, true);
+  if (st != QK_OK || M == 0) return st;
+  if (!xq || !sx || !xsum || !prepared) return QK_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(xsum) || !aligned256(prepared))
+    return QK_ERR_MISALIGNED;
+  if ((st = check_w4_product(Wp, wscale, woffset, bias, y)) != QK_OK) return st;
+  if ((st = check_device()) != QK_OK) return st;
+  return from_cuda(run_w4a8_prepared(xq, sx, xsum, M, K, Wp, wscale, woffset, prepared, bias, N,
+                                     y, true, stream),
+                   "w4a8 prepared");
+}
+
+qk_status qk_w4a8_linear_prepared(const uint16_t* x, int64_t M, int64_t K, const uint8_t* Wp,
+                                  const uint16_t* wscale, const uint16_t* woffset,
+                                  const void* prepared, const float* bias, int64_t N,
+                                  uint16_t* y, void* workspace, size_t ws_bytes,
+                                  qk_stream_t stream) {
+  qk_status st = check_shape(M, K, N, true);
+  if (st != QK_OK || M == 0) return st;
+  if (!x || !prepared) return QK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned256(prepared)) return QK_ERR_MISALIGNED;
+  if ((st = check_w4_product(Wp, wscale, woffset, bias, y)) != QK_OK) return st;
+  if ((st = check_device()) != QK_OK) return st;
+  if (gemv_quant_fits(M, K, N)) {
+    // small M: as qk_w4a8_linear (the GEMV quantizes x itself; `prepared` unused)
+    if (workspace != nullptr && (ws_bytes < qk_w4a8_workspace_size(M, K) ||
+                                 (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+      return QK_ERR_WORKSPACE;
+    return from_cuda(launch_w4a8_gemv_quant(x, M, K, Wp, wscale, woffset, bias, N, y, true,
+                                            stream),
+                     "w4a8 gemv");
+  }
+  Workspace ws;
+  if ((st = ws.init(workspace, ws_bytes, M, K, true, stream)) != QK_OK) return st;
+  const bool pdl_quant = !w4a8_takes_gemv(QK_ROUTE_AUTO, M, K, N);  // as in qk_w4a8_linear
+  if ((st = from_cuda(launch_quant_act(x, M, K, ws.xq, ws.sx, ws.xsum, stream, pdl_quant),
+                      "quant_act")) != QK_OK)
+    return st;
+  return from_cuda(run_w4a8_prepared(ws.xq, ws.sx, ws.xsum, M, K, Wp, wscale, woffset, prepared,
+                                     bias, N, y, true, stream),
+                   "w4a8 prepared");
+}
+
 qk_status qk_check_device_error(qk_stream_t stream) {
   qk_status st = check_device();
   if (st != QK_OK) return st;

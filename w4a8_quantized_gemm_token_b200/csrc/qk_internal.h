@@ -113,6 +113,22 @@ cudaError_t launch_w4a8_gemm(const int8_t* xq, const float* sx, const int32_t* x
                              const float* bias, int64_t N, uint16_t* y, void* scratch, bool pdl,
                              cudaStream_t s);
 
+// The prepared form of a weight for the GEMM route (the layout of
+// w4a8_plane_scratch_bytes(N, K)): the count and build once, with a fixed
+// epoch, after zeroing the words.  With `planes` non-null, synchronizes `s`
+// and writes the plane count (1..3, or 255: the per-group fold computes).
+cudaError_t launch_w4a8_prepare(const uint8_t* Wp, const uint16_t* ws, const uint16_t* wo,
+                                int64_t N, int64_t K, void* prepared, int* planes,
+                                cudaStream_t s);
+
+// The GEMM route on a prepared weight: the gated per-group fold and the plane
+// GEMM (two launches).
+cudaError_t launch_w4a8_gemm_prepared(const int8_t* xq, const float* sx, const int32_t* xsum,
+                                      int64_t M, int64_t K, const uint8_t* Wp,
+                                      const uint16_t* ws, const uint16_t* wo,
+                                      const void* prepared, const float* bias, int64_t N,
+                                      uint16_t* y, bool pdl, cudaStream_t s);
+
 // W4A8 weight-streaming GEMV (M <= 16; its per-CTA working set -- the weight
 // slice of R rows x one K slice, xq, scales -- must fit shared memory, see
 // gemv_fits); per-group accumulator dump as above.
