@@ -33,25 +33,35 @@
 //    maximum, or 255 when some row needs more than 3 bytes or holds a
 //    non-finite value) goes into a 64-bit word as (epoch << 8) | P, with the
 //    launch's epoch (a value never reused): a word of another epoch is
-//    replaced, one of this epoch raised, so the word needs no clearing;
-//  * w4a8_plane_build_kernel: memory-bound; writes the P digit planes of every
-//    weight row to the scratch as rows n P + p of [P N, K] int8 (one thread per
-//    16 codes: 8 packed bytes in, P 16-byte stores out);
+//    replaced, one of this epoch raised, so the word needs no clearing.  A row
+//    that needs three digits also claims one of 8 slots in its block of 60
+//    rows (the same epoch-tagged words); a block with more sets an overflow
+//    word;
+//  * w4a8_plane_build_kernel: memory-bound; writes the digit rows of every
+//    weight row to the scratch (one thread per 16 codes: 8 packed bytes in,
+//    16-byte stores out): uniform layout, the P digit rows of row n at n P + p;
+//    mixed layout (P = 3 without overflow), the two low digit rows of every row
+//    at 2 n + p and the top digit of a three-digit row at 2 N + 8 (n / 60) +
+//    its slot (2.13 digit rows per weight row on average instead of 3);
 //  * (the per-group fold kernel of gemm_w4a8.cu, gated by the same word: it
 //    computes only when P > 3);
-//  * w4a8_planes_kernel: the W8A8 GEMM's structure on those planes -- CTA pairs
+//  * w4a8_planes_kernel: the W8A8 GEMM's structure on those rows -- CTA pairs
 //    (clusters of 2) run tcgen05.mma.cta_group::2 kind::i8 with M = 256 rows of
-//    xq and N = P R plane rows (R = 256 / P weight rows; 64 for P = 3), both
-//    operands loaded by TMA into a 6-stage ring, one MMA covering every plane
-//    so that a row's P sums sit in adjacent accumulator columns; two epilogue
+//    xq and N = 256 digit rows (uniform: 256 / P weight rows, 64 for P = 3;
+//    mixed: 120 weight rows, each CTA's half holding its 60 rows' low digits
+//    and its 8 top-digit rows), both operands loaded by TMA into a 5-stage
+//    ring, one MMA covering every digit row of the tile; two epilogue
 //    warpgroups, one per TMEM accumulator (so consecutive tiles drain in
-//    parallel), tcgen05.ld the P sums of 16 outputs at a time, form Y exactly
-//    (int64), and round y = sx 2^e_n Y + bias once to bf16: in fp32 where a
-//    bound proves the result on the same side of the bf16 rounding midpoint as
-//    the exact value (so the bits are the exact value's), in fp64 otherwise;
-//    TMA stores that clip the edges write y.
+//    parallel), tcgen05.ld the digit sums of 16 outputs at a time and round
+//    y = sx 2^e_n Y + bias once to bf16: in fp32 where an error bound proves
+//    that v - err and v + err round to the same bf16 value (which is then the
+//    exact value's), else Y in int64 and one fp64 fused multiply-add for the
+//    pair of outputs; TMA stores that clip the edges write y.
 //    The plane GEMM does nothing unless the word holds 1..3 planes of this
 //    launch's epoch.
+// A prepared weight (qk_w4a8_prepare) runs the count and the build once, into
+// caller-owned memory with a fixed epoch after zeroing its words; its products
+// then run the gated fold and the plane GEMM only.
 // (Building the planes inside the GEMM was measured and not kept: a transform
 // split over the pair needs a cluster-scope handoff per stage, about a
 // microsecond of release and acquire, and one done by the issuing CTA alone
