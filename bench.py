@@ -789,7 +789,12 @@ def run_ours(args, world, rank, local):
     if single and args.workload == "dit_mlp" and not args.no_workloads:
         workloads = {}
         for name in TABLE:
-            workloads[name] = table_entry(name, local, dev, peaks, int8)
+            try:
+                workloads[name] = table_entry(name, local, dev, peaks, int8)
+            except Exception as exc:  # reported in the line; the headline stands
+                workloads[name] = {"error": f"{type(exc).__name__}: {exc}"}
+                torch.cuda.empty_cache()
+                continue
             for k in [k for k in workloads[name] if k.startswith("_")]:
                 del workloads[name][k]
 
