@@ -104,3 +104,21 @@ def test_traffic_lookup_follows_the_source_hash(tmp_path):
         other = tmp_path / src
         other.write_bytes(open(path, "rb").read() + b"\n// edited\n")
         assert bench.traffic_from_profile(tag, str(other), workload) is None
+
+
+def test_launch_counts_per_call():
+    """The launches a W4A8 call makes follow its plan: the GEMM route is the
+    quantization kernel, the plane count, the plane build, the gated fold and
+    the plane GEMM (5), on a prepared weight 3; W8A8 is the quantization
+    kernel + the GEMM."""
+    from w4a8_quantized_gemm_token_b200 import build
+
+    build.build()
+    from w4a8_quantized_gemm_token_b200 import binding as qk
+
+    assert bench.is_prepared("w4a8_m4096_prepared") and not bench.is_prepared("w4a8_m4096")
+    assert all(bench.is_w4(n) for n in bench.WORKLOADS if bench.is_prepared(n))
+    assert bench.launches_per_call(4096, 4096, 4096, True, False, qk) == 5
+    assert bench.launches_per_call(4096, 4096, 4096, True, False, qk, prepared=True) == 3
+    assert bench.launches_per_call(16384, 3072, 12288, False, False, qk) == 2
+    assert bench.launches_per_call(1, 4096, 4096, True, False, qk) == 1   # the GEMV quantizing x
