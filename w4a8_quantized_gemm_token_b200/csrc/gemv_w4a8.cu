@@ -38,7 +38,9 @@
 //    order: the quantized rows arrive by bulk copies issued by one thread.
 //  * Per-group sums fold into fp64 (exact int -> fp64 by the 2^52 magic
 //    number).  With one token the lanes first gather one group each by
-//    shuffles, so no lane folds an all-zero token column.
+//    shuffles, so no lane folds an all-zero token column.  When the kernel
+//    quantizes x itself (up to 8 tokens), the fp16 scales and offsets are
+//    first widened into an fp64 table before the dependency wait.
 //  * The partial sums of all warps of all CTAs of a cluster go, through
 //    distributed shared memory, to the CTA that owns the row (R / C rows
 //    each), which adds them in a fixed order (deterministic), applies sx and
