@@ -38,6 +38,13 @@ def test_library_exports_every_declared_symbol(qk):
         assert hasattr(qk.lib, n), n
 
 
+def test_binding_types_every_declared_call(qk):
+    """Every declared call has its argument and result types set in the binding
+    (ctypes would otherwise pass 64-bit sizes as C ints)."""
+    for n in declared_functions():
+        assert n in qk._SIGS, n
+
+
 def test_status_strings(qk):
     for s in range(8):
         assert qk.qk_status_string(s).startswith("QK_")

@@ -36,6 +36,7 @@ _SIGS = {
     "qk_w8a8_linear_fused": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w8a8_gemm": (_I, [_P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P]),
     "qk_w8a8_linear_gated": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "qk_w8a8_linear_noalloc": (_I, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P]),
     "qk_w4a8_linear": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "qk_w4a8_gemm": (_I, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I, _P]),
     "qk_w4a8_linear_plan": (_I, [_I64, _I64, _I64]),
@@ -230,6 +231,23 @@ def qk_w8a8_gemm(xq, sx, Wq, sw, bias=None, y=None, stream=None):
     y = _out(y, (M, N), torch.bfloat16, xq.device, "y")
     _check(lib.qk_w8a8_gemm(_ptr(xq), _ptr(sx), M, K, _ptr(Wq), _ptr(sw), _ptr(bias), N, _ptr(y),
                             _stream(stream)), "qk_w8a8_gemm")
+    return y
+
+
+def qk_w8a8_linear_noalloc(x, Wq, sw, bias=None, y=None, stream=None):
+    """The W8A8 linear on the library's per-device scratch (no allocation per
+    call; calls must not overlap on the device, see include/qk.h)."""
+    _need(x, torch.bfloat16, 2, "x")
+    _need(Wq, torch.int8, 2, "Wq")
+    _need(sw, torch.float32, 1, "sw")
+    if bias is not None:
+        _need(bias, torch.float32, 1, "bias")
+    M, K = x.shape
+    N = Wq.shape[0]
+    y = _out(y, (M, N), torch.bfloat16, x.device, "y")
+    _check(lib.qk_w8a8_linear_noalloc(_ptr(x), M, K, _ptr(Wq), _ptr(sw), _ptr(bias), N, _ptr(y),
+                                      _stream(stream)),
+           "qk_w8a8_linear_noalloc")
     return y
 
 
