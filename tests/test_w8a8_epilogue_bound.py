@@ -108,3 +108,50 @@ def test_extremes():
              (3, Fraction(2) ** -126, Fraction(1), f32(Fraction(2) ** -110))]
     for acc, sx, sw, bias in cases:
         check(acc, f32(sx), f32(sw), bias)
+
+
+GUARD_GATE = Fraction(1, 2 ** 13)
+
+
+def gated_fast_path(acc, sx, sw, bias, gate, res):
+    """The gated epilogue's fp32 sequence: u = fma(fl(fl(acc) sx), sw, bias),
+    y = fma(gate, u, residual), kept when |y| >= fma(2^-13 |gate|, |u| + |bias|,
+    2^-100) (each step one fp32 rounding)."""
+    u = fma(f32(f32(acc) * sx), sw, bias)
+    y = fma(gate, u, res)
+    if isinstance(y, float) or isinstance(u, float):
+        return False, None
+    z = fma(f32(GUARD_GATE * abs(gate)), f32(abs(u) + abs(bias)), TINY)
+    return abs(y) >= z, y
+
+
+def check_gated(acc, sx, sw, bias, gate, res):
+    kept, y32 = gated_fast_path(acc, sx, sw, bias, gate, res)
+    if kept:
+        y = gate * (acc * sx * sw + bias) + res
+        assert abs(bf16_ordinal(y32) - bf16_ordinal(y)) <= 1, (acc, sx, sw, bias, gate, res)
+    return kept
+
+
+def bf16_value(v: float) -> Fraction:
+    return round_binary(Fraction(float(v)), 8, -126, 127)
+
+
+def test_gated_outputs():
+    """The gated residual epilogue y = residual + gate (acc sx sw + bias):
+    random outputs and residuals that cancel most of the update."""
+    rng = np.random.default_rng(14)
+    kept = 0
+    for i in range(4000):
+        acc = int(rng.normal(0, 64 * 40 * 40))
+        sx, sw = rand_scales(rng)
+        u = acc * sx * sw
+        bias = f32(Fraction(float(rng.normal(0, 1))) * (abs(u) or Fraction(1)))
+        gate = f32(Fraction(float(rng.normal(0, 0.5))))
+        if i % 2:
+            res = bf16_value(float(rng.normal(0, 1)) * float(abs(u + bias) or 1))
+        else:  # the residual cancels the update to a small relative remainder
+            rel = Fraction(float(rng.uniform(-1, 1))) * Fraction(2) ** int(rng.integers(-20, 0))
+            res = bf16_value(float(-gate * (u + bias) * (1 + rel)))
+        kept += check_gated(acc, sx, sw, bias, gate, res)
+    assert kept > 2000
